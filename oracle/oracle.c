@@ -1,0 +1,318 @@
+/*
+ * oracle.c -- fp64 CPU oracle for batched decode attention over a paged
+ * KV cache, for the page-append scatter, and for the merge of partial
+ * attention states.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load or call this code.  The CUDA
+ * library never links, includes or calls it, and it shares no source with
+ * the CUDA library: the two meet only through the seeded inputs.
+ *
+ * What it computes (every function below cites the passage it follows):
+ *
+ *   decode: for request b and query head h, the exact single-row attention
+ *     o = softmax(scale * q K^T) V,   lse = log(sum_t exp(scale * q.k_t)),
+ *     with K, V the request's cached keys/values gathered in logical order
+ *     through the page table.  This is the standard attention formula
+ *     Attention(Q,K,V) = softmax(QK^T/sqrt(d))V ("大模型推理极致优化：
+ *     FlashAttention+PageAttention联合调优", section 2.1) restricted to one
+ *     query row; FlashAttention is stated there (section 1 and 2.2) to be
+ *     mathematically equivalent to it, so the oracle is the definition
+ *     written out, not the tiled algorithm.
+ *
+ *   append: the integer scatter of new tokens into the page slots their
+ *     logical positions map to (page = position / page_size through the
+ *     page table, "Flash Attention与Paged KV Cache优化大模型推理实战",
+ *     section 3.2, and on-demand page allocation, "大模型推理极致优化：
+ *     FlashAttention+PageAttention联合调优", section 3.2).
+ *
+ *   merge: combining attention states of disjoint key sets by their
+ *     log-sum-exp weights -- the exact form of the blockwise combination
+ *     that "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署"
+ *     section 4.2 sketches (that sketch averages per-block softmax
+ *     outputs, which is not exact; this oracle uses the exact weights).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - pool layout pool[page][K=0|V=1][kv_head][slot][dim], one pool per layer;
+ *   - query head h reads KV head h / (Hq/Hkv) (consecutive query heads share);
+ *   - page table in CSR form: page_indptr[B+1], page_indices[], and
+ *     last_page_len[B]; request b holds (np-1)*page_size + last_page_len[b]
+ *     tokens when it owns np > 0 pages, and 0 tokens otherwise;
+ *   - a request with no tokens yields o = 0 and lse = -inf;
+ *   - lse is the natural-log log-sum-exp of the scaled scores.
+ *
+ * Precision: the 16-bit stored values (fp16 or bf16) are widened to double
+ * exactly; all arithmetic is in double.  Slots past a request's length are
+ * never read (they may hold anything, including NaN).
+ *
+ * Parallelism: OpenMP over independent (request, head) rows only; each row
+ * is computed by one thread in a fixed order, so results do not depend on
+ * the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_F16 = 0, ORACLE_BF16 = 1 };
+
+/* Status codes: 0 ok, otherwise the table or arguments break an invariant
+ * that the pages state (valid length within a page, page ids inside the
+ * pool: "Flash Attention与Paged KV Cache优化大模型推理实战", section 6.2). */
+enum {
+  ORACLE_OK = 0,
+  ORACLE_BAD_ARG = 1,
+  ORACLE_BAD_INDPTR = 2,
+  ORACLE_BAD_LAST_LEN = 3,
+  ORACLE_BAD_PAGE_ID = 4,
+  ORACLE_BAD_APPEND = 5,
+  ORACLE_NO_MEMORY = 6
+};
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* Exact widening of a stored bf16 value: bf16 is the top half of an IEEE
+ * binary32, so shifting it into the high bits gives the same number. */
+static double widen_bf16(uint16_t bits) {
+  uint32_t u = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Exact widening of a stored IEEE binary16 value, from its definition:
+ * sign, 5-bit exponent with bias 15, 10-bit fraction, subnormals at e=0. */
+static double widen_f16(uint16_t bits) {
+  int sign = (bits >> 15) & 1;
+  int e = (bits >> 10) & 0x1f;
+  int frac = bits & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)frac, -24);               /* frac * 2^-10 * 2^-14 */
+  } else if (e == 31) {
+    v = frac ? NAN : INFINITY;
+  } else {
+    v = ldexp((double)(frac | 0x400), e - 25);  /* (1 + frac/1024) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+static double widen(uint16_t bits, int dtype) {
+  return dtype == ORACLE_BF16 ? widen_bf16(bits) : widen_f16(bits);
+}
+
+/* Tokens held by request b under the CSR page table.  Returns -1 when the
+ * table breaks an invariant. */
+static int64_t request_len(int b, int page_size, const int32_t* page_indptr,
+                           const int32_t* last_page_len, int* why) {
+  int64_t np = (int64_t)page_indptr[b + 1] - (int64_t)page_indptr[b];
+  if (page_indptr[b] < 0 || np < 0) { *why = ORACLE_BAD_INDPTR; return -1; }
+  if (np == 0) return 0;
+  if (last_page_len[b] < 1 || last_page_len[b] > page_size) {
+    *why = ORACLE_BAD_LAST_LEN;
+    return -1;
+  }
+  return (np - 1) * (int64_t)page_size + last_page_len[b];
+}
+
+/* Element offset of (page, kv, head, slot, dim 0) in the pool. */
+static size_t pool_offset(int64_t page, int kv, int head, int64_t slot,
+                          int num_kv_heads, int page_size, int head_dim) {
+  return ((((size_t)page * 2 + (size_t)kv) * (size_t)num_kv_heads + (size_t)head) *
+              (size_t)page_size + (size_t)slot) * (size_t)head_dim;
+}
+
+/* Validate the whole table once (so worker threads never fail midway). */
+static int check_table(int64_t num_pages, int page_size, int batch,
+                       const int32_t* page_indptr, const int32_t* page_indices,
+                       const int32_t* last_page_len) {
+  for (int b = 0; b < batch; ++b) {
+    int why = ORACLE_OK;
+    if (request_len(b, page_size, page_indptr, last_page_len, &why) < 0) return why;
+    for (int32_t i = page_indptr[b]; i < page_indptr[b + 1]; ++i) {
+      if (page_indices[i] < 0 || (int64_t)page_indices[i] >= num_pages) return ORACLE_BAD_PAGE_ID;
+    }
+  }
+  return ORACLE_OK;
+}
+
+/*
+ * oracle_decode -- exact decode attention, one query token per request.
+ *
+ * q        [batch][num_qo_heads][head_dim]   16-bit stored values
+ * pool     [num_pages][2][num_kv_heads][page_size][head_dim]   16-bit
+ * out      [batch][num_qo_heads][head_dim]   double, written
+ * lse      [batch][num_qo_heads]             double, written (natural log)
+ *
+ * For each (b, h): s_t = scale * sum_d q[d] K[t][d]; m = max_t s_t;
+ * l = sum_t exp(s_t - m); o[d] = sum_t exp(s_t - m) V[t][d] / l;
+ * lse = m + log(l).  Subtracting m changes nothing mathematically (the
+ * factor exp(-m) cancels between numerator and l); it only keeps exp()
+ * in range.
+ */
+int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
+                  int64_t num_pages, int page_size, int num_kv_heads, int head_dim,
+                  int batch, int num_qo_heads,
+                  const int32_t* page_indptr, const int32_t* page_indices,
+                  const int32_t* last_page_len, double scale,
+                  double* out, double* lse) {
+  if (batch < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1 ||
+      num_qo_heads < num_kv_heads || num_qo_heads % num_kv_heads != 0 ||
+      (dtype != ORACLE_F16 && dtype != ORACLE_BF16))
+    return ORACLE_BAD_ARG;
+  int rc = check_table(num_pages, page_size, batch, page_indptr, page_indices, last_page_len);
+  if (rc != ORACLE_OK) return rc;
+  const int group = num_qo_heads / num_kv_heads;
+  const int64_t rows = (int64_t)batch * num_qo_heads;
+  int failed = 0;
+
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t row = 0; row < rows; ++row) {
+    const int b = (int)(row / num_qo_heads);
+    const int h = (int)(row % num_qo_heads);
+    const int g = h / group;
+    int why = ORACLE_OK;
+    const int64_t len = request_len(b, page_size, page_indptr, last_page_len, &why);
+    double* o = out + (size_t)row * head_dim;
+    if (len == 0) {
+      for (int d = 0; d < head_dim; ++d) o[d] = 0.0;
+      lse[row] = -INFINITY;
+      continue;
+    }
+    double* qd = (double*)malloc(sizeof(double) * (size_t)head_dim);
+    double* s = (double*)malloc(sizeof(double) * (size_t)len);
+    if (!qd || !s) {
+      free(qd); free(s);
+#pragma omp atomic write
+      failed = 1;
+      continue;
+    }
+    for (int d = 0; d < head_dim; ++d) qd[d] = widen(q[(size_t)row * head_dim + d], dtype);
+
+    /* scores, in logical token order */
+    for (int64_t t = 0; t < len; ++t) {
+      const int64_t page = page_indices[page_indptr[b] + t / page_size];
+      const uint16_t* k = pool + pool_offset(page, 0, g, t % page_size,
+                                             num_kv_heads, page_size, head_dim);
+      double dot = 0.0;
+      for (int d = 0; d < head_dim; ++d) dot += qd[d] * widen(k[d], dtype);
+      s[t] = scale * dot;
+    }
+    double m = -INFINITY;
+    for (int64_t t = 0; t < len; ++t) if (s[t] > m) m = s[t];
+
+    double l = 0.0;
+    for (int d = 0; d < head_dim; ++d) o[d] = 0.0;
+    for (int64_t t = 0; t < len; ++t) {
+      const double w = exp(s[t] - m);
+      const int64_t page = page_indices[page_indptr[b] + t / page_size];
+      const uint16_t* v = pool + pool_offset(page, 1, g, t % page_size,
+                                             num_kv_heads, page_size, head_dim);
+      l += w;
+      for (int d = 0; d < head_dim; ++d) o[d] += w * widen(v[d], dtype);
+    }
+    for (int d = 0; d < head_dim; ++d) o[d] /= l;
+    lse[row] = m + log(l);
+    free(qd);
+    free(s);
+  }
+  return failed ? ORACLE_NO_MEMORY : ORACLE_OK;
+}
+
+/*
+ * oracle_append -- scatter new tokens into their pages (in place).
+ *
+ * The table passed is the table AFTER the append: the caller has already
+ * allocated any page the new tokens need.  Request b appends the
+ * n_b = append_indptr[b+1] - append_indptr[b] rows
+ * k_new/v_new[append_indptr[b] + i] (i < n_b, each [num_kv_heads][head_dim])
+ * at logical positions len_b - n_b + i, where len_b is its length after the
+ * append.  Position p lives in page page_indices[page_indptr[b] + p / page_size]
+ * at slot p % page_size.  Pure copies of the 16-bit patterns; every other
+ * byte of the pool is left as it was.
+ */
+int oracle_append(uint16_t* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                  int head_dim, int batch,
+                  const int32_t* page_indptr, const int32_t* page_indices,
+                  const int32_t* last_page_len,
+                  const uint16_t* k_new, const uint16_t* v_new,
+                  const int32_t* append_indptr) {
+  if (batch < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1) return ORACLE_BAD_ARG;
+  int rc = check_table(num_pages, page_size, batch, page_indptr, page_indices, last_page_len);
+  if (rc != ORACLE_OK) return rc;
+  if (append_indptr[0] < 0) return ORACLE_BAD_APPEND;
+  for (int b = 0; b < batch; ++b) {
+    int why = ORACLE_OK;
+    const int64_t len = request_len(b, page_size, page_indptr, last_page_len, &why);
+    const int64_t n_new = (int64_t)append_indptr[b + 1] - append_indptr[b];
+    if (n_new < 0 || n_new > len) return ORACLE_BAD_APPEND;
+  }
+  const size_t row = (size_t)num_kv_heads * (size_t)head_dim;
+  for (int b = 0; b < batch; ++b) {
+    int why = ORACLE_OK;
+    const int64_t len = request_len(b, page_size, page_indptr, last_page_len, &why);
+    const int64_t n_new = (int64_t)append_indptr[b + 1] - append_indptr[b];
+    for (int64_t i = 0; i < n_new; ++i) {
+      const int64_t pos = len - n_new + i;
+      const int64_t page = page_indices[page_indptr[b] + pos / page_size];
+      const int64_t slot = pos % page_size;
+      const size_t src = ((size_t)append_indptr[b] + (size_t)i) * row;
+      for (int h = 0; h < num_kv_heads; ++h) {
+        memcpy(pool + pool_offset(page, 0, h, slot, num_kv_heads, page_size, head_dim),
+               k_new + src + (size_t)h * head_dim, sizeof(uint16_t) * (size_t)head_dim);
+        memcpy(pool + pool_offset(page, 1, h, slot, num_kv_heads, page_size, head_dim),
+               v_new + src + (size_t)h * head_dim, sizeof(uint16_t) * (size_t)head_dim);
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+/*
+ * oracle_merge -- combine S attention states per (row, head).
+ *
+ * v [rows][S][H][D] are normalised partial outputs, s [rows][S][H] their
+ * natural-log log-sum-exp values.  With M = max_j s_j and w_j = exp(s_j - M):
+ *   v_out = sum_j w_j v_j / sum_j w_j,   s_out = M + log(sum_j w_j).
+ * A state with s = -inf has weight 0; if every state has s = -inf the
+ * result is v_out = 0, s_out = -inf (the value of attention over no keys).
+ */
+void oracle_merge(const double* v, const double* s, int64_t rows, int num_states,
+                  int num_heads, int head_dim, double* v_out, double* s_out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int h = 0; h < num_heads; ++h) {
+      double m = -INFINITY;
+      for (int j = 0; j < num_states; ++j) {
+        const double sj = s[((size_t)r * num_states + j) * num_heads + h];
+        if (sj > m) m = sj;
+      }
+      double* o = v_out + ((size_t)r * num_heads + h) * head_dim;
+      for (int d = 0; d < head_dim; ++d) o[d] = 0.0;
+      if (m == -INFINITY) {
+        s_out[(size_t)r * num_heads + h] = -INFINITY;
+        continue;
+      }
+      double wsum = 0.0;
+      for (int j = 0; j < num_states; ++j) {
+        const double sj = s[((size_t)r * num_states + j) * num_heads + h];
+        if (sj == -INFINITY) continue;           /* weight exactly 0 */
+        const double w = exp(sj - m);
+        const double* vj = v + (((size_t)r * num_states + j) * num_heads + h) * head_dim;
+        wsum += w;
+        for (int d = 0; d < head_dim; ++d) o[d] += w * vj[d];
+      }
+      for (int d = 0; d < head_dim; ++d) o[d] /= wsum;
+      s_out[(size_t)r * num_heads + h] = m + log(wsum);
+    }
+  }
+}
