@@ -1,0 +1,234 @@
+/*
+ * pkv.h -- C ABI of libpkv: batched decode attention over a paged KV cache
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation (PagedAttention computed FlashAttention-style):
+ *   For each request b and query head h, one new query token q[b][h][:]
+ *   attends over the request's cached keys and values:
+ *       o[b][h] = softmax(sm_scale * q K^T) V,   lse[b][h] = log sum_t exp(sm_scale * q.k_t)
+ *   which is the standard attention Attention(Q,K,V) = softmax(QK^T/sqrt(d))V
+ *   ("大模型推理极致优化：FlashAttention+PageAttention联合调优", section 2.1)
+ *   for one query row.  K and V sit in fixed-size physical pages reached
+ *   through a per-request page table ("上下文窗口优化实战：如何用PagedAttention+FlashInfer
+ *   将Llama3-70B的128K上下文吞吐提升3.8倍？", chapter 1 and section 2.3: the decode
+ *   kernel takes the page table and the block size directly).  Scores are
+ *   never written to memory: softmax is computed online over blocks of keys
+ *   ("大模型推理极致优化：FlashAttention+PageAttention联合调优", section 2.2).
+ *
+ * Memory layout (all arrays are the caller's, row-major, on the device
+ * unless a name ends in _h):
+ *   pool            [num_pages][2][num_kv_heads][page_size][head_dim]  fp16/bf16
+ *                   index 0 of the second axis holds K, index 1 holds V.
+ *   page_indptr     int32 [batch+1]   request b owns page_indices[page_indptr[b] ..
+ *                                     page_indptr[b+1]) in logical order
+ *   page_indices    int32 [page_indptr[batch]]   physical page ids in [0, num_pages)
+ *   last_page_len   int32 [batch]     tokens in the request's last page, in
+ *                                     [1, page_size] when it owns a page
+ *   The request holds len_b = (np_b - 1) * page_size + last_page_len[b] tokens,
+ *   np_b = page_indptr[b+1] - page_indptr[b]; len_b = 0 when np_b = 0.  The
+ *   same physical page may appear in several requests (a shared prefix).
+ *   q, out          [batch][num_qo_heads][head_dim], same 16-bit type as the pool
+ *   lse             float [batch][num_qo_heads], natural log
+ *   Query head h reads KV head h / (num_qo_heads / num_kv_heads).
+ *
+ * Ownership and errors: the library allocates no memory and never
+ * synchronises the stream (except pkv_read_error_word).  Every call checks
+ * its scalar arguments on the host and returns a status without launching
+ * when they are invalid; pkv_last_error() then describes the problem.
+ * Table CONTENTS live on the device and are checked by the kernels: a bad
+ * page id, indptr or last_page_len sets a bit in the optional caller-owned
+ * device word `error_word` (PKV_DEVERR_*), the offending page or request is
+ * skipped, and the kernel still completes.  No kernel traps or waits without
+ * a time limit; a wait that runs past its limit sets PKV_DEVERR_TIMEOUT.
+ * `stream` is a cudaStream_t (NULL = the legacy default stream).
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PKV_API __attribute__((visibility("default")))
+#else
+#define PKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1,   /* a scalar argument or pointer is invalid */
+  PKV_ERR_UNSUPPORTED = 2,   /* valid, but outside what the kernels implement */
+  PKV_ERR_WORKSPACE = 3,     /* workspace too small or misaligned */
+  PKV_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  PKV_ERR_DEVICE = 5         /* pkv_read_error_word found device error bits */
+} pkv_status;
+
+typedef enum pkv_dtype {
+  PKV_F16 = 0,
+  PKV_BF16 = 1,
+  PKV_F32 = 2                /* only as the output type of pkv_merge_states */
+} pkv_dtype;
+
+/* Bits the kernels OR into *error_word. */
+#define PKV_DEVERR_PAGE_ID   0x01  /* page id outside [0, num_pages): page skipped */
+#define PKV_DEVERR_INDPTR    0x02  /* page_indptr decreasing or negative: request treated as empty */
+#define PKV_DEVERR_LAST_LEN  0x04  /* last_page_len outside [1, page_size]: request treated as empty */
+#define PKV_DEVERR_APPEND    0x08  /* append_indptr malformed or more new tokens than the request holds */
+#define PKV_DEVERR_TIMEOUT   0x10  /* an internal wait ran past its time limit; outputs invalid */
+
+/* Human-readable name of a status code (static string). */
+PKV_API const char* pkv_status_string(int status);
+
+/* Detail of the last non-OK status returned on this host thread ("" if none). */
+PKV_API const char* pkv_last_error(void);
+
+/* Number of split-KV partitions pkv_decode uses when num_partitions = 0 on
+ * `device`: one persistent CTA per SM.  Returns a value < 0 on error. */
+PKV_API int pkv_default_partitions(int device);
+
+/*
+ * Workspace bytes pkv_decode needs for these shapes and this partition
+ * count (num_partitions = 0 means pkv_default_partitions(current device)).
+ * The workspace holds one arrival counter per partition and at most two
+ * partial (o, lse) states per partition.  It must be 256-byte aligned and
+ * ZERO-FILLED before its first use; pkv_decode leaves the counters at zero
+ * when it returns, so the same workspace can be reused by later calls on
+ * the same stream without clearing.  Returns 0 for invalid shapes.
+ */
+PKV_API size_t pkv_decode_workspace_bytes(int batch, int num_qo_heads, int num_kv_heads,
+                                  int head_dim, int num_partitions);
+
+/*
+ * pkv_append -- scatter new tokens' K and V into their pages
+ * (a1 of the decode step: pages are allocated on demand by the caller,
+ * "大模型推理极致优化：FlashAttention+PageAttention联合调优" section 3.2;
+ * position p of a request lives at page page_indices[page_indptr[b] + p / page_size],
+ * slot p % page_size, "Flash Attention与Paged KV Cache优化大模型推理实战" section 3.2).
+ *
+ *   pool                the KV pool (written in place)
+ *   page_indptr, page_indices, last_page_len, batch
+ *                       the page table AFTER the append (pages already allocated)
+ *   k_new, v_new        [nnz_new][num_kv_heads][head_dim] in the pool's dtype
+ *   append_indptr       int32 [batch+1]; request b appends rows
+ *                       append_indptr[b] .. append_indptr[b+1]) at its last
+ *                       n_b positions: len_b - n_b + i
+ *   nnz_new             append_indptr[batch] (rows in k_new / v_new)
+ * Bit-exact copies; no other byte of the pool changes.  head_dim must be a
+ * multiple of 8 and all data pointers 16-byte aligned.
+ */
+PKV_API pkv_status pkv_append(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                      int head_dim, int dtype,
+                      const int32_t* page_indptr, const int32_t* page_indices,
+                      const int32_t* last_page_len, int batch,
+                      const void* k_new, const void* v_new, const int32_t* append_indptr,
+                      int64_t nnz_new, int32_t* error_word, void* stream);
+
+/*
+ * pkv_decode -- batched decode attention over the paged KV cache.
+ *
+ *   q                [batch][num_qo_heads][head_dim], dtype = pool dtype, 16-byte aligned
+ *   pool, num_pages, page_size, num_kv_heads, head_dim, dtype
+ *                    the KV pool (16-byte aligned); head_dim must be 128,
+ *                    page_size one of 16, 32, 64, 128, 256,
+ *                    num_qo_heads / num_kv_heads (the GQA group) in 1..8
+ *   page_indptr, page_indices, last_page_len, batch   the page table (device)
+ *   sm_scale         score scale (1/sqrt(head_dim) for standard attention)
+ *   num_partitions   split-KV partitions, 0 = pkv_default_partitions().  The
+ *                    flattened work (request, kv head, 16-token tile) is cut
+ *                    into this many equal contiguous shares, one per CTA; a
+ *                    (request, kv head) cut across shares is merged exactly
+ *                    by log-sum-exp weights inside the same launch.  Results
+ *                    depend on the partition count only through fp32
+ *                    rounding; for a fixed count they are bitwise
+ *                    reproducible and independent of physical page placement.
+ *   workspace        see pkv_decode_workspace_bytes (device, zero-filled once)
+ *   out              [batch][num_qo_heads][head_dim] in dtype (must not alias q or pool)
+ *   lse              float [batch][num_qo_heads] or NULL
+ *   error_word       int32 device word for PKV_DEVERR_* bits, or NULL
+ * A request with no tokens gets out = 0 and lse = -inf.
+ */
+PKV_API pkv_status pkv_decode(const void* q, int num_qo_heads,
+                      const void* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                      int head_dim, int dtype,
+                      const int32_t* page_indptr, const int32_t* page_indices,
+                      const int32_t* last_page_len, int batch,
+                      float sm_scale, int num_partitions,
+                      void* workspace, size_t workspace_bytes,
+                      void* out, float* lse, int32_t* error_word, void* stream);
+
+/*
+ * pkv_merge_states -- merge attention states of disjoint key sets.
+ *
+ *   v       float [num_rows][num_states][num_heads][head_dim]  normalised partial outputs
+ *   s       float [num_rows][num_states][num_heads]            their natural-log lse
+ *   v_out   [num_rows][num_heads][head_dim] in out_dtype (PKV_F32, PKV_F16, PKV_BF16)
+ *   s_out   float [num_rows][num_heads] or NULL
+ * With M = max_j s_j, w_j = exp(s_j - M): v_out = sum_j w_j v_j / sum_j w_j,
+ * s_out = M + log sum_j w_j.  A state with s = -inf carries no weight; if all
+ * do, v_out = 0 and s_out = -inf.  This is the exact form of the blockwise
+ * combination sketched in "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署"
+ * section 4.2 (that sketch averages per-block softmax outputs, which is not exact).
+ */
+PKV_API pkv_status pkv_merge_states(const float* v, const float* s, int64_t num_rows, int num_states,
+                            int num_heads, int head_dim, void* v_out, int out_dtype,
+                            float* s_out, void* stream);
+
+/*
+ * pkv_read_error_word -- synchronise `stream`, copy the device error word to
+ * *value (host), and zero it on the device when `clear` is non-zero.
+ * Returns PKV_ERR_DEVICE when any bit is set, PKV_OK otherwise.
+ */
+PKV_API pkv_status pkv_read_error_word(int32_t* error_word, int32_t* value, int clear, void* stream);
+
+/*
+ * pkv_check_table -- host-side check of a page table the caller holds on the
+ * host (the consistency rules of "Flash Attention与Paged KV Cache优化大模型推理实战"
+ * section 6.2: a page's valid length never exceeds the page size; plus
+ * monotone indptr and page ids inside the pool).  No GPU needed.
+ */
+PKV_API pkv_status pkv_check_table(const int32_t* page_indptr_h, const int32_t* page_indices_h,
+                           const int32_t* last_page_len_h, int batch, int64_t num_pages,
+                           int page_size);
+
+/*
+ * pkv_plan_segments -- host mirror of the device-side split-KV partition, for
+ * inspection and tests (no GPU needed).  For the table held on the host it
+ * lists every segment the `num_partitions` CTAs of pkv_decode process, seven
+ * int64 per segment: partition, request, kv head, first tile, end tile
+ * (16-token tiles), partial-state slot (-1 when the segment covers its whole
+ * (request, kv head) and writes the output directly), partitions covering
+ * that (request, kv head).  Writes at most max_segments rows to `segments`
+ * and returns the total number of segments, or -1 on invalid arguments.
+ */
+PKV_API int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page_len_h,
+                          int batch, int page_size, int num_kv_heads, int num_partitions,
+                          int64_t* segments, int64_t max_segments);
+
+/* The same three operations under the names used in the paged-attention literature. */
+PKV_API pkv_status paged_kv_append(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                           int head_dim, int dtype,
+                           const int32_t* page_indptr, const int32_t* page_indices,
+                           const int32_t* last_page_len, int batch,
+                           const void* k_new, const void* v_new, const int32_t* append_indptr,
+                           int64_t nnz_new, int32_t* error_word, void* stream);
+PKV_API pkv_status paged_decode_attention(const void* q, int num_qo_heads,
+                                  const void* pool, int64_t num_pages, int page_size,
+                                  int num_kv_heads, int head_dim, int dtype,
+                                  const int32_t* page_indptr, const int32_t* page_indices,
+                                  const int32_t* last_page_len, int batch,
+                                  float sm_scale, int num_partitions,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* out, float* lse, int32_t* error_word, void* stream);
+PKV_API pkv_status merge_states(const float* v, const float* s, int64_t num_rows, int num_states,
+                        int num_heads, int head_dim, void* v_out, int out_dtype,
+                        float* s_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,42 @@
+"""paged_kv_cache_479_b200 -- batched decode attention over a paged KV cache on B200.
+
+A thin Python binding of libpkv (include/pkv.h).  Every function marshals
+torch tensors into the C ABI (data pointers, sizes, the current CUDA
+stream) and calls the library; all arithmetic runs in the library's CUDA
+kernels.  There is no CPU fallback: if libpkv.so is missing or cannot be
+loaded, importing the binding's functions raises.
+
+Functions (C names in parentheses):
+  paged_kv_append        (pkv_append)          scatter new tokens into pages
+  paged_decode_attention (pkv_decode)          decode attention + split-KV merge
+  merge_states           (pkv_merge_states)    merge (o, lse) states
+  decode_workspace_bytes (pkv_decode_workspace_bytes)
+  default_partitions     (pkv_default_partitions)
+  read_error_word        (pkv_read_error_word)
+  check_table            (pkv_check_table)     host-side table check
+  plan_segments          (pkv_plan_segments)   host mirror of the split-KV partition
+"""
+from ._binding import (  # noqa: F401
+    BF16,
+    F16,
+    F32,
+    PkvError,
+    check_table,
+    decode_workspace_bytes,
+    default_partitions,
+    lib,
+    merge_states,
+    paged_decode_attention,
+    paged_kv_append,
+    plan_segments,
+    read_error_word,
+    DEVERR_APPEND,
+    DEVERR_INDPTR,
+    DEVERR_LAST_LEN,
+    DEVERR_PAGE_ID,
+    DEVERR_TIMEOUT,
+)
+
+pkv_append = paged_kv_append
+pkv_decode = paged_decode_attention
+pkv_merge_states = merge_states

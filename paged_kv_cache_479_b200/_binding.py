@@ -1,0 +1,215 @@
+"""ctypes binding of libpkv.so: argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+F16, BF16, F32 = 0, 1, 2
+DEVERR_PAGE_ID = 0x01
+DEVERR_INDPTR = 0x02
+DEVERR_LAST_LEN = 0x04
+DEVERR_APPEND = 0x08
+DEVERR_TIMEOUT = 0x10
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkv.so")
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F32 = ctypes.c_float
+
+_SIGNATURES = {
+    "pkv_status_string": ([_I32], ctypes.c_char_p),
+    "pkv_last_error": ([], ctypes.c_char_p),
+    "pkv_default_partitions": ([_I32], _I32),
+    "pkv_decode_workspace_bytes": ([_I32, _I32, _I32, _I32, _I32], _SZ),
+    "pkv_append": ([_P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I32, _P, _P, _P, _I64, _P, _P], _I32),
+    "pkv_decode": ([_P, _I32, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I32, _F32, _I32,
+                    _P, _SZ, _P, _P, _P, _P], _I32),
+    "pkv_merge_states": ([_P, _P, _I64, _I32, _I32, _I32, _P, _I32, _P, _P], _I32),
+    "pkv_read_error_word": ([_P, _P, _I32, _P], _I32),
+    "pkv_check_table": ([_P, _P, _P, _I32, _I64, _I32], _I32),
+    "pkv_plan_segments": ([_P, _P, _I32, _I32, _I32, _I32, _P, _I64], _I64),
+}
+_SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
+_SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
+_SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
+
+_lib = None
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(what)
+
+
+def lib():
+    """The loaded libpkv.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_479_b200.build` "
+                "(there is no CPU fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        L = lib()
+        raise PkvError(status, f"{what}: {L.pkv_status_string(status).decode()}: "
+                               f"{L.pkv_last_error().decode()}")
+
+
+_DTYPES = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev_tensor(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+    return t
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def default_partitions(device=None) -> int:
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index or 0
+    n = lib().pkv_default_partitions(dev)
+    if n <= 0:
+        raise PkvError(4, "pkv_default_partitions failed")
+    return n
+
+
+def decode_workspace_bytes(batch: int, num_qo_heads: int, num_kv_heads: int,
+                           head_dim: int = 128, num_partitions: int = 0) -> int:
+    n = lib().pkv_decode_workspace_bytes(batch, num_qo_heads, num_kv_heads, head_dim,
+                                          num_partitions)
+    if n == 0:
+        raise PkvError(1, "pkv_decode_workspace_bytes: invalid shapes")
+    return int(n)
+
+
+def paged_kv_append(pool, page_indptr, page_indices, last_page_len, k_new, v_new,
+                    append_indptr, error_word=None, stream=None) -> None:
+    """Scatter k_new / v_new [nnz, Hkv, D] into `pool` [P, 2, Hkv, ps, D] (C: pkv_append).
+    The page table is the table after the append."""
+    _dev_tensor(pool, "pool")
+    P, two, hkv, ps, d = pool.shape
+    if two != 2:
+        raise ValueError("pool must be [P, 2, Hkv, ps, D]")
+    for name, t in (("page_indptr", page_indptr), ("page_indices", page_indices),
+                    ("last_page_len", last_page_len), ("append_indptr", append_indptr)):
+        _dev_tensor(t, name, torch.int32)
+    _dev_tensor(k_new, "k_new", pool.dtype)
+    _dev_tensor(v_new, "v_new", pool.dtype)
+    batch = last_page_len.numel()
+    st = lib().pkv_append(_ptr(pool), P, ps, hkv, d, _DTYPES[pool.dtype], _ptr(page_indptr),
+                          _ptr(page_indices), _ptr(last_page_len), batch, _ptr(k_new),
+                          _ptr(v_new), _ptr(append_indptr), k_new.shape[0], _ptr(error_word),
+                          _stream(stream, pool.device))
+    _check(st, "pkv_append")
+
+
+def paged_decode_attention(q, pool, page_indptr, page_indices, last_page_len, workspace,
+                           out=None, lse=None, sm_scale=None, num_partitions: int = 0,
+                           error_word=None, stream=None, return_lse: bool = True):
+    """Decode attention of q [B, Hq, D] over the paged pool (C: pkv_decode).
+    Returns (out [B, Hq, D] in q's dtype, lse [B, Hq] float32 or None)."""
+    _dev_tensor(q, "q", pool.dtype)
+    _dev_tensor(pool, "pool")
+    _dev_tensor(workspace, "workspace")
+    for name, t in (("page_indptr", page_indptr), ("page_indices", page_indices),
+                    ("last_page_len", last_page_len)):
+        _dev_tensor(t, name, torch.int32)
+    B, hq, d = q.shape
+    P, _, hkv, ps, dp = pool.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_decode(_ptr(q), hq, _ptr(pool), P, ps, hkv, dp, _DTYPES[pool.dtype],
+                          _ptr(page_indptr), _ptr(page_indices), _ptr(last_page_len), B, scale,
+                          num_partitions, _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
+                          _ptr(error_word), _stream(stream, q.device))
+    _check(st, "pkv_decode")
+    return out, lse
+
+
+def merge_states(v, s, out_dtype=torch.float32, v_out=None, s_out=None, stream=None,
+                 return_lse: bool = True):
+    """Merge states v [N, S, H, D] float32 with lse s [N, S, H] (C: pkv_merge_states)."""
+    _dev_tensor(v, "v", torch.float32)
+    _dev_tensor(s, "s", torch.float32)
+    N, S, H, D = v.shape
+    if v_out is None:
+        v_out = torch.empty((N, H, D), dtype=out_dtype, device=v.device)
+    if s_out is None and return_lse:
+        s_out = torch.empty((N, H), dtype=torch.float32, device=v.device)
+    st = lib().pkv_merge_states(_ptr(v), _ptr(s), N, S, H, D, _ptr(v_out), _DTYPES[v_out.dtype],
+                                _ptr(s_out), _stream(stream, v.device))
+    _check(st, "pkv_merge_states")
+    return v_out, s_out
+
+
+def read_error_word(error_word, clear: bool = True, stream=None) -> int:
+    """Synchronise and return the device error word (PKV_DEVERR_* bits)."""
+    val = ctypes.c_int32(0)
+    st = lib().pkv_read_error_word(_ptr(error_word), ctypes.byref(val), int(clear),
+                                   _stream(stream, error_word.device))
+    if st not in (0, 5):
+        _check(st, "pkv_read_error_word")
+    return int(val.value)
+
+
+def check_table(page_indptr, page_indices, last_page_len, num_pages: int, page_size: int) -> None:
+    """Host-side table check (C: pkv_check_table); raises PkvError when invalid."""
+    ip = np.ascontiguousarray(page_indptr, np.int32)
+    ix = np.ascontiguousarray(page_indices, np.int32)
+    ll = np.ascontiguousarray(last_page_len, np.int32)
+    st = lib().pkv_check_table(ip.ctypes.data_as(_P), ix.ctypes.data_as(_P) if ix.size else None,
+                               ll.ctypes.data_as(_P), len(ll), int(num_pages), int(page_size))
+    _check(st, "pkv_check_table")
+
+
+def plan_segments(page_indptr, last_page_len, page_size: int, num_kv_heads: int,
+                  num_partitions: int) -> np.ndarray:
+    """Host mirror of the decode kernel's split-KV partition (C: pkv_plan_segments).
+    Rows: partition, request, kv head, first tile, end tile, state slot (-1 =
+    direct output), partitions covering the pair."""
+    ip = np.ascontiguousarray(page_indptr, np.int32)
+    ll = np.ascontiguousarray(last_page_len, np.int32)
+    L = lib()
+    n = L.pkv_plan_segments(ip.ctypes.data_as(_P), ll.ctypes.data_as(_P), len(ll), page_size,
+                            num_kv_heads, num_partitions, None, 0)
+    if n < 0:
+        raise PkvError(1, "pkv_plan_segments: invalid arguments")
+    out = np.zeros((max(n, 1), 7), np.int64)
+    L.pkv_plan_segments(ip.ctypes.data_as(_P), ll.ctypes.data_as(_P), len(ll), page_size,
+                        num_kv_heads, num_partitions, out.ctypes.data_as(_P), n)
+    return out[:n]

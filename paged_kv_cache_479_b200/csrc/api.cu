@@ -1,0 +1,436 @@
+// api.cu -- the C ABI of libpkv (declared in include/pkv.h): host-side
+// argument checks, workspace sizing, the bulk-tensor map of the KV pool, and
+// kernel launches.  No memory is allocated and no stream is synchronised
+// here, except in pkv_read_error_word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "partition.cuh"
+#include "pkv.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+pkv_status fail(pkv_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+pkv_status ok() {
+  g_err[0] = '\0';
+  return PKV_OK;
+}
+
+pkv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+bool valid_page_size(int ps) { return ps == 16 || ps == 32 || ps == 64 || ps == 128 || ps == 256; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kDecodeHeadDim = 128;
+constexpr int kMaxGroup = 8;
+constexpr int kMaxPartitions = 1 << 20;
+
+// workspace layout: counters int32[N] | part_lse float[2N][G] | part_o float[2N][G][128]
+struct WsLayout {
+  size_t counters, part_lse, part_o, total;
+};
+
+WsLayout ws_layout(int group, int N) {
+  WsLayout w;
+  w.counters = 0;
+  w.part_lse = align_up((size_t)N * 4, 256);
+  w.part_o = w.part_lse + align_up((size_t)2 * N * group * 4, 256);
+  w.total = w.part_o + align_up((size_t)2 * N * group * kDecodeHeadDim * 4, 256);
+  return w;
+}
+
+int current_device_partitions() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return pkv_default_partitions(dev);
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void* pool;
+  long long pages;
+  int ps, hkv, dtype, device;
+  bool operator==(const MapKey& o) const {
+    return pool == o.pool && pages == o.pages && ps == o.ps && hkv == o.hkv && dtype == o.dtype &&
+           device == o.device;
+  }
+};
+
+// The pool viewed as a 4-D tensor (dim, slot, kv*Hkv + head, page), boxes of
+// [16 slots][64 dims] with 128-byte swizzle: two boxes make one tile's K or V.
+pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, int dtype,
+                           CUtensorMap* out) {
+  static std::mutex mu;
+  static MapKey keys[16];
+  static CUtensorMap maps[16];
+  static int used = 0, next = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const MapKey key{pool, pages, ps, hkv, dtype, dev};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < used; ++i)
+      if (keys[i] == key) {
+        *out = maps[i];
+        return PKV_OK;
+      }
+  }
+  auto encode = get_encode();
+  if (!encode) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  CUtensorMap m;
+  const cuuint64_t esz = 2;
+  cuuint64_t dims[4] = {(cuuint64_t)kDecodeHeadDim, (cuuint64_t)ps, (cuuint64_t)2 * hkv,
+                        (cuuint64_t)pages};
+  cuuint64_t strides[3] = {kDecodeHeadDim * esz, (cuuint64_t)ps * kDecodeHeadDim * esz,
+                           (cuuint64_t)2 * hkv * ps * kDecodeHeadDim * esz};
+  cuuint32_t box[4] = {64, (cuuint32_t)pkv::kTileTokens, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(&m,
+                      dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                      4, const_cast<void*>(pool), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    keys[next] = key;
+    maps[next] = m;
+    next = (next + 1) % 16;
+    if (used < 16) ++used;
+  }
+  *out = m;
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_string(int status) {
+  switch (status) {
+    case PKV_OK: return "PKV_OK";
+    case PKV_ERR_INVALID_ARG: return "PKV_ERR_INVALID_ARG";
+    case PKV_ERR_UNSUPPORTED: return "PKV_ERR_UNSUPPORTED";
+    case PKV_ERR_WORKSPACE: return "PKV_ERR_WORKSPACE";
+    case PKV_ERR_CUDA: return "PKV_ERR_CUDA";
+    case PKV_ERR_DEVICE: return "PKV_ERR_DEVICE";
+    default: return "PKV_ERR_UNKNOWN";
+  }
+}
+
+const char* pkv_last_error(void) { return g_err; }
+
+int pkv_default_partitions(int device) {
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return -1;
+  return sms;  // one persistent CTA per SM (the decode CTA uses ~167 KB of shared memory)
+}
+
+size_t pkv_decode_workspace_bytes(int batch, int num_qo_heads, int num_kv_heads, int head_dim,
+                                  int num_partitions) {
+  if (batch < 0 || num_kv_heads < 1 || num_qo_heads < num_kv_heads ||
+      num_qo_heads % num_kv_heads != 0 || head_dim != kDecodeHeadDim)
+    return 0;
+  const int group = num_qo_heads / num_kv_heads;
+  if (group > kMaxGroup) return 0;
+  int N = num_partitions;
+  if (N == 0) N = current_device_partitions();
+  if (N <= 0 || N > kMaxPartitions) return 0;
+  return ws_layout(group, N).total;
+}
+
+pkv_status pkv_check_table(const int32_t* page_indptr_h, const int32_t* page_indices_h,
+                           const int32_t* last_page_len_h, int batch, int64_t num_pages,
+                           int page_size) {
+  if (batch < 0 || page_size < 1 || num_pages < 0)
+    return fail(PKV_ERR_INVALID_ARG, "batch, page_size or num_pages out of range");
+  if (batch > 0 && (!page_indptr_h || !last_page_len_h))
+    return fail(PKV_ERR_INVALID_ARG, "null table pointer");
+  if (batch == 0) return ok();
+  if (page_indptr_h[0] < 0) return fail(PKV_ERR_INVALID_ARG, "page_indptr[0] < 0");
+  for (int b = 0; b < batch; ++b) {
+    const pkv::ReqInfo r = pkv::request_info(page_indptr_h, last_page_len_h, b, page_size);
+    if (r.err & pkv::kErrIndptr)
+      return fail(PKV_ERR_INVALID_ARG, "page_indptr decreases at request %d", b);
+    if (r.err & pkv::kErrLastLen)
+      return fail(PKV_ERR_INVALID_ARG, "last_page_len[%d] = %d outside [1, %d]", b,
+                  last_page_len_h[b], page_size);
+  }
+  if (page_indptr_h[batch] > 0 && !page_indices_h)
+    return fail(PKV_ERR_INVALID_ARG, "null page_indices");
+  for (int32_t i = page_indptr_h[0]; i < page_indptr_h[batch]; ++i)
+    if (page_indices_h[i] < 0 || page_indices_h[i] >= num_pages)
+      return fail(PKV_ERR_INVALID_ARG, "page_indices[%d] = %d outside [0, %lld)", i,
+                  page_indices_h[i], (long long)num_pages);
+  return ok();
+}
+
+int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page_len_h,
+                          int batch, int page_size, int num_kv_heads, int num_partitions,
+                          int64_t* segments, int64_t max_segments) {
+  if (batch < 0 || !valid_page_size(page_size) || num_kv_heads < 1 || num_partitions < 1 ||
+      num_partitions > kMaxPartitions || (batch > 0 && (!page_indptr_h || !last_page_len_h)))
+    return -1;
+  long long total = 0;
+  for (int b = 0; b < batch; ++b)
+    total += pkv::request_info(page_indptr_h, last_page_len_h, b, page_size).tiles;
+  const long long W = (long long)num_kv_heads * total;
+  if (W == 0) return 0;
+  // the kernel uses min(num_partitions, W) partitions: none of them is empty
+  const int N = W < num_partitions ? (int)W : num_partitions;
+  int64_t count = 0;
+  for (int c = 0; c < N; ++c) {
+    const long long f0 = pkv::part_start(W, N, c), f1 = pkv::part_start(W, N, c + 1);
+    if (f0 >= f1) continue;
+    // locate the request holding f0 (the device does this with a block scan)
+    long long Cb = 0;
+    int b0 = -1;
+    pkv::ReqInfo r0{};
+    for (int b = 0; b < batch; ++b) {
+      const pkv::ReqInfo r = pkv::request_info(page_indptr_h, last_page_len_h, b, page_size);
+      if (r.tiles > 0 && (long long)num_kv_heads * Cb <= f0 &&
+          f0 < (long long)num_kv_heads * (Cb + r.tiles)) {
+        b0 = b;
+        r0 = r;
+        break;
+      }
+      Cb += r.tiles;
+    }
+    if (b0 < 0) return -1;
+    pkv::Walk wk;
+    wk.indptr = page_indptr_h;
+    wk.last_len = last_page_len_h;
+    wk.B = batch;
+    wk.ps = page_size;
+    wk.Hkv = num_kv_heads;
+    wk.start(b0, Cb, r0, f0, f1);
+    while (!wk.done()) {
+      const long long n = wk.seg_tiles();
+      const pkv::SegPlace pl = pkv::seg_place(W, N, wk.pair_start(), wk.ri.tiles, c);
+      if (segments && count < max_segments) {
+        int64_t* row = segments + 7 * count;
+        row[0] = c;
+        row[1] = wk.b;
+        row[2] = wk.kvh;
+        row[3] = wk.t;
+        row[4] = wk.t + n;
+        row[5] = pl.slot;
+        row[6] = pl.ncover;
+      }
+      ++count;
+      wk.advance();
+    }
+  }
+  return count;
+}
+
+pkv_status pkv_append(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                      int head_dim, int dtype, const int32_t* page_indptr,
+                      const int32_t* page_indices, const int32_t* last_page_len, int batch,
+                      const void* k_new, const void* v_new, const int32_t* append_indptr,
+                      int64_t nnz_new, int32_t* error_word, void* stream) {
+  if (batch < 0 || nnz_new < 0 || num_pages < 0 || page_size < 1 || num_kv_heads < 1)
+    return fail(PKV_ERR_INVALID_ARG, "negative or zero size");
+  if (dtype != PKV_F16 && dtype != PKV_BF16)
+    return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
+  if (head_dim < 8 || head_dim % 8 != 0)
+    return fail(PKV_ERR_UNSUPPORTED, "append needs head_dim a positive multiple of 8");
+  if (nnz_new == 0 || batch == 0) return ok();
+  if (!pool || !page_indptr || !page_indices || !last_page_len || !k_new || !v_new ||
+      !append_indptr)
+    return fail(PKV_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(PKV_ERR_INVALID_ARG, "pool, k_new and v_new must be 16-byte aligned");
+  if (nnz_new * (int64_t)num_kv_heads > (int64_t)1 << 40)
+    return fail(PKV_ERR_UNSUPPORTED, "too many new rows");
+  pkv::AppendArgs a;
+  a.pool = pool;
+  a.indptr = page_indptr;
+  a.indices = page_indices;
+  a.last_len = last_page_len;
+  a.append_indptr = append_indptr;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.err = reinterpret_cast<int*>(error_word);
+  a.num_pages = num_pages;
+  a.nnz = nnz_new;
+  a.batch = batch;
+  a.hkv = num_kv_heads;
+  a.head_dim = head_dim;
+  a.page_size = page_size;
+  cudaError_t e = pkv::launch_append(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return ok();
+}
+
+pkv_status pkv_decode(const void* q, int num_qo_heads, const void* pool, int64_t num_pages,
+                      int page_size, int num_kv_heads, int head_dim, int dtype,
+                      const int32_t* page_indptr, const int32_t* page_indices,
+                      const int32_t* last_page_len, int batch, float sm_scale,
+                      int num_partitions, void* workspace, size_t workspace_bytes, void* out,
+                      float* lse, int32_t* error_word, void* stream) {
+  if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1)
+    return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
+  if (dtype != PKV_F16 && dtype != PKV_BF16)
+    return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
+  if (num_qo_heads % num_kv_heads != 0)
+    return fail(PKV_ERR_INVALID_ARG, "num_qo_heads must be a multiple of num_kv_heads");
+  if (head_dim != kDecodeHeadDim) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 128");
+  const int group = num_qo_heads / num_kv_heads;
+  if (group > kMaxGroup) return fail(PKV_ERR_UNSUPPORTED, "GQA group must be 1..8");
+  if (!valid_page_size(page_size))
+    return fail(PKV_ERR_UNSUPPORTED, "page_size must be 16, 32, 64, 128 or 256");
+  if (num_pages > 0x7fffffffLL) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31-1 pages");
+  if (!std::isfinite(sm_scale)) return fail(PKV_ERR_INVALID_ARG, "sm_scale is not finite");
+  if (num_partitions < 0 || num_partitions > kMaxPartitions)
+    return fail(PKV_ERR_INVALID_ARG, "num_partitions out of range");
+  if (batch == 0) return ok();
+  if (!q || !pool || !page_indptr || !page_indices || !last_page_len || !out || !workspace)
+    return fail(PKV_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(q, 16) || !aligned(pool, 16) || !aligned(out, 16))
+    return fail(PKV_ERR_INVALID_ARG, "q, pool and out must be 16-byte aligned");
+  if (out == q || out == pool) return fail(PKV_ERR_INVALID_ARG, "out aliases q or pool");
+  int N = num_partitions;
+  if (N == 0) N = current_device_partitions();
+  if (N <= 0) return fail(PKV_ERR_CUDA, "cannot query the SM count");
+  const WsLayout L = ws_layout(group, N);
+  if (!aligned(workspace, 256)) return fail(PKV_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, L.total);
+
+  CUtensorMap tmap;
+  pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, &tmap);
+  if (st != PKV_OK) return st;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pkv::DecodeArgs a;
+  a.q = q;
+  a.out = out;
+  a.lse = lse;
+  a.indptr = page_indptr;
+  a.indices = page_indices;
+  a.last_len = last_page_len;
+  a.counters = reinterpret_cast<int*>(ws + L.counters);
+  a.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
+  a.part_o = reinterpret_cast<float*>(ws + L.part_o);
+  a.err = reinterpret_cast<int*>(error_word);
+  a.num_pages = num_pages;
+  a.batch = batch;
+  a.hq = num_qo_heads;
+  a.hkv = num_kv_heads;
+  a.group = group;
+  a.page_size = page_size;
+  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  cudaError_t e = pkv::launch_decode(tmap, a, dtype == PKV_BF16, N, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
+pkv_status pkv_merge_states(const float* v, const float* s, int64_t num_rows, int num_states,
+                            int num_heads, int head_dim, void* v_out, int out_dtype,
+                            float* s_out, void* stream) {
+  if (num_rows < 0 || num_states < 1 || num_heads < 1 || head_dim < 1)
+    return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
+  if (out_dtype != PKV_F16 && out_dtype != PKV_BF16 && out_dtype != PKV_F32)
+    return fail(PKV_ERR_INVALID_ARG, "out_dtype must be PKV_F16, PKV_BF16 or PKV_F32");
+  if (num_rows == 0) return ok();
+  if (!v || !s || !v_out) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+  pkv::MergeArgs a;
+  a.v = v;
+  a.s = s;
+  a.v_out = v_out;
+  a.s_out = s_out;
+  a.rows = num_rows;
+  a.states = num_states;
+  a.heads = num_heads;
+  a.head_dim = head_dim;
+  a.out_dtype = out_dtype;
+  cudaError_t e = pkv::launch_merge(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return ok();
+}
+
+pkv_status pkv_read_error_word(int32_t* error_word, int32_t* value, int clear, void* stream) {
+  if (!error_word || !value) return fail(PKV_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(value, error_word, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  if (clear && *value) {
+    e = cudaMemsetAsync(error_word, 0, sizeof(int32_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  }
+  if (*value) return fail(PKV_ERR_DEVICE, "device error bits 0x%x", *value);
+  return ok();
+}
+
+pkv_status paged_kv_append(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                           int head_dim, int dtype, const int32_t* page_indptr,
+                           const int32_t* page_indices, const int32_t* last_page_len,
+                           int batch, const void* k_new, const void* v_new,
+                           const int32_t* append_indptr, int64_t nnz_new, int32_t* error_word,
+                           void* stream) {
+  return pkv_append(pool, num_pages, page_size, num_kv_heads, head_dim, dtype, page_indptr,
+                    page_indices, last_page_len, batch, k_new, v_new, append_indptr, nnz_new,
+                    error_word, stream);
+}
+
+pkv_status paged_decode_attention(const void* q, int num_qo_heads, const void* pool,
+                                  int64_t num_pages, int page_size, int num_kv_heads,
+                                  int head_dim, int dtype, const int32_t* page_indptr,
+                                  const int32_t* page_indices, const int32_t* last_page_len,
+                                  int batch, float sm_scale, int num_partitions,
+                                  void* workspace, size_t workspace_bytes, void* out, float* lse,
+                                  int32_t* error_word, void* stream) {
+  return pkv_decode(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
+                    page_indptr, page_indices, last_page_len, batch, sm_scale, num_partitions,
+                    workspace, workspace_bytes, out, lse, error_word, stream);
+}
+
+pkv_status merge_states(const float* v, const float* s, int64_t num_rows, int num_states,
+                        int num_heads, int head_dim, void* v_out, int out_dtype, float* s_out,
+                        void* stream) {
+  return pkv_merge_states(v, s, num_rows, num_states, num_heads, head_dim, v_out, out_dtype,
+                          s_out, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,572 @@
+// decode.cu -- batched decode attention over the paged KV cache, sm_100a.
+//
+// One persistent CTA per partition (see partition.cuh): 8 consumer warps and
+// 1 producer warp.
+//
+//  producer warp   walks the partition's (request, kv head, tile) sequence,
+//                  looks the physical page up in the page table and issues
+//                  bulk-tensor (TMA) loads of the tile's K and V
+//                  ([16 tokens][128 dims] each, two 128-byte-swizzled boxes
+//                  of 64 dims) into a 16-slot shared-memory ring guarded by
+//                  full/empty mbarriers.  This is the "load the next block
+//                  while the current one is being computed" pipeline of
+//                  "大模型推理极致优化：FlashAttention+PageAttention联合调优"
+//                  section 5.2, with the K/V of each page reached through the
+//                  page table ("上下文窗口优化实战：如何用PagedAttention+FlashInfer
+//                  将Llama3-70B的128K上下文吞吐提升3.8倍？", section 4.3 names this
+//                  gather as the decode hot spot).
+//  consumer warps  take ring slots round-robin.  Per tile, with tokens on the
+//                  MMA's M axis and the (up to 8) query heads of the GQA group
+//                  on N, one warp computes
+//                      S^T[16 x 8]  = K_tile[16 x 128] . Q_g^T   (m16n8k16, fp32 acc)
+//                  applies the online-softmax update (running max and sum in
+//                  log2 units, "大模型推理极致优化：FlashAttention+PageAttention
+//                  联合调优" section 2.2: recursive block-wise softmax), turns
+//                  P^T into the B operand of the second MMA with movmatrix,
+//                  and accumulates
+//                      O^T[128 x 8] += V_tile^T[128 x 16] . P^T[16 x 8]
+//                  so every K/V element read from HBM serves all G query
+//                  heads of its KV head (GQA reuse).  For bf16, P is split
+//                  into a bf16 high part and a bf16 remainder (two MMAs) so
+//                  the probabilities keep ~16 significant bits.
+//                  At the end of each (request, kv head) segment the 8 warps'
+//                  states are merged through shared memory (rows padded from
+//                  128 to 132 floats against bank conflicts, the padding trick of
+//                  "Flash Attention与Paged KV Cache优化大模型推理实战" section 3.1),
+//                  then either written as the final output or, when the pair
+//                  spans several partitions, as a partial (o, lse) state; the
+//                  last partition to arrive (atomic counter, no waiting)
+//                  merges the partial states by their log-sum-exp weights.
+//
+// Tokens past a request's length in its last tile are excluded by setting
+// their scores to -inf (a select, never a multiply) and zeroing their V rows
+// in shared memory, so whatever those slots hold (even NaN) never reaches
+// the output.  Every wait has a time limit; see common.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "partition.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kStages = 16;
+constexpr int kHalfBytes = kTileTokens * 64 * 2;  // one [16][64] box: 2 KiB
+constexpr int kTileBytes = 2 * kHalfBytes;        // K or V of one tile: 4 KiB
+constexpr int kSlotBytes = 2 * kTileBytes;        // K + V: 8 KiB
+constexpr int kSegRecs = 8;
+constexpr int kMaxGroup = 8;
+constexpr int kScratchStride = kD + 4;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// TileMeta bits
+constexpr int kMetaValid = 0x1f;
+constexpr int kMetaSegLast = 1 << 8;
+constexpr int kMetaEnd = 1 << 9;
+constexpr int kMetaSegShift = 12;
+
+struct SegRec {
+  int b, kvh, slot, c_first, ncover, pad;
+  long long pair_start;
+};
+
+struct __align__(16) Ctl {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t cons;                      // consumer-only barrier (256 arrivals)
+  int meta[kStages];
+  SegRec seg[kSegRecs];
+  long long warp_tot[kDecodeThreads / 32];
+  long long Cb0;
+  int b0;
+  int abort;
+  int merge_last;
+  int pad_;
+};
+
+struct Scratch {
+  float m[kConsumerWarps][kMaxGroup];
+  float l[kConsumerWarps][kMaxGroup];
+  float o[kConsumerWarps][kMaxGroup][kScratchStride];
+};
+
+constexpr size_t kRingBytes = (size_t)kStages * kSlotBytes;
+constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + sizeof(Ctl) + sizeof(Scratch);
+
+// inclusive scan over the whole block (kDecodeThreads threads); returns the
+// prefix for this thread and the block total in *total
+__device__ long long block_incl_scan(long long v, long long* warp_tot, long long* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  long long before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kDecodeThreads / 32; ++w) {
+    const long long t = warp_tot[w];
+    if (w < warp) before += t;
+    all += t;
+  }
+  __syncthreads();
+  *total = all;
+  return x + before;
+}
+
+__device__ __forceinline__ uint32_t ld_u32(const void* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+
+// all 256 consumer threads meet; bounded
+__device__ __forceinline__ bool cons_sync(Ctl& ctl, uint32_t& phase, int* err) {
+  mbar_arrive(smem_u32(&ctl.cons));
+  const bool ok = mbar_wait_bounded(smem_u32(&ctl.cons), phase, &ctl.abort, err);
+  phase ^= 1u;
+  return ok;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte-swizzled TMA boxes need 1024-byte aligned shared addresses
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* ring = smem;
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + kRingBytes);
+  Scratch& scr = *reinterpret_cast<Scratch*>(smem + kRingBytes + sizeof(Ctl));
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int c = blockIdx.x;
+  const int B = a.batch;
+  const int Hkv = a.hkv;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl.full[s]), 1);
+      mbar_init(smem_u32(&ctl.empty[s]), 32);
+    }
+    mbar_init(smem_u32(&ctl.cons), kConsumerThreads);
+    ctl.abort = 0;
+    ctl.b0 = -1;
+    fence_barrier_init();
+  }
+  if (warp == kConsumerWarps && lane == 0) prefetch_tensormap(&tmap);
+
+  // ---- prologue: total work W, this partition's share [f0, f1), its first request
+  long long mine = 0;
+  int errs = 0;
+  for (int b = tid; b < B; b += kDecodeThreads) {
+    const ReqInfo r = request_info(a.indptr, a.last_len, b, a.page_size);
+    mine += r.tiles;
+    errs |= r.err;
+  }
+  if (errs && c == 0 && a.err) atomicOr(a.err, errs);
+  long long total_tiles;
+  (void)block_incl_scan(mine, ctl.warp_tot, &total_tiles);
+  const long long W = (long long)Hkv * total_tiles;
+  // with fewer tiles than CTAs only the first W partitions get work, so that
+  // every partition that covers a (request, kv head) pair is non-empty
+  const int N = W < (long long)gridDim.x ? (int)W : (int)gridDim.x;
+  const long long f0 = c < N ? part_start(W, N, c) : 0;
+  const long long f1 = c < N ? part_start(W, N, c + 1) : 0;
+
+  long long carry = 0;
+  for (int base = 0; base < B; base += kDecodeThreads) {
+    const int b = base + tid;
+    ReqInfo r;
+    r.tiles = 0;
+    r.len = 0;
+    if (b < B) r = request_info(a.indptr, a.last_len, b, a.page_size);
+    long long chunk_total;
+    const long long incl = block_incl_scan(r.tiles, ctl.warp_tot, &chunk_total);
+    const long long excl = incl - r.tiles;
+    if (b < B && r.tiles > 0 && f0 < f1) {
+      const long long s0 = (long long)Hkv * (carry + excl), s1 = (long long)Hkv * (carry + incl);
+      if (s0 <= f0 && f0 < s1) {
+        ctl.b0 = b;
+        ctl.Cb0 = carry + excl;
+      }
+    }
+    if (b < B && r.tiles == 0 && (b % (int)gridDim.x) == c) {
+      // a request with no tokens: attention over no keys -> o = 0, lse = -inf
+      uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)b * a.hq * kD);
+      for (int k = 0; k < a.hq * kD / 8; ++k) o4[k] = make_uint4(0, 0, 0, 0);
+      if (a.lse)
+        for (int h = 0; h < a.hq; ++h) a.lse[(size_t)b * a.hq + h] = -INFINITY;
+    }
+    carry += chunk_total;
+  }
+  __syncthreads();
+  if (f0 >= f1 || ctl.b0 < 0) return;
+
+  const int G = a.group;
+
+  if (warp == kConsumerWarps) {
+    // =========================== producer ===========================
+    Walk wk;
+    wk.indptr = a.indptr;
+    wk.last_len = a.last_len;
+    wk.B = B;
+    wk.ps = a.page_size;
+    wk.Hkv = Hkv;
+    wk.start(ctl.b0, ctl.Cb0, request_info(a.indptr, a.last_len, ctl.b0, a.page_size), f0, f1);
+    uint32_t i = 0;
+    int seg = 0;
+    bool ok = true;
+    const uint32_t ring0 = smem_u32(ring);
+    while (ok && !wk.done()) {
+      const long long n = wk.seg_tiles();
+      if (n <= 0) {  // only possible if the table changed under the kernel
+        if (lane == 0) {
+          if (a.err) atomicOr(a.err, kErrIndptr);
+          ctl.abort = 1;
+        }
+        ok = false;
+        break;
+      }
+      const long long n_pad = (n + kConsumerWarps - 1) / kConsumerWarps * kConsumerWarps;
+      const long long pstart = wk.pair_start();
+      if (lane == 0) {
+        const SegPlace pl = seg_place(W, N, pstart, wk.ri.tiles, c);
+        SegRec& r = ctl.seg[seg & (kSegRecs - 1)];
+        r.b = wk.b;
+        r.kvh = wk.kvh;
+        r.slot = pl.slot;
+        r.c_first = pl.c_first;
+        r.ncover = pl.ncover;
+        r.pair_start = pstart;
+      }
+      for (long long k0 = 0; ok && k0 < n_pad; k0 += 32) {
+        const long long k = k0 + lane;
+        int page = -1, yoff = 0, valid = 0;
+        if (k < n) {
+          const long long tok0 = (wk.t + k) * kTileTokens;
+          page = a.indices[(long long)wk.ri.page_base + tok0 / a.page_size];
+          if (page < 0 || (long long)page >= a.num_pages) {
+            if (a.err) atomicOr(a.err, kErrPageId);
+            page = -1;
+          }
+          yoff = (int)(tok0 % a.page_size);
+          const long long left = wk.ri.len - tok0;
+          valid = left < kTileTokens ? (int)left : kTileTokens;
+        }
+        const int cnt = (int)((n_pad - k0) < 32 ? (n_pad - k0) : 32);
+        for (int j = 0; j < cnt; ++j) {
+          const int pg = __shfl_sync(0xffffffffu, page, j);
+          const int y = __shfl_sync(0xffffffffu, yoff, j);
+          const int v = __shfl_sync(0xffffffffu, valid, j);
+          const int s = (int)(i % kStages);
+          int okl = 1;
+          if (lane == 0) {
+            okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((i / kStages) & 1u) ^ 1u,
+                                    &ctl.abort, a.err);
+            if (okl) {
+              const int flags = ((k0 + j >= n_pad - kConsumerWarps) ? kMetaSegLast : 0) |
+                                ((seg & (kSegRecs - 1)) << kMetaSegShift);
+              const uint32_t full = smem_u32(&ctl.full[s]);
+              if (pg >= 0 && v > 0) {
+                ctl.meta[s] = v | flags;
+                mbar_arrive_expect_tx(full, kSlotBytes);
+                const uint32_t dst = ring0 + (uint32_t)s * kSlotBytes;
+                const int zk = wk.kvh, zv = Hkv + wk.kvh;
+                tma_load_4d(dst, &tmap, 0, y, zk, pg, full);
+                tma_load_4d(dst + kHalfBytes, &tmap, 64, y, zk, pg, full);
+                tma_load_4d(dst + 2 * kHalfBytes, &tmap, 0, y, zv, pg, full);
+                tma_load_4d(dst + 3 * kHalfBytes, &tmap, 64, y, zv, pg, full);
+              } else {
+                ctl.meta[s] = flags;  // no data: padding, or a skipped bad page
+                mbar_arrive(full);
+              }
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+          if (!ok) break;
+          ++i;
+        }
+      }
+      ++seg;
+      wk.advance();
+    }
+    // one end marker per consumer warp
+    for (int j = 0; ok && j < kConsumerWarps; ++j) {
+      const int s = (int)(i % kStages);
+      int okl = 1;
+      if (lane == 0) {
+        okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((i / kStages) & 1u) ^ 1u, &ctl.abort,
+                                a.err);
+        if (okl) {
+          ctl.meta[s] = kMetaEnd;
+          mbar_arrive(smem_u32(&ctl.full[s]));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+      ++i;
+    }
+    if (!ok && lane == 0) {
+      // aborted: let the copies already issued land before the CTA exits
+      const uint32_t first = i > (uint32_t)kStages ? i - kStages : 0;
+      for (uint32_t k = first; k < i; ++k) {
+        const uint32_t bar = smem_u32(&ctl.full[k % kStages]);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar, (k / kStages) & 1u) &&
+               global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+    return;
+  }
+
+  // =========================== consumers ===========================
+  const int g = lane >> 2;     // MMA row group: token g / g+8 of the tile, head g of P^T
+  const int cq = lane & 3;     // MMA column pair: heads 2cq, 2cq+1 of S^T
+  const int mi = lane >> 3;    // ldmatrix: which 8x8 matrix this lane addresses
+  const int r8 = lane & 7;     // ldmatrix: row within it
+  const float sl2 = a.scale_log2;
+  const int ct = warp * 32 + lane;
+  const uint32_t ring0 = smem_u32(ring);
+
+  uint32_t qf[8][2];
+  float o[8][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  int cur_seg = -1;
+  SegRec rec;
+  rec.b = 0;
+  rec.kvh = 0;
+  uint32_t cons_phase = 0;
+
+  for (uint32_t i = warp;; i += kConsumerWarps) {
+    const int s = (int)(i % kStages);
+    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kStages) & 1u, &ctl.abort, a.err)) break;
+    const int info = ctl.meta[s];
+    if (info & kMetaEnd) break;
+    const int sid = (info >> kMetaSegShift) & (kSegRecs - 1);
+    if (sid != cur_seg) {
+      cur_seg = sid;
+      rec = ctl.seg[sid];
+      const int h = rec.kvh * G + g;
+      if (g < G) {
+        const uint16_t* qp =
+            static_cast<const uint16_t*>(a.q) + ((size_t)rec.b * a.hq + h) * kD + 2 * cq;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          qf[j][0] = ld_u32(qp + j * 16);
+          qf[j][1] = ld_u32(qp + j * 16 + 8);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) qf[j][0] = qf[j][1] = 0u;
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+    const int valid = info & kMetaValid;
+    const uint32_t kb = ring0 + (uint32_t)s * kSlotBytes;
+    const uint32_t vb = kb + kTileBytes;
+    bool wrote_smem = false;
+    if (valid > 0) {
+      // ---- S^T = K_tile . Q^T  (tokens on M, heads on N)
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int tok = ((mi & 1) << 3) + r8;
+        const uint32_t rowb = kb + (uint32_t)tok * 128u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int chunk = 2 * j + (mi >> 1);
+          const uint32_t addr =
+              rowb + (uint32_t)(j >> 2) * kHalfBytes + (uint32_t)(((chunk & 7) ^ r8) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(addr, a0, a1, a2, a3);
+          if (j & 1)
+            mma_16816<BF16>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+          else
+            mma_16816<BF16>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+        }
+      }
+      // ---- mask tokens past the request's end, online softmax (log2 units)
+      const bool v_lo = g < valid, v_hi = g + 8 < valid;
+      const float x0 = v_lo ? (sa[0] + sb[0]) * sl2 : -INFINITY;  // token g,   head 2cq
+      const float x1 = v_lo ? (sa[1] + sb[1]) * sl2 : -INFINITY;  // token g,   head 2cq+1
+      const float x2 = v_hi ? (sa[2] + sb[2]) * sl2 : -INFINITY;  // token g+8, head 2cq
+      const float x3 = v_hi ? (sa[3] + sb[3]) * sl2 : -INFINITY;  // token g+8, head 2cq+1
+      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+      const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1);
+      const float p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
+      l0 = l0 * al0 + (p0 + p2);
+      l1 = l1 * al1 + (p1 + p3);
+      m0 = mn0;
+      m1 = mn1;
+      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          o[mt][0] *= al0;
+          o[mt][1] *= al1;
+          o[mt][2] *= al0;
+          o[mt][3] *= al1;
+        }
+      }
+      // ---- P^T as the B operand of the PV MMA (movmatrix transposes S^T's layout)
+      const uint32_t ph0 = pack2<BF16>(p0, p1), ph1 = pack2<BF16>(p2, p3);
+      const uint32_t bh0 = movmatrix_trans(ph0), bh1 = movmatrix_trans(ph1);
+      uint32_t bl0 = 0, bl1 = 0;
+      if constexpr (BF16) {
+        const float2 f0 = unpack2<true>(ph0), f1 = unpack2<true>(ph1);
+        bl0 = movmatrix_trans(pack2<true>(p0 - f0.x, p1 - f0.y));
+        bl1 = movmatrix_trans(pack2<true>(p2 - f1.x, p3 - f1.y));
+      }
+      // ---- zero V rows past the end (their slots may hold anything, even NaN)
+      if (valid < kTileTokens) {
+        uint8_t* vrow = ring + (size_t)s * kSlotBytes + kTileBytes;
+        for (int idx = lane; idx < (kTileTokens - valid) * 16; idx += 32) {
+          const int tok = valid + (idx >> 4), half = (idx >> 3) & 1, ch = idx & 7;
+          *reinterpret_cast<uint4*>(vrow + half * kHalfBytes + tok * 128 + ch * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+        wrote_smem = true;
+        __syncwarp();
+      }
+      // ---- O^T += V_tile^T . P^T   (dims on M, heads on N, tokens on K)
+      {
+        const int tok = ((mi >> 1) << 3) + r8;
+        const uint32_t rowb = vb + (uint32_t)tok * 128u;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int chunk = 2 * mt + (mi & 1);
+          const uint32_t addr =
+              rowb + (uint32_t)(mt >> 2) * kHalfBytes + (uint32_t)(((chunk & 7) ^ r8) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4_trans(addr, a0, a1, a2, a3);
+          mma_16816<BF16>(o[mt], a0, a1, a2, a3, bh0, bh1);
+          if constexpr (BF16) mma_16816<BF16>(o[mt], a0, a1, a2, a3, bl0, bl1);
+        }
+      }
+    }
+    if (wrote_smem) fence_proxy_async_smem();
+    __syncwarp();
+    mbar_arrive(smem_u32(&ctl.empty[s]));
+
+    if (info & kMetaSegLast) {
+      // ================= end of segment: merge the 8 warps' states =================
+      if (!cons_sync(ctl, cons_phase, a.err)) break;  // previous merge done with scratch
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      if (g == 0) {
+        scr.m[warp][2 * cq] = m0;
+        scr.m[warp][2 * cq + 1] = m1;
+        scr.l[warp][2 * cq] = l0;
+        scr.l[warp][2 * cq + 1] = l1;
+      }
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        scr.o[warp][2 * cq][mt * 16 + g] = o[mt][0];
+        scr.o[warp][2 * cq + 1][mt * 16 + g] = o[mt][1];
+        scr.o[warp][2 * cq][mt * 16 + g + 8] = o[mt][2];
+        scr.o[warp][2 * cq + 1][mt * 16 + g + 8] = o[mt][3];
+      }
+      if (!cons_sync(ctl, cons_phase, a.err)) break;
+      const bool direct = rec.ncover == 1;
+      for (int e = ct; e < G * kD; e += kConsumerThreads) {
+        const int h = e >> 7, d = e & (kD - 1);
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, scr.m[w][h]);
+        float L = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float wt = ex2(scr.m[w][h] - M);
+          L += wt * scr.l[w][h];
+          acc += wt * scr.o[w][h][d];
+        }
+        const float val = acc / L;
+        if (direct) {
+          const size_t row = (size_t)rec.b * a.hq + (size_t)rec.kvh * G + h;
+          static_cast<uint16_t*>(a.out)[row * kD + d] = to_bits16<BF16>(val);
+          if (d == 0 && a.lse) a.lse[row] = (M + log2f(L)) * kLn2;
+        } else {
+          a.part_o[((size_t)rec.slot * G + h) * kD + d] = val;
+          if (d == 0) a.part_lse[(size_t)rec.slot * G + h] = M + log2f(L);
+        }
+      }
+      if (!direct) {
+        __threadfence();
+        if (!cons_sync(ctl, cons_phase, a.err)) break;
+        if (ct == 0) {
+          const int old = atomicAdd(&a.counters[rec.c_first], 1);
+          ctl.merge_last = (old == rec.ncover - 1);
+        }
+        if (!cons_sync(ctl, cons_phase, a.err)) break;
+        if (ctl.merge_last) {
+          // this partition arrived last: merge the pair's partial states
+          __threadfence();
+          const long long pstart = rec.pair_start;
+          for (int e = ct; e < G * kD; e += kConsumerThreads) {
+            const int h = e >> 7, d = e & (kD - 1);
+            float M = -INFINITY;
+            for (int k = 0; k < rec.ncover; ++k) {
+              const int sl = state_slot(W, N, pstart, rec.c_first, rec.c_first + k);
+              M = fmaxf(M, __ldcg(a.part_lse + (size_t)sl * G + h));
+            }
+            float L = 0.f, acc = 0.f;
+            for (int k = 0; k < rec.ncover; ++k) {
+              const int sl = state_slot(W, N, pstart, rec.c_first, rec.c_first + k);
+              const float wt = ex2(__ldcg(a.part_lse + (size_t)sl * G + h) - M);
+              L += wt;
+              acc += wt * __ldcg(a.part_o + ((size_t)sl * G + h) * kD + d);
+            }
+            const size_t row = (size_t)rec.b * a.hq + (size_t)rec.kvh * G + h;
+            static_cast<uint16_t*>(a.out)[row * kD + d] = to_bits16<BF16>(acc / L);
+            if (d == 0 && a.lse) a.lse[row] = (M + log2f(L)) * kLn2;
+          }
+          if (ct == 0) a.counters[rec.c_first] = 0;  // ready for the next launch
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t decode_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int grid,
+                          cudaStream_t stream) {
+  static_assert(sizeof(Ctl) % 16 == 0, "Ctl must keep Scratch 16-byte aligned");
+  auto kern = bf16 ? decode_kernel<true> : decode_kernel<false>;
+  // the shared-memory opt-in is per function and device; do it once each
+  static bool attr_set[2][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !attr_set[bf16][dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[bf16][dev] = true;
+  }
+  kern<<<grid, kDecodeThreads, kSmemBytes, stream>>>(tmap, a);
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -1,0 +1,57 @@
+// internal.h -- launch entry points shared between the kernel files and the
+// C ABI layer (api.cu).  Not installed; the public interface is include/pkv.h.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pkv {
+
+struct DecodeArgs {
+  const void* q;          // [B][Hq][128]
+  void* out;              // [B][Hq][128]
+  float* lse;             // [B][Hq] or null
+  const int32_t* indptr;  // [B+1]
+  const int32_t* indices;
+  const int32_t* last_len;  // [B]
+  int* counters;          // [N] arrival counters (zero between launches)
+  float* part_lse;        // [2N][G], log2 domain
+  float* part_o;          // [2N][G][128]
+  int* err;               // device error word or null
+  long long num_pages;
+  int batch, hq, hkv, group, page_size;
+  float scale_log2;       // sm_scale * log2(e)
+};
+
+constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp
+
+size_t decode_smem_bytes();
+cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int grid,
+                          cudaStream_t stream);
+
+struct AppendArgs {
+  void* pool;
+  const int32_t* indptr;
+  const int32_t* indices;
+  const int32_t* last_len;
+  const int32_t* append_indptr;
+  const void* k_new;
+  const void* v_new;
+  int* err;
+  long long num_pages;
+  long long nnz;
+  int batch, hkv, head_dim, page_size;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+
+struct MergeArgs {
+  const float* v;
+  const float* s;
+  void* v_out;
+  float* s_out;
+  long long rows;
+  int states, heads, head_dim, out_dtype;
+};
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream);
+
+}  // namespace pkv

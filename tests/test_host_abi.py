@@ -1,0 +1,163 @@
+"""Host-only checks of the C ABI (no GPU): the library loads and exports every
+symbol include/pkv.h declares, host helpers behave, arguments are rejected
+before any launch, and the split-KV partition mirror covers the work
+exactly once with balanced shares."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import paged_kv_cache_479_b200 as pkv
+from paged_kv_cache_479_b200 import workloads as wl
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "pkv.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"^PKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 13
+    L = ctypes.CDLL(pkv._binding.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), f"libpkv.so does not export {n}"
+    assert {"pkv_append", "pkv_decode", "pkv_merge_states",
+            "paged_kv_append", "paged_decode_attention", "merge_states"} <= set(names)
+
+
+def test_status_strings():
+    L = pkv.lib()
+    assert L.pkv_status_string(0) == b"PKV_OK"
+    assert L.pkv_status_string(3) == b"PKV_ERR_WORKSPACE"
+    assert L.pkv_status_string(99) == b"PKV_ERR_UNKNOWN"
+
+
+def test_workspace_bytes():
+    L = pkv.lib()
+    assert L.pkv_decode_workspace_bytes(8, 64, 8, 128, 148) > 0
+    assert L.pkv_decode_workspace_bytes(8, 64, 8, 64, 148) == 0     # head_dim 128 only
+    assert L.pkv_decode_workspace_bytes(8, 128, 8, 128, 148) == 0    # group 16 > 8
+    assert L.pkv_decode_workspace_bytes(8, 30, 8, 128, 148) == 0     # Hq % Hkv != 0
+    a = L.pkv_decode_workspace_bytes(8, 64, 8, 128, 100)
+    b = L.pkv_decode_workspace_bytes(8, 64, 8, 128, 200)
+    assert b > a and a % 256 == 0
+
+
+def _decode_args(**over):
+    args = dict(q=ctypes.c_void_p(4096), hq=8, pool=ctypes.c_void_p(4096), P=64, ps=16, hkv=2,
+                d=128, dtype=pkv.F16, ip=ctypes.c_void_p(4096), ix=ctypes.c_void_p(4096),
+                ll=ctypes.c_void_p(4096), B=4, scale=0.1, N=8, ws=ctypes.c_void_p(4096),
+                wsb=1 << 30, out=ctypes.c_void_p(8192), lse=None, err=None, stream=None)
+    args.update(over)
+    return list(args.values())
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(d=64), 2), (dict(hq=32, hkv=2), 2), (dict(ps=24), 2), (dict(hq=9), 1),
+    (dict(dtype=7), 1), (dict(scale=float("inf")), 1), (dict(N=-1), 1),
+    (dict(q=ctypes.c_void_p(4097)), 1), (dict(out=None), 1), (dict(ws=ctypes.c_void_p(4100)), 3),
+    (dict(wsb=100), 3), (dict(out=ctypes.c_void_p(4096)), 1),
+])
+def test_decode_rejects_bad_arguments_before_launch(over, status):
+    L = pkv.lib()
+    assert L.pkv_decode(*_decode_args(**over)) == status
+    assert L.pkv_last_error() != b""
+
+
+def test_append_and_merge_reject_bad_arguments():
+    L = pkv.lib()
+    p = ctypes.c_void_p(4096)
+    assert L.pkv_append(p, 8, 16, 2, 12, pkv.F16, p, p, p, 2, p, p, p, 3, None, None) == 2
+    assert L.pkv_append(p, 8, 16, 2, 128, 5, p, p, p, 2, p, p, p, 3, None, None) == 1
+    assert L.pkv_append(ctypes.c_void_p(4098), 8, 16, 2, 128, pkv.F16, p, p, p, 2, p, p, p, 3,
+                        None, None) == 1
+    # nothing to append is a no-op, not an error
+    assert L.pkv_append(None, 8, 16, 2, 128, pkv.F16, None, None, None, 2, None, None, None, 0,
+                        None, None) == 0
+    assert L.pkv_merge_states(p, p, 4, 0, 2, 128, p, pkv.F32, None, None) == 1
+    assert L.pkv_merge_states(p, p, 4, 2, 2, 128, p, 9, None, None) == 1
+    assert L.pkv_merge_states(None, None, 0, 2, 2, 128, None, pkv.F32, None, None) == 0
+
+
+def test_check_table():
+    w = wl.named(2)
+    pkv.check_table(w.page_indptr, w.page_indices, w.last_page_len, w.num_pages, 16)
+    bad = w.last_page_len.copy(); bad[3] = 17
+    with pytest.raises(pkv.PkvError, match="last_page_len"):
+        pkv.check_table(w.page_indptr, w.page_indices, bad, w.num_pages, 16)
+    bad = w.page_indices.copy(); bad[5] = w.num_pages
+    with pytest.raises(pkv.PkvError, match="page_indices"):
+        pkv.check_table(w.page_indptr, bad, w.last_page_len, w.num_pages, 16)
+    bad = w.page_indptr.copy(); bad[4] = bad[3] - 1
+    with pytest.raises(pkv.PkvError, match="decreases"):
+        pkv.check_table(bad, w.page_indices, w.last_page_len, w.num_pages, 16)
+
+
+def _tiles(w):
+    return [int(-(-int(L) // 16)) for L in w.kv_lens]
+
+
+def check_plan(w, N):
+    seg = pkv.plan_segments(w.page_indptr, w.last_page_len, w.page_size, w.num_kv_heads, N)
+    tiles = _tiles(w)
+    W = w.num_kv_heads * sum(tiles)
+    N = min(N, W)          # partitions beyond the tile count get no work
+    # every (request, kv head, tile) exactly once
+    cover = {}
+    for c, b, g, t0, t1, slot, ncov in seg:
+        assert 0 <= t0 < t1 <= tiles[b]
+        for t in range(t0, t1):
+            key = (b, g, t)
+            assert key not in cover
+            cover[key] = c
+    assert len(cover) == W
+    # each partition streams floor((c+1)W/N) - floor(cW/N) tiles, in flat order
+    per = np.zeros(N, np.int64)
+    for c, b, g, t0, t1, *_ in seg:
+        per[c] += t1 - t0
+    expect = np.array([(c + 1) * W // N - c * W // N for c in range(N)])
+    assert np.array_equal(per, expect)
+    assert per.max() - per.min() <= 1
+    # state slots: unique, < 2N, present exactly when the pair is split
+    pairs = {}
+    slots = set()
+    for c, b, g, t0, t1, slot, ncov in seg:
+        pairs.setdefault((b, g), []).append((c, slot, ncov))
+        if ncov == 1:
+            assert slot == -1
+        else:
+            assert 0 <= slot < 2 * N and slot // 2 == c and slot not in slots
+            slots.add(slot)
+    for (b, g), parts in pairs.items():
+        assert all(p[2] == len(parts) for p in parts)
+        cs = [p[0] for p in parts]
+        assert cs == list(range(cs[0], cs[0] + len(cs)))
+    return seg
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 4, 5])
+@pytest.mark.parametrize("N", [1, 2, 7, 148, 1000])
+def test_partition_covers_work_exactly_once(cfg, N):
+    check_plan(wl.named(cfg), N)
+
+
+def test_partition_with_empty_and_tiny_requests():
+    w = wl.make_workload("t", [0, 1, 0, 0, 17, 300, 0, 16, 2], num_qo_heads=4, num_kv_heads=2,
+                         page_size=16, dtype="f16", seed=1)
+    for N in (1, 3, 5, 8, 40, 148, 500):
+        check_plan(w, N)
+    w = wl.make_workload("t", [0, 0], num_qo_heads=4, num_kv_heads=2, page_size=16,
+                         dtype="f16", seed=1)
+    assert len(pkv.plan_segments(w.page_indptr, w.last_page_len, 16, 2, 4)) == 0
+
+
+def test_partition_long_single_sequence_fills_all_partitions():
+    w = wl.named(4)
+    seg = check_plan(w, 148)
+    assert set(seg[:, 0].tolist()) == set(range(148))
+    assert (seg[:, 6] > 1).all()   # every pair is split, so every segment merges
