@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark: batched decode attention over a paged KV cache on B200.
+
+One step = one pass of the whole decode hot path over one batch: append the
+step's new K/V token(s) into their pages (when the workload appends), then
+decode attention for every request with the split-KV partition and the
+in-kernel merge.  Default workload: the Llama-3-8B-shaped decode layer
+(batch 64, KV lengths U[512,4096] + 1 appended token, 32 q / 8 kv heads,
+head_dim 128, page size 16, bf16, pool 1.25x the pages needed).
+
+Metric: KV HBM GB/s (algorithmic bytes: unique K/V once + q + out + page
+table + lse, plus the append's rows), with us/step and decoded tokens/s.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload 1..5] [--impl reference]
+
+N > 1 (launched by torch.distributed.run, one rank per GPU): every rank runs
+its own independent batch of the same shape (weak scaling; no collective on
+the data path; the barrier and the max-over-ranks timing use NCCL).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_479_b200 import workloads as wl  # noqa: E402
+
+METRIC = "paged decode attn: KV HBM GB/s (% of B200 peak), µs/step, tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ["csrc/decode.cu", "csrc/common.cuh", "csrc/partition.cuh"]
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
+    p.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    p.add_argument("--partitions", type=int, default=0, help="split-KV partitions (0 = one per SM)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for cpu_baseline")
+    p.add_argument("--ref-seconds", type=float, default=150.0, help="oracle time budget of the reference arm")
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash():
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_479_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_id):
+    """DRAM bytes per decode launch from a committed ncu summary, only while the
+    kernel sources are the ones that summary was taken on."""
+    path = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_hash") != decode_source_hash():
+        return None
+    entry = rec.get("workloads", {}).get(str(workload_id))
+    return None if entry is None else int(entry["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_index):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ident, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[0]), float(parts[1]),
+                                     float(parts[2]) if parts[2] not in ("[N/A]", "N/A") else 0.0,
+                                     [p == "Active" for p in parts[3:]]))
+            except ValueError:
+                continue
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if not inside:
+            inside = self.samples
+            window = "whole run (timed region shorter than the 100 ms sampling period)"
+        if not inside:
+            return None
+        mhz = [s[1] for s in inside]
+        reasons = sorted({self.REASONS[i] for s in inside for i, a in enumerate(s[4]) if a})
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(s[2] for s in inside),
+                "reasons": reasons, "samples": len(inside), "window": window,
+                "power_w_max": max(s[3] for s in inside)}
+
+
+def algorithmic_bytes(w):
+    return wl.decode_bytes(w) + wl.append_bytes(w)
+
+
+def workload_config(w, args, rotation, partitions):
+    cfg = {"workload": w.name, "batch": w.batch, "kv_tokens": int(w.kv_lens.sum()),
+           "num_qo_heads": w.num_qo_heads, "num_kv_heads": w.num_kv_heads,
+           "head_dim": w.head_dim, "page_size": w.page_size, "pool_pages": w.num_pages,
+           "appended_tokens": w.nnz_new, "partitions": partitions,
+           "algorithmic_bytes_per_step": algorithmic_bytes(w),
+           "unique_kv_bytes": wl.kv_cache_bytes(1, w.num_kv_heads, w.head_dim, wl.unique_kv_tokens(w)),
+           "logical_kv_bytes": wl.logical_kv_bytes(w),
+           "l2": (f"inputs larger than L2: {rotation} rotating batch copies of "
+                  f"{wl.logical_kv_bytes(w) / 1e6:.0f} MB K/V each"),
+           "parallelism": f"dp{args.gpus} (independent batches per GPU)"}
+    if w.note:
+        cfg["values"] = w.note
+    return cfg
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline; never tuned)
+# --------------------------------------------------------------------------
+
+def head_workload(w, n):
+    """The first n requests of a workload (same shapes and value recipe)."""
+    prefix = w.shared_prefix_pages * w.page_size
+    return wl.make_workload(f"{w.name} [first {n} requests]", w.kv_lens[:n],
+                            num_qo_heads=w.num_qo_heads, num_kv_heads=w.num_kv_heads,
+                            head_dim=w.head_dim, page_size=w.page_size, dtype=w.dtype,
+                            seed=w.seed, pool_factor=1.0, shared_prefix_len=prefix,
+                            append_counts=w.append_counts[:n], q_std=w.q_std,
+                            key_offset_std=w.key_offset_std, note=w.note)
+
+
+def time_oracle(w, q_bits, pool_bits):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.decode(q_bits, pool_bits, oracle.BF16 if w.dtype == "bf16" else oracle.F16,
+                  w.page_indptr, w.page_indices, w.last_page_len, w.sm_scale)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(w, budget_s):
+    """Pick the first n requests so the oracle runs about budget_s; returns
+    (workload, q_bits, pool_bits, seconds of one run)."""
+    n = 1
+    while True:
+        ws = head_workload(w, n)
+        q, pool, _, _ = wl.make_tensors(ws, "cpu")
+        qb, pb = wl.bits(q), wl.bits(pool)
+        t = time_oracle(ws, qb, pb)
+        if n >= w.batch or t * 1.5 >= budget_s:
+            return ws, qb, pb, t
+        n = min(w.batch, max(n + 1, int(n * budget_s / max(t, 1e-3) * 0.8)))
+
+
+def cpu_baseline(w, budget_s):
+    import oracle
+    ws, qb, pb, t = oracle_sample(w, budget_s)
+    kv = wl.kv_cache_bytes(1, ws.num_kv_heads, ws.head_dim, wl.unique_kv_tokens(ws))
+    return {"value": round(kv / t / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"fp64 C oracle (OpenMP) on the first {ws.batch} of {w.batch} requests "
+                       f"({int(ws.kv_lens.sum())} KV tokens, {kv / 1e6:.1f} MB K/V), {t:.2f} s"),
+            "seconds": round(t, 3)}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, as it stands, on the machine's host
+    cores, on a bounded sample of the same workload per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = wl.named(args.workload)
+    per_step = max(0.05, args.ref_seconds / max(1, args.steps + args.warmup))
+    ws, qb, pb, _ = oracle_sample(w, per_step)
+    for _ in range(args.warmup):
+        time_oracle(ws, qb, pb)
+    times = [time_oracle(ws, qb, pb) for _ in range(args.steps)]
+    total = sum(times)
+    kv = wl.kv_cache_bytes(1, ws.num_kv_heads, ws.head_dim, wl.unique_kv_tokens(ws))
+    value = kv * args.steps / total / 1e9
+    sample = (f"first {ws.batch} of {w.batch} requests per step "
+              f"({int(ws.kv_lens.sum())} KV tokens, {kv / 1e6:.1f} MB K/V)")
+    cfg = workload_config(w, args, 1, 0)
+    cfg["reference_sample"] = sample
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": cfg, "impl": "reference",
+            "us_per_step": round(total / args.steps * 1e6, 1),
+            "tokens_per_s": round(ws.batch * args.steps / total, 2),
+            "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "sample": sample,
+                             "value": round(value, 4), "unit": "GB/s"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# the GPU arm
+# --------------------------------------------------------------------------
+
+class Batch:
+    """One copy of the workload's tensors on the device."""
+
+    def __init__(self, w, dev, value_seed):
+        wv = wl.Workload(**{**w.__dict__, "seed": value_seed})
+        self.q, self.pool, self.k_new, self.v_new = wl.make_tensors(wv, dev)
+
+
+def run_pkv(args):
+    import paged_kv_cache_479_b200 as pkv
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                             device_id=dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    w = wl.named(args.workload)
+    N = args.partitions or pkv.default_partitions(local)
+    kv_bytes = wl.logical_kv_bytes(w)
+    rotation = 2 if kv_bytes < (2 << 30) else 1
+    batches = [Batch(w, dev, w.seed + 1000 * rank + r) for r in range(rotation)]
+    t = lambda a: torch.as_tensor(a, device=dev)
+    indptr, indices, last = t(w.page_indptr), t(w.page_indices), t(w.last_page_len)
+    app = t(w.append_indptr)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.zeros(pkv.decode_workspace_bytes(w.batch, w.num_qo_heads, w.num_kv_heads, 128, N) // 4 + 64,
+                     dtype=torch.int32, device=dev)
+    out = torch.empty_like(batches[0].q)
+    lse = torch.empty((w.batch, w.num_qo_heads), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 1 + (1 if w.nnz_new else 0)
+
+    def step(bt, ev0=None, ev1=None):
+        if w.nnz_new:
+            pkv.paged_kv_append(bt.pool, indptr, indices, last, bt.k_new, bt.v_new, app,
+                                error_word=err, stream=stream)
+        if ev0 is not None:
+            ev0.record(stream)
+        pkv.paged_decode_attention(bt.q, bt.pool, indptr, indices, last, ws, out=out, lse=lse,
+                                   sm_scale=w.sm_scale, num_partitions=N, error_word=err,
+                                   stream=stream)
+        if ev1 is not None:
+            ev1.record(stream)
+
+    clocks = ClockSampler(local)
+    for i in range(args.warmup):
+        step(batches[i % rotation])
+    torch.cuda.synchronize()
+    if pkv.read_error_word(err) != 0:
+        raise RuntimeError("device error bits set during warm-up")
+
+    K = args.steps
+    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_host0 = time.time()
+    start.record(stream)
+    for i in range(K):
+        step(batches[i % rotation], d0[i], d1[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    barrier()
+    ms_local = start.elapsed_time(end)
+    decode_ms = sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K
+    ms = max_over_ranks(ms_local)
+    decode_ms_max = max_over_ranks(decode_ms)
+    if pkv.read_error_word(err) != 0:
+        raise RuntimeError("device error bits set during the timed steps")
+
+    step_bytes = algorithmic_bytes(w)
+    s_per_step = ms / 1e3 / K
+    value = step_bytes * world / s_per_step / 1e9
+    dec_bytes = wl.decode_bytes(w)
+    peak, peak_kind = measured_hbm()
+    achieved = dec_bytes / (decode_ms_max / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        src = batches[0]
+        pin = lambda x: x.detach().cpu().pin_memory()
+        q_h, k_h, v_h = pin(src.q), pin(src.k_new), pin(src.v_new)
+        ip_h, ix_h, ll_h, ap_h = (torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+                                  for a in (w.page_indptr, w.page_indices, w.last_page_len,
+                                            w.append_indptr))
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        q_d, k_d, v_d = (torch.empty_like(x, device=dev) for x in (q_h, k_h, v_h))
+        ip_d, ix_d, ll_d, ap_d = (torch.empty_like(x, device=dev) for x in (ip_h, ix_h, ll_h, ap_h))
+        h2d = sum(x.numel() * x.element_size() for x in (q_h, k_h, v_h, ip_h, ix_h, ll_h, ap_h))
+        d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+
+        def e2e_step():
+            for d, h in ((q_d, q_h), (k_d, k_h), (v_d, v_h), (ip_d, ip_h), (ix_d, ix_h),
+                         (ll_d, ll_h), (ap_d, ap_h)):
+                d.copy_(h, non_blocking=True)
+            if w.nnz_new:
+                pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d, error_word=err,
+                                    stream=stream)
+            pkv.paged_decode_attention(q_d, src.pool, ip_d, ix_d, ll_d, ws, out=out, lse=lse,
+                                       sm_scale=w.sm_scale, num_partitions=N, error_word=err,
+                                       stream=stream)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+            stream.synchronize()   # the caller needs the result before the next step
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": round(step_bytes * world / (e_ms / 1e3 / K) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "us_per_step": round(e_ms / K * 1e3, 2)}
+    clocks.stop()
+
+    if rank == 0:
+        traffic = recorded_traffic(args.workload)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f16", "data": "synthetic",
+            "config": workload_config(w, args, rotation, N),
+            "us_per_step": round(ms / K * 1e3, 2),
+            "tokens_per_s": round(w.batch * world / s_per_step, 1),
+            "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+            "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6650 GB/s",
+                         "traffic": traffic, "algorithmic_bytes_per_launch": dec_bytes,
+                         "avg_launch_us": round(decode_ms_max * 1e3, 2)},
+            "gpu_launches": K * launches_per_step,
+            "e2e": e2e,
+            "clocks": clocks.summary(t_host0, t_host1),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_pkv(args)
+
+
+if __name__ == "__main__":
+    main()

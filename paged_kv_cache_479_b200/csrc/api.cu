@@ -92,13 +92,19 @@ struct MapKey {
   }
 };
 
-// The pool viewed as a 4-D tensor (dim, slot, kv*Hkv + head, page), boxes of
-// [16 slots][64 dims] with 128-byte swizzle: two boxes make one tile's K or V.
+// Tensor map of the pool for the decode kernel's bulk-tensor loads.  Preferred
+// form, 5-D: (dim % 64, slot, dim / 64, kv * Hkv + head, page) with boxes of
+// [2][16 slots][64 dims] -- one load brings a tile's whole K (or V) into
+// shared memory as two 128-byte-swizzled [16][64] halves.  The dim/64 axis
+// has a smaller stride than the slot axis; if the driver rejects that order,
+// the 4-D form (dim, slot, kv * Hkv + head, page) with [16][64] boxes is used
+// (two loads per K or V tile, same shared-memory layout).
 pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, int dtype,
-                           CUtensorMap* out) {
+                           CUtensorMap* out, int* one_box) {
   static std::mutex mu;
   static MapKey keys[16];
   static CUtensorMap maps[16];
+  static int kinds[16];
   static int used = 0, next = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -108,34 +114,52 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
     for (int i = 0; i < used; ++i)
       if (keys[i] == key) {
         *out = maps[i];
+        *one_box = kinds[i];
         return PKV_OK;
       }
   }
   auto encode = get_encode();
   if (!encode) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const CUtensorMapDataType dt =
+      dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t row = (cuuint64_t)kDecodeHeadDim * 2;  // bytes of one token's K (or V) row
   CUtensorMap m;
-  const cuuint64_t esz = 2;
-  cuuint64_t dims[4] = {(cuuint64_t)kDecodeHeadDim, (cuuint64_t)ps, (cuuint64_t)2 * hkv,
-                        (cuuint64_t)pages};
-  cuuint64_t strides[3] = {kDecodeHeadDim * esz, (cuuint64_t)ps * kDecodeHeadDim * esz,
-                           (cuuint64_t)2 * hkv * ps * kDecodeHeadDim * esz};
-  cuuint32_t box[4] = {64, (cuuint32_t)pkv::kTileTokens, 1, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = encode(&m,
-                      dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                      4, const_cast<void*>(pool), dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  int kind = 0;
+  CUresult r = CUDA_ERROR_INVALID_VALUE;
+#ifndef PKV_FORCE_4D_MAP
+  {
+    cuuint64_t dims[5] = {64, (cuuint64_t)ps, 2, (cuuint64_t)2 * hkv, (cuuint64_t)pages};
+    cuuint64_t strides[4] = {row, 128, (cuuint64_t)ps * row, (cuuint64_t)2 * hkv * ps * row};
+    cuuint32_t box[5] = {64, (cuuint32_t)pkv::kTileTokens, 2, 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    r = encode(&m, dt, 5, const_cast<void*>(pool), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    kind = 1;
+  }
+#endif
+  if (r != CUDA_SUCCESS) {
+    cuuint64_t dims[4] = {(cuuint64_t)kDecodeHeadDim, (cuuint64_t)ps, (cuuint64_t)2 * hkv,
+                          (cuuint64_t)pages};
+    cuuint64_t strides[3] = {row, (cuuint64_t)ps * row, (cuuint64_t)2 * hkv * ps * row};
+    cuuint32_t box[4] = {64, (cuuint32_t)pkv::kTileTokens, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    r = encode(&m, dt, 4, const_cast<void*>(pool), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    kind = 0;
+  }
   if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   {
     std::lock_guard<std::mutex> lk(mu);
     keys[next] = key;
     maps[next] = m;
+    kinds[next] = kind;
     next = (next + 1) % 16;
     if (used < 16) ++used;
   }
   *out = m;
+  *one_box = kind;
   return PKV_OK;
 }
 
@@ -161,7 +185,7 @@ int pkv_default_partitions(int device) {
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
     return -1;
-  return sms;  // one persistent CTA per SM (the decode CTA uses ~167 KB of shared memory)
+  return sms * pkv::kDecodeCtasPerSm;  // persistent decode CTAs resident at once
 }
 
 size_t pkv_decode_workspace_bytes(int batch, int num_qo_heads, int num_kv_heads, int head_dim,
@@ -337,7 +361,8 @@ pkv_status pkv_decode(const void* q, int num_qo_heads, const void* pool, int64_t
     return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, L.total);
 
   CUtensorMap tmap;
-  pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, &tmap);
+  int one_box = 0;
+  pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, &tmap, &one_box);
   if (st != PKV_OK) return st;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -359,6 +384,7 @@ pkv_status pkv_decode(const void* q, int num_qo_heads, const void* pool, int64_t
   a.group = group;
   a.page_size = page_size;
   a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.one_box = one_box;
   cudaError_t e = pkv::launch_decode(tmap, a, dtype == PKV_BF16, N, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();

@@ -56,7 +56,15 @@ namespace {
 constexpr int kD = 128;
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kStages = 16;
+constexpr int kStages = kDecodeStages;
+constexpr int kIssueLanes = kStages < 16 ? kStages : 16;  // producer lanes issuing at once
+// Consumer warp w takes ring positions w, w+8, w+16, ...  With the slot count
+// a multiple of the warp count, every slot has ONE consumer warp, so a warp
+// only ever waits on the next round of a slot it has itself finished.  (A
+// parity wait cannot tell the round before last from the next one: if another
+// warp could still own the current round, the wait might return early.)
+static_assert(kStages % kConsumerWarps == 0 && 32 % kIssueLanes == 0,
+              "each ring slot must have a single consumer warp");
 constexpr int kHalfBytes = kTileTokens * 64 * 2;  // one [16][64] box: 2 KiB
 constexpr int kTileBytes = 2 * kHalfBytes;        // K or V of one tile: 4 KiB
 constexpr int kSlotBytes = 2 * kTileBytes;        // K + V: 8 KiB
@@ -136,7 +144,7 @@ __device__ __forceinline__ bool cons_sync(Ctl& ctl, uint32_t& phase, int* err) {
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
+__global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   // 128-byte-swizzled TMA boxes need 1024-byte aligned shared addresses
@@ -222,10 +230,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     wk.ps = a.page_size;
     wk.Hkv = Hkv;
     wk.start(ctl.b0, ctl.Cb0, request_info(a.indptr, a.last_len, ctl.b0, a.page_size), f0, f1);
-    uint32_t i = 0;
+    const uint32_t ring0 = smem_u32(ring);
+    const long long ps = a.page_size;
+    uint32_t i = 0;  // tiles handed to the ring so far
     int seg = 0;
     bool ok = true;
-    const uint32_t ring0 = smem_u32(ring);
     while (ok && !wk.done()) {
       const long long n = wk.seg_tiles();
       if (n <= 0) {  // only possible if the table changed under the kernel
@@ -247,72 +256,92 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         r.c_first = pl.c_first;
         r.ncover = pl.ncover;
         r.pair_start = pstart;
+        // last segment of this request: warm L2 with the next request's table entries
+        if (wk.kvh == Hkv - 1 && wk.b + 1 < B) {
+          prefetch_l2(a.indptr + wk.b + 2);
+          prefetch_l2(a.last_len + wk.b + 1);
+          prefetch_l2(a.indices + wk.ri.page_base + (wk.ri.len + ps - 1) / ps);
+        }
       }
+      __syncwarp();  // the record is written before any lane publishes a tile of it
+      // page ids, one tile per lane, loaded one 32-tile batch ahead of their use
+      const int* idx = a.indices + wk.ri.page_base;
+      int page_next = -1;
+      if (lane < n) page_next = idx[(wk.t + lane) * kTileTokens / ps];
       for (long long k0 = 0; ok && k0 < n_pad; k0 += 32) {
+        int page = page_next;
+        if (k0 + 32 + lane < n) page_next = idx[(wk.t + k0 + 32 + lane) * kTileTokens / ps];
         const long long k = k0 + lane;
-        int page = -1, yoff = 0, valid = 0;
+        int yoff = 0, valid = 0;
         if (k < n) {
-          const long long tok0 = (wk.t + k) * kTileTokens;
-          page = a.indices[(long long)wk.ri.page_base + tok0 / a.page_size];
           if (page < 0 || (long long)page >= a.num_pages) {
             if (a.err) atomicOr(a.err, kErrPageId);
             page = -1;
           }
-          yoff = (int)(tok0 % a.page_size);
+          const long long tok0 = (wk.t + k) * kTileTokens;
+          yoff = (int)(tok0 % ps);
           const long long left = wk.ri.len - tok0;
           valid = left < kTileTokens ? (int)left : kTileTokens;
+        } else {
+          page = -1;
         }
+        const int flags = ((k >= n_pad - kConsumerWarps) ? kMetaSegLast : 0) |
+                          ((seg & (kSegRecs - 1)) << kMetaSegShift);
         const int cnt = (int)((n_pad - k0) < 32 ? (n_pad - k0) : 32);
-        for (int j = 0; j < cnt; ++j) {
-          const int pg = __shfl_sync(0xffffffffu, page, j);
-          const int y = __shfl_sync(0xffffffffu, yoff, j);
-          const int v = __shfl_sync(0xffffffffu, valid, j);
-          const int s = (int)(i % kStages);
+        // lanes [jb, jb + kIssueLanes) publish their tiles concurrently (distinct ring slots)
+        for (int jb = 0; jb < cnt; jb += kIssueLanes) {
           int okl = 1;
-          if (lane == 0) {
-            okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((i / kStages) & 1u) ^ 1u,
+          if (lane >= jb && lane < jb + kIssueLanes && lane < cnt) {
+            const uint32_t it = i + (uint32_t)(lane - jb);
+            const int s = (int)(it % kStages);
+            okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kStages) & 1u) ^ 1u,
                                     &ctl.abort, a.err);
             if (okl) {
-              const int flags = ((k0 + j >= n_pad - kConsumerWarps) ? kMetaSegLast : 0) |
-                                ((seg & (kSegRecs - 1)) << kMetaSegShift);
               const uint32_t full = smem_u32(&ctl.full[s]);
-              if (pg >= 0 && v > 0) {
-                ctl.meta[s] = v | flags;
+              if (page >= 0 && valid > 0) {
+                ctl.meta[s] = valid | flags;
                 mbar_arrive_expect_tx(full, kSlotBytes);
                 const uint32_t dst = ring0 + (uint32_t)s * kSlotBytes;
                 const int zk = wk.kvh, zv = Hkv + wk.kvh;
-                tma_load_4d(dst, &tmap, 0, y, zk, pg, full);
-                tma_load_4d(dst + kHalfBytes, &tmap, 64, y, zk, pg, full);
-                tma_load_4d(dst + 2 * kHalfBytes, &tmap, 0, y, zv, pg, full);
-                tma_load_4d(dst + 3 * kHalfBytes, &tmap, 64, y, zv, pg, full);
+                if (a.one_box) {
+                  tma_load_5d(dst, &tmap, 0, yoff, 0, zk, page, full);
+                  tma_load_5d(dst + kTileBytes, &tmap, 0, yoff, 0, zv, page, full);
+                } else {
+                  tma_load_4d(dst, &tmap, 0, yoff, zk, page, full);
+                  tma_load_4d(dst + kHalfBytes, &tmap, 64, yoff, zk, page, full);
+                  tma_load_4d(dst + 2 * kHalfBytes, &tmap, 0, yoff, zv, page, full);
+                  tma_load_4d(dst + 3 * kHalfBytes, &tmap, 64, yoff, zv, page, full);
+                }
               } else {
                 ctl.meta[s] = flags;  // no data: padding, or a skipped bad page
                 mbar_arrive(full);
               }
             }
           }
-          ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+          ok = __all_sync(0xffffffffu, okl) != 0;
+          const int issued = (cnt - jb) < kIssueLanes ? (cnt - jb) : kIssueLanes;
+          i += (uint32_t)issued;
           if (!ok) break;
-          ++i;
         }
       }
       ++seg;
       wk.advance();
     }
     // one end marker per consumer warp
-    for (int j = 0; ok && j < kConsumerWarps; ++j) {
-      const int s = (int)(i % kStages);
+    if (ok) {
       int okl = 1;
-      if (lane == 0) {
-        okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((i / kStages) & 1u) ^ 1u, &ctl.abort,
+      if (lane < kConsumerWarps) {
+        const uint32_t it = i + lane;
+        const int s = (int)(it % kStages);
+        okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kStages) & 1u) ^ 1u, &ctl.abort,
                                 a.err);
         if (okl) {
           ctl.meta[s] = kMetaEnd;
           mbar_arrive(smem_u32(&ctl.full[s]));
         }
       }
-      ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
-      ++i;
+      ok = __all_sync(0xffffffffu, okl) != 0;
+      i += kConsumerWarps;
     }
     if (!ok && lane == 0) {
       // aborted: let the copies already issued land before the CTA exits
@@ -355,6 +384,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     if (sid != cur_seg) {
       cur_seg = sid;
       rec = ctl.seg[sid];
+      if ((unsigned)rec.b >= (unsigned)B || (unsigned)rec.kvh >= (unsigned)Hkv) {
+        // never expected: a corrupted record would address out of bounds
+        if (lane == 0 && a.err) atomicOr(a.err, kErrTimeout);
+        ctl.abort = 1;
+        break;
+      }
       const int h = rec.kvh * G + g;
       if (g < G) {
         const uint16_t* qp =
@@ -373,7 +408,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
     }
-    const int valid = info & kMetaValid;
+    const int valid = (info & kMetaValid) > kTileTokens ? kTileTokens : (info & kMetaValid);
     const uint32_t kb = ring0 + (uint32_t)s * kSlotBytes;
     const uint32_t vb = kb + kTileBytes;
     bool wrote_smem = false;

@@ -21,9 +21,18 @@ struct DecodeArgs {
   long long num_pages;
   int batch, hq, hkv, group, page_size;
   float scale_log2;       // sm_scale * log2(e)
+  int one_box;            // 1: 5-D tensor map, one box per K/V tile; 0: 4-D map, two boxes
 };
 
 constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp
+#ifndef PKV_STAGES
+#define PKV_STAGES 16
+#endif
+#ifndef PKV_CTAS_PER_SM
+#define PKV_CTAS_PER_SM 1
+#endif
+constexpr int kDecodeStages = PKV_STAGES;        // K/V ring slots (8 KiB each) per CTA
+constexpr int kDecodeCtasPerSm = PKV_CTAS_PER_SM; // resident decode CTAs per SM
 
 size_t decode_smem_bytes();
 cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int grid,
