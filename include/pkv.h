@@ -208,6 +208,39 @@ PKV_API int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* l
                           int batch, int page_size, int num_kv_heads, int num_partitions,
                           int64_t* segments, int64_t max_segments);
 
+/*
+ * pkv_decode_static_workspace -- pkv_decode without a caller-provided workspace.
+ *
+ * The pages describe no such call; it exists for users of this library who
+ * cannot allocate device memory at the point where they decode, and have no
+ * spare device buffer to lend as workspace -- for example a serving engine
+ * that reserved all free HBM for its KV pool up front, a plugin running
+ * inside a host framework whose allocator it cannot reach, or a
+ * latency-critical loop where cudaMalloc (which can synchronise the device)
+ * is not allowed.
+ *
+ * Same arguments and results as pkv_decode, minus workspace and
+ * workspace_bytes.  The scratch is a file-scope device array of 4 MiB inside
+ * libpkv, present on every GPU that loads the library until the process
+ * exits; it fits the default partition count for up to 8 query heads per KV
+ * head (about 1.2 MiB on a 148-SM B200).  Calls needing more return
+ * PKV_ERR_WORKSPACE without launching.  The call allocates nothing: its first
+ * call on a device looks the array's device address up (make that first call
+ * before any stream capture), and every call clears the part of the array it
+ * uses with cudaMemsetAsync on `stream` before the kernel.  All calls share
+ * the one array, which keeps the last call's contents: calls that can
+ * overlap on the GPU (different streams, or different host threads) race on
+ * it and must be serialised by the caller.
+ */
+PKV_API pkv_status pkv_decode_static_workspace(const void* q, int num_qo_heads,
+                                               const void* pool, int64_t num_pages,
+                                               int page_size, int num_kv_heads, int head_dim,
+                                               int dtype, const int32_t* page_indptr,
+                                               const int32_t* page_indices,
+                                               const int32_t* last_page_len, int batch,
+                                               float sm_scale, int num_partitions, void* out,
+                                               float* lse, int32_t* error_word, void* stream);
+
 /* The same three operations under the names used in the paged-attention literature. */
 PKV_API pkv_status paged_kv_append(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
                            int head_dim, int dtype,

@@ -15,6 +15,7 @@ Functions (C names in parentheses):
   read_error_word        (pkv_read_error_word)
   check_table            (pkv_check_table)     host-side table check
   plan_segments          (pkv_plan_segments)   host mirror of the split-KV partition
+  decode_static_workspace (pkv_decode_static_workspace)  decode on the library's own scratch
 """
 from ._binding import (  # noqa: F401
     BF16,
@@ -22,6 +23,7 @@ from ._binding import (  # noqa: F401
     F32,
     PkvError,
     check_table,
+    decode_static_workspace,
     decode_workspace_bytes,
     default_partitions,
     lib,
@@ -39,4 +41,5 @@ from ._binding import (  # noqa: F401
 
 pkv_append = paged_kv_append
 pkv_decode = paged_decode_attention
+pkv_decode_static_workspace = decode_static_workspace
 pkv_merge_states = merge_states

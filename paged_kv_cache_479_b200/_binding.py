@@ -37,6 +37,8 @@ _SIGNATURES = {
     "pkv_check_table": ([_P, _P, _P, _I32, _I64, _I32], _I32),
     "pkv_plan_segments": ([_P, _P, _I32, _I32, _I32, _I32, _P, _I64], _I64),
 }
+_SIGNATURES["pkv_decode_static_workspace"] = (
+    [_P, _I32, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I32, _F32, _I32, _P, _P, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
 _SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
 _SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
@@ -158,6 +160,32 @@ def paged_decode_attention(q, pool, page_indptr, page_indices, last_page_len, wo
                           workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
                           _ptr(error_word), _stream(stream, q.device))
     _check(st, "pkv_decode")
+    return out, lse
+
+
+def decode_static_workspace(q, pool, page_indptr, page_indices, last_page_len, out, lse=None,
+                            sm_scale=None, num_partitions: int = 0, error_word=None,
+                            stream=None):
+    """Decode attention like paged_decode_attention, for callers that cannot
+    allocate device memory: the library's own static scratch replaces the
+    workspace, and the caller passes the output buffers (nothing is allocated
+    here).  Calls sharing that scratch must not overlap on the GPU
+    (C: pkv_decode_static_workspace)."""
+    _dev_tensor(q, "q", pool.dtype)
+    _dev_tensor(pool, "pool")
+    _dev_tensor(out, "out", pool.dtype)
+    for name, t in (("page_indptr", page_indptr), ("page_indices", page_indices),
+                    ("last_page_len", last_page_len)):
+        _dev_tensor(t, name, torch.int32)
+    B, hq, d = q.shape
+    P, _, hkv, ps, dp = pool.shape
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_decode_static_workspace(_ptr(q), hq, _ptr(pool), P, ps, hkv, dp,
+                                           _DTYPES[pool.dtype], _ptr(page_indptr),
+                                           _ptr(page_indices), _ptr(last_page_len), B, scale,
+                                           num_partitions, _ptr(out), _ptr(lse),
+                                           _ptr(error_word), _stream(stream, q.device))
+    _check(st, "pkv_decode_static_workspace")
     return out, lse
 
 

@@ -165,6 +165,14 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
 
 }  // namespace
 
+pkv_status pkv::set_error(pkv_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
 extern "C" {
 
 const char* pkv_status_string(int status) {

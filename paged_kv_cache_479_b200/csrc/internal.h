@@ -5,7 +5,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "pkv.h"
+
 namespace pkv {
+
+// record the detail that pkv_last_error() reports on this thread; returns s
+pkv_status set_error(pkv_status s, const char* fmt, ...);
 
 struct DecodeArgs {
   const void* q;          // [B][Hq][128]
