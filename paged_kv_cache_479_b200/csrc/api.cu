@@ -243,7 +243,7 @@ int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page
     return -1;
   long long total = 0;
   for (int b = 0; b < batch; ++b)
-    total += pkv::request_info(page_indptr_h, last_page_len_h, b, page_size).tiles;
+    total += pkv::request_info(page_indptr_h, last_page_len_h, b, page_size).units;
   const long long W = (long long)num_kv_heads * total;
   if (W == 0) return 0;
   // the kernel uses min(num_partitions, W) partitions: none of them is empty
@@ -258,13 +258,13 @@ int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page
     pkv::ReqInfo r0{};
     for (int b = 0; b < batch; ++b) {
       const pkv::ReqInfo r = pkv::request_info(page_indptr_h, last_page_len_h, b, page_size);
-      if (r.tiles > 0 && (long long)num_kv_heads * Cb <= f0 &&
-          f0 < (long long)num_kv_heads * (Cb + r.tiles)) {
+      if (r.units > 0 && (long long)num_kv_heads * Cb <= f0 &&
+          f0 < (long long)num_kv_heads * (Cb + r.units)) {
         b0 = b;
         r0 = r;
         break;
       }
-      Cb += r.tiles;
+      Cb += r.units;
     }
     if (b0 < 0) return -1;
     pkv::Walk wk;
@@ -275,19 +275,21 @@ int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page
     wk.Hkv = num_kv_heads;
     wk.start(b0, Cb, r0, f0, f1);
     while (!wk.done()) {
-      const long long n = wk.seg_tiles();
-      const pkv::SegPlace pl = pkv::seg_place(W, N, wk.pair_start(), wk.ri.tiles, c);
-      if (segments && count < max_segments) {
-        int64_t* row = segments + 7 * count;
-        row[0] = c;
-        row[1] = wk.b;
-        row[2] = wk.kvh;
-        row[3] = wk.t;
-        row[4] = wk.t + n;
-        row[5] = pl.slot;
-        row[6] = pl.ncover;
+      const long long t0 = wk.t0(), t1 = wk.t1();
+      if (t1 > t0) {
+        const pkv::SegPlace pl = pkv::seg_place(W, N, wk.pair_start(), wk.ri.units, c);
+        if (segments && count < max_segments) {
+          int64_t* row = segments + 7 * count;
+          row[0] = c;
+          row[1] = wk.b;
+          row[2] = wk.kvh;
+          row[3] = t0;
+          row[4] = t1;
+          row[5] = pl.slot;
+          row[6] = pl.ncover;
+        }
+        ++count;
       }
-      ++count;
       wk.advance();
     }
   }

@@ -1,14 +1,15 @@
 // append.cu -- scatter newly decoded tokens' K and V into their pages.
 //
-// One warp per (new token, kv head): the warp finds the token's request by
-// binary search over append_indptr, maps its logical position to
-// (page, slot) through the page table -- page = page_indices[indptr[b] + pos / page_size],
-// slot = pos % page_size, the O(1) translation of "Flash Attention与Paged KV Cache
-// 优化大模型推理实战" section 3.2 -- and copies the head's K row and V row with
-// 16-byte vector loads and stores.  Pure copies: the pool is bit-identical to
-// what a byte-wise scatter would produce.
+// Blocks take requests (grid-stride over b, blockIdx.y splits a request's new
+// rows further when requests append many tokens); a warp copies one
+// (new token, kv head) row pair.  Position pos of request b lives at page
+// page_indices[indptr[b] + pos / page_size], slot pos % page_size -- the O(1)
+// translation of "Flash Attention与Paged KV Cache优化大模型推理实战" section 3.2.
+// The K row and the V row are copied with 16-byte vector loads and stores;
+// the pool ends up bit-identical to a byte-wise scatter.
 #include <cuda_runtime.h>
 
+#include "common.cuh"
 #include "internal.h"
 #include "partition.cuh"
 
@@ -18,58 +19,71 @@ namespace {
 constexpr int kWarps = 8;
 
 __global__ void __launch_bounds__(kWarps * 32) append_kernel(const AppendArgs a) {
+  // PDL: the next kernel (the decode) may start its prologue now; this one
+  // waits for the kernel before it, which may have produced k_new / v_new
+  grid_dependents_launch();
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
-  const long long gw = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (gw >= a.nnz * a.hkv) return;
-  const long long i = gw / a.hkv;     // new token
-  const int h = (int)(gw % a.hkv);    // kv head
-
-  // request b: append_indptr[b] <= i < append_indptr[b+1]
-  int lo = 0, hi = a.batch;           // invariant: append_indptr[lo] <= i < append_indptr[hi]
-  if (a.append_indptr[0] > i || a.append_indptr[a.batch] <= i) {
-    if (lane == 0 && a.err) atomicOr(a.err, kErrAppend);
-    return;
-  }
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (a.append_indptr[mid] <= i) lo = mid; else hi = mid;
-  }
-  const int b = lo;
-  const ReqInfo r = request_info(a.indptr, a.last_len, b, a.page_size);
-  const long long n_new = (long long)a.append_indptr[b + 1] - a.append_indptr[b];
-  const long long pos = r.len - n_new + (i - a.append_indptr[b]);
-  if (r.err || pos < 0 || pos >= r.len) {
-    if (lane == 0 && a.err) atomicOr(a.err, r.err ? r.err : kErrAppend);
-    return;
-  }
-  const int page = a.indices[(long long)r.page_base + pos / a.page_size];
-  if (page < 0 || (long long)page >= a.num_pages) {
-    if (lane == 0 && a.err) atomicOr(a.err, kErrPageId);
-    return;
-  }
-  const long long slot = pos % a.page_size;
-  const int vecs = a.head_dim / 8;    // 16-byte vectors per row
-  const size_t src = ((size_t)i * a.hkv + h) * a.head_dim;
-  const size_t dk = ((((size_t)page * 2 + 0) * a.hkv + h) * a.page_size + slot) * a.head_dim;
-  const size_t dv = ((((size_t)page * 2 + 1) * a.hkv + h) * a.page_size + slot) * a.head_dim;
-  const uint16_t* kn = static_cast<const uint16_t*>(a.k_new);
-  const uint16_t* vn = static_cast<const uint16_t*>(a.v_new);
-  uint16_t* pool = static_cast<uint16_t*>(a.pool);
-  for (int e = lane; e < 2 * vecs; e += 32) {
-    const bool is_v = e >= vecs;
-    const int x = (is_v ? e - vecs : e) * 8;
-    const uint4 val = *reinterpret_cast<const uint4*>((is_v ? vn : kn) + src + x);
-    *reinterpret_cast<uint4*>(pool + (is_v ? dv : dk) + x) = val;
+  const int warp = threadIdx.x >> 5;
+  for (int b = blockIdx.x; b < a.batch; b += gridDim.x) {
+    const int a0 = a.append_indptr[b], a1 = a.append_indptr[b + 1];
+    const ReqInfo r = request_info(a.indptr, a.last_len, b, a.page_size);
+    const long long n_new = (long long)a1 - a0;
+    if (n_new == 0) continue;
+    if (a0 < 0 || n_new < 0 || a1 > a.nnz || r.err || n_new > r.len) {
+      if (threadIdx.x == 0 && blockIdx.y == 0 && a.err) atomicOr(a.err, r.err ? r.err : kErrAppend);
+      continue;
+    }
+    const long long rows = n_new * a.hkv;
+    for (long long row = (long long)blockIdx.y * kWarps + warp; row < rows;
+         row += (long long)gridDim.y * kWarps) {
+      const long long i = row / a.hkv;  // new token within the request
+      const int h = (int)(row % a.hkv);
+      const long long pos = r.len - n_new + i;
+      const int page = a.indices[(long long)r.page_base + pos / a.page_size];
+      if (page < 0 || (long long)page >= a.num_pages) {
+        if (lane == 0 && a.err) atomicOr(a.err, kErrPageId);
+        continue;
+      }
+      const long long slot = pos % a.page_size;
+      const int vecs = a.head_dim / 8;  // 16-byte vectors per row
+      const size_t src = ((size_t)(a0 + i) * a.hkv + h) * a.head_dim;
+      const size_t dk = ((((size_t)page * 2 + 0) * a.hkv + h) * a.page_size + slot) * a.head_dim;
+      const size_t dv = ((((size_t)page * 2 + 1) * a.hkv + h) * a.page_size + slot) * a.head_dim;
+      const uint16_t* kn = static_cast<const uint16_t*>(a.k_new);
+      const uint16_t* vn = static_cast<const uint16_t*>(a.v_new);
+      uint16_t* pool = static_cast<uint16_t*>(a.pool);
+      for (int e = lane; e < 2 * vecs; e += 32) {
+        const bool is_v = e >= vecs;
+        const int x = (is_v ? e - vecs : e) * 8;
+        const uint4 val = *reinterpret_cast<const uint4*>((is_v ? vn : kn) + src + x);
+        *reinterpret_cast<uint4*>(pool + (is_v ? dv : dk) + x) = val;
+      }
+    }
   }
 }
 
 }  // namespace
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
-  const long long warps = a.nnz * a.hkv;
-  if (warps == 0) return cudaSuccess;
-  const long long blocks = (warps + kWarps - 1) / kWarps;
-  append_kernel<<<(unsigned)blocks, kWarps * 32, 0, stream>>>(a);
+  if (a.nnz == 0 || a.batch == 0) return cudaSuccess;
+  const unsigned gx = (unsigned)(a.batch < 65535 ? a.batch : 65535);
+  // split a request's rows over more blocks when the average request appends many
+  const long long avg_rows = (a.nnz * a.hkv + a.batch - 1) / a.batch;
+  long long gy = (avg_rows + 4 * kWarps - 1) / (4 * kWarps);
+  gy = gy < 1 ? 1 : (gy > 1024 ? 1024 : gy);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(gx, (unsigned)gy);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, append_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

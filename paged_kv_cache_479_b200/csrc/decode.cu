@@ -70,8 +70,13 @@ constexpr int kTileBytes = 2 * kHalfBytes;        // K or V of one tile: 4 KiB
 constexpr int kSlotBytes = 2 * kTileBytes;        // K + V: 8 KiB
 constexpr int kSegRecs = 8;
 constexpr int kMaxGroup = 8;
+constexpr int kQBufs = 4;                         // staged query blocks in flight
+constexpr int kQBufBytes = kMaxGroup * 128 * 2;   // G query rows: up to 2 KiB
 constexpr int kScratchStride = kD + 4;
 constexpr float kLn2 = 0.6931471805599453f;
+
+// a partition's first and last pair are the only ones it can share with others
+constexpr int kMaxPending = 2;
 
 // TileMeta bits
 constexpr int kMetaValid = 0x1f;
@@ -88,13 +93,16 @@ struct __align__(16) Ctl {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t cons;                      // consumer-only barrier (256 arrivals)
+  uint64_t qfull[kQBufs];             // a segment's query rows landed in qbuf[i]
   int meta[kStages];
   SegRec seg[kSegRecs];
   long long warp_tot[kDecodeThreads / 32];
   long long Cb0;
+  SegRec pend[kMaxPending];   // split pairs this CTA wrote partial states for
+  int pend_last[kMaxPending]; // 1 when this CTA arrived last for that pair
+  int npend;
   int b0;
   int abort;
-  int merge_last;
   int pad_;
 };
 
@@ -105,7 +113,8 @@ struct Scratch {
 };
 
 constexpr size_t kRingBytes = (size_t)kStages * kSlotBytes;
-constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + sizeof(Ctl) + sizeof(Scratch);
+constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + (size_t)kQBufs * kQBufBytes +
+                              sizeof(Ctl) + sizeof(Scratch);
 
 // inclusive scan over the whole block (kDecodeThreads threads); returns the
 // prefix for this thread and the block total in *total
@@ -150,8 +159,9 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   // 128-byte-swizzled TMA boxes need 1024-byte aligned shared addresses
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* ring = smem;
-  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + kRingBytes);
-  Scratch& scr = *reinterpret_cast<Scratch*>(smem + kRingBytes + sizeof(Ctl));
+  uint8_t* qbuf = smem + kRingBytes;
+  Ctl& ctl = *reinterpret_cast<Ctl*>(qbuf + (size_t)kQBufs * kQBufBytes);
+  Scratch& scr = *reinterpret_cast<Scratch*>(reinterpret_cast<uint8_t*>(&ctl) + sizeof(Ctl));
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -166,25 +176,31 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       mbar_init(smem_u32(&ctl.empty[s]), 32);
     }
     mbar_init(smem_u32(&ctl.cons), kConsumerThreads);
+    for (int i = 0; i < kQBufs; ++i) mbar_init(smem_u32(&ctl.qfull[i]), 1);
     ctl.abort = 0;
     ctl.b0 = -1;
+    ctl.npend = 0;
     fence_barrier_init();
   }
   if (warp == kConsumerWarps && lane == 0) prefetch_tensormap(&tmap);
+  // With programmatic dependent launch this CTA may start while the previous
+  // kernel in the stream still runs; everything above touched no input.
+  grid_dependency_wait();
+  grid_dependents_launch();
 
   // ---- prologue: total work W, this partition's share [f0, f1), its first request
   long long mine = 0;
   int errs = 0;
   for (int b = tid; b < B; b += kDecodeThreads) {
     const ReqInfo r = request_info(a.indptr, a.last_len, b, a.page_size);
-    mine += r.tiles;
+    mine += r.units;
     errs |= r.err;
   }
   if (errs && c == 0 && a.err) atomicOr(a.err, errs);
-  long long total_tiles;
-  (void)block_incl_scan(mine, ctl.warp_tot, &total_tiles);
-  const long long W = (long long)Hkv * total_tiles;
-  // with fewer tiles than CTAs only the first W partitions get work, so that
+  long long total_units;
+  (void)block_incl_scan(mine, ctl.warp_tot, &total_units);
+  const long long W = (long long)Hkv * total_units;
+  // with fewer units than CTAs only the first W partitions get work, so that
   // every partition that covers a (request, kv head) pair is non-empty
   const int N = W < (long long)gridDim.x ? (int)W : (int)gridDim.x;
   const long long f0 = c < N ? part_start(W, N, c) : 0;
@@ -195,12 +211,13 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     const int b = base + tid;
     ReqInfo r;
     r.tiles = 0;
+    r.units = 0;
     r.len = 0;
     if (b < B) r = request_info(a.indptr, a.last_len, b, a.page_size);
     long long chunk_total;
-    const long long incl = block_incl_scan(r.tiles, ctl.warp_tot, &chunk_total);
-    const long long excl = incl - r.tiles;
-    if (b < B && r.tiles > 0 && f0 < f1) {
+    const long long incl = block_incl_scan(r.units, ctl.warp_tot, &chunk_total);
+    const long long excl = incl - r.units;
+    if (b < B && r.units > 0 && f0 < f1) {
       const long long s0 = (long long)Hkv * (carry + excl), s1 = (long long)Hkv * (carry + incl);
       if (s0 <= f0 && f0 < s1) {
         ctl.b0 = b;
@@ -236,8 +253,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     int seg = 0;
     bool ok = true;
     while (ok && !wk.done()) {
-      const long long n = wk.seg_tiles();
-      if (n <= 0) {  // only possible if the table changed under the kernel
+      if (wk.seg_units() <= 0) {  // only possible if the table changed under the kernel
         if (lane == 0) {
           if (a.err) atomicOr(a.err, kErrIndptr);
           ctl.abort = 1;
@@ -245,10 +261,16 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         ok = false;
         break;
       }
+      const long long t0 = wk.t0();
+      const long long n = wk.t1() - t0;
+      if (n == 0) {  // this share of the pair holds only its fixed-cost units
+        wk.advance();
+        continue;
+      }
       const long long n_pad = (n + kConsumerWarps - 1) / kConsumerWarps * kConsumerWarps;
       const long long pstart = wk.pair_start();
       if (lane == 0) {
-        const SegPlace pl = seg_place(W, N, pstart, wk.ri.tiles, c);
+        const SegPlace pl = seg_place(W, N, pstart, wk.ri.units, c);
         SegRec& r = ctl.seg[seg & (kSegRecs - 1)];
         r.b = wk.b;
         r.kvh = wk.kvh;
@@ -256,6 +278,15 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         r.c_first = pl.c_first;
         r.ncover = pl.ncover;
         r.pair_start = pstart;
+        // stage the segment's G query rows (contiguous in q) for the consumers
+        const int qb = seg & (kQBufs - 1);
+        const uint32_t qbar = smem_u32(&ctl.qfull[qb]);
+        const uint32_t qbytes = (uint32_t)a.group * kD * 2;
+        mbar_arrive_expect_tx(qbar, qbytes);
+        bulk_load(smem_u32(qbuf + (size_t)qb * kQBufBytes),
+                  static_cast<const uint16_t*>(a.q) +
+                      ((size_t)wk.b * a.hq + (size_t)wk.kvh * a.group) * kD,
+                  qbytes, qbar);
         // last segment of this request: warm L2 with the next request's table entries
         if (wk.kvh == Hkv - 1 && wk.b + 1 < B) {
           prefetch_l2(a.indptr + wk.b + 2);
@@ -267,10 +298,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       // page ids, one tile per lane, loaded one 32-tile batch ahead of their use
       const int* idx = a.indices + wk.ri.page_base;
       int page_next = -1;
-      if (lane < n) page_next = idx[(wk.t + lane) * kTileTokens / ps];
+      if (lane < n) page_next = idx[(t0 + lane) * kTileTokens / ps];
       for (long long k0 = 0; ok && k0 < n_pad; k0 += 32) {
         int page = page_next;
-        if (k0 + 32 + lane < n) page_next = idx[(wk.t + k0 + 32 + lane) * kTileTokens / ps];
+        if (k0 + 32 + lane < n) page_next = idx[(t0 + k0 + 32 + lane) * kTileTokens / ps];
         const long long k = k0 + lane;
         int yoff = 0, valid = 0;
         if (k < n) {
@@ -278,7 +309,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
             if (a.err) atomicOr(a.err, kErrPageId);
             page = -1;
           }
-          const long long tok0 = (wk.t + k) * kTileTokens;
+          const long long tok0 = (t0 + k) * kTileTokens;
           yoff = (int)(tok0 % ps);
           const long long left = wk.ri.len - tok0;
           valid = left < kTileTokens ? (int)left : kTileTokens;
@@ -353,6 +384,14 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
                global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
+      for (int qb = 0; qb < kQBufs && qb < seg; ++qb) {
+        const int last = seg - 1 - ((seg - 1 - qb) % kQBufs);  // latest segment using qbuf qb
+        const uint32_t bar = smem_u32(&ctl.qfull[qb]);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bar, (uint32_t)(last / kQBufs) & 1u) &&
+               global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
     }
     return;
   }
@@ -374,10 +413,14 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   rec.b = 0;
   rec.kvh = 0;
   uint32_t cons_phase = 0;
+  bool clean = true;
 
   for (uint32_t i = warp;; i += kConsumerWarps) {
     const int s = (int)(i % kStages);
-    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kStages) & 1u, &ctl.abort, a.err)) break;
+    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kStages) & 1u, &ctl.abort, a.err)) {
+      clean = false;
+      break;
+    }
     const int info = ctl.meta[s];
     if (info & kMetaEnd) break;
     const int sid = (info >> kMetaSegShift) & (kSegRecs - 1);
@@ -388,12 +431,19 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         // never expected: a corrupted record would address out of bounds
         if (lane == 0 && a.err) atomicOr(a.err, kErrTimeout);
         ctl.abort = 1;
+        clean = false;
         break;
       }
-      const int h = rec.kvh * G + g;
+      // the segment's query rows, staged by the producer
+      const int qb = sid & (kQBufs - 1);
+      if (!mbar_wait_bounded(smem_u32(&ctl.qfull[qb]), (uint32_t)(sid >> 2) & 1u, &ctl.abort,
+                             a.err)) {
+        clean = false;
+        break;
+      }
       if (g < G) {
         const uint16_t* qp =
-            static_cast<const uint16_t*>(a.q) + ((size_t)rec.b * a.hq + h) * kD + 2 * cq;
+            reinterpret_cast<const uint16_t*>(qbuf + (size_t)qb * kQBufBytes) + g * kD + 2 * cq;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           qf[j][0] = ld_u32(qp + j * 16);
@@ -502,7 +552,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 
     if (info & kMetaSegLast) {
       // ================= end of segment: merge the 8 warps' states =================
-      if (!cons_sync(ctl, cons_phase, a.err)) break;  // previous merge done with scratch
+      if (!cons_sync(ctl, cons_phase, a.err)) {  // previous merge done with scratch
+        clean = false;
+        break;
+      }
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, off);
@@ -521,7 +574,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         scr.o[warp][2 * cq][mt * 16 + g + 8] = o[mt][2];
         scr.o[warp][2 * cq + 1][mt * 16 + g + 8] = o[mt][3];
       }
-      if (!cons_sync(ctl, cons_phase, a.err)) break;
+      if (!cons_sync(ctl, cons_phase, a.err)) {
+        clean = false;
+        break;
+      }
       const bool direct = rec.ncover == 1;
       for (int e = ct; e < G * kD; e += kConsumerThreads) {
         const int h = e >> 7, d = e & (kD - 1);
@@ -545,40 +601,69 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           if (d == 0) a.part_lse[(size_t)rec.slot * G + h] = M + log2f(L);
         }
       }
-      if (!direct) {
-        __threadfence();
-        if (!cons_sync(ctl, cons_phase, a.err)) break;
-        if (ct == 0) {
-          const int old = atomicAdd(&a.counters[rec.c_first], 1);
-          ctl.merge_last = (old == rec.ncover - 1);
-        }
-        if (!cons_sync(ctl, cons_phase, a.err)) break;
-        if (ctl.merge_last) {
-          // this partition arrived last: merge the pair's partial states
-          __threadfence();
-          const long long pstart = rec.pair_start;
-          for (int e = ct; e < G * kD; e += kConsumerThreads) {
-            const int h = e >> 7, d = e & (kD - 1);
-            float M = -INFINITY;
-            for (int k = 0; k < rec.ncover; ++k) {
-              const int sl = state_slot(W, N, pstart, rec.c_first, rec.c_first + k);
-              M = fmaxf(M, __ldcg(a.part_lse + (size_t)sl * G + h));
-            }
-            float L = 0.f, acc = 0.f;
-            for (int k = 0; k < rec.ncover; ++k) {
-              const int sl = state_slot(W, N, pstart, rec.c_first, rec.c_first + k);
-              const float wt = ex2(__ldcg(a.part_lse + (size_t)sl * G + h) - M);
-              L += wt;
-              acc += wt * __ldcg(a.part_o + ((size_t)sl * G + h) * kD + d);
-            }
-            const size_t row = (size_t)rec.b * a.hq + (size_t)rec.kvh * G + h;
-            static_cast<uint16_t*>(a.out)[row * kD + d] = to_bits16<BF16>(acc / L);
-            if (d == 0 && a.lse) a.lse[row] = (M + log2f(L)) * kLn2;
-          }
-          if (ct == 0) a.counters[rec.c_first] = 0;  // ready for the next launch
+      if (!direct && ct == 0 && ctl.npend < kMaxPending) ctl.pend[ctl.npend++] = rec;
+    }
+  }
+  if (!clean || ctl.abort) return;
+
+  // ============ end of the partition: split pairs, last arrival merges ============
+  __threadfence();  // this CTA's partial states are visible before it counts itself in
+  if (!cons_sync(ctl, cons_phase, a.err)) return;
+  const int npend = ctl.npend;
+  if (ct == 0)
+    for (int k = 0; k < npend; ++k) {
+      const int old = atomicAdd(&a.counters[ctl.pend[k].c_first], 1);
+      ctl.pend_last[k] = (old == ctl.pend[k].ncover - 1);
+      // the last arrival is the pair's only remaining user of the counter
+      if (ctl.pend_last[k]) a.counters[ctl.pend[k].c_first] = 0;
+    }
+  if (!cons_sync(ctl, cons_phase, a.err)) return;
+  __threadfence();
+  // one warp per (pair, head); lane L owns dims 4L .. 4L+3
+  for (int item = warp; item < npend * G; item += kConsumerWarps) {
+    const int k = item / G, h = item % G;
+    if (!ctl.pend_last[k]) continue;
+    const SegRec pr = ctl.pend[k];
+    auto slot_of = [&](int j) { return state_slot(pr.c_first, j); };
+    float M = -INFINITY;
+    for (int j = lane; j < pr.ncover; j += 32)
+      M = fmaxf(M, __ldcg(a.part_lse + (size_t)slot_of(j) * G + h));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    constexpr int kBatch = 8;  // partial states loaded together
+    for (int j0 = 0; j0 < pr.ncover; j0 += kBatch) {
+      float wt[kBatch];
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = j0 + u;
+        if (j < pr.ncover) {
+          const int sl = slot_of(j);
+          wt[u] = __ldcg(a.part_lse + (size_t)sl * G + h);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * G + h) * kD) + lane);
+        } else {
+          wt[u] = -INFINITY;
+          v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const float w = ex2(wt[u] - M);
+        L += w;
+        acc.x += w * v[u].x;
+        acc.y += w * v[u].y;
+        acc.z += w * v[u].z;
+        acc.w += w * v[u].w;
+      }
     }
+    const float inv = 1.f / L;
+    const size_t row = (size_t)pr.b * a.hq + (size_t)pr.kvh * G + h;
+    uint16_t* op = static_cast<uint16_t*>(a.out) + row * kD + 4 * lane;
+    *reinterpret_cast<uint2*>(op) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv),
+                                               pack2<BF16>(acc.z * inv, acc.w * inv));
+    if (lane == 0 && a.lse) a.lse[row] = (M + log2f(L)) * kLn2;
   }
 }
 
@@ -600,7 +685,20 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[bf16][dev] = true;
   }
-  kern<<<grid, kDecodeThreads, kSmemBytes, stream>>>(tmap, a);
+  // programmatic dependent launch: CTAs may become resident while the previous
+  // kernel drains; the kernel waits for it before reading any input
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmap, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -102,41 +102,61 @@ def _tiles(w):
     return [int(-(-int(L) // 16)) for L in w.kv_lens]
 
 
+def reference_plan(w, N, cost):
+    """The split-KV partition written out from its definition: pair (b, g)
+    occupies `cost` fixed units followed by its tiles in the flattened (b, g)
+    order; partition c takes units [floor(cW/N), floor((c+1)W/N)); a pair's
+    partial-state slot is 2c + 1 in its first covering partition, 2c in the
+    others, and -1 when one partition holds all its tiles."""
+    tiles = _tiles(w)
+    units = [t + cost if t else 0 for t in tiles]
+    W = w.num_kv_heads * sum(units)
+    if W == 0:
+        return []
+    N = min(N, W)
+    bounds = [c * W // N for c in range(N + 1)]
+    rows = []
+    start = 0
+    for b in range(w.batch):
+        for g in range(w.num_kv_heads):
+            lo_real, hi_real = start + cost, start + units[b]
+            parts = []
+            for c in range(N):
+                lo, hi = max(bounds[c], lo_real), min(bounds[c + 1], hi_real)
+                if lo < hi:
+                    parts.append((c, lo - lo_real, hi - lo_real))
+            for j, (c, t0, t1) in enumerate(parts):
+                slot = -1 if len(parts) == 1 else 2 * c + (1 if j == 0 else 0)
+                rows.append((c, b, g, t0, t1, slot, len(parts)))
+            start += units[b]
+    return sorted(rows)
+
+
+def library_cost():
+    """The fixed per-pair cost the library charges, recovered from a probe plan."""
+    w = wl.make_workload("probe", [16, 1, 40, 300, 17], num_qo_heads=4, num_kv_heads=2,
+                         page_size=16, dtype="f16", seed=2)
+    got = sorted(map(tuple, pkv.plan_segments(w.page_indptr, w.last_page_len, 16, 2, 7).tolist()))
+    costs = [k for k in range(0, 65) if reference_plan(w, 7, k) == got]
+    assert len(costs) == 1, costs
+    return costs[0]
+
+
 def check_plan(w, N):
     seg = pkv.plan_segments(w.page_indptr, w.last_page_len, w.page_size, w.num_kv_heads, N)
+    got = sorted(map(tuple, seg.tolist()))
+    assert got == reference_plan(w, N, library_cost())
     tiles = _tiles(w)
-    W = w.num_kv_heads * sum(tiles)
-    N = min(N, W)          # partitions beyond the tile count get no work
     # every (request, kv head, tile) exactly once
-    cover = {}
-    for c, b, g, t0, t1, slot, ncov in seg:
-        assert 0 <= t0 < t1 <= tiles[b]
+    cover = set()
+    for c, b, g, t0, t1, slot, ncov in got:
         for t in range(t0, t1):
-            key = (b, g, t)
-            assert key not in cover
-            cover[key] = c
-    assert len(cover) == W
-    # each partition streams floor((c+1)W/N) - floor(cW/N) tiles, in flat order
-    per = np.zeros(N, np.int64)
-    for c, b, g, t0, t1, *_ in seg:
-        per[c] += t1 - t0
-    expect = np.array([(c + 1) * W // N - c * W // N for c in range(N)])
-    assert np.array_equal(per, expect)
-    assert per.max() - per.min() <= 1
-    # state slots: unique, < 2N, present exactly when the pair is split
-    pairs = {}
-    slots = set()
-    for c, b, g, t0, t1, slot, ncov in seg:
-        pairs.setdefault((b, g), []).append((c, slot, ncov))
-        if ncov == 1:
-            assert slot == -1
-        else:
-            assert 0 <= slot < 2 * N and slot // 2 == c and slot not in slots
-            slots.add(slot)
-    for (b, g), parts in pairs.items():
-        assert all(p[2] == len(parts) for p in parts)
-        cs = [p[0] for p in parts]
-        assert cs == list(range(cs[0], cs[0] + len(cs)))
+            assert (b, g, t) not in cover
+            cover.add((b, g, t))
+    assert len(cover) == w.num_kv_heads * sum(tiles)
+    # state slots unique and below 2N
+    slots = [r[5] for r in got if r[5] >= 0]
+    assert len(slots) == len(set(slots)) and all(0 <= x < 2 * N for x in slots)
     return seg
 
 
@@ -161,3 +181,18 @@ def test_partition_long_single_sequence_fills_all_partitions():
     seg = check_plan(w, 148)
     assert set(seg[:, 0].tolist()) == set(range(148))
     assert (seg[:, 6] > 1).all()   # every pair is split, so every segment merges
+    per = np.bincount(seg[:, 0], weights=seg[:, 4] - seg[:, 3])
+    assert per.max() - per.min() <= library_cost() + 1
+
+
+def test_partition_balances_time_weighted_work():
+    # each partition's tiles plus the fixed cost of the pairs it starts is the
+    # same up to one pair's fixed cost and rounding
+    w = wl.named(5)
+    N = 148
+    seg = check_plan(w, N)
+    cost = library_cost()
+    work = np.zeros(N)
+    for c, b, g, t0, t1, slot, ncov in seg:
+        work[c] += (t1 - t0) + (cost if t0 == 0 else 0)
+    assert work.max() - work.min() <= 2 * cost + 2
