@@ -64,6 +64,26 @@ def dist_env():
     return rank, world, local
 
 
+def rank_value_seed(base_seed, rank, copy):
+    """Seed of the values of batch copy `copy` on `rank`: every rank decodes its own
+    independent batch of the same shape (weak scaling)."""
+    return base_seed + 1000 * rank + copy
+
+
+def max_over_ranks(x, world, device):
+    """Max of a float over all ranks (the slowest rank times the job)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step_per_rank, world, ms_total, steps):
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
+    return bytes_per_step_per_rank * world / (ms_total / 1e3 / steps) / 1e9
+
+
 def measured_hbm():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -299,18 +319,11 @@ def run_pkv(args):
         if world > 1:
             torch.distributed.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
-
     w = wl.named(args.workload)
     N = args.partitions or pkv.default_partitions(local)
     kv_bytes = wl.logical_kv_bytes(w)
     rotation = 2 if kv_bytes < (2 << 30) else 1
-    batches = [Batch(w, dev, w.seed + 1000 * rank + r) for r in range(rotation)]
+    batches = [Batch(w, dev, rank_value_seed(w.seed, rank, r)) for r in range(rotation)]
     t = lambda a: torch.as_tensor(a, device=dev)
     indptr, indices, last = t(w.page_indptr), t(w.page_indices), t(w.last_page_len)
     app = t(w.append_indptr)
@@ -357,14 +370,14 @@ def run_pkv(args):
     barrier()
     ms_local = start.elapsed_time(end)
     decode_ms = sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K
-    ms = max_over_ranks(ms_local)
-    decode_ms_max = max_over_ranks(decode_ms)
+    ms = max_over_ranks(ms_local, world, dev)
+    decode_ms_max = max_over_ranks(decode_ms, world, dev)
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during the timed steps")
 
     step_bytes = algorithmic_bytes(w)
     s_per_step = ms / 1e3 / K
-    value = step_bytes * world / s_per_step / 1e9
+    value = job_throughput(step_bytes, world, ms, K)
     dec_bytes = wl.decode_bytes(w)
     peak, peak_kind = measured_hbm()
     achieved = dec_bytes / (decode_ms_max / 1e3) / 1e9
@@ -406,8 +419,8 @@ def run_pkv(args):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": round(step_bytes * world / (e_ms / 1e3 / K) / 1e9, 2), "unit": "GB/s",
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": round(job_throughput(step_bytes, world, e_ms, K), 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "us_per_step": round(e_ms / K * 1e3, 2),
                "path": "pinned host -> device (1 copy), append + decode, device -> pinned host "
