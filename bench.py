@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--partitions", type=int, default=0, help="split-KV partitions (0 = one per SM)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="launch every call from Python instead of replaying CUDA graphs")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for cpu_baseline")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="oracle time budget of the reference arm")
     return p.parse_args()
@@ -335,24 +337,47 @@ def run_pkv(args):
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 1 + (1 if w.nnz_new else 0)
 
-    def step(bt, ev0=None, ev1=None):
+    def append_call(bt):
         if w.nnz_new:
             pkv.paged_kv_append(bt.pool, indptr, indices, last, bt.k_new, bt.v_new, app,
-                                error_word=err, stream=stream)
-        if ev0 is not None:
-            ev0.record(stream)
+                                error_word=err, stream=torch.cuda.current_stream(dev))
+
+    def decode_call(bt):
         pkv.paged_decode_attention(bt.q, bt.pool, indptr, indices, last, ws, out=out, lse=lse,
                                    sm_scale=w.sm_scale, num_partitions=N, error_word=err,
-                                   stream=stream)
-        if ev1 is not None:
-            ev1.record(stream)
+                                   stream=torch.cuda.current_stream(dev))
 
     clocks = ClockSampler(local)
     for i in range(args.warmup):
-        step(batches[i % rotation])
+        append_call(batches[i % rotation])
+        decode_call(batches[i % rotation])
     torch.cuda.synchronize()
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during warm-up")
+
+    # the same calls captured once per batch copy and replayed (no Python on the
+    # launch path); each library call is capturable: no allocation, no sync
+    def graphed(fn, bt):
+        if args.no_graph:
+            return lambda: fn(bt)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(bt)
+        return g.replay
+    app_g = [graphed(append_call, bt) if w.nnz_new else (lambda: None) for bt in batches]
+    dec_g = [graphed(decode_call, bt) for bt in batches]
+    for i in range(2 * rotation):
+        app_g[i % rotation]()
+        dec_g[i % rotation]()
+    torch.cuda.synchronize()
+
+    def step(r, ev0=None, ev1=None):
+        app_g[r]()
+        if ev0 is not None:
+            ev0.record(stream)
+        dec_g[r]()
+        if ev1 is not None:
+            ev1.record(stream)
 
     K = args.steps
     d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -363,7 +388,7 @@ def run_pkv(args):
     t_host0 = time.time()
     start.record(stream)
     for i in range(K):
-        step(batches[i % rotation], d0[i], d1[i])
+        step(i % rotation, d0[i], d1[i])
     end.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.time()
@@ -397,15 +422,23 @@ def run_pkv(args):
         out_d, lse_d = d_out
         h2d, d2h = h_in[0].numel(), h_out[0].numel()
 
-        def e2e_step():
+        def e2e_calls(_):
+            cur = torch.cuda.current_stream(dev)
             h_in[1].copy_(h_in[0], non_blocking=True)
             if w.nnz_new:
                 pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d, error_word=err,
-                                    stream=stream)
+                                    stream=cur)
             pkv.paged_decode_attention(q_d, src.pool, ip_d, ix_d, ll_d, ws, out=out_d, lse=lse_d,
                                        sm_scale=w.sm_scale, num_partitions=N, error_word=err,
-                                       stream=stream)
+                                       stream=cur)
             h_out[0].copy_(h_out[1], non_blocking=True)
+
+        e2e_calls(None)
+        torch.cuda.synchronize()
+        e2e_replay = graphed(e2e_calls, None)
+
+        def e2e_step():
+            e2e_replay()
             stream.synchronize()   # the caller needs the result before the next step
 
         for _ in range(args.warmup):
@@ -424,7 +457,8 @@ def run_pkv(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "us_per_step": round(e_ms / K * 1e3, 2),
                "path": "pinned host -> device (1 copy), append + decode, device -> pinned host "
-                       "(1 copy), stream sync every step"}
+                       "(1 copy), stream sync every step" +
+                       ("" if args.no_graph else "; the step's calls replayed as one CUDA graph")}
     clocks.stop()
 
     if rank == 0:
@@ -434,7 +468,9 @@ def run_pkv(args):
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f16", "data": "synthetic",
-            "config": workload_config(w, args, rotation, N),
+            "config": {**workload_config(w, args, rotation, N),
+                       "launch": "direct calls" if args.no_graph else
+                       "append and decode each captured once per batch copy as a CUDA graph, replayed"},
             "us_per_step": round(ms / K * 1e3, 2),
             "tokens_per_s": round(w.batch * world / s_per_step, 1),
             "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
