@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--partitions", type=int, default=0, help="split-KV partitions (0 = one per SM)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cascade", action="store_true",
+                   help="decode a shared-prefix workload with pkv_cascade_decode")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every call from Python instead of replaying CUDA graphs")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for cpu_baseline")
@@ -192,6 +194,8 @@ def workload_config(w, args, rotation, partitions):
            "parallelism": f"dp{args.gpus} (independent batches per GPU)"}
     if w.note:
         cfg["values"] = w.note
+    if getattr(args, "cascade", False):
+        cfg["method"] = "shared-prefix cascade: prefix attention once per 128 query rows, own pages by the decode kernel, states merged"
     return cfg
 
 
@@ -322,6 +326,8 @@ def run_pkv(args):
             torch.distributed.barrier()
 
     w = wl.named(args.workload)
+    if args.cascade and not w.shared_prefix_pages:
+        raise SystemExit("--cascade needs a workload with a shared prefix (workload 5)")
     N = args.partitions or pkv.default_partitions(local)
     kv_bytes = wl.logical_kv_bytes(w)
     rotation = 2 if kv_bytes < (2 << 30) else 1
@@ -330,12 +336,19 @@ def run_pkv(args):
     indptr, indices, last = t(w.page_indptr), t(w.page_indices), t(w.last_page_len)
     app = t(w.append_indptr)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws = torch.zeros(pkv.decode_workspace_bytes(w.batch, w.num_qo_heads, w.num_kv_heads, 128, N) // 4 + 64,
-                     dtype=torch.int32, device=dev)
+    if args.cascade:
+        c_prefix, c_len, c_ip, c_ix, c_ll = wl.cascade_view(w)
+        c_prefix, c_ip, c_ix, c_ll = (t(np.ascontiguousarray(x, np.int32)) for x in
+                                      (c_prefix, c_ip, c_ix, c_ll))
+        ws_bytes = pkv.cascade_workspace_bytes(w.batch, w.num_qo_heads, w.num_kv_heads, c_len,
+                                               num_partitions=N)
+    else:
+        ws_bytes = pkv.decode_workspace_bytes(w.batch, w.num_qo_heads, w.num_kv_heads, 128, N)
+    ws = torch.zeros(ws_bytes // 4 + 64, dtype=torch.int32, device=dev)
     out = torch.empty_like(batches[0].q)
     lse = torch.empty((w.batch, w.num_qo_heads), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 1 + (1 if w.nnz_new else 0)
+    launches_per_step = (3 if args.cascade else 1) + (1 if w.nnz_new else 0)
 
     def append_call(bt):
         if w.nnz_new:
@@ -343,6 +356,11 @@ def run_pkv(args):
                                 error_word=err, stream=torch.cuda.current_stream(dev))
 
     def decode_call(bt):
+        if args.cascade:
+            pkv.cascade_decode(bt.q, bt.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws, out=out,
+                               lse=lse, sm_scale=w.sm_scale, num_partitions=N, error_word=err,
+                               stream=torch.cuda.current_stream(dev))
+            return
         pkv.paged_decode_attention(bt.q, bt.pool, indptr, indices, last, ws, out=out, lse=lse,
                                    sm_scale=w.sm_scale, num_partitions=N, error_word=err,
                                    stream=torch.cuda.current_stream(dev))
@@ -428,9 +446,14 @@ def run_pkv(args):
             if w.nnz_new:
                 pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d, error_word=err,
                                     stream=cur)
-            pkv.paged_decode_attention(q_d, src.pool, ip_d, ix_d, ll_d, ws, out=out_d, lse=lse_d,
-                                       sm_scale=w.sm_scale, num_partitions=N, error_word=err,
-                                       stream=cur)
+            if args.cascade:
+                pkv.cascade_decode(q_d, src.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws,
+                                   out=out_d, lse=lse_d, sm_scale=w.sm_scale, num_partitions=N,
+                                   error_word=err, stream=cur)
+            else:
+                pkv.paged_decode_attention(q_d, src.pool, ip_d, ix_d, ll_d, ws, out=out_d,
+                                           lse=lse_d, sm_scale=w.sm_scale, num_partitions=N,
+                                           error_word=err, stream=cur)
             h_out[0].copy_(h_out[1], non_blocking=True)
 
         e2e_calls(None)
@@ -462,7 +485,7 @@ def run_pkv(args):
     clocks.stop()
 
     if rank == 0:
-        traffic = recorded_traffic(args.workload)
+        traffic = None if args.cascade else recorded_traffic(args.workload)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
@@ -475,7 +498,10 @@ def run_pkv(args):
             "tokens_per_s": round(w.batch * world / s_per_step, 1),
             "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
-            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
+            "roofline": {"bound": "hbm",
+                         "kernel": ("pkv_cascade_decode (prefix + own-page decode + merge launches)"
+                                    if args.cascade else "decode_kernel"),
+                         "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",

@@ -161,6 +161,44 @@ PKV_API pkv_status pkv_decode(const void* q, int num_qo_heads,
                       void* out, float* lse, int32_t* error_word, void* stream);
 
 /*
+ * pkv_cascade_decode -- pkv_decode for a batch whose requests all begin with
+ * the same shared prefix (a system prompt stored once in shared pages: physical
+ * page sharing between requests with a common prefix, "大模型推理极致优化：
+ * FlashAttention+PageAttention联合调优" section 3.2; automatic prefix reuse,
+ * "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署" section 3.3).
+ *
+ * Request b attends over the prefix's prefix_len tokens followed by its own
+ * tokens; the result equals pkv_decode on the concatenated page lists up to
+ * fp32 rounding.  Instead of reading the prefix once per request, the prefix's
+ * K/V are read once per block of 128 (request, query head) rows and multiplied
+ * on tensor cores against all requests' queries; each request's own pages go
+ * through the decode kernel; the two attention states are merged by their
+ * log-sum-exp weights.
+ *
+ *   prefix_page_indices  device int32 [ceil(prefix_len / page_size)]: the prefix's
+ *                        pages in order (the last one holds the remainder)
+ *   prefix_len           prefix tokens (0: plain pkv_decode)
+ *   page_indptr, page_indices, last_page_len, batch
+ *                        each request's OWN pages after the prefix (CSR; a request
+ *                        with no own tokens has no pages)
+ *   workspace            pkv_cascade_workspace_bytes(), 256-byte aligned, zero-filled
+ *                        before first use (as for pkv_decode)
+ * Other arguments as pkv_decode.  Three launches on `stream`; no allocation.
+ */
+PKV_API size_t pkv_cascade_workspace_bytes(int batch, int num_qo_heads, int num_kv_heads,
+                                           int head_dim, int64_t prefix_len,
+                                           int num_partitions);
+PKV_API pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
+                                      int64_t num_pages, int page_size, int num_kv_heads,
+                                      int head_dim, int dtype,
+                                      const int32_t* prefix_page_indices, int64_t prefix_len,
+                                      const int32_t* page_indptr, const int32_t* page_indices,
+                                      const int32_t* last_page_len, int batch, float sm_scale,
+                                      int num_partitions, void* workspace,
+                                      size_t workspace_bytes, void* out, float* lse,
+                                      int32_t* error_word, void* stream);
+
+/*
  * pkv_merge_states -- merge attention states of disjoint key sets.
  *
  *   v       float [num_rows][num_states][num_heads][head_dim]  normalised partial outputs

@@ -16,12 +16,15 @@ Functions (C names in parentheses):
   check_table            (pkv_check_table)     host-side table check
   plan_segments          (pkv_plan_segments)   host mirror of the split-KV partition
   decode_static_workspace (pkv_decode_static_workspace)  decode on the library's own scratch
+  cascade_decode         (pkv_cascade_decode)  decode for a batch sharing one prefix
 """
 from ._binding import (  # noqa: F401
     BF16,
     F16,
     F32,
     PkvError,
+    cascade_decode,
+    cascade_workspace_bytes,
     check_table,
     decode_static_workspace,
     decode_workspace_bytes,
@@ -43,3 +46,4 @@ pkv_append = paged_kv_append
 pkv_decode = paged_decode_attention
 pkv_decode_static_workspace = decode_static_workspace
 pkv_merge_states = merge_states
+pkv_cascade_decode = cascade_decode

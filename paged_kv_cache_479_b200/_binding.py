@@ -39,6 +39,10 @@ _SIGNATURES = {
 }
 _SIGNATURES["pkv_decode_static_workspace"] = (
     [_P, _I32, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I32, _F32, _I32, _P, _P, _P, _P], _I32)
+_SIGNATURES["pkv_cascade_workspace_bytes"] = ([_I32, _I32, _I32, _I32, _I64, _I32], _SZ)
+_SIGNATURES["pkv_cascade_decode"] = (
+    [_P, _I32, _P, _I64, _I32, _I32, _I32, _I32, _P, _I64, _P, _P, _P, _I32, _F32, _I32, _P, _SZ,
+     _P, _P, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
 _SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
 _SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
@@ -186,6 +190,43 @@ def decode_static_workspace(q, pool, page_indptr, page_indices, last_page_len, o
                                            num_partitions, _ptr(out), _ptr(lse),
                                            _ptr(error_word), _stream(stream, q.device))
     _check(st, "pkv_decode_static_workspace")
+    return out, lse
+
+
+def cascade_workspace_bytes(batch: int, num_qo_heads: int, num_kv_heads: int, prefix_len: int,
+                            head_dim: int = 128, num_partitions: int = 0) -> int:
+    n = lib().pkv_cascade_workspace_bytes(batch, num_qo_heads, num_kv_heads, head_dim,
+                                           int(prefix_len), num_partitions)
+    if n == 0:
+        raise PkvError(1, "pkv_cascade_workspace_bytes: invalid shapes")
+    return int(n)
+
+
+def cascade_decode(q, pool, prefix_pages, prefix_len, page_indptr, page_indices, last_page_len,
+                   workspace, out=None, lse=None, sm_scale=None, num_partitions: int = 0,
+                   error_word=None, stream=None, return_lse: bool = True):
+    """Decode attention for requests that all start with one shared prefix
+    (C: pkv_cascade_decode).  The page table holds each request's own pages."""
+    _dev_tensor(q, "q", pool.dtype)
+    _dev_tensor(pool, "pool")
+    _dev_tensor(workspace, "workspace")
+    for name, t in (("prefix_pages", prefix_pages), ("page_indptr", page_indptr),
+                    ("page_indices", page_indices), ("last_page_len", last_page_len)):
+        _dev_tensor(t, name, torch.int32)
+    B, hq, d = q.shape
+    P, _, hkv, ps, dp = pool.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_cascade_decode(_ptr(q), hq, _ptr(pool), P, ps, hkv, dp, _DTYPES[pool.dtype],
+                                  _ptr(prefix_pages), int(prefix_len), _ptr(page_indptr),
+                                  _ptr(page_indices), _ptr(last_page_len), B, scale,
+                                  num_partitions, _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _ptr(out),
+                                  _ptr(lse), _ptr(error_word), _stream(stream, q.device))
+    _check(st, "pkv_cascade_decode")
     return out, lse
 
 

@@ -173,6 +173,75 @@ pkv_status pkv::set_error(pkv_status s, const char* fmt, ...) {
   return s;
 }
 
+static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool, int64_t num_pages,
+                      int page_size, int num_kv_heads, int head_dim, int dtype,
+                      const int32_t* page_indptr, const int32_t* page_indices,
+                      const int32_t* last_page_len, int batch, float sm_scale,
+                      int num_partitions, void* workspace, size_t workspace_bytes, void* out,
+                      float* lse, int32_t* error_word, void* stream, int out_f32,
+                      long long out_rs, long long lse_rs) {
+  if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1)
+    return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
+  if (dtype != PKV_F16 && dtype != PKV_BF16)
+    return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
+  if (num_qo_heads % num_kv_heads != 0)
+    return fail(PKV_ERR_INVALID_ARG, "num_qo_heads must be a multiple of num_kv_heads");
+  if (head_dim != kDecodeHeadDim) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 128");
+  const int group = num_qo_heads / num_kv_heads;
+  if (group > kMaxGroup) return fail(PKV_ERR_UNSUPPORTED, "GQA group must be 1..8");
+  if (!valid_page_size(page_size))
+    return fail(PKV_ERR_UNSUPPORTED, "page_size must be 16, 32, 64, 128 or 256");
+  if (num_pages > 0x7fffffffLL) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31-1 pages");
+  if (!std::isfinite(sm_scale)) return fail(PKV_ERR_INVALID_ARG, "sm_scale is not finite");
+  if (num_partitions < 0 || num_partitions > kMaxPartitions)
+    return fail(PKV_ERR_INVALID_ARG, "num_partitions out of range");
+  if (batch == 0) return ok();
+  if (!q || !pool || !page_indptr || !page_indices || !last_page_len || !out || !workspace)
+    return fail(PKV_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(q, 16) || !aligned(pool, 16) || !aligned(out, 16))
+    return fail(PKV_ERR_INVALID_ARG, "q, pool and out must be 16-byte aligned");
+  if (out == q || out == pool) return fail(PKV_ERR_INVALID_ARG, "out aliases q or pool");
+  int N = num_partitions;
+  if (N == 0) N = current_device_partitions();
+  if (N <= 0) return fail(PKV_ERR_CUDA, "cannot query the SM count");
+  const WsLayout L = ws_layout(group, N);
+  if (!aligned(workspace, 256)) return fail(PKV_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, L.total);
+
+  CUtensorMap tmap;
+  int one_box = 0;
+  pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, &tmap, &one_box);
+  if (st != PKV_OK) return st;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pkv::DecodeArgs a;
+  a.q = q;
+  a.out = out;
+  a.lse = lse;
+  a.indptr = page_indptr;
+  a.indices = page_indices;
+  a.last_len = last_page_len;
+  a.counters = reinterpret_cast<int*>(ws + L.counters);
+  a.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
+  a.part_o = reinterpret_cast<float*>(ws + L.part_o);
+  a.err = reinterpret_cast<int*>(error_word);
+  a.num_pages = num_pages;
+  a.batch = batch;
+  a.hq = num_qo_heads;
+  a.hkv = num_kv_heads;
+  a.group = group;
+  a.page_size = page_size;
+  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.one_box = one_box;
+  a.out_f32 = out_f32;
+  a.out_rs = out_rs;
+  a.lse_rs = lse_rs;
+  cudaError_t e = pkv::launch_decode(tmap, a, dtype == PKV_BF16, N, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return ok();
+}
+
 extern "C" {
 
 const char* pkv_status_string(int status) {
@@ -341,62 +410,164 @@ pkv_status pkv_decode(const void* q, int num_qo_heads, const void* pool, int64_t
                       const int32_t* last_page_len, int batch, float sm_scale,
                       int num_partitions, void* workspace, size_t workspace_bytes, void* out,
                       float* lse, int32_t* error_word, void* stream) {
-  if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1)
+  return decode_impl(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
+                     page_indptr, page_indices, last_page_len, batch, sm_scale, num_partitions,
+                     workspace, workspace_bytes, out, lse, error_word, stream, 0,
+                     (long long)num_qo_heads * kDecodeHeadDim, num_qo_heads);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared-prefix cascade: the prefix kernel's grid (row blocks x splits x kv
+// heads) and the fp32 attention states it and the suffix decode write.
+struct CascadePlan {
+  int row_blocks, splits, states;
+  long long tokens_per_split;
+  size_t state_o, state_lse, decode_ws, total;  // byte offsets / size
+};
+
+CascadePlan cascade_plan(int batch, int hq, int hkv, long long prefix_len, int N, int sms) {
+  CascadePlan p;
+  const int G = hq / hkv;
+  const long long rows = (long long)batch * G;
+  const int R = pkv::prefix_rows_per_cta(), T = pkv::prefix_tile_tokens();
+  p.row_blocks = (int)((rows + R - 1) / R);
+  const long long tiles = (prefix_len + T - 1) / T;
+  const long long units = (long long)p.row_blocks * hkv;
+  long long splits = units >= sms ? 1 : sms / units;  // about one wave of CTAs
+  if (splits > tiles) splits = tiles;
+  if (splits < 1) splits = 1;
+  const long long tiles_per = (tiles + splits - 1) / splits;
+  p.tokens_per_split = tiles_per * T;
+  p.splits = (int)((prefix_len + p.tokens_per_split - 1) / p.tokens_per_split);
+  if (p.splits < 1) p.splits = 1;
+  p.states = p.splits + 1;
+  p.state_o = 0;
+  p.state_lse = align_up((size_t)batch * p.states * hq * kDecodeHeadDim * 4, 256);
+  p.decode_ws = p.state_lse + align_up((size_t)batch * p.states * hq * 4, 256);
+  p.total = p.decode_ws + ws_layout(G, N).total;
+  return p;
+}
+
+int current_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return sms;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pkv_cascade_workspace_bytes(int batch, int num_qo_heads, int num_kv_heads, int head_dim,
+                                   int64_t prefix_len, int num_partitions) {
+  const size_t dec = pkv_decode_workspace_bytes(batch, num_qo_heads, num_kv_heads, head_dim,
+                                                num_partitions);
+  if (dec == 0 || prefix_len < 0) return 0;
+  if (prefix_len == 0) return dec;
+  int N = num_partitions ? num_partitions : current_device_partitions();
+  const int sms = current_sms();
+  if (N <= 0 || sms <= 0) return 0;
+  return cascade_plan(batch, num_qo_heads, num_kv_heads, prefix_len, N, sms).total;
+}
+
+pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool, int64_t num_pages,
+                              int page_size, int num_kv_heads, int head_dim, int dtype,
+                              const int32_t* prefix_page_indices, int64_t prefix_len,
+                              const int32_t* page_indptr, const int32_t* page_indices,
+                              const int32_t* last_page_len, int batch, float sm_scale,
+                              int num_partitions, void* workspace, size_t workspace_bytes,
+                              void* out, float* lse, int32_t* error_word, void* stream) {
+  if (prefix_len < 0) return fail(PKV_ERR_INVALID_ARG, "prefix_len < 0");
+  if (prefix_len == 0 || batch == 0)
+    return pkv_decode(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
+                      page_indptr, page_indices, last_page_len, batch, sm_scale, num_partitions,
+                      workspace, workspace_bytes, out, lse, error_word, stream);
+  if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1 ||
+      num_qo_heads % num_kv_heads != 0)
     return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
   if (dtype != PKV_F16 && dtype != PKV_BF16)
     return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
-  if (num_qo_heads % num_kv_heads != 0)
-    return fail(PKV_ERR_INVALID_ARG, "num_qo_heads must be a multiple of num_kv_heads");
   if (head_dim != kDecodeHeadDim) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 128");
   const int group = num_qo_heads / num_kv_heads;
   if (group > kMaxGroup) return fail(PKV_ERR_UNSUPPORTED, "GQA group must be 1..8");
   if (!valid_page_size(page_size))
     return fail(PKV_ERR_UNSUPPORTED, "page_size must be 16, 32, 64, 128 or 256");
-  if (num_pages > 0x7fffffffLL) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31-1 pages");
+  if (prefix_len > (int64_t)num_pages * page_size)
+    return fail(PKV_ERR_INVALID_ARG, "prefix longer than the pool");
   if (!std::isfinite(sm_scale)) return fail(PKV_ERR_INVALID_ARG, "sm_scale is not finite");
   if (num_partitions < 0 || num_partitions > kMaxPartitions)
     return fail(PKV_ERR_INVALID_ARG, "num_partitions out of range");
-  if (batch == 0) return ok();
-  if (!q || !pool || !page_indptr || !page_indices || !last_page_len || !out || !workspace)
+  if (!q || !pool || !prefix_page_indices || !page_indptr || !page_indices || !last_page_len ||
+      !out || !workspace)
     return fail(PKV_ERR_INVALID_ARG, "null pointer");
   if (!aligned(q, 16) || !aligned(pool, 16) || !aligned(out, 16))
     return fail(PKV_ERR_INVALID_ARG, "q, pool and out must be 16-byte aligned");
   if (out == q || out == pool) return fail(PKV_ERR_INVALID_ARG, "out aliases q or pool");
-  int N = num_partitions;
-  if (N == 0) N = current_device_partitions();
-  if (N <= 0) return fail(PKV_ERR_CUDA, "cannot query the SM count");
-  const WsLayout L = ws_layout(group, N);
   if (!aligned(workspace, 256)) return fail(PKV_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  if (workspace_bytes < L.total)
-    return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, L.total);
+  int N = num_partitions ? num_partitions : current_device_partitions();
+  const int sms = current_sms();
+  if (N <= 0 || sms <= 0) return fail(PKV_ERR_CUDA, "cannot query the SM count");
+  const CascadePlan P = cascade_plan(batch, num_qo_heads, num_kv_heads, prefix_len, N, sms);
+  if (workspace_bytes < P.total)
+    return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, P.total);
 
   CUtensorMap tmap;
   int one_box = 0;
   pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, &tmap, &one_box);
   if (st != PKV_OK) return st;
-
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  pkv::DecodeArgs a;
-  a.q = q;
-  a.out = out;
-  a.lse = lse;
-  a.indptr = page_indptr;
-  a.indices = page_indices;
-  a.last_len = last_page_len;
-  a.counters = reinterpret_cast<int*>(ws + L.counters);
-  a.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
-  a.part_o = reinterpret_cast<float*>(ws + L.part_o);
-  a.err = reinterpret_cast<int*>(error_word);
-  a.num_pages = num_pages;
-  a.batch = batch;
-  a.hq = num_qo_heads;
-  a.hkv = num_kv_heads;
-  a.group = group;
-  a.page_size = page_size;
-  a.scale_log2 = sm_scale * 1.4426950408889634f;
-  a.one_box = one_box;
-  cudaError_t e = pkv::launch_decode(tmap, a, dtype == PKV_BF16, N, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  float* state_o = reinterpret_cast<float*>(ws + P.state_o);
+  float* state_lse = reinterpret_cast<float*>(ws + P.state_lse);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // 1. the shared prefix, once for every request's queries: state slots 0 .. splits-1
+  pkv::PrefixArgs pa;
+  pa.q = q;
+  pa.prefix_pages = prefix_page_indices;
+  pa.state_o = state_o;
+  pa.state_lse = state_lse;
+  pa.err = reinterpret_cast<int*>(error_word);
+  pa.num_pages = num_pages;
+  pa.prefix_len = prefix_len;
+  pa.tokens_per_split = P.tokens_per_split;
+  pa.page_size = page_size;
+  pa.batch = batch;
+  pa.hq = num_qo_heads;
+  pa.hkv = num_kv_heads;
+  pa.group = group;
+  pa.states = P.states;
+  pa.splits = P.splits;
+  pa.scale_log2 = sm_scale * 1.4426950408889634f;
+  pa.one_box = one_box;
+  cudaError_t e = pkv::launch_prefix(tmap, pa, dtype == PKV_BF16, P.row_blocks, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
+  // 2. each request's own pages: the last state slot, as an fp32 state
+  st = decode_impl(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
+                   page_indptr, page_indices, last_page_len, batch, sm_scale, N,
+                   ws + P.decode_ws, workspace_bytes - P.decode_ws,
+                   state_o + (size_t)P.splits * num_qo_heads * kDecodeHeadDim,
+                   state_lse + (size_t)P.splits * num_qo_heads, error_word, stream, 1,
+                   (long long)P.states * num_qo_heads * kDecodeHeadDim,
+                   (long long)P.states * num_qo_heads);
+  if (st != PKV_OK) return st;
+  // 3. merge the prefix and suffix states of every (request, head)
+  pkv::MergeArgs ma;
+  ma.v = state_o;
+  ma.s = state_lse;
+  ma.v_out = out;
+  ma.s_out = lse;
+  ma.rows = batch;
+  ma.states = P.states;
+  ma.heads = num_qo_heads;
+  ma.head_dim = kDecodeHeadDim;
+  ma.out_dtype = dtype;
+  ma.vec4 = 1;
+  e = pkv::launch_merge(ma, s);
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
 }
 
@@ -419,6 +590,7 @@ pkv_status pkv_merge_states(const float* v, const float* s, int64_t num_rows, in
   a.heads = num_heads;
   a.head_dim = head_dim;
   a.out_dtype = out_dtype;
+  a.vec4 = head_dim == 128 && aligned(v, 16);
   cudaError_t e = pkv::launch_merge(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();

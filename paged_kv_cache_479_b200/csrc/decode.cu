@@ -116,6 +116,29 @@ constexpr size_t kRingBytes = (size_t)kStages * kSlotBytes;
 constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + (size_t)kQBufs * kQBufBytes +
                               sizeof(Ctl) + sizeof(Scratch);
 
+// output of (request b, query head h): 16-bit final outputs, or fp32 attention
+// states at a caller-chosen request stride (used when the result is merged later)
+template <bool BF16>
+__device__ __forceinline__ void store_out1(const DecodeArgs& a, size_t b, size_t h, int d, float v) {
+  const size_t i = b * (size_t)a.out_rs + h * kD + d;
+  if (a.out_f32) static_cast<float*>(a.out)[i] = v;
+  else static_cast<uint16_t*>(a.out)[i] = to_bits16<BF16>(v);
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store_out4(const DecodeArgs& a, size_t b, size_t h, int d, float4 v) {
+  const size_t i = b * (size_t)a.out_rs + h * kD + d;
+  if (a.out_f32)
+    *reinterpret_cast<float4*>(static_cast<float*>(a.out) + i) = v;
+  else
+    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(a.out) + i) =
+        make_uint2(pack2<BF16>(v.x, v.y), pack2<BF16>(v.z, v.w));
+}
+
+__device__ __forceinline__ void store_lse(const DecodeArgs& a, size_t b, size_t h, float v) {
+  if (a.lse) a.lse[b * (size_t)a.lse_rs + h] = v;
+}
+
 // inclusive scan over the whole block (kDecodeThreads threads); returns the
 // prefix for this thread and the block total in *total
 __device__ long long block_incl_scan(long long v, long long* warp_tot, long long* total) {
@@ -226,10 +249,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     }
     if (b < B && r.tiles == 0 && (b % (int)gridDim.x) == c) {
       // a request with no tokens: attention over no keys -> o = 0, lse = -inf
-      uint4* o4 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + (size_t)b * a.hq * kD);
-      for (int k = 0; k < a.hq * kD / 8; ++k) o4[k] = make_uint4(0, 0, 0, 0);
-      if (a.lse)
-        for (int h = 0; h < a.hq; ++h) a.lse[(size_t)b * a.hq + h] = -INFINITY;
+      for (int h = 0; h < a.hq; ++h) {
+        for (int d = 0; d < kD; d += 4) store_out4<BF16>(a, b, h, d, make_float4(0.f, 0.f, 0.f, 0.f));
+        store_lse(a, b, h, -INFINITY);
+      }
     }
     carry += chunk_total;
   }
@@ -593,9 +616,9 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         }
         const float val = acc / L;
         if (direct) {
-          const size_t row = (size_t)rec.b * a.hq + (size_t)rec.kvh * G + h;
-          static_cast<uint16_t*>(a.out)[row * kD + d] = to_bits16<BF16>(val);
-          if (d == 0 && a.lse) a.lse[row] = (M + log2f(L)) * kLn2;
+          const size_t hq = (size_t)rec.kvh * G + h;
+          store_out1<BF16>(a, rec.b, hq, d, val);
+          if (d == 0) store_lse(a, rec.b, hq, (M + log2f(L)) * kLn2);
         } else {
           a.part_o[((size_t)rec.slot * G + h) * kD + d] = val;
           if (d == 0) a.part_lse[(size_t)rec.slot * G + h] = M + log2f(L);
@@ -659,11 +682,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       }
     }
     const float inv = 1.f / L;
-    const size_t row = (size_t)pr.b * a.hq + (size_t)pr.kvh * G + h;
-    uint16_t* op = static_cast<uint16_t*>(a.out) + row * kD + 4 * lane;
-    *reinterpret_cast<uint2*>(op) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv),
-                                               pack2<BF16>(acc.z * inv, acc.w * inv));
-    if (lane == 0 && a.lse) a.lse[row] = (M + log2f(L)) * kLn2;
+    const size_t hq = (size_t)pr.kvh * G + h;
+    store_out4<BF16>(a, pr.b, hq, 4 * lane,
+                     make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
+    if (lane == 0) store_lse(a, pr.b, hq, (M + log2f(L)) * kLn2);
   }
 }
 

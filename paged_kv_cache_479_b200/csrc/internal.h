@@ -27,6 +27,9 @@ struct DecodeArgs {
   int batch, hq, hkv, group, page_size;
   float scale_log2;       // sm_scale * log2(e)
   int one_box;            // 1: 5-D tensor map, one box per K/V tile; 0: 4-D map, two boxes
+  int out_f32;            // 1: out is fp32 (an attention state for a later merge)
+  long long out_rs;       // elements of out between consecutive requests (Hq * 128 when packed)
+  long long lse_rs;       // elements of lse between consecutive requests (Hq when packed)
 };
 
 constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp
@@ -41,6 +44,26 @@ constexpr int kDecodeCtasPerSm = PKV_CTAS_PER_SM; // resident decode CTAs per SM
 
 size_t decode_smem_bytes();
 cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int grid,
+                          cudaStream_t stream);
+
+// attention of every request's queries over one shared prefix (prefix.cu)
+struct PrefixArgs {
+  const void* q;               // [B][Hq][128]
+  const int32_t* prefix_pages; // ceil(prefix_len / page_size) page ids
+  float* state_o;              // [B][states][Hq][128] fp32, slot `split` written
+  float* state_lse;            // [B][states][Hq] fp32, natural log
+  int* err;
+  long long num_pages;
+  long long prefix_len;        // tokens
+  long long tokens_per_split;  // multiple of the prefix tile
+  int page_size, batch, hq, hkv, group, states, splits;
+  float scale_log2;
+  int one_box;
+};
+size_t prefix_smem_bytes();
+int prefix_rows_per_cta();
+int prefix_tile_tokens();
+cudaError_t launch_prefix(const CUtensorMap& tmap, const PrefixArgs& a, bool bf16, int row_blocks,
                           cudaStream_t stream);
 
 struct AppendArgs {
@@ -65,6 +88,7 @@ struct MergeArgs {
   float* s_out;
   long long rows;
   int states, heads, head_dim, out_dtype;
+  int vec4;  // 1: head_dim 128 and v 16-byte aligned (float4 loads)
 };
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream);
 

@@ -8,6 +8,10 @@
 // fused into the decode kernel for its own split-KV partitions; this kernel
 // serves callers that combine states computed elsewhere (another launch, a
 // shared prefix, another GPU).
+//
+// Lane L handles dims 4L .. 4L+3 (float4 loads) when head_dim is 128, every
+// 32nd dim otherwise; the state weights are computed once per warp, 32 states
+// at a time (lane j holds state j's weight), and broadcast with shuffles.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -20,6 +24,16 @@ namespace {
 
 constexpr int kWarps = 8;
 
+__device__ __forceinline__ void store_val(const MergeArgs& a, size_t i, float v) {
+  if (a.out_dtype == 2) {
+    static_cast<float*>(a.v_out)[i] = v;
+  } else if (a.out_dtype == 1) {
+    static_cast<__nv_bfloat16*>(a.v_out)[i] = __float2bfloat16_rn(v);
+  } else {
+    static_cast<__half*>(a.v_out)[i] = __float2half_rn(v);
+  }
+}
+
 __global__ void __launch_bounds__(kWarps * 32) merge_kernel(const MergeArgs a) {
   const int lane = threadIdx.x & 31;
   const long long gw = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -27,39 +41,63 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(const MergeArgs a) {
   const long long r = gw / a.heads;
   const int h = (int)(gw % a.heads);
   const int S = a.states, H = a.heads, D = a.head_dim;
+  const float* s_row = a.s + (size_t)r * S * H + h;           // stride H between states
+  const float* v_row = a.v + ((size_t)r * S * H + h) * D;     // stride H * D between states
 
   float M = -INFINITY;
-  for (int j = 0; j < S; ++j) M = fmaxf(M, a.s[((size_t)r * S + j) * H + h]);
+  for (int j = lane; j < S; j += 32) M = fmaxf(M, s_row[(size_t)j * H]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   const size_t orow = ((size_t)r * H + h) * D;
-  if (M == -INFINITY) {
-    for (int d = lane; d < D; d += 32) {
-      if (a.out_dtype == 2) static_cast<float*>(a.v_out)[orow + d] = 0.f;
-      else static_cast<uint16_t*>(a.v_out)[orow + d] = 0;
-    }
+  if (M == -INFINITY) {  // no keys at all
+    for (int d = lane; d < D; d += 32) store_val(a, orow + d, 0.f);
     if (lane == 0 && a.s_out) a.s_out[(size_t)r * H + h] = -INFINITY;
     return;
   }
+  const bool vec = a.vec4 != 0;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);  // vec: dims 4L..4L+3
+  float accs[4] = {0.f, 0.f, 0.f, 0.f};          // otherwise: dims L, L+32, L+64, L+96
   float wsum = 0.f;
-  for (int j = 0; j < S; ++j) {
-    const float sj = a.s[((size_t)r * S + j) * H + h];
-    if (sj != -INFINITY) wsum += expf(sj - M);
-  }
-  for (int d = lane; d < D; d += 32) {
-    float acc = 0.f;
-    for (int j = 0; j < S; ++j) {
-      const float sj = a.s[((size_t)r * S + j) * H + h];
-      if (sj == -INFINITY) continue;  // no weight, whatever its values hold
-      acc += expf(sj - M) * a.v[(((size_t)r * S + j) * H + h) * D + d];
+  for (int j0 = 0; j0 < S; j0 += 32) {
+    const int j = j0 + lane;
+    const float sj = j < S ? s_row[(size_t)j * H] : -INFINITY;
+    const float wj = sj == -INFINITY ? 0.f : expf(sj - M);  // a state with no keys: weight 0
+    wsum += wj;
+    const int cnt = S - j0 < 32 ? S - j0 : 32;
+    for (int k = 0; k < cnt; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, wj, k);
+      if (wk == 0.f) continue;  // (uniform) its values may be anything, even NaN
+      const float* vj = v_row + (size_t)(j0 + k) * H * D;
+      if (vec) {
+        const float4 v = *reinterpret_cast<const float4*>(vj + 4 * lane);
+        acc.x += wk * v.x;
+        acc.y += wk * v.y;
+        acc.z += wk * v.z;
+        acc.w += wk * v.w;
+      } else {
+        for (int i = 0, d = lane; d < D && i < 4; ++i, d += 32) accs[i] += wk * vj[d];
+      }
     }
-    const float val = acc / wsum;
-    if (a.out_dtype == 2) {
-      static_cast<float*>(a.v_out)[orow + d] = val;
-    } else if (a.out_dtype == 1) {
-      __nv_bfloat16 x = __float2bfloat16_rn(val);
-      static_cast<__nv_bfloat16*>(a.v_out)[orow + d] = x;
-    } else {
-      __half x = __float2half_rn(val);
-      static_cast<__half*>(a.v_out)[orow + d] = x;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+  const float inv = 1.f / wsum;
+  if (vec) {
+    store_val(a, orow + 4 * lane + 0, acc.x * inv);
+    store_val(a, orow + 4 * lane + 1, acc.y * inv);
+    store_val(a, orow + 4 * lane + 2, acc.z * inv);
+    store_val(a, orow + 4 * lane + 3, acc.w * inv);
+  } else {
+    for (int i = 0, d = lane; d < D && i < 4; ++i, d += 32) store_val(a, orow + d, accs[i] * inv);
+    // head_dim above 128: the remaining dims, one state pass each
+    for (int d = lane + 128; d < D; d += 32) {
+      float x = 0.f;
+      for (int j = 0; j < S; ++j) {
+        const float sj = s_row[(size_t)j * H];
+        if (sj == -INFINITY) continue;
+        x += expf(sj - M) * v_row[(size_t)j * H * D + d];
+      }
+      store_val(a, orow + d, x * inv);
     }
   }
   if (lane == 0 && a.s_out) a.s_out[(size_t)r * H + h] = M + logf(wsum);

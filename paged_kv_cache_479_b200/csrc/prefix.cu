@@ -1,0 +1,341 @@
+// prefix.cu -- attention of many requests' queries over ONE shared prefix.
+//
+// When requests share a prefix (a system prompt stored once in shared pages:
+// "大模型推理极致优化：FlashAttention+PageAttention联合调优" section 3.2; automatic
+// prefix sharing, "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署"
+// section 3.3), decoding each request separately re-reads the prefix's K/V
+// once per request.  Here the prefix is read once per block of 128 query
+// rows, where a row is one (request, query head) of one KV head's group:
+// B * G rows per KV head become the M dimension of a dense contraction,
+//     S[128 x 64]  = Q[128 x 128] . K_tile^T      (m16n8k16, fp32 accumulate)
+//     O[128 x 128] += P[128 x 64] . V_tile         (P split into bf16 high + low)
+// with online softmax over the prefix tokens (FlashAttention-style, "大模型推理
+// 极致优化：FlashAttention+PageAttention联合调优" section 2.2).  The prefix tokens are
+// cut into `splits` chunks so the grid fills the GPU; each CTA writes its rows'
+// normalised partial state (o, natural-log lse) as fp32 into state slot
+// `split` of [B][S][Hq][128]; the states are merged with the requests' own
+// (suffix) attention afterwards (pkv_merge_states).
+//
+// CTA: 8 consumer warps (16 query rows each) and 1 producer warp issuing the
+// K/V of 64-token tiles as 16-token bulk-tensor boxes into a 3-stage ring.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "partition.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kWarps = 8;                       // consumer warps
+constexpr int kRows = kWarps * 16;              // query rows per CTA
+constexpr int kTile = 64;                       // prefix tokens per stage
+constexpr int kBoxes = kTile / kTileTokens;     // 16-token boxes per K (or V) tile
+constexpr int kBoxBytes = kTileTokens * kD * 2; // 4 KiB
+constexpr int kHalf = kBoxBytes / 2;            // one [16][64] half of a box
+constexpr int kKVBytes = kBoxes * kBoxBytes;    // 16 KiB for K (and for V) of a tile
+constexpr int kStageBytes = 2 * kKVBytes;
+constexpr int kStages = 3;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct __align__(16) Ctl {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  int valid[kStages];  // prefix tokens present in the stage's tile
+  int abort;
+};
+
+constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Ctl);
+
+// byte offset of (token t of the tile, 16-byte chunk c of its 128 dims) in a
+// K or V area made of kBoxes 128-byte-swizzled [2][16][64] boxes
+__device__ __forceinline__ uint32_t tile_off(int t, int c) {
+  const int bx = t >> 4, tt = t & 15;
+  return (uint32_t)(bx * kBoxBytes + (c >> 3) * kHalf + tt * 128 + (((c & 7) ^ (tt & 7)) << 4));
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__((kWarps + 1) * 32, 1)
+    prefix_kernel(const __grid_constant__ CUtensorMap tmap, const PrefixArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + (size_t)kStages * kStageBytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rb = blockIdx.x, split = blockIdx.y, kvh = blockIdx.z;
+  const int G = a.group;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl.full[s]), 1);
+      mbar_init(smem_u32(&ctl.empty[s]), kWarps * 32);
+    }
+    ctl.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarps && lane == 0) prefetch_tensormap(&tmap);
+  grid_dependency_wait();
+  __syncthreads();
+
+  const long long t_begin = (long long)split * a.tokens_per_split;
+  const long long t_end = t_begin + a.tokens_per_split < a.prefix_len
+                              ? t_begin + a.tokens_per_split : a.prefix_len;
+  const int ntiles = t_end > t_begin ? (int)((t_end - t_begin + kTile - 1) / kTile) : 0;
+
+  if (warp == kWarps) {
+    // =========================== producer ===========================
+    const uint32_t ring0 = smem_u32(smem);
+    bool ok = true;
+    for (int i = 0; ok && i < ntiles; ++i) {
+      const int s = i % kStages;
+      const long long t0 = t_begin + (long long)i * kTile;
+      const int valid = (int)((t_end - t0) < kTile ? (t_end - t0) : kTile);
+      // lanes 0..kBoxes-1 each handle one 16-token box
+      int page = -1, yoff = 0;
+      if (lane < kBoxes && lane * kTileTokens < valid) {
+        const long long tok = t0 + lane * kTileTokens;
+        page = a.prefix_pages[tok / a.page_size];
+        if (page < 0 || (long long)page >= a.num_pages) {
+          if (a.err) atomicOr(a.err, kErrPageId);
+          page = -1;
+        }
+        yoff = (int)(tok % a.page_size);
+      }
+      const unsigned have = __ballot_sync(0xffffffffu, page >= 0);
+      int okl = 1;
+      if (lane == 0) {
+        okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((i / kStages) & 1) ^ 1, &ctl.abort, a.err);
+        if (okl) {
+          ctl.valid[s] = valid;
+          mbar_arrive_expect_tx(smem_u32(&ctl.full[s]), (uint32_t)__popc(have) * 2 * kBoxBytes);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+      if (!ok) break;
+      if (page >= 0) {
+        const uint32_t full = smem_u32(&ctl.full[s]);
+        const uint32_t kdst = ring0 + (uint32_t)s * kStageBytes + (uint32_t)lane * kBoxBytes;
+        const uint32_t vdst = kdst + kKVBytes;
+        if (a.one_box) {
+          tma_load_5d(kdst, &tmap, 0, yoff, 0, kvh, page, full);
+          tma_load_5d(vdst, &tmap, 0, yoff, 0, a.hkv + kvh, page, full);
+        } else {
+          tma_load_4d(kdst, &tmap, 0, yoff, kvh, page, full);
+          tma_load_4d(kdst + kHalf, &tmap, 64, yoff, kvh, page, full);
+          tma_load_4d(vdst, &tmap, 0, yoff, a.hkv + kvh, page, full);
+          tma_load_4d(vdst + kHalf, &tmap, 64, yoff, a.hkv + kvh, page, full);
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // aborted: let the copies already issued land before the CTA exits
+      for (int s = 0; s < kStages; ++s) {
+        const uint64_t t0 = global_timer_ns();
+        const uint32_t bar = smem_u32(&ctl.full[s]);
+        for (int ph = 0; ph < 2; ++ph)
+          while (!mbar_try_wait(bar, ph) && global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+      }
+    }
+    return;
+  }
+
+  // =========================== consumers ===========================
+  const int g = lane >> 2, cq = lane & 3, mi = lane >> 3, r8 = lane & 7;
+  const long long nrows = (long long)a.batch * G;
+  const long long row0 = (long long)rb * kRows + warp * 16;  // this warp's first row
+  // query rows as A fragments: row r -> request r / G, query head kvh * G + r % G
+  uint32_t qa[8][4];
+  {
+    const uint16_t* qp[2];
+    bool qv[2];
+    for (int hr = 0; hr < 2; ++hr) {
+      const long long r = row0 + g + 8 * hr;
+      qv[hr] = r < nrows;
+      const long long b = qv[hr] ? r / G : 0, hh = qv[hr] ? r % G : 0;
+      qp[hr] = static_cast<const uint16_t*>(a.q) + ((size_t)b * a.hq + (size_t)kvh * G + hh) * kD;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int d0 = j * 16 + 2 * cq;
+      qa[j][0] = qv[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + d0) : 0u;
+      qa[j][1] = qv[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + d0) : 0u;
+      qa[j][2] = qv[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + d0 + 8) : 0u;
+      qa[j][3] = qv[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + d0 + 8) : 0u;
+    }
+  }
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows g and g + 8
+  const float sl2 = a.scale_log2;
+  const uint32_t ring0 = smem_u32(smem);
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % kStages;
+    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kStages) & 1, &ctl.abort, a.err)) return;
+    const int valid = ctl.valid[s];
+    const uint32_t kb = ring0 + (uint32_t)s * kStageBytes, vb = kb + kKVBytes;
+    // ---- S = Q K^T for 64 tokens (8 n-tiles of 8)
+    float sc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {  // n-tile pair (2np, 2np+1)
+        const int tok = np * 16 + (mi >> 1) * 8 + r8;
+        const int chunk = j * 2 + (mi & 1);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4(kb + tile_off(tok, chunk), b0, b1, b2, b3);
+        mma_16816<BF16>(sc[2 * np], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
+        mma_16816<BF16>(sc[2 * np + 1], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b2, b3);
+      }
+    }
+    // ---- mask tokens past the prefix, online softmax (log2 units)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int t = n * 8 + 2 * cq;
+      sc[n][0] = t < valid ? sc[n][0] * sl2 : -INFINITY;
+      sc[n][1] = t + 1 < valid ? sc[n][1] * sl2 : -INFINITY;
+      sc[n][2] = t < valid ? sc[n][2] * sl2 : -INFINITY;
+      sc[n][3] = t + 1 < valid ? sc[n][3] * sl2 : -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(sc[n][0], sc[n][1]));
+      mx1 = fmaxf(mx1, fmaxf(sc[n][2], sc[n][3]));
+    }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float al0 = mn0 == -INFINITY ? 1.f : ex2(m0 - mn0);
+    const float al1 = mn1 == -INFINITY ? 1.f : ex2(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      sc[n][0] = ex2(sc[n][0] - mn0);
+      sc[n][1] = ex2(sc[n][1] - mn0);
+      sc[n][2] = ex2(sc[n][2] - mn1);
+      sc[n][3] = ex2(sc[n][3] - mn1);
+      ps0 += sc[n][0] + sc[n][1];
+      ps1 += sc[n][2] + sc[n][3];
+    }
+    l0 = l0 * al0 + ps0;
+    l1 = l1 * al1 + ps1;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      o[n][0] *= al0;
+      o[n][1] *= al0;
+      o[n][2] *= al1;
+      o[n][3] *= al1;
+    }
+    // ---- V rows past the prefix may hold anything (even NaN): zero them
+    if (valid < kTile) {
+      uint8_t* vrow = smem + (size_t)s * kStageBytes + kKVBytes;
+      for (int idx = lane; idx < (kTile - valid) * 16; idx += 32) {
+        const int t = valid + (idx >> 4), c = idx & 15;
+        *reinterpret_cast<uint4*>(vrow + tile_off(t, c)) = make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+    // ---- O += P V  (P of two adjacent n-tiles is the A fragment of one k-step)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t ah[4], al[4];
+      {
+        const float* p0 = sc[2 * kk];
+        const float* p1 = sc[2 * kk + 1];
+        ah[0] = pack2<BF16>(p0[0], p0[1]);
+        ah[1] = pack2<BF16>(p0[2], p0[3]);
+        ah[2] = pack2<BF16>(p1[0], p1[1]);
+        ah[3] = pack2<BF16>(p1[2], p1[3]);
+        if constexpr (BF16) {
+          float2 f;
+          f = unpack2<true>(ah[0]); al[0] = pack2<true>(p0[0] - f.x, p0[1] - f.y);
+          f = unpack2<true>(ah[1]); al[1] = pack2<true>(p0[2] - f.x, p0[3] - f.y);
+          f = unpack2<true>(ah[2]); al[2] = pack2<true>(p1[0] - f.x, p1[1] - f.y);
+          f = unpack2<true>(ah[3]); al[3] = pack2<true>(p1[2] - f.x, p1[3] - f.y);
+        }
+      }
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {  // dim n-tile pair (2np, 2np+1)
+        const int tok = kk * 16 + (mi & 1) * 8 + r8;
+        const int chunk = 2 * np + (mi >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldmatrix_x4_trans(vb + tile_off(tok, chunk), b0, b1, b2, b3);
+        mma_16816<BF16>(o[2 * np], ah[0], ah[1], ah[2], ah[3], b0, b1);
+        mma_16816<BF16>(o[2 * np + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
+        if constexpr (BF16) {
+          mma_16816<BF16>(o[2 * np], al[0], al[1], al[2], al[3], b0, b1);
+          mma_16816<BF16>(o[2 * np + 1], al[0], al[1], al[2], al[3], b2, b3);
+        }
+      }
+    }
+    if (valid < kTile) fence_proxy_async_smem();
+    __syncwarp();
+    mbar_arrive(smem_u32(&ctl.empty[s]));
+  }
+
+  // ---- rows' partial states: o / l (fp32) and lse (natural log)
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  for (int hr = 0; hr < 2; ++hr) {
+    const long long r = row0 + g + 8 * hr;
+    if (r >= nrows) continue;
+    const long long b = r / G, h = (long long)kvh * G + r % G;
+    const float l = hr ? l1 : l0, m = hr ? m1 : m0;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float* op = a.state_o + (((size_t)b * a.states + split) * a.hq + h) * kD;
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<float2*>(op + n * 8 + 2 * cq) =
+          make_float2(o[n][2 * hr] * inv, o[n][2 * hr + 1] * inv);
+    if (cq == 0)
+      a.state_lse[((size_t)b * a.states + split) * a.hq + h] =
+          l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+  }
+}
+
+}  // namespace
+
+size_t prefix_smem_bytes() { return kSmemBytes; }
+int prefix_rows_per_cta() { return kRows; }
+int prefix_tile_tokens() { return kTile; }
+
+cudaError_t launch_prefix(const CUtensorMap& tmap, const PrefixArgs& a, bool bf16, int row_blocks,
+                          cudaStream_t stream) {
+  auto kern = bf16 ? prefix_kernel<true> : prefix_kernel<false>;
+  static bool attr_set[2][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !attr_set[bf16][dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[bf16][dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)row_blocks, (unsigned)a.splits, (unsigned)a.hkv);
+  cfg.blockDim = dim3((kWarps + 1) * 32);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmap, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -312,6 +312,23 @@ def from_bits(a: np.ndarray, dtype: str) -> torch.Tensor:
     return t.view(torch.float16 if dtype == "f16" else torch.bfloat16)
 
 
+def cascade_view(w: Workload):
+    """Split w's table into its shared prefix and each request's own pages:
+    (prefix page ids, prefix tokens, own indptr, own indices, own last_page_len)."""
+    k = w.shared_prefix_pages
+    prefix = w.pages_of(0)[:k].astype(np.int32) if w.batch else np.zeros(0, np.int32)
+    indptr = np.zeros(w.batch + 1, np.int32)
+    chunks = []
+    last = np.zeros(w.batch, np.int32)
+    for b in range(w.batch):
+        own = w.pages_of(b)[k:]
+        chunks.append(own)
+        indptr[b + 1] = indptr[b] + len(own)
+        last[b] = w.last_page_len[b] if len(own) else 0
+    indices = np.concatenate(chunks).astype(np.int32) if chunks else np.zeros(0, np.int32)
+    return prefix, k * w.page_size, indptr, indices, last
+
+
 def subset(w: Workload, requests, pool_bits_of_pages):
     """A compact copy of requests `requests` of workload w: the returned table
     renumbers their pages 0..n-1 in order of first use; `pool_bits_of_pages(ids)`

@@ -197,10 +197,12 @@ def test_append_overflow_sets_error_bit():
 
 # ------------------------------------------------------------------ merge
 
-@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16, torch.float16])
-def test_merge_states_matches_oracle(out_dtype):
+@pytest.mark.parametrize("out_dtype,S,D", [(torch.float32, 5, 128), (torch.bfloat16, 5, 128),
+                                           (torch.float16, 5, 128), (torch.float32, 40, 128),
+                                           (torch.float32, 3, 64), (torch.float32, 7, 200)])
+def test_merge_states_matches_oracle(out_dtype, S, D):
     g = torch.Generator().manual_seed(9)
-    N, S, H, D = 37, 5, 8, 128
+    N, H = 37, 8
     v = torch.randn((N, S, H, D), generator=g)
     s = torch.randn((N, S, H), generator=g) * 4
     s[3, 2] = -float("inf")
