@@ -245,6 +245,13 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       if (s0 <= f0 && f0 < s1) {
         ctl.b0 = b;
         ctl.Cb0 = carry + excl;
+        // warm L2 with the first page ids and query rows this partition needs,
+        // while the rest of the prologue runs
+        const long long u = (f0 - s0) % r.units;
+        const long long t0 = u > kSegmentCost ? u - kSegmentCost : 0;
+        const int kvh0 = (int)((f0 - s0) / r.units);
+        prefetch_l2(a.indices + r.page_base + (t0 * kTileTokens) / a.page_size);
+        prefetch_l2(static_cast<const uint16_t*>(a.q) + ((size_t)b * a.hq + (size_t)kvh0 * a.group) * kD);
       }
     }
     if (b < B && r.tiles == 0 && (b % (int)gridDim.x) == c) {
@@ -272,6 +279,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     wk.start(ctl.b0, ctl.Cb0, request_info(a.indptr, a.last_len, ctl.b0, a.page_size), f0, f1);
     const uint32_t ring0 = smem_u32(ring);
     const long long ps = a.page_size;
+    const int ps_shift = __ffs(a.page_size) - 1;  // page sizes are powers of two
     uint32_t i = 0;  // tiles handed to the ring so far
     int seg = 0;
     bool ok = true;
@@ -321,10 +329,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       // page ids, one tile per lane, loaded one 32-tile batch ahead of their use
       const int* idx = a.indices + wk.ri.page_base;
       int page_next = -1;
-      if (lane < n) page_next = idx[(t0 + lane) * kTileTokens / ps];
+      if (lane < n) page_next = idx[((t0 + lane) * kTileTokens) >> ps_shift];
       for (long long k0 = 0; ok && k0 < n_pad; k0 += 32) {
         int page = page_next;
-        if (k0 + 32 + lane < n) page_next = idx[(t0 + k0 + 32 + lane) * kTileTokens / ps];
+        if (k0 + 32 + lane < n)
+          page_next = idx[((t0 + k0 + 32 + lane) * kTileTokens) >> ps_shift];
         const long long k = k0 + lane;
         int yoff = 0, valid = 0;
         if (k < n) {
@@ -333,7 +342,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
             page = -1;
           }
           const long long tok0 = (t0 + k) * kTileTokens;
-          yoff = (int)(tok0 % ps);
+          yoff = (int)(tok0 & (ps - 1));
           const long long left = wk.ri.len - tok0;
           valid = left < kTileTokens ? (int)left : kTileTokens;
         } else {

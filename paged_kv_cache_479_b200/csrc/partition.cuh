@@ -32,7 +32,7 @@
 #endif
 
 #ifndef PKV_SEG_COST
-#define PKV_SEG_COST 12
+#define PKV_SEG_COST 16
 #endif
 
 namespace pkv {
