@@ -133,13 +133,17 @@ def reference_plan(w, N, cost):
 
 
 def library_cost():
-    """The fixed per-pair cost the library charges, recovered from a probe plan."""
-    w = wl.make_workload("probe", [16, 1, 40, 300, 17], num_qo_heads=4, num_kv_heads=2,
-                         page_size=16, dtype="f16", seed=2)
-    got = sorted(map(tuple, pkv.plan_segments(w.page_indptr, w.last_page_len, 16, 2, 7).tolist()))
-    costs = [k for k in range(0, 65) if reference_plan(w, 7, k) == got]
-    assert len(costs) == 1, costs
-    return costs[0]
+    """The fixed per-pair cost the library charges, recovered from probe plans: the
+    one value in 0..64 for which the definition reproduces every probe."""
+    w = wl.make_workload("probe", [16, 1, 40, 300, 17, 5, 90, 33, 2, 160], num_qo_heads=4,
+                         num_kv_heads=2, page_size=16, dtype="f16", seed=2)
+    costs = set(range(0, 65))
+    for N in (7, 13, 29, 61, 97):
+        got = sorted(map(tuple, pkv.plan_segments(w.page_indptr, w.last_page_len, 16, 2,
+                                                  N).tolist()))
+        costs &= {k for k in costs if reference_plan(w, N, k) == got}
+    assert len(costs) == 1, sorted(costs)
+    return costs.pop()
 
 
 def check_plan(w, N):
