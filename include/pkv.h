@@ -73,12 +73,57 @@ typedef enum pkv_dtype {
   PKV_F32 = 2                /* only as the output type of pkv_merge_states */
 } pkv_dtype;
 
+/* Pool layouts (the simple calls use HND). */
+typedef enum pkv_layout {
+  PKV_LAYOUT_HND = 0,  /* pool[page][2][kv_head][slot][head_dim]: one head's slots contiguous */
+  PKV_LAYOUT_NHD = 1   /* pool[page][2][slot][kv_head][head_dim]: one slot's heads contiguous */
+} pkv_layout;
+
+/* A KV pool: `data` holds num_pages pages of 2 (K, V) x num_kv_heads x page_size
+ * x head_dim elements of `dtype`, in `layout` order. */
+typedef struct pkv_pool_desc {
+  void* data;
+  int64_t num_pages;
+  int32_t page_size;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t dtype;   /* pkv_dtype */
+  int32_t layout;  /* pkv_layout */
+  int32_t reserved;
+} pkv_pool_desc;
+
+/* Page-table forms. */
+typedef enum pkv_table_kind {
+  PKV_TABLE_CSR = 0,   /* page_indptr / page_indices / last_page_len, as in the simple calls */
+  PKV_TABLE_BLOCK = 1  /* dense block table + context lengths (the vLLM form, "上下文窗口优化实战：
+                          如何用PagedAttention+FlashInfer将Llama3-70B的128K上下文吞吐提升3.8倍？"
+                          section 4.3: block_table [batch, max_blocks_per_seq], context_lens [batch]) */
+} pkv_table_kind;
+
+/* A page table (device arrays).  CSR: request b owns page_indices[page_indptr[b] ..
+ * page_indptr[b+1]) and holds (np-1)*page_size + last_page_len[b] tokens.  BLOCK:
+ * request b owns block_table[b][0 .. ceil(context_lens[b]/page_size)) and holds
+ * context_lens[b] tokens (at most max_blocks_per_seq * page_size; more sets
+ * PKV_DEVERR_CONTEXT_LEN and the request is treated as empty). */
+typedef struct pkv_table_desc {
+  int32_t kind;   /* pkv_table_kind */
+  int32_t batch;
+  const int32_t* page_indptr;
+  const int32_t* page_indices;
+  const int32_t* last_page_len;
+  const int32_t* block_table;
+  const int32_t* context_lens;
+  int32_t max_blocks_per_seq;
+  int32_t reserved;
+} pkv_table_desc;
+
 /* Bits the kernels OR into *error_word. */
 #define PKV_DEVERR_PAGE_ID   0x01  /* page id outside [0, num_pages): page skipped */
 #define PKV_DEVERR_INDPTR    0x02  /* page_indptr decreasing or negative: request treated as empty */
 #define PKV_DEVERR_LAST_LEN  0x04  /* last_page_len outside [1, page_size]: request treated as empty */
 #define PKV_DEVERR_APPEND    0x08  /* append_indptr malformed or more new tokens than the request holds */
 #define PKV_DEVERR_TIMEOUT   0x10  /* an internal wait ran past its time limit; outputs invalid */
+#define PKV_DEVERR_CONTEXT_LEN 0x20 /* block table: context_lens[b] < 0 or beyond its row: request treated as empty */
 
 /* Human-readable name of a status code (static string). */
 PKV_API const char* pkv_status_string(int status);
@@ -159,6 +204,23 @@ PKV_API pkv_status pkv_decode(const void* q, int num_qo_heads,
                       float sm_scale, int num_partitions,
                       void* workspace, size_t workspace_bytes,
                       void* out, float* lse, int32_t* error_word, void* stream);
+
+/*
+ * pkv_decode_ex / pkv_append_ex -- pkv_decode / pkv_append on a pool and a page
+ * table given by descriptors, which adds the NHD pool layout and the dense
+ * block-table form.  Same semantics, workspace (pkv_decode_workspace_bytes)
+ * and error behaviour as the simple calls; with PKV_TABLE_BLOCK the table to
+ * pass to pkv_append_ex is the table after the append (context_lens counts
+ * the new tokens).
+ */
+PKV_API pkv_status pkv_decode_ex(const void* q, int num_qo_heads, const pkv_pool_desc* pool,
+                                 const pkv_table_desc* table, float sm_scale, int num_partitions,
+                                 void* workspace, size_t workspace_bytes, void* out, float* lse,
+                                 int32_t* error_word, void* stream);
+PKV_API pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc* table,
+                                 const void* k_new, const void* v_new,
+                                 const int32_t* append_indptr, int64_t nnz_new,
+                                 int32_t* error_word, void* stream);
 
 /*
  * pkv_cascade_decode -- pkv_decode for a batch whose requests all begin with

@@ -17,29 +17,43 @@ Functions (C names in parentheses):
   plan_segments          (pkv_plan_segments)   host mirror of the split-KV partition
   decode_static_workspace (pkv_decode_static_workspace)  decode on the library's own scratch
   cascade_decode         (pkv_cascade_decode)  decode for a batch sharing one prefix
+  paged_decode_attention_ex / paged_kv_append_ex (pkv_decode_ex / pkv_append_ex)
+                         NHD pools and dense (vLLM-style) block tables
 """
 from ._binding import (  # noqa: F401
     BF16,
     F16,
     F32,
     PkvError,
+    PoolDesc,
+    TableDesc,
+    block_table,
     cascade_decode,
     cascade_workspace_bytes,
     check_table,
+    csr_table,
     decode_static_workspace,
     decode_workspace_bytes,
     default_partitions,
     lib,
     merge_states,
     paged_decode_attention,
+    paged_decode_attention_ex,
     paged_kv_append,
+    paged_kv_append_ex,
+    pool_desc,
     plan_segments,
     read_error_word,
     DEVERR_APPEND,
+    DEVERR_CONTEXT_LEN,
     DEVERR_INDPTR,
     DEVERR_LAST_LEN,
     DEVERR_PAGE_ID,
     DEVERR_TIMEOUT,
+    LAYOUT_HND,
+    LAYOUT_NHD,
+    TABLE_BLOCK,
+    TABLE_CSR,
 )
 
 pkv_append = paged_kv_append
@@ -47,3 +61,5 @@ pkv_decode = paged_decode_attention
 pkv_decode_static_workspace = decode_static_workspace
 pkv_merge_states = merge_states
 pkv_cascade_decode = cascade_decode
+pkv_decode_ex = paged_decode_attention_ex
+pkv_append_ex = paged_kv_append_ex

@@ -14,6 +14,9 @@ DEVERR_INDPTR = 0x02
 DEVERR_LAST_LEN = 0x04
 DEVERR_APPEND = 0x08
 DEVERR_TIMEOUT = 0x10
+DEVERR_CONTEXT_LEN = 0x20
+LAYOUT_HND, LAYOUT_NHD = 0, 1
+TABLE_CSR, TABLE_BLOCK = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpkv.so")
@@ -43,6 +46,27 @@ _SIGNATURES["pkv_cascade_workspace_bytes"] = ([_I32, _I32, _I32, _I32, _I64, _I3
 _SIGNATURES["pkv_cascade_decode"] = (
     [_P, _I32, _P, _I64, _I32, _I32, _I32, _I32, _P, _I64, _P, _P, _P, _I32, _F32, _I32, _P, _SZ,
      _P, _P, _P, _P], _I32)
+class PoolDesc(ctypes.Structure):
+    """pkv_pool_desc"""
+    _fields_ = [("data", ctypes.c_void_p), ("num_pages", ctypes.c_int64),
+                ("page_size", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("layout", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class TableDesc(ctypes.Structure):
+    """pkv_table_desc"""
+    _fields_ = [("kind", ctypes.c_int32), ("batch", ctypes.c_int32),
+                ("page_indptr", ctypes.c_void_p), ("page_indices", ctypes.c_void_p),
+                ("last_page_len", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("context_lens", ctypes.c_void_p), ("max_blocks_per_seq", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_PP = ctypes.POINTER(PoolDesc)
+_TP = ctypes.POINTER(TableDesc)
+_SIGNATURES["pkv_decode_ex"] = ([_P, _I32, _PP, _TP, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
+_SIGNATURES["pkv_append_ex"] = ([_PP, _TP, _P, _P, _P, _I64, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
 _SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
 _SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
@@ -228,6 +252,73 @@ def cascade_decode(q, pool, prefix_pages, prefix_len, page_indptr, page_indices,
                                   _ptr(lse), _ptr(error_word), _stream(stream, q.device))
     _check(st, "pkv_cascade_decode")
     return out, lse
+
+
+def pool_desc(pool, layout: str = "HND") -> PoolDesc:
+    """Descriptor of a pool tensor: HND [P, 2, Hkv, ps, D] or NHD [P, 2, ps, Hkv, D]."""
+    _dev_tensor(pool, "pool")
+    if layout == "HND":
+        P, two, hkv, ps, d = pool.shape
+    elif layout == "NHD":
+        P, two, ps, hkv, d = pool.shape
+    else:
+        raise ValueError("layout must be 'HND' or 'NHD'")
+    if two != 2:
+        raise ValueError("the second pool axis must be (K, V)")
+    return PoolDesc(pool.data_ptr(), P, ps, hkv, d, _DTYPES[pool.dtype],
+                    LAYOUT_HND if layout == "HND" else LAYOUT_NHD, 0)
+
+
+def csr_table(page_indptr, page_indices, last_page_len) -> TableDesc:
+    for name, t in (("page_indptr", page_indptr), ("page_indices", page_indices),
+                    ("last_page_len", last_page_len)):
+        _dev_tensor(t, name, torch.int32)
+    return TableDesc(TABLE_CSR, last_page_len.numel(), page_indptr.data_ptr(),
+                     page_indices.data_ptr(), last_page_len.data_ptr(), None, None, 0, 0)
+
+
+def block_table(table, context_lens) -> TableDesc:
+    """Dense [batch, max_blocks_per_seq] block table + context lengths (tokens)."""
+    _dev_tensor(table, "block_table", torch.int32)
+    _dev_tensor(context_lens, "context_lens", torch.int32)
+    if table.dim() != 2 or table.shape[0] != context_lens.numel():
+        raise ValueError("block_table must be [batch, max_blocks_per_seq]")
+    return TableDesc(TABLE_BLOCK, table.shape[0], None, None, None, table.data_ptr(),
+                     context_lens.data_ptr(), table.shape[1], 0)
+
+
+def paged_decode_attention_ex(q, pool, table: TableDesc, workspace, layout: str = "HND",
+                              out=None, lse=None, sm_scale=None, num_partitions: int = 0,
+                              error_word=None, stream=None, return_lse: bool = True):
+    """pkv_decode_ex: decode on an HND/NHD pool with a CSR or dense block table."""
+    _dev_tensor(q, "q", pool.dtype)
+    _dev_tensor(workspace, "workspace")
+    pd = pool_desc(pool, layout)
+    B, hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_decode_ex(_ptr(q), hq, ctypes.byref(pd), ctypes.byref(table), scale,
+                             num_partitions, _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _ptr(out), _ptr(lse),
+                             _ptr(error_word), _stream(stream, q.device))
+    _check(st, "pkv_decode_ex")
+    return out, lse
+
+
+def paged_kv_append_ex(pool, table: TableDesc, k_new, v_new, append_indptr, layout: str = "HND",
+                       error_word=None, stream=None) -> None:
+    """pkv_append_ex: append on an HND/NHD pool with a CSR or dense block table."""
+    pd = pool_desc(pool, layout)
+    _dev_tensor(k_new, "k_new", pool.dtype)
+    _dev_tensor(v_new, "v_new", pool.dtype)
+    _dev_tensor(append_indptr, "append_indptr", torch.int32)
+    st = lib().pkv_append_ex(ctypes.byref(pd), ctypes.byref(table), _ptr(k_new), _ptr(v_new),
+                             _ptr(append_indptr), k_new.shape[0], _ptr(error_word),
+                             _stream(stream, pool.device))
+    _check(st, "pkv_append_ex")
 
 
 def merge_states(v, s, out_dtype=torch.float32, v_out=None, s_out=None, stream=None,

@@ -85,21 +85,23 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 struct MapKey {
   const void* pool;
   long long pages;
-  int ps, hkv, dtype, device;
+  int ps, hkv, dtype, layout, device;
   bool operator==(const MapKey& o) const {
     return pool == o.pool && pages == o.pages && ps == o.ps && hkv == o.hkv && dtype == o.dtype &&
-           device == o.device;
+           layout == o.layout && device == o.device;
   }
 };
 
-// Tensor map of the pool for the decode kernel's bulk-tensor loads.  Preferred
-// form, 5-D: (dim % 64, slot, dim / 64, kv * Hkv + head, page) with boxes of
+// Tensor map of the pool for the kernels' bulk-tensor loads.  Preferred form,
+// 5-D: (dim % 64, slot, dim / 64, kv head, 2 page + K/V) with boxes of
 // [2][16 slots][64 dims] -- one load brings a tile's whole K (or V) into
-// shared memory as two 128-byte-swizzled [16][64] halves.  The dim/64 axis
-// has a smaller stride than the slot axis; if the driver rejects that order,
-// the 4-D form (dim, slot, kv * Hkv + head, page) with [16][64] boxes is used
-// (two loads per K or V tile, same shared-memory layout).
-pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, int dtype,
+// shared memory as two 128-byte-swizzled [16][64] halves.  Both pool layouts
+// (HND [page][2][head][slot][dim], NHD [page][2][slot][head][dim]) are this
+// view with different strides.  If the driver rejected the 5-D form (its
+// strides are not increasing), the HND pool falls back to the 4-D form
+// (dim, slot, K/V * Hkv + head, page) with [16][64] boxes: two loads per K or
+// V tile, same shared-memory layout.
+pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, int dtype, int layout,
                            CUtensorMap* out, int* one_box) {
   static std::mutex mu;
   static MapKey keys[16];
@@ -108,7 +110,7 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
   static int used = 0, next = 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  const MapKey key{pool, pages, ps, hkv, dtype, dev};
+  const MapKey key{pool, pages, ps, hkv, dtype, layout, dev};
   {
     std::lock_guard<std::mutex> lk(mu);
     for (int i = 0; i < used; ++i)
@@ -128,8 +130,10 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
   CUresult r = CUDA_ERROR_INVALID_VALUE;
 #ifndef PKV_FORCE_4D_MAP
   {
-    cuuint64_t dims[5] = {64, (cuuint64_t)ps, 2, (cuuint64_t)2 * hkv, (cuuint64_t)pages};
-    cuuint64_t strides[4] = {row, 128, (cuuint64_t)ps * row, (cuuint64_t)2 * hkv * ps * row};
+    const bool nhd = layout == PKV_LAYOUT_NHD;
+    cuuint64_t dims[5] = {64, (cuuint64_t)ps, 2, (cuuint64_t)hkv, (cuuint64_t)2 * pages};
+    cuuint64_t strides[4] = {nhd ? (cuuint64_t)hkv * row : row, 128,
+                             nhd ? row : (cuuint64_t)ps * row, (cuuint64_t)hkv * ps * row};
     cuuint32_t box[5] = {64, (cuuint32_t)pkv::kTileTokens, 2, 1, 1};
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     r = encode(&m, dt, 5, const_cast<void*>(pool), dims, strides, box, estr,
@@ -138,6 +142,8 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
     kind = 1;
   }
 #endif
+  if (r != CUDA_SUCCESS && layout == PKV_LAYOUT_NHD)
+    return fail(PKV_ERR_UNSUPPORTED, "the driver rejected the 5-D tensor map the NHD layout needs");
   if (r != CUDA_SUCCESS) {
     cuuint64_t dims[4] = {(cuuint64_t)kDecodeHeadDim, (cuuint64_t)ps, (cuuint64_t)2 * hkv,
                           (cuuint64_t)pages};
@@ -174,9 +180,8 @@ pkv_status pkv::set_error(pkv_status s, const char* fmt, ...) {
 }
 
 static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool, int64_t num_pages,
-                      int page_size, int num_kv_heads, int head_dim, int dtype,
-                      const int32_t* page_indptr, const int32_t* page_indices,
-                      const int32_t* last_page_len, int batch, float sm_scale,
+                      int page_size, int num_kv_heads, int head_dim, int dtype, int layout,
+                      const pkv::TableView& tv, const int32_t* page_ids, int batch, float sm_scale,
                       int num_partitions, void* workspace, size_t workspace_bytes, void* out,
                       float* lse, int32_t* error_word, void* stream, int out_f32,
                       long long out_rs, long long lse_rs) {
@@ -195,9 +200,12 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   if (!std::isfinite(sm_scale)) return fail(PKV_ERR_INVALID_ARG, "sm_scale is not finite");
   if (num_partitions < 0 || num_partitions > kMaxPartitions)
     return fail(PKV_ERR_INVALID_ARG, "num_partitions out of range");
+  if (layout != PKV_LAYOUT_HND && layout != PKV_LAYOUT_NHD)
+    return fail(PKV_ERR_INVALID_ARG, "layout must be PKV_LAYOUT_HND or PKV_LAYOUT_NHD");
   if (batch == 0) return ok();
-  if (!q || !pool || !page_indptr || !page_indices || !last_page_len || !out || !workspace)
-    return fail(PKV_ERR_INVALID_ARG, "null pointer");
+  if (!q || !pool || !page_ids || !out || !workspace ||
+      (tv.indptr ? !tv.last_len : (!tv.context_lens || tv.max_blocks < 1)))
+    return fail(PKV_ERR_INVALID_ARG, "null pointer or empty block table");
   if (!aligned(q, 16) || !aligned(pool, 16) || !aligned(out, 16))
     return fail(PKV_ERR_INVALID_ARG, "q, pool and out must be 16-byte aligned");
   if (out == q || out == pool) return fail(PKV_ERR_INVALID_ARG, "out aliases q or pool");
@@ -211,7 +219,8 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
 
   CUtensorMap tmap;
   int one_box = 0;
-  pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, &tmap, &one_box);
+  pkv_status st =
+      pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, layout, &tmap, &one_box);
   if (st != PKV_OK) return st;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -219,9 +228,8 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.q = q;
   a.out = out;
   a.lse = lse;
-  a.indptr = page_indptr;
-  a.indices = page_indices;
-  a.last_len = last_page_len;
+  a.tv = tv;
+  a.indices = page_ids;
   a.counters = reinterpret_cast<int*>(ws + L.counters);
   a.part_lse = reinterpret_cast<float*>(ws + L.part_lse);
   a.part_o = reinterpret_cast<float*>(ws + L.part_o);
@@ -240,6 +248,67 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   cudaError_t e = pkv::launch_decode(tmap, a, dtype == PKV_BF16, N, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
+}
+
+static pkv_status append_impl(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                              int head_dim, int dtype, int layout, const pkv::TableView& tv,
+                              const int32_t* page_ids, int batch, const void* k_new,
+                              const void* v_new, const int32_t* append_indptr, int64_t nnz_new,
+                              int32_t* error_word, void* stream) {
+  if (batch < 0 || nnz_new < 0 || num_pages < 0 || page_size < 1 || num_kv_heads < 1)
+    return fail(PKV_ERR_INVALID_ARG, "negative or zero size");
+  if (dtype != PKV_F16 && dtype != PKV_BF16)
+    return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
+  if (layout != PKV_LAYOUT_HND && layout != PKV_LAYOUT_NHD)
+    return fail(PKV_ERR_INVALID_ARG, "layout must be PKV_LAYOUT_HND or PKV_LAYOUT_NHD");
+  if (head_dim < 8 || head_dim % 8 != 0)
+    return fail(PKV_ERR_UNSUPPORTED, "append needs head_dim a positive multiple of 8");
+  if (nnz_new == 0 || batch == 0) return ok();
+  if (!pool || !page_ids || !k_new || !v_new || !append_indptr ||
+      (tv.indptr ? !tv.last_len : (!tv.context_lens || tv.max_blocks < 1)))
+    return fail(PKV_ERR_INVALID_ARG, "null pointer or empty block table");
+  if (!aligned(pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
+    return fail(PKV_ERR_INVALID_ARG, "pool, k_new and v_new must be 16-byte aligned");
+  if (nnz_new * (int64_t)num_kv_heads > (int64_t)1 << 40)
+    return fail(PKV_ERR_UNSUPPORTED, "too many new rows");
+  pkv::AppendArgs a;
+  a.pool = pool;
+  a.tv = tv;
+  a.indices = page_ids;
+  a.append_indptr = append_indptr;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.err = reinterpret_cast<int*>(error_word);
+  a.num_pages = num_pages;
+  a.nnz = nnz_new;
+  a.batch = batch;
+  a.hkv = num_kv_heads;
+  a.head_dim = head_dim;
+  a.page_size = page_size;
+  a.layout = layout;
+  cudaError_t e = pkv::launch_append(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  return ok();
+}
+
+// unpack the descriptors of the _ex calls
+static pkv_status table_view(const pkv_table_desc* t, pkv::TableView* tv, const int32_t** ids) {
+  if (!t) return fail(PKV_ERR_INVALID_ARG, "null table descriptor");
+  if (t->kind == PKV_TABLE_CSR) {
+    *tv = pkv::csr_view(t->page_indptr, t->last_page_len);
+    *ids = t->page_indices;
+    if (t->batch > 0 && !t->page_indptr) return fail(PKV_ERR_INVALID_ARG, "null page_indptr");
+    return PKV_OK;
+  }
+  if (t->kind == PKV_TABLE_BLOCK) {
+    tv->indptr = nullptr;
+    tv->last_len = nullptr;
+    tv->context_lens = t->context_lens;
+    tv->max_blocks = t->max_blocks_per_seq;
+    *ids = t->block_table;
+    return PKV_OK;
+  }
+  return fail(PKV_ERR_INVALID_ARG, "table kind must be PKV_TABLE_CSR or PKV_TABLE_BLOCK");
 }
 
 extern "C" {
@@ -288,7 +357,7 @@ pkv_status pkv_check_table(const int32_t* page_indptr_h, const int32_t* page_ind
   if (batch == 0) return ok();
   if (page_indptr_h[0] < 0) return fail(PKV_ERR_INVALID_ARG, "page_indptr[0] < 0");
   for (int b = 0; b < batch; ++b) {
-    const pkv::ReqInfo r = pkv::request_info(page_indptr_h, last_page_len_h, b, page_size);
+    const pkv::ReqInfo r = pkv::request_info(pkv::csr_view(page_indptr_h, last_page_len_h), b, page_size);
     if (r.err & pkv::kErrIndptr)
       return fail(PKV_ERR_INVALID_ARG, "page_indptr decreases at request %d", b);
     if (r.err & pkv::kErrLastLen)
@@ -312,7 +381,7 @@ int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page
     return -1;
   long long total = 0;
   for (int b = 0; b < batch; ++b)
-    total += pkv::request_info(page_indptr_h, last_page_len_h, b, page_size).units;
+    total += pkv::request_info(pkv::csr_view(page_indptr_h, last_page_len_h), b, page_size).units;
   const long long W = (long long)num_kv_heads * total;
   if (W == 0) return 0;
   // the kernel uses min(num_partitions, W) partitions: none of them is empty
@@ -326,7 +395,7 @@ int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page
     int b0 = -1;
     pkv::ReqInfo r0{};
     for (int b = 0; b < batch; ++b) {
-      const pkv::ReqInfo r = pkv::request_info(page_indptr_h, last_page_len_h, b, page_size);
+      const pkv::ReqInfo r = pkv::request_info(pkv::csr_view(page_indptr_h, last_page_len_h), b, page_size);
       if (r.units > 0 && (long long)num_kv_heads * Cb <= f0 &&
           f0 < (long long)num_kv_heads * (Cb + r.units)) {
         b0 = b;
@@ -337,8 +406,7 @@ int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page
     }
     if (b0 < 0) return -1;
     pkv::Walk wk;
-    wk.indptr = page_indptr_h;
-    wk.last_len = last_page_len_h;
+    wk.tv = pkv::csr_view(page_indptr_h, last_page_len_h);
     wk.B = batch;
     wk.ps = page_size;
     wk.Hkv = num_kv_heads;
@@ -370,38 +438,9 @@ pkv_status pkv_append(void* pool, int64_t num_pages, int page_size, int num_kv_h
                       const int32_t* page_indices, const int32_t* last_page_len, int batch,
                       const void* k_new, const void* v_new, const int32_t* append_indptr,
                       int64_t nnz_new, int32_t* error_word, void* stream) {
-  if (batch < 0 || nnz_new < 0 || num_pages < 0 || page_size < 1 || num_kv_heads < 1)
-    return fail(PKV_ERR_INVALID_ARG, "negative or zero size");
-  if (dtype != PKV_F16 && dtype != PKV_BF16)
-    return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
-  if (head_dim < 8 || head_dim % 8 != 0)
-    return fail(PKV_ERR_UNSUPPORTED, "append needs head_dim a positive multiple of 8");
-  if (nnz_new == 0 || batch == 0) return ok();
-  if (!pool || !page_indptr || !page_indices || !last_page_len || !k_new || !v_new ||
-      !append_indptr)
-    return fail(PKV_ERR_INVALID_ARG, "null pointer");
-  if (!aligned(pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16))
-    return fail(PKV_ERR_INVALID_ARG, "pool, k_new and v_new must be 16-byte aligned");
-  if (nnz_new * (int64_t)num_kv_heads > (int64_t)1 << 40)
-    return fail(PKV_ERR_UNSUPPORTED, "too many new rows");
-  pkv::AppendArgs a;
-  a.pool = pool;
-  a.indptr = page_indptr;
-  a.indices = page_indices;
-  a.last_len = last_page_len;
-  a.append_indptr = append_indptr;
-  a.k_new = k_new;
-  a.v_new = v_new;
-  a.err = reinterpret_cast<int*>(error_word);
-  a.num_pages = num_pages;
-  a.nnz = nnz_new;
-  a.batch = batch;
-  a.hkv = num_kv_heads;
-  a.head_dim = head_dim;
-  a.page_size = page_size;
-  cudaError_t e = pkv::launch_append(a, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "append launch");
-  return ok();
+  return append_impl(pool, num_pages, page_size, num_kv_heads, head_dim, dtype, PKV_LAYOUT_HND,
+                     pkv::csr_view(page_indptr, last_page_len), page_indices, batch, k_new, v_new,
+                     append_indptr, nnz_new, error_word, stream);
 }
 
 pkv_status pkv_decode(const void* q, int num_qo_heads, const void* pool, int64_t num_pages,
@@ -411,9 +450,39 @@ pkv_status pkv_decode(const void* q, int num_qo_heads, const void* pool, int64_t
                       int num_partitions, void* workspace, size_t workspace_bytes, void* out,
                       float* lse, int32_t* error_word, void* stream) {
   return decode_impl(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
-                     page_indptr, page_indices, last_page_len, batch, sm_scale, num_partitions,
-                     workspace, workspace_bytes, out, lse, error_word, stream, 0,
-                     (long long)num_qo_heads * kDecodeHeadDim, num_qo_heads);
+                     PKV_LAYOUT_HND, pkv::csr_view(page_indptr, last_page_len), page_indices,
+                     batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
+                     error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
+                     num_qo_heads);
+}
+
+pkv_status pkv_decode_ex(const void* q, int num_qo_heads, const pkv_pool_desc* pool,
+                         const pkv_table_desc* table, float sm_scale, int num_partitions,
+                         void* workspace, size_t workspace_bytes, void* out, float* lse,
+                         int32_t* error_word, void* stream) {
+  if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
+  pkv::TableView tv;
+  const int32_t* ids = nullptr;
+  pkv_status st = table_view(table, &tv, &ids);
+  if (st != PKV_OK) return st;
+  return decode_impl(q, num_qo_heads, pool->data, pool->num_pages, pool->page_size,
+                     pool->num_kv_heads, pool->head_dim, pool->dtype, pool->layout, tv, ids,
+                     table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
+                     error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
+                     num_qo_heads);
+}
+
+pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc* table,
+                         const void* k_new, const void* v_new, const int32_t* append_indptr,
+                         int64_t nnz_new, int32_t* error_word, void* stream) {
+  if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
+  pkv::TableView tv;
+  const int32_t* ids = nullptr;
+  pkv_status st = table_view(table, &tv, &ids);
+  if (st != PKV_OK) return st;
+  return append_impl(pool->data, pool->num_pages, pool->page_size, pool->num_kv_heads,
+                     pool->head_dim, pool->dtype, pool->layout, tv, ids, table->batch, k_new,
+                     v_new, append_indptr, nnz_new, error_word, stream);
 }
 
 }  // extern "C"
@@ -517,7 +586,8 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
 
   CUtensorMap tmap;
   int one_box = 0;
-  pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, &tmap, &one_box);
+  pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, PKV_LAYOUT_HND,
+                                  &tmap, &one_box);
   if (st != PKV_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* state_o = reinterpret_cast<float*>(ws + P.state_o);
@@ -547,7 +617,8 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
   if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
   // 2. each request's own pages: the last state slot, as an fp32 state
   st = decode_impl(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
-                   page_indptr, page_indices, last_page_len, batch, sm_scale, N,
+                   PKV_LAYOUT_HND, pkv::csr_view(page_indptr, last_page_len), page_indices,
+                   batch, sm_scale, N,
                    ws + P.decode_ws, workspace_bytes - P.decode_ws,
                    state_o + (size_t)P.splits * num_qo_heads * kDecodeHeadDim,
                    state_lse + (size_t)P.splits * num_qo_heads, error_word, stream, 1,

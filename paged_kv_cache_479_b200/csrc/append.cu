@@ -1,5 +1,8 @@
 // append.cu -- scatter newly decoded tokens' K and V into their pages.
 //
+// Works on either page-table form (CSR or dense block table) and either pool
+// layout (HND or NHD).
+//
 // Blocks take requests (grid-stride over b, blockIdx.y splits a request's new
 // rows further when requests append many tokens); a warp copies one
 // (new token, kv head) row pair.  Position pos of request b lives at page
@@ -27,7 +30,7 @@ __global__ void __launch_bounds__(kWarps * 32) append_kernel(const AppendArgs a)
   const int warp = threadIdx.x >> 5;
   for (int b = blockIdx.x; b < a.batch; b += gridDim.x) {
     const int a0 = a.append_indptr[b], a1 = a.append_indptr[b + 1];
-    const ReqInfo r = request_info(a.indptr, a.last_len, b, a.page_size);
+    const ReqInfo r = request_info(a.tv, b, a.page_size);
     const long long n_new = (long long)a1 - a0;
     if (n_new == 0) continue;
     if (a0 < 0 || n_new < 0 || a1 > a.nnz || r.err || n_new > r.len) {
@@ -48,8 +51,11 @@ __global__ void __launch_bounds__(kWarps * 32) append_kernel(const AppendArgs a)
       const long long slot = pos % a.page_size;
       const int vecs = a.head_dim / 8;  // 16-byte vectors per row
       const size_t src = ((size_t)(a0 + i) * a.hkv + h) * a.head_dim;
-      const size_t dk = ((((size_t)page * 2 + 0) * a.hkv + h) * a.page_size + slot) * a.head_dim;
-      const size_t dv = ((((size_t)page * 2 + 1) * a.hkv + h) * a.page_size + slot) * a.head_dim;
+      // HND: [page][K/V][head][slot][dim]; NHD: [page][K/V][slot][head][dim]
+      const size_t dk = a.layout == PKV_LAYOUT_NHD
+          ? ((((size_t)page * 2 + 0) * a.page_size + slot) * a.hkv + h) * a.head_dim
+          : ((((size_t)page * 2 + 0) * a.hkv + h) * a.page_size + slot) * a.head_dim;
+      const size_t dv = dk + (size_t)a.hkv * a.page_size * a.head_dim;
       const uint16_t* kn = static_cast<const uint16_t*>(a.k_new);
       const uint16_t* vn = static_cast<const uint16_t*>(a.v_new);
       uint16_t* pool = static_cast<uint16_t*>(a.pool);

@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   long long mine = 0;
   int errs = 0;
   for (int b = tid; b < B; b += kDecodeThreads) {
-    const ReqInfo r = request_info(a.indptr, a.last_len, b, a.page_size);
+    const ReqInfo r = request_info(a.tv, b, a.page_size);
     mine += r.units;
     errs |= r.err;
   }
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     r.tiles = 0;
     r.units = 0;
     r.len = 0;
-    if (b < B) r = request_info(a.indptr, a.last_len, b, a.page_size);
+    if (b < B) r = request_info(a.tv, b, a.page_size);
     long long chunk_total;
     const long long incl = block_incl_scan(r.units, ctl.warp_tot, &chunk_total);
     const long long excl = incl - r.units;
@@ -271,12 +271,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   if (warp == kConsumerWarps) {
     // =========================== producer ===========================
     Walk wk;
-    wk.indptr = a.indptr;
-    wk.last_len = a.last_len;
+    wk.tv = a.tv;
     wk.B = B;
     wk.ps = a.page_size;
     wk.Hkv = Hkv;
-    wk.start(ctl.b0, ctl.Cb0, request_info(a.indptr, a.last_len, ctl.b0, a.page_size), f0, f1);
+    wk.start(ctl.b0, ctl.Cb0, request_info(a.tv, ctl.b0, a.page_size), f0, f1);
     const uint32_t ring0 = smem_u32(ring);
     const long long ps = a.page_size;
     const int ps_shift = __ffs(a.page_size) - 1;  // page sizes are powers of two
@@ -320,9 +319,14 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
                   qbytes, qbar);
         // last segment of this request: warm L2 with the next request's table entries
         if (wk.kvh == Hkv - 1 && wk.b + 1 < B) {
-          prefetch_l2(a.indptr + wk.b + 2);
-          prefetch_l2(a.last_len + wk.b + 1);
-          prefetch_l2(a.indices + wk.ri.page_base + (wk.ri.len + ps - 1) / ps);
+          if (a.tv.indptr) {
+            prefetch_l2(a.tv.indptr + wk.b + 2);
+            prefetch_l2(a.tv.last_len + wk.b + 1);
+            prefetch_l2(a.indices + wk.ri.page_base + (wk.ri.len + ps - 1) / ps);
+          } else {
+            prefetch_l2(a.tv.context_lens + wk.b + 1);
+            prefetch_l2(a.indices + wk.ri.page_base + a.tv.max_blocks);
+          }
         }
       }
       __syncwarp();  // the record is written before any lane publishes a tile of it
@@ -366,10 +370,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
                 mbar_arrive_expect_tx(full, kSlotBytes);
                 const uint32_t dst = ring0 + (uint32_t)s * kSlotBytes;
                 const int zk = wk.kvh, zv = Hkv + wk.kvh;
-                if (a.one_box) {
-                  tma_load_5d(dst, &tmap, 0, yoff, 0, zk, page, full);
-                  tma_load_5d(dst + kTileBytes, &tmap, 0, yoff, 0, zv, page, full);
-                } else {
+                if (a.one_box) {  // 5-D view: (dim % 64, slot, dim / 64, kv head, 2 page + K/V)
+                  tma_load_5d(dst, &tmap, 0, yoff, 0, wk.kvh, 2 * page, full);
+                  tma_load_5d(dst + kTileBytes, &tmap, 0, yoff, 0, wk.kvh, 2 * page + 1, full);
+                } else {  // 4-D view of the HND layout: (dim, slot, K/V * Hkv + head, page)
                   tma_load_4d(dst, &tmap, 0, yoff, zk, page, full);
                   tma_load_4d(dst + kHalfBytes, &tmap, 64, yoff, zk, page, full);
                   tma_load_4d(dst + 2 * kHalfBytes, &tmap, 0, yoff, zv, page, full);

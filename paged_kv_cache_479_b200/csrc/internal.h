@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "partition.cuh"
 #include "pkv.h"
 
 namespace pkv {
@@ -16,9 +17,8 @@ struct DecodeArgs {
   const void* q;          // [B][Hq][128]
   void* out;              // [B][Hq][128]
   float* lse;             // [B][Hq] or null
-  const int32_t* indptr;  // [B+1]
-  const int32_t* indices;
-  const int32_t* last_len;  // [B]
+  TableView tv;           // page table (CSR or dense block table)
+  const int32_t* indices; // page ids: CSR indices, or the [B][max_blocks] block table
   int* counters;          // [N] arrival counters (zero between launches)
   float* part_lse;        // [2N][G], log2 domain
   float* part_o;          // [2N][G][128]
@@ -68,9 +68,8 @@ cudaError_t launch_prefix(const CUtensorMap& tmap, const PrefixArgs& a, bool bf1
 
 struct AppendArgs {
   void* pool;
-  const int32_t* indptr;
+  TableView tv;
   const int32_t* indices;
-  const int32_t* last_len;
   const int32_t* append_indptr;
   const void* k_new;
   const void* v_new;
@@ -78,6 +77,7 @@ struct AppendArgs {
   long long num_pages;
   long long nnz;
   int batch, hkv, head_dim, page_size;
+  int layout;  // PKV_LAYOUT_HND or PKV_LAYOUT_NHD
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 

@@ -46,38 +46,70 @@ constexpr int kErrIndptr = 0x02;
 constexpr int kErrLastLen = 0x04;
 constexpr int kErrAppend = 0x08;
 constexpr int kErrTimeout = 0x10;
+constexpr int kErrContextLen = 0x20;
+
+// A page table in one of two forms:
+//   CSR:   request b owns ids[indptr[b] .. indptr[b+1]) and holds
+//          (np - 1) * page_size + last_len[b] tokens;
+//   dense: request b owns ids[b * max_blocks ..] (a [batch][max_blocks] block
+//          table, vLLM-style) and holds context_lens[b] tokens.
+struct TableView {
+  const int32_t* indptr;        // CSR, or null for the dense form
+  const int32_t* last_len;      // CSR
+  const int32_t* context_lens;  // dense
+  int max_blocks;               // dense: row length of the block table
+};
 
 struct ReqInfo {
-  int32_t page_base;  // page_indptr[b]
+  int64_t page_base;  // first entry of the request's page ids
   int32_t err;        // error bits (request then counts as empty)
   int64_t len;        // tokens
   int64_t tiles;      // ceil(len / 16)
   int64_t units;      // kSegmentCost + tiles per kv head, 0 for an empty request
 };
 
-// Length of request b from the CSR table: (np - 1) * page_size + last_page_len.
-PKV_HD ReqInfo request_info(const int32_t* indptr, const int32_t* last_len, int b, int ps) {
+PKV_HD ReqInfo request_info(const TableView& tv, int b, int ps) {
   ReqInfo r;
-  r.page_base = indptr[b];
   r.err = 0;
   r.len = 0;
   r.tiles = 0;
   r.units = 0;
-  const int64_t np = (int64_t)indptr[b + 1] - (int64_t)r.page_base;
-  if (r.page_base < 0 || np < 0) {
-    r.err = kErrIndptr;
-    return r;
+  if (tv.indptr) {
+    r.page_base = tv.indptr[b];
+    const int64_t np = (int64_t)tv.indptr[b + 1] - r.page_base;
+    if (r.page_base < 0 || np < 0) {
+      r.err = kErrIndptr;
+      return r;
+    }
+    if (np == 0) return r;
+    const int ll = tv.last_len[b];
+    if (ll < 1 || ll > ps) {
+      r.err = kErrLastLen;
+      return r;
+    }
+    r.len = (np - 1) * (int64_t)ps + ll;
+  } else {
+    r.page_base = (int64_t)b * tv.max_blocks;
+    const int64_t len = tv.context_lens[b];
+    if (len < 0 || len > (int64_t)tv.max_blocks * ps) {
+      r.err = kErrContextLen;
+      return r;
+    }
+    r.len = len;
   }
-  if (np == 0) return r;
-  const int ll = last_len[b];
-  if (ll < 1 || ll > ps) {
-    r.err = kErrLastLen;
-    return r;
-  }
-  r.len = (np - 1) * (int64_t)ps + ll;
   r.tiles = (r.len + kTileTokens - 1) / kTileTokens;
-  r.units = r.tiles + kSegmentCost;
+  r.units = r.len ? r.tiles + kSegmentCost : 0;
   return r;
+}
+
+// CSR view of (indptr, last_len)
+PKV_HD TableView csr_view(const int32_t* indptr, const int32_t* last_len) {
+  TableView t;
+  t.indptr = indptr;
+  t.last_len = last_len;
+  t.context_lens = nullptr;
+  t.max_blocks = 0;
+  return t;
 }
 
 // First flat unit of partition c.
@@ -110,8 +142,7 @@ PKV_HD SegPlace seg_place(int64_t W, int N, int64_t pair_start, int64_t pair_uni
 // host or device memory (whichever side runs the walk).  A segment whose
 // share of the pair holds only fixed-cost units has no tiles (t0 == t1).
 struct Walk {
-  const int32_t* indptr;
-  const int32_t* last_len;
+  TableView tv;
   int B, ps, Hkv;
   int b, kvh;
   int64_t u;      // unit within the pair
@@ -152,7 +183,7 @@ struct Walk {
     if (f >= f1) return;
     do {
       ++b;
-      ri = request_info(indptr, last_len, b, ps);
+      ri = request_info(tv, b, ps);
     } while (ri.units == 0 && b + 1 < B);
   }
 };

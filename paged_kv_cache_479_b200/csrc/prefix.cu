@@ -118,9 +118,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
         const uint32_t full = smem_u32(&ctl.full[s]);
         const uint32_t kdst = ring0 + (uint32_t)s * kStageBytes + (uint32_t)lane * kBoxBytes;
         const uint32_t vdst = kdst + kKVBytes;
-        if (a.one_box) {
-          tma_load_5d(kdst, &tmap, 0, yoff, 0, kvh, page, full);
-          tma_load_5d(vdst, &tmap, 0, yoff, 0, a.hkv + kvh, page, full);
+        if (a.one_box) {  // 5-D view: (dim % 64, slot, dim / 64, kv head, 2 page + K/V)
+          tma_load_5d(kdst, &tmap, 0, yoff, 0, kvh, 2 * page, full);
+          tma_load_5d(vdst, &tmap, 0, yoff, 0, kvh, 2 * page + 1, full);
         } else {
           tma_load_4d(kdst, &tmap, 0, yoff, kvh, page, full);
           tma_load_4d(kdst + kHalf, &tmap, 64, yoff, kvh, page, full);

@@ -91,7 +91,8 @@ def errors(out, lse, ref_o, ref_l, rows=None):
     lse_err = 0.0
     if l is not None and l.size:
         both_inf = np.isneginf(l) & np.isneginf(ref_l)
-        d = np.where(both_inf, 0.0, l - ref_l)
+        with np.errstate(invalid="ignore"):
+            d = np.where(both_inf, 0.0, l - ref_l)
         lse_err = float(np.abs(d).max())
     return dict(finite=bool(finite), max_abs=max_abs, rel_l2=rel, lse_abs=lse_err)
 

@@ -200,3 +200,26 @@ def test_partition_balances_time_weighted_work():
     for c, b, g, t0, t1, slot, ncov in seg:
         work[c] += (t1 - t0) + (cost if t0 == 0 else 0)
     assert work.max() - work.min() <= 2 * cost + 2
+
+
+def test_descriptor_calls_reject_bad_arguments():
+    L = pkv.lib()
+    p = ctypes.c_void_p(4096)
+    pool = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.BF16, 0, 0)
+    csr = pkv.TableDesc(pkv.TABLE_CSR if hasattr(pkv, "TABLE_CSR") else 0, 4, 4096, 4096, 4096,
+                        None, None, 0, 0)
+    args = lambda pool, table: [p, 8, ctypes.byref(pool) if pool is not None else None,
+                                ctypes.byref(table) if table is not None else None, 0.1, 8, p,
+                                1 << 30, ctypes.c_void_p(8192), None, None, None]
+    assert L.pkv_decode_ex(*args(None, csr)) == 1
+    assert L.pkv_decode_ex(*args(pool, None)) == 1
+    bad_layout = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.BF16, 7, 0)
+    assert L.pkv_decode_ex(*args(bad_layout, csr)) == 1
+    bad_kind = pkv.TableDesc(5, 4, 4096, 4096, 4096, None, None, 0, 0)
+    assert L.pkv_decode_ex(*args(pool, bad_kind)) == 1
+    empty_block = pkv.TableDesc(1, 4, None, None, None, 4096, 4096, 0, 0)
+    assert L.pkv_decode_ex(*args(pool, empty_block)) == 1   # max_blocks_per_seq 0
+    hd64 = pkv.PoolDesc(4096, 64, 16, 2, 64, pkv.BF16, 1, 0)
+    assert L.pkv_decode_ex(*args(hd64, csr)) == 2
+    assert L.pkv_append_ex(None, ctypes.byref(csr), p, p, p, 3, None, None) == 1
+    assert L.pkv_append_ex(ctypes.byref(bad_layout), ctypes.byref(csr), p, p, p, 3, None, None) == 1
