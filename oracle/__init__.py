@@ -18,6 +18,7 @@ from . import build as _build
 
 F16 = 0
 BF16 = 1
+FP8_E4M3 = 3
 
 _STATUS = {
     0: "ok",
@@ -45,6 +46,17 @@ def _load():
         lib.oracle_append.restype = i32
         lib.oracle_merge.argtypes = [p, p, i64, i32, i32, i32, p, p]
         lib.oracle_merge.restype = None
+        f32 = ctypes.c_float
+        lib.oracle_decode_fp8.argtypes = [p, i32, p, f32, f32, i64, i32, i32, i32, i32, i32,
+                                          p, p, p, dbl, p, p]
+        lib.oracle_decode_fp8.restype = i32
+        lib.oracle_append_fp8.argtypes = [p, f32, f32, i64, i32, i32, i32, i32, p, p, p,
+                                          p, p, i32, p]
+        lib.oracle_append_fp8.restype = i32
+        lib.oracle_e4m3_decode.argtypes = [p, i64, p]
+        lib.oracle_e4m3_decode.restype = i32
+        lib.oracle_e4m3_encode.argtypes = [p, i64, f32, p]
+        lib.oracle_e4m3_encode.restype = i32
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -135,3 +147,76 @@ def merge(v, s):
     _load().oracle_merge(vp, sp, N, S, H, D, vo.ctypes.data_as(ctypes.c_void_p),
                          so.ctypes.data_as(ctypes.c_void_p))
     return vo, so
+
+
+def e4m3_values(codes):
+    """Exact value of every E4M3 code (NaN for 0x7f / 0xff), float64."""
+    codes, cp = _c(codes, np.uint8)
+    out = np.zeros(codes.shape, np.float64)
+    _load().oracle_e4m3_decode(cp, codes.size, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def e4m3_encode(x, scale=1.0):
+    """E4M3 codes of float32(x) / float32(scale): nearest, ties to even, saturating."""
+    x, xp = _c(x, np.float32)
+    codes = np.zeros(x.shape, np.uint8)
+    rc = _load().oracle_e4m3_encode(xp, x.size, float(scale),
+                                    codes.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise OracleError(f"oracle_e4m3_encode: {_STATUS.get(rc, rc)}")
+    return codes
+
+
+def decode_fp8(q_bits, q_dtype, pool_codes, k_scale, v_scale, page_indptr, page_indices,
+               last_page_len, scale):
+    """Exact decode attention over an E4M3 pool.
+
+    q_bits     uint16 [B, Hq, D]  fp16/bf16 bits (q_dtype)
+    pool_codes uint8 [P, 2, Hkv, ps, D]; K = code value * k_scale, V = * v_scale
+    Returns (out float64 [B, Hq, D], lse float64 [B, Hq]).
+    """
+    q_bits, qp = _c(q_bits, np.uint16)
+    pool_codes, pp = _c(pool_codes, np.uint8)
+    if pool_codes.ndim != 5 or pool_codes.shape[1] != 2:
+        raise ValueError("pool must be [P, 2, Hkv, ps, D]")
+    P, _, hkv, ps, d = pool_codes.shape
+    B, hq, dq = q_bits.shape
+    if dq != d:
+        raise ValueError("q head_dim does not match pool head_dim")
+    indptr, ip = _c(page_indptr, np.int32)
+    indices, xp = _c(page_indices if len(page_indices) else np.zeros(1, np.int32), np.int32)
+    last, lp = _c(last_page_len if len(last_page_len) else np.zeros(1, np.int32), np.int32)
+    out = np.zeros((B, hq, d), np.float64)
+    lse = np.zeros((B, hq), np.float64)
+    rc = _load().oracle_decode_fp8(qp, int(q_dtype), pp, float(k_scale), float(v_scale), P, ps,
+                                   hkv, d, B, hq, ip, xp, lp, float(scale),
+                                   out.ctypes.data_as(ctypes.c_void_p),
+                                   lse.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise OracleError(f"oracle_decode_fp8: {_STATUS.get(rc, rc)}")
+    return out, lse
+
+
+def append_fp8(pool_codes, k_scale, v_scale, page_indptr, page_indices, last_page_len,
+               k_new_bits, v_new_bits, new_dtype, append_indptr):
+    """Return a copy of an E4M3 pool with the new 16-bit rows quantised in.
+
+    pool_codes uint8 [P, 2, Hkv, ps, D] (not modified); k/v_new uint16 [nnz, Hkv, D]
+    of type new_dtype; element x is stored as e4m3(float32(x) / scale).
+    """
+    pool = np.array(pool_codes, dtype=np.uint8, copy=True, order="C")
+    P, _, hkv, ps, d = pool.shape
+    B = len(page_indptr) - 1
+    indptr, ip = _c(page_indptr, np.int32)
+    indices, xp = _c(page_indices if len(page_indices) else np.zeros(1, np.int32), np.int32)
+    last, lp = _c(last_page_len if len(last_page_len) else np.zeros(1, np.int32), np.int32)
+    kn, kp = _c(k_new_bits if np.size(k_new_bits) else np.zeros(1, np.uint16), np.uint16)
+    vn, vp = _c(v_new_bits if np.size(v_new_bits) else np.zeros(1, np.uint16), np.uint16)
+    ap, app = _c(append_indptr, np.int32)
+    rc = _load().oracle_append_fp8(pool.ctypes.data_as(ctypes.c_void_p), float(k_scale),
+                                   float(v_scale), P, ps, hkv, d, B, ip, xp, lp, kp, vp,
+                                   int(new_dtype), app)
+    if rc != 0:
+        raise OracleError(f"oracle_append_fp8: {_STATUS.get(rc, rc)}")
+    return pool

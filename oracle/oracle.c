@@ -32,6 +32,13 @@
  *     section 4.2 sketches (that sketch averages per-block softmax
  *     outputs, which is not exact; this oracle uses the exact weights).
  *
+ *   fp8 KV cache: the same decode and append over a pool of E4M3 codes
+ *     ("fp8_e4m3" KV cache of the serving configurations in "上下文窗口优化实战：
+ *     如何用PagedAttention+FlashInfer将Llama3-70B的128K上下文吞吐提升3.8倍？"
+ *     section 4.1); a key element is code_value * k_scale, a value element
+ *     code_value * v_scale, and append stores e4m3(float(x) / scale), round to
+ *     nearest even, saturating at +-448.
+ *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - pool layout pool[page][K=0|V=1][kv_head][slot][dim], one pool per layer;
  *   - query head h reads KV head h / (Hq/Hkv) (consecutive query heads share);
@@ -39,7 +46,9 @@
  *     last_page_len[B]; request b holds (np-1)*page_size + last_page_len[b]
  *     tokens when it owns np > 0 pages, and 0 tokens otherwise;
  *   - a request with no tokens yields o = 0 and lse = -inf;
- *   - lse is the natural-log log-sum-exp of the scaled scores.
+ *   - lse is the natural-log log-sum-exp of the scaled scores;
+ *   - fp8: one binary32 scale for all of K and one for all of V (per-tensor),
+ *     the query stays 16-bit, and quantisation divides in binary32 first.
  *
  * Precision: the 16-bit stored values (fp16 or bf16) are widened to double
  * exactly; all arithmetic is in double.  Slots past a request's length are
@@ -57,7 +66,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F16 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F16 = 0, ORACLE_BF16 = 1, ORACLE_FP8_E4M3 = 3 };
 
 /* Status codes: 0 ok, otherwise the table or arguments break an invariant
  * that the pages state (valid length within a page, page ids inside the
@@ -110,6 +119,69 @@ static double widen(uint16_t bits, int dtype) {
   return dtype == ORACLE_BF16 ? widen_bf16(bits) : widen_f16(bits);
 }
 
+/*
+ * FP8 E4M3 ("e4m3fn"): sign, 4-bit exponent with bias 7, 3-bit fraction;
+ * e = 0 is subnormal (fraction * 2^-9); the code S.1111.111 is NaN and there
+ * is no infinity, so the largest finite magnitude is 1.75 * 2^8 = 448.  This
+ * is the 8-bit KV-cache format ("fp8_e4m3" in the serving configurations of
+ * "上下文窗口优化实战：如何用PagedAttention+FlashInfer将Llama3-70B的128K上下文吞吐提升3.8倍？"
+ * section 4.1 and "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署"
+ * section 3.2); a stored code means code_value * scale, one scale for all K and
+ * one for all V.
+ */
+static double widen_e4m3(uint8_t code) {
+  const int sign = code >> 7, e = (code >> 3) & 0xf, frac = code & 7;
+  double v;
+  if (e == 15 && frac == 7) return NAN;
+  if (e == 0) v = ldexp((double)frac, -9);
+  else v = ldexp((double)(frac | 8), e - 10);  /* (1 + frac/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+int oracle_e4m3_decode(const uint8_t* codes, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = widen_e4m3(codes[i]);
+  return ORACLE_OK;
+}
+
+/*
+ * Encode x / scale (both binary32; the quotient rounded once to binary32) as
+ * E4M3: round to the nearest representable value, ties to the even code;
+ * magnitudes beyond 448 saturate to +-448; NaN stays NaN.  The nearest value
+ * is found by comparing against every finite code -- slow, and plainly the
+ * definition.
+ */
+static uint8_t encode_e4m3(float x, float scale) {
+  const float q = x / scale;
+  if (isnan(q)) return 0x7f;
+  const double v = (double)q;
+  const int neg = signbit(q) ? 1 : 0;
+  const double a = fabs(v);
+  if (a >= 448.0) return (uint8_t)((neg << 7) | 0x7e);
+  int best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c < 0x7f; ++c) {           /* non-negative finite codes */
+    const double err = fabs(widen_e4m3((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && (c & 1) == 0)) {
+      best = c;
+      best_err = err;
+    }
+  }
+  return (uint8_t)((neg << 7) | best);
+}
+
+int oracle_e4m3_encode(const float* x, int64_t n, float scale, uint8_t* codes) {
+  if (!(scale > 0.0f) || isinf(scale)) return ORACLE_BAD_ARG;
+  for (int64_t i = 0; i < n; ++i) codes[i] = encode_e4m3(x[i], scale);
+  return ORACLE_OK;
+}
+
+/* Element idx of a pool of 16-bit (fp16 / bf16) or 8-bit (E4M3) values, widened
+ * exactly (E4M3 codes are multiplied by their scale afterwards). */
+static double kv_elem(const void* pool, int kv_dtype, size_t idx) {
+  if (kv_dtype == ORACLE_FP8_E4M3) return widen_e4m3(((const uint8_t*)pool)[idx]);
+  return widen(((const uint16_t*)pool)[idx], kv_dtype);
+}
+
 /* Tokens held by request b under the CSR page table.  Returns -1 when the
  * table breaks an invariant. */
 static int64_t request_len(int b, int page_size, const int32_t* page_indptr,
@@ -159,15 +231,17 @@ static int check_table(int64_t num_pages, int page_size, int batch,
  * factor exp(-m) cancels between numerator and l); it only keeps exp()
  * in range.
  */
-int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
-                  int64_t num_pages, int page_size, int num_kv_heads, int head_dim,
-                  int batch, int num_qo_heads,
-                  const int32_t* page_indptr, const int32_t* page_indices,
-                  const int32_t* last_page_len, double scale,
-                  double* out, double* lse) {
+static int decode_rows(const uint16_t* q, int q_dtype, const void* pool, int kv_dtype,
+                       double k_scale, double v_scale,
+                       int64_t num_pages, int page_size, int num_kv_heads, int head_dim,
+                       int batch, int num_qo_heads,
+                       const int32_t* page_indptr, const int32_t* page_indices,
+                       const int32_t* last_page_len, double scale,
+                       double* out, double* lse) {
   if (batch < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1 ||
       num_qo_heads < num_kv_heads || num_qo_heads % num_kv_heads != 0 ||
-      (dtype != ORACLE_F16 && dtype != ORACLE_BF16))
+      (q_dtype != ORACLE_F16 && q_dtype != ORACLE_BF16) ||
+      (kv_dtype != ORACLE_F16 && kv_dtype != ORACLE_BF16 && kv_dtype != ORACLE_FP8_E4M3))
     return ORACLE_BAD_ARG;
   int rc = check_table(num_pages, page_size, batch, page_indptr, page_indices, last_page_len);
   if (rc != ORACLE_OK) return rc;
@@ -196,15 +270,15 @@ int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
       failed = 1;
       continue;
     }
-    for (int d = 0; d < head_dim; ++d) qd[d] = widen(q[(size_t)row * head_dim + d], dtype);
+    for (int d = 0; d < head_dim; ++d) qd[d] = widen(q[(size_t)row * head_dim + d], q_dtype);
 
     /* scores, in logical token order */
     for (int64_t t = 0; t < len; ++t) {
       const int64_t page = page_indices[page_indptr[b] + t / page_size];
-      const uint16_t* k = pool + pool_offset(page, 0, g, t % page_size,
-                                             num_kv_heads, page_size, head_dim);
+      const size_t k = pool_offset(page, 0, g, t % page_size,
+                                   num_kv_heads, page_size, head_dim);
       double dot = 0.0;
-      for (int d = 0; d < head_dim; ++d) dot += qd[d] * widen(k[d], dtype);
+      for (int d = 0; d < head_dim; ++d) dot += qd[d] * (kv_elem(pool, kv_dtype, k + d) * k_scale);
       s[t] = scale * dot;
     }
     double m = -INFINITY;
@@ -215,10 +289,10 @@ int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
     for (int64_t t = 0; t < len; ++t) {
       const double w = exp(s[t] - m);
       const int64_t page = page_indices[page_indptr[b] + t / page_size];
-      const uint16_t* v = pool + pool_offset(page, 1, g, t % page_size,
-                                             num_kv_heads, page_size, head_dim);
+      const size_t v = pool_offset(page, 1, g, t % page_size,
+                                   num_kv_heads, page_size, head_dim);
       l += w;
-      for (int d = 0; d < head_dim; ++d) o[d] += w * widen(v[d], dtype);
+      for (int d = 0; d < head_dim; ++d) o[d] += w * (kv_elem(pool, kv_dtype, v + d) * v_scale);
     }
     for (int d = 0; d < head_dim; ++d) o[d] /= l;
     lse[row] = m + log(l);
@@ -226,6 +300,33 @@ int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
     free(s);
   }
   return failed ? ORACLE_NO_MEMORY : ORACLE_OK;
+}
+
+int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
+                  int64_t num_pages, int page_size, int num_kv_heads, int head_dim,
+                  int batch, int num_qo_heads,
+                  const int32_t* page_indptr, const int32_t* page_indices,
+                  const int32_t* last_page_len, double scale,
+                  double* out, double* lse) {
+  if (dtype == ORACLE_FP8_E4M3) return ORACLE_BAD_ARG;
+  return decode_rows(q, dtype, pool, dtype, 1.0, 1.0, num_pages, page_size, num_kv_heads,
+                     head_dim, batch, num_qo_heads, page_indptr, page_indices, last_page_len,
+                     scale, out, lse);
+}
+
+/*
+ * oracle_decode_fp8 -- the same attention over an E4M3 pool: key element =
+ * code_value * k_scale, value element = code_value * v_scale (exact in
+ * double); q is fp16 or bf16 (q_dtype).
+ */
+int oracle_decode_fp8(const uint16_t* q, int q_dtype, const uint8_t* pool, float k_scale,
+                      float v_scale, int64_t num_pages, int page_size, int num_kv_heads,
+                      int head_dim, int batch, int num_qo_heads,
+                      const int32_t* page_indptr, const int32_t* page_indices,
+                      const int32_t* last_page_len, double scale, double* out, double* lse) {
+  return decode_rows(q, q_dtype, pool, ORACLE_FP8_E4M3, (double)k_scale, (double)v_scale,
+                     num_pages, page_size, num_kv_heads, head_dim, batch, num_qo_heads,
+                     page_indptr, page_indices, last_page_len, scale, out, lse);
 }
 
 /*
@@ -240,13 +341,15 @@ int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
  * at slot p % page_size.  Pure copies of the 16-bit patterns; every other
  * byte of the pool is left as it was.
  */
-int oracle_append(uint16_t* pool, int64_t num_pages, int page_size, int num_kv_heads,
-                  int head_dim, int batch,
-                  const int32_t* page_indptr, const int32_t* page_indices,
-                  const int32_t* last_page_len,
-                  const uint16_t* k_new, const uint16_t* v_new,
-                  const int32_t* append_indptr) {
+static int append_rows(void* pool, int kv_dtype, float k_scale, float v_scale,
+                       int64_t num_pages, int page_size, int num_kv_heads,
+                       int head_dim, int batch,
+                       const int32_t* page_indptr, const int32_t* page_indices,
+                       const int32_t* last_page_len,
+                       const uint16_t* k_new, const uint16_t* v_new, int new_dtype,
+                       const int32_t* append_indptr) {
   if (batch < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1) return ORACLE_BAD_ARG;
+  if (kv_dtype != ORACLE_FP8_E4M3 && kv_dtype != new_dtype) return ORACLE_BAD_ARG;
   int rc = check_table(num_pages, page_size, batch, page_indptr, page_indices, last_page_len);
   if (rc != ORACLE_OK) return rc;
   if (append_indptr[0] < 0) return ORACLE_BAD_APPEND;
@@ -267,14 +370,54 @@ int oracle_append(uint16_t* pool, int64_t num_pages, int page_size, int num_kv_h
       const int64_t slot = pos % page_size;
       const size_t src = ((size_t)append_indptr[b] + (size_t)i) * row;
       for (int h = 0; h < num_kv_heads; ++h) {
-        memcpy(pool + pool_offset(page, 0, h, slot, num_kv_heads, page_size, head_dim),
-               k_new + src + (size_t)h * head_dim, sizeof(uint16_t) * (size_t)head_dim);
-        memcpy(pool + pool_offset(page, 1, h, slot, num_kv_heads, page_size, head_dim),
-               v_new + src + (size_t)h * head_dim, sizeof(uint16_t) * (size_t)head_dim);
+        const size_t dk = pool_offset(page, 0, h, slot, num_kv_heads, page_size, head_dim);
+        const size_t dv = pool_offset(page, 1, h, slot, num_kv_heads, page_size, head_dim);
+        const uint16_t* ks = k_new + src + (size_t)h * head_dim;
+        const uint16_t* vs = v_new + src + (size_t)h * head_dim;
+        if (kv_dtype == ORACLE_FP8_E4M3) {
+          /* quantise: the 16-bit value widened to binary32, divided by the scale */
+          uint8_t* p8 = (uint8_t*)pool;
+          for (int d = 0; d < head_dim; ++d) {
+            p8[dk + d] = encode_e4m3((float)widen(ks[d], new_dtype), k_scale);
+            p8[dv + d] = encode_e4m3((float)widen(vs[d], new_dtype), v_scale);
+          }
+        } else {
+          memcpy((uint16_t*)pool + dk, ks, sizeof(uint16_t) * (size_t)head_dim);
+          memcpy((uint16_t*)pool + dv, vs, sizeof(uint16_t) * (size_t)head_dim);
+        }
       }
     }
   }
   return ORACLE_OK;
+}
+
+int oracle_append(uint16_t* pool, int64_t num_pages, int page_size, int num_kv_heads,
+                  int head_dim, int batch,
+                  const int32_t* page_indptr, const int32_t* page_indices,
+                  const int32_t* last_page_len,
+                  const uint16_t* k_new, const uint16_t* v_new,
+                  const int32_t* append_indptr) {
+  /* the 16-bit type is irrelevant to a bit copy; BF16 stands for either */
+  return append_rows(pool, ORACLE_BF16, 1.0f, 1.0f, num_pages, page_size, num_kv_heads,
+                     head_dim, batch, page_indptr, page_indices, last_page_len, k_new, v_new,
+                     ORACLE_BF16, append_indptr);
+}
+
+/*
+ * oracle_append_fp8 -- the same scatter into an E4M3 pool: every new element
+ * is quantised as encode(value / scale) (k_scale for K, v_scale for V).
+ */
+int oracle_append_fp8(uint8_t* pool, float k_scale, float v_scale, int64_t num_pages,
+                      int page_size, int num_kv_heads, int head_dim, int batch,
+                      const int32_t* page_indptr, const int32_t* page_indices,
+                      const int32_t* last_page_len, const uint16_t* k_new,
+                      const uint16_t* v_new, int new_dtype, const int32_t* append_indptr) {
+  if (!(k_scale > 0.0f) || !(v_scale > 0.0f) || isinf(k_scale) || isinf(v_scale))
+    return ORACLE_BAD_ARG;
+  if (new_dtype != ORACLE_F16 && new_dtype != ORACLE_BF16) return ORACLE_BAD_ARG;
+  return append_rows(pool, ORACLE_FP8_E4M3, k_scale, v_scale, num_pages, page_size,
+                     num_kv_heads, head_dim, batch, page_indptr, page_indices, last_page_len,
+                     k_new, v_new, new_dtype, append_indptr);
 }
 
 /*

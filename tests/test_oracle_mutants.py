@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+import test_oracle_fp8 as fp8pins
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -31,6 +32,18 @@ MUTANTS = {
                           "const int64_t slot = (pos + 1) % page_size;"),
     "append_page_of_next": ("page_indices[page_indptr[b] + pos / page_size];\n      const int64_t slot",
                             "page_indices[page_indptr[b] + (pos / page_size + 1) % (page_indptr[b + 1] - page_indptr[b])];\n      const int64_t slot"),
+    "e4m3_exponent_bias": ("ldexp((double)(frac | 8), e - 10)", "ldexp((double)(frac | 8), e - 9)"),
+    "e4m3_subnormal_scale": ("if (e == 0) v = ldexp((double)frac, -9);",
+                             "if (e == 0) v = ldexp((double)frac, -10);"),
+    "e4m3_ties_to_odd": ("(c & 1) == 0", "(c & 1) == 1"),
+    "e4m3_saturates_to_nan": ("(uint8_t)((neg << 7) | 0x7e)", "(uint8_t)((neg << 7) | 0x7f)"),
+    "e4m3_scale_multiplies": ("const float q = x / scale;", "const float q = x * scale;"),
+    "fp8_keys_take_v_scale": ("(kv_elem(pool, kv_dtype, k + d) * k_scale)",
+                              "(kv_elem(pool, kv_dtype, k + d) * v_scale)"),
+    "fp8_values_unscaled": ("(kv_elem(pool, kv_dtype, v + d) * v_scale)",
+                            "(kv_elem(pool, kv_dtype, v + d))"),
+    "fp8_append_v_takes_k_scale": ("encode_e4m3((float)widen(vs[d], new_dtype), v_scale)",
+                                   "encode_e4m3((float)widen(vs[d], new_dtype), k_scale)"),
 }
 
 PINS = [
@@ -46,6 +59,13 @@ PINS = [
     pins.test_merge_closed_forms,
     pins.test_append_hand_derived_positions,
     pins.test_append_extends_the_logical_sequence,
+    fp8pins.test_code_values_from_the_format_definition,
+    fp8pins.test_encode_matches_torch_round_to_nearest_even,
+    fp8pins.test_encode_saturates_and_keeps_nan,
+    fp8pins.test_encode_divides_by_the_scale_in_binary32,
+    lambda: [fp8pins.test_fp8_decode_matches_dense_sdpa_on_dequantised_values(c)
+             for c in range(len(fp8pins.FP8_CASES))],
+    fp8pins.test_fp8_append_positions_and_codes,
 ]
 
 
@@ -61,7 +81,9 @@ def test_pins_catch_mutant(name, tmp_path, monkeypatch):
                     "-o", str(so), "-lm"], check=True)
     real = oracle._load()
     lib = ctypes.CDLL(str(so))
-    for fn in ("oracle_decode", "oracle_append", "oracle_merge", "oracle_num_threads"):
+    for fn in ("oracle_decode", "oracle_append", "oracle_merge", "oracle_num_threads",
+               "oracle_decode_fp8", "oracle_append_fp8", "oracle_e4m3_decode",
+               "oracle_e4m3_encode"):
         getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         getattr(lib, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", lib)
