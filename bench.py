@@ -56,6 +56,9 @@ def parse():
                    help="decode a shared-prefix workload with pkv_cascade_decode")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every call from Python instead of replaying CUDA graphs")
+    p.add_argument("--kv", choices=["16bit", "fp8"], default="16bit",
+                   help="KV pool type: the workload's 16-bit type, or FP8 E4M3 codes with "
+                        "per-tensor K/V scales (q and out stay 16-bit)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for cpu_baseline")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="oracle time budget of the reference arm")
     return p.parse_args()
@@ -177,8 +180,18 @@ class ClockSampler:
                 "power_w_max": max(s[3] for s in inside)}
 
 
-def algorithmic_bytes(w):
-    return wl.decode_bytes(w) + wl.append_bytes(w)
+# scales of the E4M3 pools (typical codes have magnitude ~16: keys ~1, values ~0.1)
+FP8_K_SCALE = 1.0 / 16
+FP8_V_SCALE = 0.0071
+
+
+def kv_elem_bytes(args):
+    return 1 if getattr(args, "kv", "16bit") == "fp8" else None
+
+
+def algorithmic_bytes(w, args=None):
+    kvb = kv_elem_bytes(args)
+    return wl.decode_bytes(w, kvb) + wl.append_bytes(w, kvb)
 
 
 def workload_config(w, args, rotation, partitions):
@@ -186,14 +199,18 @@ def workload_config(w, args, rotation, partitions):
            "num_qo_heads": w.num_qo_heads, "num_kv_heads": w.num_kv_heads,
            "head_dim": w.head_dim, "page_size": w.page_size, "pool_pages": w.num_pages,
            "appended_tokens": w.nnz_new, "partitions": partitions,
-           "algorithmic_bytes_per_step": algorithmic_bytes(w),
-           "unique_kv_bytes": wl.kv_cache_bytes(1, w.num_kv_heads, w.head_dim, wl.unique_kv_tokens(w)),
-           "logical_kv_bytes": wl.logical_kv_bytes(w),
+           "algorithmic_bytes_per_step": algorithmic_bytes(w, args),
+           "unique_kv_bytes": wl.kv_cache_bytes(1, w.num_kv_heads, w.head_dim, wl.unique_kv_tokens(w),
+                                                kv_elem_bytes(args) or w.elem_bytes),
+           "logical_kv_bytes": wl.logical_kv_bytes(w, kv_elem_bytes(args)),
            "l2": (f"inputs larger than L2: {rotation} rotating batch copies of "
-                  f"{wl.logical_kv_bytes(w) / 1e6:.0f} MB K/V each"),
+                  f"{wl.logical_kv_bytes(w, kv_elem_bytes(args)) / 1e6:.0f} MB K/V each"),
            "parallelism": f"dp{args.gpus} (independent batches per GPU)"}
     if w.note:
         cfg["values"] = w.note
+    if getattr(args, "kv", "16bit") == "fp8":
+        cfg["kv_cache"] = (f"FP8 E4M3 codes, k_scale {FP8_K_SCALE}, v_scale {FP8_V_SCALE}; "
+                           f"q / out {w.dtype}; append quantises the new {w.dtype} rows")
     if getattr(args, "cascade", False):
         cfg["method"] = "shared-prefix cascade: prefix attention once per 128 query rows, own pages by the decode kernel, states merged"
     return cfg
@@ -305,9 +322,10 @@ def pack(tensors, dev):
 class Batch:
     """One copy of the workload's tensors on the device."""
 
-    def __init__(self, w, dev, value_seed):
+    def __init__(self, w, dev, value_seed, fp8=False):
         wv = wl.Workload(**{**w.__dict__, "seed": value_seed})
-        self.q, self.pool, self.k_new, self.v_new = wl.make_tensors(wv, dev)
+        make = wl.make_fp8_tensors if fp8 else wl.make_tensors
+        self.q, self.pool, self.k_new, self.v_new = make(wv, dev)
 
 
 def run_pkv(args):
@@ -328,10 +346,13 @@ def run_pkv(args):
     w = wl.named(args.workload)
     if args.cascade and not w.shared_prefix_pages:
         raise SystemExit("--cascade needs a workload with a shared prefix (workload 5)")
+    fp8 = args.kv == "fp8"
+    if fp8 and args.cascade:
+        raise SystemExit("--cascade runs on 16-bit pools only")
     N = args.partitions or pkv.default_partitions(local)
-    kv_bytes = wl.logical_kv_bytes(w)
+    kv_bytes = wl.logical_kv_bytes(w, kv_elem_bytes(args))
     rotation = 2 if kv_bytes < (2 << 30) else 1
-    batches = [Batch(w, dev, rank_value_seed(w.seed, rank, r)) for r in range(rotation)]
+    batches = [Batch(w, dev, rank_value_seed(w.seed, rank, r), fp8) for r in range(rotation)]
     t = lambda a: torch.as_tensor(a, device=dev)
     indptr, indices, last = t(w.page_indptr), t(w.page_indices), t(w.last_page_len)
     app = t(w.append_indptr)
@@ -350,12 +371,24 @@ def run_pkv(args):
     stream = torch.cuda.current_stream(dev)
     launches_per_step = (3 if args.cascade else 1) + (1 if w.nnz_new else 0)
 
+    table = pkv.csr_table(indptr, indices, last)
+
     def append_call(bt):
-        if w.nnz_new:
+        if w.nnz_new and fp8:
+            pkv.paged_kv_append_fp8(bt.pool, table, bt.k_new, bt.v_new, app, FP8_K_SCALE,
+                                    FP8_V_SCALE, error_word=err,
+                                    stream=torch.cuda.current_stream(dev))
+        elif w.nnz_new:
             pkv.paged_kv_append(bt.pool, indptr, indices, last, bt.k_new, bt.v_new, app,
                                 error_word=err, stream=torch.cuda.current_stream(dev))
 
     def decode_call(bt):
+        if fp8:
+            pkv.paged_decode_attention_fp8(bt.q, bt.pool, table, ws, FP8_K_SCALE, FP8_V_SCALE,
+                                           out=out, lse=lse, sm_scale=w.sm_scale,
+                                           num_partitions=N, error_word=err,
+                                           stream=torch.cuda.current_stream(dev))
+            return
         if args.cascade:
             pkv.cascade_decode(bt.q, bt.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws, out=out,
                                lse=lse, sm_scale=w.sm_scale, num_partitions=N, error_word=err,
@@ -418,10 +451,10 @@ def run_pkv(args):
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during the timed steps")
 
-    step_bytes = algorithmic_bytes(w)
+    step_bytes = algorithmic_bytes(w, args)
     s_per_step = ms / 1e3 / K
     value = job_throughput(step_bytes, world, ms, K)
-    dec_bytes = wl.decode_bytes(w)
+    dec_bytes = wl.decode_bytes(w, kv_elem_bytes(args))
     peak, peak_kind = measured_hbm()
     achieved = dec_bytes / (decode_ms_max / 1e3) / 1e9
 
@@ -440,20 +473,31 @@ def run_pkv(args):
         out_d, lse_d = d_out
         h2d, d2h = h_in[0].numel(), h_out[0].numel()
 
+        e2e_table = pkv.csr_table(ip_d, ix_d, ll_d)
+
         def e2e_calls(_):
             cur = torch.cuda.current_stream(dev)
             h_in[1].copy_(h_in[0], non_blocking=True)
-            if w.nnz_new:
-                pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d, error_word=err,
-                                    stream=cur)
-            if args.cascade:
-                pkv.cascade_decode(q_d, src.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws,
-                                   out=out_d, lse=lse_d, sm_scale=w.sm_scale, num_partitions=N,
-                                   error_word=err, stream=cur)
+            if fp8:
+                if w.nnz_new:
+                    pkv.paged_kv_append_fp8(src.pool, e2e_table, k_d, v_d, ap_d, FP8_K_SCALE,
+                                            FP8_V_SCALE, error_word=err, stream=cur)
+                pkv.paged_decode_attention_fp8(q_d, src.pool, e2e_table, ws, FP8_K_SCALE,
+                                               FP8_V_SCALE, out=out_d, lse=lse_d,
+                                               sm_scale=w.sm_scale, num_partitions=N,
+                                               error_word=err, stream=cur)
             else:
-                pkv.paged_decode_attention(q_d, src.pool, ip_d, ix_d, ll_d, ws, out=out_d,
-                                           lse=lse_d, sm_scale=w.sm_scale, num_partitions=N,
-                                           error_word=err, stream=cur)
+                if w.nnz_new:
+                    pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d,
+                                        error_word=err, stream=cur)
+                if args.cascade:
+                    pkv.cascade_decode(q_d, src.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws,
+                                       out=out_d, lse=lse_d, sm_scale=w.sm_scale,
+                                       num_partitions=N, error_word=err, stream=cur)
+                else:
+                    pkv.paged_decode_attention(q_d, src.pool, ip_d, ix_d, ll_d, ws, out=out_d,
+                                               lse=lse_d, sm_scale=w.sm_scale, num_partitions=N,
+                                               error_word=err, stream=cur)
             h_out[0].copy_(h_out[1], non_blocking=True)
 
         e2e_calls(None)
@@ -485,12 +529,13 @@ def run_pkv(args):
     clocks.stop()
 
     if rank == 0:
-        traffic = None if args.cascade else recorded_traffic(args.workload)
+        traffic = None if (args.cascade or fp8) else recorded_traffic(args.workload)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if w.dtype == "bf16" else "f16", "data": "synthetic",
+            "dtype": ("e4m3 KV widened to f16, f32 accumulate" if fp8 else
+                      ("bf16" if w.dtype == "bf16" else "f16")), "data": "synthetic",
             "config": {**workload_config(w, args, rotation, N),
                        "launch": "direct calls" if args.no_graph else
                        "append and decode each captured once per batch copy as a CUDA graph, replayed"},
@@ -500,7 +545,8 @@ def run_pkv(args):
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
             "roofline": {"bound": "hbm",
                          "kernel": ("pkv_cascade_decode (prefix + own-page decode + merge launches)"
-                                    if args.cascade else "decode_kernel"),
+                                    if args.cascade else
+                                    ("decode_kernel (E4M3 pool)" if fp8 else "decode_kernel")),
                          "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
@@ -511,7 +557,7 @@ def run_pkv(args):
             "e2e": e2e,
             "clocks": clocks.summary(t_host0, t_host1),
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not fp8:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:

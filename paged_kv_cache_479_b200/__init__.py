@@ -19,11 +19,14 @@ Functions (C names in parentheses):
   cascade_decode         (pkv_cascade_decode)  decode for a batch sharing one prefix
   paged_decode_attention_ex / paged_kv_append_ex (pkv_decode_ex / pkv_append_ex)
                          NHD pools and dense (vLLM-style) block tables
+  paged_decode_attention_fp8 / paged_kv_append_fp8 (pkv_decode_fp8 / pkv_append_fp8)
+                         the 8-bit (FP8 E4M3) KV cache with per-tensor K / V scales
 """
 from ._binding import (  # noqa: F401
     BF16,
     F16,
     F32,
+    FP8_E4M3,
     PkvError,
     PoolDesc,
     TableDesc,
@@ -39,8 +42,10 @@ from ._binding import (  # noqa: F401
     merge_states,
     paged_decode_attention,
     paged_decode_attention_ex,
+    paged_decode_attention_fp8,
     paged_kv_append,
     paged_kv_append_ex,
+    paged_kv_append_fp8,
     pool_desc,
     plan_segments,
     read_error_word,
@@ -63,3 +68,5 @@ pkv_merge_states = merge_states
 pkv_cascade_decode = cascade_decode
 pkv_decode_ex = paged_decode_attention_ex
 pkv_append_ex = paged_kv_append_ex
+pkv_decode_fp8 = paged_decode_attention_fp8
+pkv_append_fp8 = paged_kv_append_fp8

@@ -8,7 +8,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-F16, BF16, F32 = 0, 1, 2
+F16, BF16, F32, FP8_E4M3 = 0, 1, 2, 3
 DEVERR_PAGE_ID = 0x01
 DEVERR_INDPTR = 0x02
 DEVERR_LAST_LEN = 0x04
@@ -67,6 +67,9 @@ _PP = ctypes.POINTER(PoolDesc)
 _TP = ctypes.POINTER(TableDesc)
 _SIGNATURES["pkv_decode_ex"] = ([_P, _I32, _PP, _TP, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["pkv_append_ex"] = ([_PP, _TP, _P, _P, _P, _I64, _P, _P], _I32)
+_SIGNATURES["pkv_decode_fp8"] = (
+    [_P, _I32, _I32, _PP, _F32, _F32, _TP, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
+_SIGNATURES["pkv_append_fp8"] = ([_PP, _F32, _F32, _TP, _P, _P, _I32, _P, _I64, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
 _SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
 _SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
@@ -104,7 +107,8 @@ def _check(status: int, what: str):
                                f"{L.pkv_last_error().decode()}")
 
 
-_DTYPES = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
+_DTYPES = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32,
+           torch.uint8: FP8_E4M3, torch.float8_e4m3fn: FP8_E4M3}
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -319,6 +323,54 @@ def paged_kv_append_ex(pool, table: TableDesc, k_new, v_new, append_indptr, layo
                              _ptr(append_indptr), k_new.shape[0], _ptr(error_word),
                              _stream(stream, pool.device))
     _check(st, "pkv_append_ex")
+
+
+def _fp8_pool(pool, layout):
+    if pool.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise ValueError("an E4M3 pool must be a uint8 or float8_e4m3fn tensor")
+    return pool_desc(pool, layout)
+
+
+def paged_decode_attention_fp8(q, pool, table: TableDesc, workspace, k_scale: float,
+                               v_scale: float, layout: str = "HND", out=None, lse=None,
+                               sm_scale=None, num_partitions: int = 0, error_word=None,
+                               stream=None, return_lse: bool = True):
+    """pkv_decode_fp8: decode over an E4M3 pool (key = code * k_scale, value = code * v_scale);
+    q and out are fp16 or bf16."""
+    _dev_tensor(q, "q")
+    if q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("q must be fp16 or bf16")
+    _dev_tensor(workspace, "workspace")
+    pd = _fp8_pool(pool, layout)
+    B, hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_decode_fp8(_ptr(q), _DTYPES[q.dtype], hq, ctypes.byref(pd), float(k_scale),
+                              float(v_scale), ctypes.byref(table), scale, num_partitions,
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _ptr(out), _ptr(lse), _ptr(error_word), _stream(stream, q.device))
+    _check(st, "pkv_decode_fp8")
+    return out, lse
+
+
+def paged_kv_append_fp8(pool, table: TableDesc, k_new, v_new, append_indptr, k_scale: float,
+                        v_scale: float, layout: str = "HND", error_word=None,
+                        stream=None) -> None:
+    """pkv_append_fp8: quantise fp16/bf16 rows into an E4M3 pool (x -> e4m3(x / scale))."""
+    pd = _fp8_pool(pool, layout)
+    _dev_tensor(k_new, "k_new")
+    _dev_tensor(v_new, "v_new", k_new.dtype)
+    if k_new.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("k_new / v_new must be fp16 or bf16")
+    _dev_tensor(append_indptr, "append_indptr", torch.int32)
+    st = lib().pkv_append_fp8(ctypes.byref(pd), float(k_scale), float(v_scale),
+                              ctypes.byref(table), _ptr(k_new), _ptr(v_new), _DTYPES[k_new.dtype],
+                              _ptr(append_indptr), k_new.shape[0], _ptr(error_word),
+                              _stream(stream, pool.device))
+    _check(st, "pkv_append_fp8")
 
 
 def merge_states(v, s, out_dtype=torch.float32, v_out=None, s_out=None, stream=None,

@@ -122,6 +122,33 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
   }
   auto encode = get_encode();
   if (!encode) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  if (dtype == PKV_FP8_E4M3) {
+    // E4M3 pool: 4-D view (byte of the row, slot, kv head, 2 page + K/V) with
+    // [2][16 slots][128 bytes] boxes -- one load brings a tile's K and V
+    const bool nhd = layout == PKV_LAYOUT_NHD;
+    const cuuint64_t row = kDecodeHeadDim;  // one token's K (or V) row: 128 bytes
+    cuuint64_t dims[4] = {row, (cuuint64_t)ps, (cuuint64_t)hkv, (cuuint64_t)2 * pages};
+    cuuint64_t strides[3] = {nhd ? (cuuint64_t)hkv * row : row, nhd ? row : (cuuint64_t)ps * row,
+                             (cuuint64_t)hkv * ps * row};
+    cuuint32_t box[4] = {(cuuint32_t)row, (cuuint32_t)pkv::kTileTokens, 1, 2};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMap m8;
+    const CUresult r8 = encode(&m8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(pool), dims,
+                               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r8 != CUDA_SUCCESS)
+      return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed for the E4M3 pool (%d)", (int)r8);
+    std::lock_guard<std::mutex> lk(mu);
+    keys[next] = key;
+    maps[next] = m8;
+    kinds[next] = 2;
+    next = (next + 1) % 16;
+    if (used < 16) ++used;
+    *out = m8;
+    *one_box = 2;
+    return PKV_OK;
+  }
   const CUtensorMapDataType dt =
       dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const cuuint64_t row = (cuuint64_t)kDecodeHeadDim * 2;  // bytes of one token's K (or V) row
@@ -179,16 +206,25 @@ pkv_status pkv::set_error(pkv_status s, const char* fmt, ...) {
   return s;
 }
 
+// dtype: type of q and out; kv_dtype: the pool's (dtype, or PKV_FP8_E4M3 with
+// k_scale / v_scale)
 static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool, int64_t num_pages,
                       int page_size, int num_kv_heads, int head_dim, int dtype, int layout,
                       const pkv::TableView& tv, const int32_t* page_ids, int batch, float sm_scale,
                       int num_partitions, void* workspace, size_t workspace_bytes, void* out,
                       float* lse, int32_t* error_word, void* stream, int out_f32,
-                      long long out_rs, long long lse_rs) {
+                      long long out_rs, long long lse_rs, int kv_dtype = -1,
+                      float k_scale = 1.f, float v_scale = 1.f) {
+  if (kv_dtype < 0) kv_dtype = dtype;
   if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1)
     return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
   if (dtype != PKV_F16 && dtype != PKV_BF16)
     return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
+  if (kv_dtype != dtype && kv_dtype != PKV_FP8_E4M3)
+    return fail(PKV_ERR_INVALID_ARG, "the pool must hold q's type or PKV_FP8_E4M3 codes");
+  if (kv_dtype == PKV_FP8_E4M3 &&
+      !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+    return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
   if (num_qo_heads % num_kv_heads != 0)
     return fail(PKV_ERR_INVALID_ARG, "num_qo_heads must be a multiple of num_kv_heads");
   if (head_dim != kDecodeHeadDim) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 128");
@@ -220,7 +256,7 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   CUtensorMap tmap;
   int one_box = 0;
   pkv_status st =
-      pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, layout, &tmap, &one_box);
+      pool_tensor_map(pool, num_pages, page_size, num_kv_heads, kv_dtype, layout, &tmap, &one_box);
   if (st != PKV_OK) return st;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -240,25 +276,37 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.hkv = num_kv_heads;
   a.group = group;
   a.page_size = page_size;
-  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  const bool fp8 = kv_dtype == PKV_FP8_E4M3;
+  a.scale_log2 = (float)((double)sm_scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
+  a.v_scale = fp8 ? v_scale : 1.f;
   a.one_box = one_box;
   a.out_f32 = out_f32;
   a.out_rs = out_rs;
   a.lse_rs = lse_rs;
-  cudaError_t e = pkv::launch_decode(tmap, a, dtype == PKV_BF16, N, static_cast<cudaStream_t>(stream));
+  cudaError_t e =
+      pkv::launch_decode(tmap, a, dtype == PKV_BF16, fp8, N, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }
 
+// dtype: type of k_new / v_new; kv_dtype: the pool's (dtype, or PKV_FP8_E4M3:
+// the rows are quantised with k_scale / v_scale)
 static pkv_status append_impl(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
                               int head_dim, int dtype, int layout, const pkv::TableView& tv,
                               const int32_t* page_ids, int batch, const void* k_new,
                               const void* v_new, const int32_t* append_indptr, int64_t nnz_new,
-                              int32_t* error_word, void* stream) {
+                              int32_t* error_word, void* stream, int kv_dtype = -1,
+                              float k_scale = 1.f, float v_scale = 1.f) {
+  if (kv_dtype < 0) kv_dtype = dtype;
   if (batch < 0 || nnz_new < 0 || num_pages < 0 || page_size < 1 || num_kv_heads < 1)
     return fail(PKV_ERR_INVALID_ARG, "negative or zero size");
   if (dtype != PKV_F16 && dtype != PKV_BF16)
     return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
+  if (kv_dtype != dtype && kv_dtype != PKV_FP8_E4M3)
+    return fail(PKV_ERR_INVALID_ARG, "the pool must hold the rows' type or PKV_FP8_E4M3 codes");
+  if (kv_dtype == PKV_FP8_E4M3 &&
+      !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+    return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
   if (layout != PKV_LAYOUT_HND && layout != PKV_LAYOUT_NHD)
     return fail(PKV_ERR_INVALID_ARG, "layout must be PKV_LAYOUT_HND or PKV_LAYOUT_NHD");
   if (head_dim < 8 || head_dim % 8 != 0)
@@ -286,6 +334,10 @@ static pkv_status append_impl(void* pool, int64_t num_pages, int page_size, int 
   a.head_dim = head_dim;
   a.page_size = page_size;
   a.layout = layout;
+  a.fp8 = kv_dtype == PKV_FP8_E4M3;
+  a.in_bf16 = dtype == PKV_BF16;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
   cudaError_t e = pkv::launch_append(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
   return ok();
@@ -465,6 +517,8 @@ pkv_status pkv_decode_ex(const void* q, int num_qo_heads, const pkv_pool_desc* p
   const int32_t* ids = nullptr;
   pkv_status st = table_view(table, &tv, &ids);
   if (st != PKV_OK) return st;
+  if (pool->dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_INVALID_ARG, "an E4M3 pool needs pkv_decode_fp8 (it carries the scales)");
   return decode_impl(q, num_qo_heads, pool->data, pool->num_pages, pool->page_size,
                      pool->num_kv_heads, pool->head_dim, pool->dtype, pool->layout, tv, ids,
                      table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
@@ -480,9 +534,44 @@ pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc* table,
   const int32_t* ids = nullptr;
   pkv_status st = table_view(table, &tv, &ids);
   if (st != PKV_OK) return st;
+  if (pool->dtype == PKV_FP8_E4M3)
+    return fail(PKV_ERR_INVALID_ARG, "an E4M3 pool needs pkv_append_fp8 (it carries the scales)");
   return append_impl(pool->data, pool->num_pages, pool->page_size, pool->num_kv_heads,
                      pool->head_dim, pool->dtype, pool->layout, tv, ids, table->batch, k_new,
                      v_new, append_indptr, nnz_new, error_word, stream);
+}
+
+pkv_status pkv_decode_fp8(const void* q, int q_dtype, int num_qo_heads, const pkv_pool_desc* pool,
+                          float k_scale, float v_scale, const pkv_table_desc* table,
+                          float sm_scale, int num_partitions, void* workspace,
+                          size_t workspace_bytes, void* out, float* lse, int32_t* error_word,
+                          void* stream) {
+  if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
+  if (pool->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_FP8_E4M3");
+  pkv::TableView tv;
+  const int32_t* ids = nullptr;
+  pkv_status st = table_view(table, &tv, &ids);
+  if (st != PKV_OK) return st;
+  return decode_impl(q, num_qo_heads, pool->data, pool->num_pages, pool->page_size,
+                     pool->num_kv_heads, pool->head_dim, q_dtype, pool->layout, tv, ids,
+                     table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
+                     error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
+                     num_qo_heads, PKV_FP8_E4M3, k_scale, v_scale);
+}
+
+pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, float v_scale,
+                          const pkv_table_desc* table, const void* k_new, const void* v_new,
+                          int new_dtype, const int32_t* append_indptr, int64_t nnz_new,
+                          int32_t* error_word, void* stream) {
+  if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
+  if (pool->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_FP8_E4M3");
+  pkv::TableView tv;
+  const int32_t* ids = nullptr;
+  pkv_status st = table_view(table, &tv, &ids);
+  if (st != PKV_OK) return st;
+  return append_impl(pool->data, pool->num_pages, pool->page_size, pool->num_kv_heads,
+                     pool->head_dim, new_dtype, pool->layout, tv, ids, table->batch, k_new, v_new,
+                     append_indptr, nnz_new, error_word, stream, PKV_FP8_E4M3, k_scale, v_scale);
 }
 
 }  // extern "C"

@@ -202,6 +202,32 @@ __device__ __forceinline__ uint16_t to_bits16(float x) {
   }
 }
 
+// ---- FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 fraction bits; no
+// infinity, S.1111.111 is NaN).  Every E4M3 value is exact in fp16, so the
+// widening below loses nothing.
+
+// two E4M3 codes (low byte -> low half) widened to an fp16 pair, exactly
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t codes) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(codes));
+  return r;
+}
+
+// byte permute: result byte k = byte (sel >> 4k) & 7 of {b:a}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// two fp32 values (lo -> low byte) rounded to nearest even E4M3, saturating
+// at +-448 (satfinite); NaN stays NaN
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // 2^x, PTX ex2.approx (relative error about 2^-22); ex2(-inf) = +0
 __device__ __forceinline__ float ex2(float x) {
   float y;

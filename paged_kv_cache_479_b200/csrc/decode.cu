@@ -66,12 +66,25 @@ constexpr int kIssueLanes = kStages < 16 ? kStages : 16;  // producer lanes issu
 static_assert(kStages % kConsumerWarps == 0 && 32 % kIssueLanes == 0,
               "each ring slot must have a single consumer warp");
 constexpr int kHalfBytes = kTileTokens * 64 * 2;  // one [16][64] box: 2 KiB
-constexpr int kTileBytes = 2 * kHalfBytes;        // K or V of one tile: 4 KiB
+constexpr int kTileBytes = 2 * kHalfBytes;        // K or V of one 16-bit tile: 4 KiB
 constexpr int kSlotBytes = 2 * kTileBytes;        // K + V: 8 KiB
-constexpr int kSegRecs = 8;
+// An 8-bit (E4M3) tile is half the bytes; its ring has twice the slots, so the
+// same bytes are in flight.
+constexpr int kMaxStages = 2 * kStages;
+constexpr int kSegRecs = 16;                      // segment records in flight
 constexpr int kMaxGroup = 8;
-constexpr int kQBufs = 4;                         // staged query blocks in flight
+constexpr int kQBufs = 8;                         // staged query blocks in flight
 constexpr int kQBufBytes = kMaxGroup * 128 * 2;   // G query rows: up to 2 KiB
+// The producer refills query buffer (and record) seg % n for segment seg + n
+// only after issuing every tile of segments seg .. seg+n-1 (each a multiple of
+// 8 tiles, at least 8).  With S ring slots that means the tiles up to
+// start(seg) + 8n - 1 - S have been released, which includes every consumer
+// warp's first tile of segment seg -- where it reads the buffer -- as long as
+// S <= 8 (n - 1).  The consumer's parity (sid / kQBufs) & 1 needs the record
+// index to run over at least two buffer rounds.
+static_assert(kMaxStages <= kConsumerWarps * (kQBufs - 1) &&
+                  kMaxStages <= kConsumerWarps * (kSegRecs - 1) && kSegRecs % (2 * kQBufs) == 0,
+              "a query buffer or segment record could be refilled before every warp read it");
 constexpr int kScratchStride = kD + 4;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -90,11 +103,11 @@ struct SegRec {
 };
 
 struct __align__(16) Ctl {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t cons;                      // consumer-only barrier (256 arrivals)
   uint64_t qfull[kQBufs];             // a segment's query rows landed in qbuf[i]
-  int meta[kStages];
+  int meta[kMaxStages];
   SegRec seg[kSegRecs];
   long long warp_tot[kDecodeThreads / 32];
   long long Cb0;
@@ -175,9 +188,19 @@ __device__ __forceinline__ bool cons_sync(Ctl& ctl, uint32_t& phase, int* err) {
   return ok;
 }
 
-template <bool BF16>
+template <bool BF16, bool FP8>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
+  // ring geometry of this KV type (16-bit: 16 slots of 8 KiB; E4M3: 32 of 4 KiB)
+  constexpr int kSt = FP8 ? 2 * kStages : kStages;
+  constexpr int kTileB = FP8 ? kTileBytes / 2 : kTileBytes;
+  constexpr int kSlotB = 2 * kTileB;
+  constexpr int kIssue = kSt < 16 ? kSt : 16;
+  static_assert(kSt % kConsumerWarps == 0 && 32 % kIssue == 0 && kSt <= kMaxStages,
+                "each ring slot must have a single consumer warp");
+  // MMA operand type: 16-bit pools use their own type; E4M3 codes are widened
+  // to fp16 (exact), so those tiles run the fp16 MMA
+  constexpr bool kMmaBF16 = BF16 && !FP8;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte-swizzled TMA boxes need 1024-byte aligned shared addresses
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -194,7 +217,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   const int Hkv = a.hkv;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(smem_u32(&ctl.full[s]), 1);
       mbar_init(smem_u32(&ctl.empty[s]), 32);
     }
@@ -355,24 +378,28 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         const int flags = ((k >= n_pad - kConsumerWarps) ? kMetaSegLast : 0) |
                           ((seg & (kSegRecs - 1)) << kMetaSegShift);
         const int cnt = (int)((n_pad - k0) < 32 ? (n_pad - k0) : 32);
-        // lanes [jb, jb + kIssueLanes) publish their tiles concurrently (distinct ring slots)
-        for (int jb = 0; jb < cnt; jb += kIssueLanes) {
+        // lanes [jb, jb + kIssue) publish their tiles concurrently (distinct ring slots)
+        for (int jb = 0; jb < cnt; jb += kIssue) {
           int okl = 1;
-          if (lane >= jb && lane < jb + kIssueLanes && lane < cnt) {
+          if (lane >= jb && lane < jb + kIssue && lane < cnt) {
             const uint32_t it = i + (uint32_t)(lane - jb);
-            const int s = (int)(it % kStages);
-            okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kStages) & 1u) ^ 1u,
+            const int s = (int)(it % kSt);
+            okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kSt) & 1u) ^ 1u,
                                     &ctl.abort, a.err);
             if (okl) {
               const uint32_t full = smem_u32(&ctl.full[s]);
               if (page >= 0 && valid > 0) {
                 ctl.meta[s] = valid | flags;
-                mbar_arrive_expect_tx(full, kSlotBytes);
-                const uint32_t dst = ring0 + (uint32_t)s * kSlotBytes;
+                mbar_arrive_expect_tx(full, kSlotB);
+                const uint32_t dst = ring0 + (uint32_t)s * kSlotB;
                 const int zk = wk.kvh, zv = Hkv + wk.kvh;
-                if (a.one_box) {  // 5-D view: (dim % 64, slot, dim / 64, kv head, 2 page + K/V)
+                if constexpr (FP8) {
+                  // 4-D view (byte of the row, slot, kv head, 2 page + K/V): one
+                  // [2][16][128] box brings the tile's K and V
+                  tma_load_4d(dst, &tmap, 0, yoff, wk.kvh, 2 * page, full);
+                } else if (a.one_box) {  // 5-D view: (dim % 64, slot, dim / 64, kv head, 2 page + K/V)
                   tma_load_5d(dst, &tmap, 0, yoff, 0, wk.kvh, 2 * page, full);
-                  tma_load_5d(dst + kTileBytes, &tmap, 0, yoff, 0, wk.kvh, 2 * page + 1, full);
+                  tma_load_5d(dst + kTileB, &tmap, 0, yoff, 0, wk.kvh, 2 * page + 1, full);
                 } else {  // 4-D view of the HND layout: (dim, slot, K/V * Hkv + head, page)
                   tma_load_4d(dst, &tmap, 0, yoff, zk, page, full);
                   tma_load_4d(dst + kHalfBytes, &tmap, 64, yoff, zk, page, full);
@@ -386,7 +413,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
             }
           }
           ok = __all_sync(0xffffffffu, okl) != 0;
-          const int issued = (cnt - jb) < kIssueLanes ? (cnt - jb) : kIssueLanes;
+          const int issued = (cnt - jb) < kIssue ? (cnt - jb) : kIssue;
           i += (uint32_t)issued;
           if (!ok) break;
         }
@@ -399,8 +426,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       int okl = 1;
       if (lane < kConsumerWarps) {
         const uint32_t it = i + lane;
-        const int s = (int)(it % kStages);
-        okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kStages) & 1u) ^ 1u, &ctl.abort,
+        const int s = (int)(it % kSt);
+        okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kSt) & 1u) ^ 1u, &ctl.abort,
                                 a.err);
         if (okl) {
           ctl.meta[s] = kMetaEnd;
@@ -412,11 +439,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     }
     if (!ok && lane == 0) {
       // aborted: let the copies already issued land before the CTA exits
-      const uint32_t first = i > (uint32_t)kStages ? i - kStages : 0;
+      const uint32_t first = i > (uint32_t)kSt ? i - kSt : 0;
       for (uint32_t k = first; k < i; ++k) {
-        const uint32_t bar = smem_u32(&ctl.full[k % kStages]);
+        const uint32_t bar = smem_u32(&ctl.full[k % kSt]);
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bar, (k / kStages) & 1u) &&
+        while (!mbar_try_wait(bar, (k / kSt) & 1u) &&
                global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
@@ -442,6 +469,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   const uint32_t ring0 = smem_u32(ring);
 
   uint32_t qf[8][2];
+  float qsc0 = sl2, qsc1 = sl2;  // score scale of S^T columns 2cq, 2cq+1 (E4M3 pools)
   float o[8][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   int cur_seg = -1;
@@ -452,8 +480,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   bool clean = true;
 
   for (uint32_t i = warp;; i += kConsumerWarps) {
-    const int s = (int)(i % kStages);
-    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kStages) & 1u, &ctl.abort, a.err)) {
+    const int s = (int)(i % kSt);
+    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kSt) & 1u, &ctl.abort, a.err)) {
       clean = false;
       break;
     }
@@ -472,12 +500,59 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       }
       // the segment's query rows, staged by the producer
       const int qb = sid & (kQBufs - 1);
-      if (!mbar_wait_bounded(smem_u32(&ctl.qfull[qb]), (uint32_t)(sid >> 2) & 1u, &ctl.abort,
+      if (!mbar_wait_bounded(smem_u32(&ctl.qfull[qb]), (uint32_t)(sid / kQBufs) & 1u, &ctl.abort,
                              a.err)) {
         clean = false;
         break;
       }
-      if (g < G) {
+      if constexpr (FP8) {
+        // B fragments of the fp16 MMA against widened E4M3 keys.  Head g's dims
+        // are taken in the order the 8-bit K fragments deliver them: k slots
+        // 2cq, 2cq+1, 2cq+8, 2cq+9 of chunk ch are dims 16ch + 4cq + 0..3.  A
+        // bf16 row is first multiplied by a power of two that puts its largest
+        // magnitude in [2^14, 2^15) (inside fp16's range; only elements 2^28
+        // below that maximum lose bits), and the score scale undoes it.
+        uint2 raw[8];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) raw[ch] = make_uint2(0u, 0u);
+        if (g < G) {
+          const uint8_t* qp = qbuf + (size_t)qb * kQBufBytes + ((size_t)g * kD + 4 * cq) * 2;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) raw[ch] = *reinterpret_cast<const uint2*>(qp + ch * 32);
+        }
+        int qexp = 0;  // head g's row was multiplied by 2^qexp
+        if constexpr (BF16) {
+          float mx = 0.f;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const float2 u = unpack2<true>(raw[ch].x), v = unpack2<true>(raw[ch].y);
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(u.x), fabsf(u.y)), fmaxf(fabsf(v.x), fabsf(v.y))));
+          }
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          int e = (mx > 0.f && mx <= 3.0e38f) ? ((__float_as_int(mx) >> 23) & 0xff) - 127 : 0;
+          e = e < -100 ? -100 : e;
+          qexp = 14 - e;
+          const float f = __int_as_float((127 + qexp) << 23);
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const float2 u = unpack2<true>(raw[ch].x), v = unpack2<true>(raw[ch].y);
+            qf[ch][0] = pack2<false>(u.x * f, u.y * f);
+            qf[ch][1] = pack2<false>(v.x * f, v.y * f);
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            qf[ch][0] = raw[ch].x;
+            qf[ch][1] = raw[ch].y;
+          }
+        }
+        // this lane's S^T columns are heads 2cq and 2cq+1 (held by lanes 8cq and 8cq+4)
+        const int e0 = __shfl_sync(0xffffffffu, qexp, 8 * cq);
+        const int e1 = __shfl_sync(0xffffffffu, qexp, 8 * cq + 4);
+        qsc0 = sl2 * __int_as_float((127 - e0) << 23);
+        qsc1 = sl2 * __int_as_float((127 - e1) << 23);
+      } else if (g < G) {
         const uint16_t* qp =
             reinterpret_cast<const uint16_t*>(qbuf + (size_t)qb * kQBufBytes) + g * kD + 2 * cq;
 #pragma unroll
@@ -495,13 +570,30 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       l0 = l1 = 0.f;
     }
     const int valid = (info & kMetaValid) > kTileTokens ? kTileTokens : (info & kMetaValid);
-    const uint32_t kb = ring0 + (uint32_t)s * kSlotBytes;
-    const uint32_t vb = kb + kTileBytes;
+    const uint32_t kb = ring0 + (uint32_t)s * kSlotB;
+    const uint32_t vb = kb + kTileB;
     bool wrote_smem = false;
     if (valid > 0) {
       // ---- S^T = K_tile . Q^T  (tokens on M, heads on N)
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-      {
+      if constexpr (FP8) {
+        // one ldmatrix.x4 = tokens (0-7 | 8-15) x chunks (2jj | 2jj+1) of 16 codes;
+        // lane (g, cq) gets codes 4cq .. 4cq+3 of token g's chunk, widened in pairs
+        const int tok = ((mi & 1) << 3) + r8;
+        const uint32_t rowb = kb + (uint32_t)tok * 128u;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int chunk = 2 * jj + (mi >> 1);
+          uint32_t r0, r1, r2, r3;
+          ldmatrix_x4(rowb + (uint32_t)(((chunk & 7) ^ r8) << 4), r0, r1, r2, r3);
+          mma_16816<false>(sa, e4m3x2_to_f16x2((uint16_t)r0), e4m3x2_to_f16x2((uint16_t)r1),
+                           e4m3x2_to_f16x2((uint16_t)(r0 >> 16)), e4m3x2_to_f16x2((uint16_t)(r1 >> 16)),
+                           qf[2 * jj][0], qf[2 * jj][1]);
+          mma_16816<false>(sb, e4m3x2_to_f16x2((uint16_t)r2), e4m3x2_to_f16x2((uint16_t)r3),
+                           e4m3x2_to_f16x2((uint16_t)(r2 >> 16)), e4m3x2_to_f16x2((uint16_t)(r3 >> 16)),
+                           qf[2 * jj + 1][0], qf[2 * jj + 1][1]);
+        }
+      } else {
         const int tok = ((mi & 1) << 3) + r8;
         const uint32_t rowb = kb + (uint32_t)tok * 128u;
 #pragma unroll
@@ -519,10 +611,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       }
       // ---- mask tokens past the request's end, online softmax (log2 units)
       const bool v_lo = g < valid, v_hi = g + 8 < valid;
-      const float x0 = v_lo ? (sa[0] + sb[0]) * sl2 : -INFINITY;  // token g,   head 2cq
-      const float x1 = v_lo ? (sa[1] + sb[1]) * sl2 : -INFINITY;  // token g,   head 2cq+1
-      const float x2 = v_hi ? (sa[2] + sb[2]) * sl2 : -INFINITY;  // token g+8, head 2cq
-      const float x3 = v_hi ? (sa[3] + sb[3]) * sl2 : -INFINITY;  // token g+8, head 2cq+1
+      const float sc0 = FP8 ? qsc0 : sl2, sc1 = FP8 ? qsc1 : sl2;
+      const float x0 = v_lo ? (sa[0] + sb[0]) * sc0 : -INFINITY;  // token g,   head 2cq
+      const float x1 = v_lo ? (sa[1] + sb[1]) * sc1 : -INFINITY;  // token g,   head 2cq+1
+      const float x2 = v_hi ? (sa[2] + sb[2]) * sc0 : -INFINITY;  // token g+8, head 2cq
+      const float x3 = v_hi ? (sa[3] + sb[3]) * sc1 : -INFINITY;  // token g+8, head 2cq+1
       float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -547,27 +640,56 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         }
       }
       // ---- P^T as the B operand of the PV MMA (movmatrix transposes S^T's layout)
-      const uint32_t ph0 = pack2<BF16>(p0, p1), ph1 = pack2<BF16>(p2, p3);
+      const uint32_t ph0 = pack2<kMmaBF16>(p0, p1), ph1 = pack2<kMmaBF16>(p2, p3);
       const uint32_t bh0 = movmatrix_trans(ph0), bh1 = movmatrix_trans(ph1);
       uint32_t bl0 = 0, bl1 = 0;
-      if constexpr (BF16) {
+      if constexpr (kMmaBF16) {
         const float2 f0 = unpack2<true>(ph0), f1 = unpack2<true>(ph1);
         bl0 = movmatrix_trans(pack2<true>(p0 - f0.x, p1 - f0.y));
         bl1 = movmatrix_trans(pack2<true>(p2 - f1.x, p3 - f1.y));
       }
       // ---- zero V rows past the end (their slots may hold anything, even NaN)
       if (valid < kTileTokens) {
-        uint8_t* vrow = ring + (size_t)s * kSlotBytes + kTileBytes;
-        for (int idx = lane; idx < (kTileTokens - valid) * 16; idx += 32) {
-          const int tok = valid + (idx >> 4), half = (idx >> 3) & 1, ch = idx & 7;
-          *reinterpret_cast<uint4*>(vrow + half * kHalfBytes + tok * 128 + ch * 16) =
-              make_uint4(0, 0, 0, 0);
+        uint8_t* vrow = ring + (size_t)s * kSlotB + kTileB;
+        if constexpr (FP8) {  // one [16][128]-byte box
+          for (int idx = lane; idx < (kTileTokens - valid) * 8; idx += 32) {
+            const int tok = valid + (idx >> 3), ch = idx & 7;
+            *reinterpret_cast<uint4*>(vrow + tok * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+          }
+        } else {  // two [16][64]-element boxes
+          for (int idx = lane; idx < (kTileTokens - valid) * 16; idx += 32) {
+            const int tok = valid + (idx >> 4), half = (idx >> 3) & 1, ch = idx & 7;
+            *reinterpret_cast<uint4*>(vrow + half * kHalfBytes + tok * 128 + ch * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
         }
         wrote_smem = true;
         __syncwarp();
       }
       // ---- O^T += V_tile^T . P^T   (dims on M, heads on N, tokens on K)
-      {
+      if constexpr (FP8) {
+        // ldmatrix.trans of tokens (0-7 | 8-15) x chunks (2jj | 2jj+1) hands lane
+        // (g, cq) codes V[2cq][2g], V[2cq][2g+1], V[2cq+1][2g], V[2cq+1][2g+1];
+        // a byte permute pairs them by dim, so accumulator o[2jj] holds dims
+        // 32jj + 2g (row g) and 32jj + 16 + 2g (row g+8), o[2jj+1] those + 1
+        const int tok = ((mi >> 1) << 3) + r8;
+        const uint32_t rowb = vb + (uint32_t)tok * 128u;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int chunk = 2 * jj + (mi & 1);
+          uint32_t r0, r1, r2, r3;
+          ldmatrix_x4_trans(rowb + (uint32_t)(((chunk & 7) ^ r8) << 4), r0, r1, r2, r3);
+          r0 = prmt(r0, 0u, 0x3120u);
+          r1 = prmt(r1, 0u, 0x3120u);
+          r2 = prmt(r2, 0u, 0x3120u);
+          r3 = prmt(r3, 0u, 0x3120u);
+          mma_16816<false>(o[2 * jj], e4m3x2_to_f16x2((uint16_t)r0), e4m3x2_to_f16x2((uint16_t)r1),
+                           e4m3x2_to_f16x2((uint16_t)r2), e4m3x2_to_f16x2((uint16_t)r3), bh0, bh1);
+          mma_16816<false>(o[2 * jj + 1], e4m3x2_to_f16x2((uint16_t)(r0 >> 16)),
+                           e4m3x2_to_f16x2((uint16_t)(r1 >> 16)), e4m3x2_to_f16x2((uint16_t)(r2 >> 16)),
+                           e4m3x2_to_f16x2((uint16_t)(r3 >> 16)), bh0, bh1);
+        }
+      } else {
         const int tok = ((mi >> 1) << 3) + r8;
         const uint32_t rowb = vb + (uint32_t)tok * 128u;
 #pragma unroll
@@ -605,10 +727,13 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       }
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        scr.o[warp][2 * cq][mt * 16 + g] = o[mt][0];
-        scr.o[warp][2 * cq + 1][mt * 16 + g] = o[mt][1];
-        scr.o[warp][2 * cq][mt * 16 + g + 8] = o[mt][2];
-        scr.o[warp][2 * cq + 1][mt * 16 + g + 8] = o[mt][3];
+        // dims of accumulator rows g and g+8 (see the PV MMA of each KV type)
+        const int d0 = FP8 ? 32 * (mt >> 1) + 2 * g + (mt & 1) : mt * 16 + g;
+        const int d1 = FP8 ? d0 + 16 : d0 + 8;
+        scr.o[warp][2 * cq][d0] = o[mt][0];
+        scr.o[warp][2 * cq + 1][d0] = o[mt][1];
+        scr.o[warp][2 * cq][d1] = o[mt][2];
+        scr.o[warp][2 * cq + 1][d1] = o[mt][3];
       }
       if (!cons_sync(ctl, cons_phase, a.err)) {
         clean = false;
@@ -627,7 +752,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           L += wt * scr.l[w][h];
           acc += wt * scr.o[w][h][d];
         }
-        const float val = acc / L;
+        const float val = FP8 ? acc * a.v_scale / L : acc / L;
         if (direct) {
           const size_t hq = (size_t)rec.kvh * G + h;
           store_out1<BF16>(a, rec.b, hq, d, val);
@@ -706,19 +831,21 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 
 size_t decode_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int grid,
-                          cudaStream_t stream) {
+cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, bool fp8,
+                          int grid, cudaStream_t stream) {
   static_assert(sizeof(Ctl) % 16 == 0, "Ctl must keep Scratch 16-byte aligned");
-  auto kern = bf16 ? decode_kernel<true> : decode_kernel<false>;
+  const int variant = (fp8 ? 2 : 0) + (bf16 ? 1 : 0);
+  auto kern = fp8 ? (bf16 ? decode_kernel<true, true> : decode_kernel<false, true>)
+                  : (bf16 ? decode_kernel<true, false> : decode_kernel<false, false>);
   // the shared-memory opt-in is per function and device; do it once each
-  static bool attr_set[2][64] = {};
+  static bool attr_set[4][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !attr_set[bf16][dev]) {
+  if (dev >= 64 || !attr_set[variant][dev]) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set[bf16][dev] = true;
+    if (dev < 64) attr_set[variant][dev] = true;
   }
   // programmatic dependent launch: CTAs may become resident while the previous
   // kernel drains; the kernel waits for it before reading any input

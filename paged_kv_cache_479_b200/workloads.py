@@ -112,24 +112,29 @@ def unique_kv_tokens(w: Workload) -> int:
     return int(w.kv_lens.sum() - prefix * max(w.batch - 1, 0)) if prefix else int(w.kv_lens.sum())
 
 
-def decode_bytes(w: Workload) -> int:
+def decode_bytes(w: Workload, kv_elem_bytes: Optional[int] = None) -> int:
     """Algorithmic HBM bytes of one decode launch: unique K/V once, q in, out,
-    the page table, and the fp32 lse."""
-    kv = kv_cache_bytes(1, w.num_kv_heads, w.head_dim, unique_kv_tokens(w), w.elem_bytes)
+    the page table, and the fp32 lse.  kv_elem_bytes: bytes of a cached
+    element (1 for an E4M3 pool; default the workload's 16-bit type)."""
+    kvb = w.elem_bytes if kv_elem_bytes is None else kv_elem_bytes
+    kv = kv_cache_bytes(1, w.num_kv_heads, w.head_dim, unique_kv_tokens(w), kvb)
     qo = 2 * w.batch * w.num_qo_heads * w.head_dim * w.elem_bytes
     table = 4 * (w.batch + 1 + len(w.page_indices) + w.batch)
     lse = 4 * w.batch * w.num_qo_heads
     return kv + qo + table + lse
 
 
-def append_bytes(w: Workload) -> int:
-    """Algorithmic bytes of one append launch: new rows read, then written."""
-    rows = 2 * w.nnz_new * w.num_kv_heads * w.head_dim * w.elem_bytes
-    return 2 * rows + 4 * (w.batch + 1) if w.nnz_new else 0
+def append_bytes(w: Workload, kv_elem_bytes: Optional[int] = None) -> int:
+    """Algorithmic bytes of one append launch: new 16-bit rows read, then
+    written into the pool (kv_elem_bytes each)."""
+    kvb = w.elem_bytes if kv_elem_bytes is None else kv_elem_bytes
+    elems = 2 * w.nnz_new * w.num_kv_heads * w.head_dim
+    return elems * (w.elem_bytes + kvb) + 4 * (w.batch + 1) if w.nnz_new else 0
 
 
-def logical_kv_bytes(w: Workload) -> int:
-    return kv_cache_bytes(1, w.num_kv_heads, w.head_dim, int(w.kv_lens.sum()), w.elem_bytes)
+def logical_kv_bytes(w: Workload, kv_elem_bytes: Optional[int] = None) -> int:
+    kvb = w.elem_bytes if kv_elem_bytes is None else kv_elem_bytes
+    return kv_cache_bytes(1, w.num_kv_heads, w.head_dim, int(w.kv_lens.sum()), kvb)
 
 
 # --------------------------------------------------------------------------
@@ -299,6 +304,57 @@ def make_tensors(w: Workload, device="cpu"):
     k_new = torch.empty((w.nnz_new, w.num_kv_heads, w.head_dim), dtype=dt, device=device)
     v_new = torch.empty_like(k_new)
     _fill(pool, q, k_new, v_new, w, gen, device)
+    return q, pool, k_new, v_new
+
+
+# --------------------------------------------------------------------------
+# 8-bit (E4M3) pools
+# --------------------------------------------------------------------------
+
+FP8_CANARY = 0x7F  # an E4M3 NaN code: fills every slot that holds no token
+FP8_EXP_MEAN = 11  # exponent field of a typical code: magnitude 2^(11-7) = 16
+
+
+def e4m3_codes(shape, gen, device, exp_mean=FP8_EXP_MEAN, exp_std=1.25):
+    """Random E4M3 codes assembled field by field (no conversion arithmetic):
+    sign uniform, exponent field round(N(exp_mean, exp_std)) clipped to
+    [0, 15] (0 gives subnormals), fraction uniform; the NaN codes S.1111.111
+    are never drawn (they become S.1111.110 = +-448)."""
+    sign = torch.randint(0, 2, shape, generator=gen, device=device, dtype=torch.int32)
+    e = torch.randn(shape, generator=gen, device=device) * exp_std + exp_mean
+    e = e.round().clamp(0, 15).to(torch.int32)
+    m = torch.randint(0, 8, shape, generator=gen, device=device, dtype=torch.int32)
+    code = (sign << 7) | (e << 3) | m
+    code = torch.where((code & 0x7F) == 0x7F, code - 1, code)
+    return code.to(torch.uint8)
+
+
+def make_fp8_tensors(w: Workload, device="cpu"):
+    """q [B,Hq,D] and new rows [nnz,Hkv,D] in the workload's 16-bit dtype, and
+    an E4M3 pool [P,2,Hkv,ps,D] (uint8 codes; state before the append) whose
+    slots that hold no token carry FP8_CANARY."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(w.seed) + 8)
+    dt = w.torch_dtype
+    q = (torch.randn((w.batch, w.num_qo_heads, w.head_dim), generator=gen, device=device)
+         * w.q_std).to(dt)
+    pool = torch.empty(w.pool_shape, dtype=torch.uint8, device=device)
+    chunk = max(1, (1 << 26) // (2 * w.num_kv_heads * w.page_size * w.head_dim))
+    for p0 in range(0, w.num_pages, chunk):
+        p1 = min(w.num_pages, p0 + chunk)
+        pool[p0:p1] = e4m3_codes((p1 - p0,) + tuple(w.pool_shape[1:]), gen, device)
+    k_new = torch.randn((w.nnz_new, w.num_kv_heads, w.head_dim), generator=gen,
+                        device=device).to(dt)
+    v_new = torch.randn((w.nnz_new, w.num_kv_heads, w.head_dim), generator=gen,
+                        device=device).to(dt)
+    unused, pairs = _canary_mask_slots(w)
+    if len(unused):
+        pool[torch.as_tensor(unused, device=device)] = FP8_CANARY
+    if len(pairs):
+        pg = torch.as_tensor(pairs[:, 0], device=device)
+        sl = torch.as_tensor(pairs[:, 1], device=device)
+        pool[pg, :, :, sl, :] = FP8_CANARY
     return q, pool, k_new, v_new
 
 

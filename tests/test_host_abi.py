@@ -223,3 +223,33 @@ def test_descriptor_calls_reject_bad_arguments():
     assert L.pkv_decode_ex(*args(hd64, csr)) == 2
     assert L.pkv_append_ex(None, ctypes.byref(csr), p, p, p, 3, None, None) == 1
     assert L.pkv_append_ex(ctypes.byref(bad_layout), ctypes.byref(csr), p, p, p, 3, None, None) == 1
+
+
+def test_fp8_calls_reject_bad_arguments():
+    L = pkv.lib()
+    p = ctypes.c_void_p(4096)
+    fp8 = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.FP8_E4M3, 0, 0)
+    bf16 = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.BF16, 0, 0)
+    csr = pkv.TableDesc(0, 4, 4096, 4096, 4096, None, None, 0, 0)
+
+    def dec(pool, q_dtype=pkv.BF16, ks=0.5, vs=0.5):
+        return L.pkv_decode_fp8(p, q_dtype, 8, ctypes.byref(pool), ks, vs, ctypes.byref(csr), 0.1,
+                                8, p, 1 << 30, ctypes.c_void_p(8192), None, None, None)
+
+    def app(pool, new_dtype=pkv.BF16, ks=0.5, vs=0.5):
+        return L.pkv_append_fp8(ctypes.byref(pool), ks, vs, ctypes.byref(csr), p, p, new_dtype, p,
+                                3, None, None)
+
+    for ks, vs in ((0.0, 1.0), (1.0, -1.0), (float("inf"), 1.0), (1.0, float("nan"))):
+        assert dec(fp8, ks=ks, vs=vs) == 1
+        assert app(fp8, ks=ks, vs=vs) == 1
+    assert dec(bf16) == 1                       # the fp8 calls need an E4M3 pool
+    assert app(bf16) == 1
+    assert dec(fp8, q_dtype=pkv.F32) == 1       # q is fp16 or bf16
+    assert dec(fp8, q_dtype=pkv.FP8_E4M3) == 1
+    assert app(fp8, new_dtype=pkv.FP8_E4M3) == 1
+    # the descriptor calls without scales refuse an E4M3 pool
+    assert L.pkv_decode_ex(p, 8, ctypes.byref(fp8), ctypes.byref(csr), 0.1, 8, p, 1 << 30,
+                           ctypes.c_void_p(8192), None, None, None) == 1
+    assert L.pkv_append_ex(ctypes.byref(fp8), ctypes.byref(csr), p, p, p, 3, None, None) == 1
+    assert b"pkv_append_fp8" in L.pkv_last_error()
