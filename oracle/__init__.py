@@ -53,6 +53,9 @@ def _load():
         lib.oracle_append_fp8.argtypes = [p, f32, f32, i64, i32, i32, i32, i32, p, p, p,
                                           p, p, i32, p]
         lib.oracle_append_fp8.restype = i32
+        lib.oracle_append_attention.argtypes = [p, p, i32, i64, i32, i32, i32, i32, i32,
+                                                p, p, p, p, i32, i32, dbl, p, p]
+        lib.oracle_append_attention.restype = i32
         lib.oracle_e4m3_decode.argtypes = [p, i64, p]
         lib.oracle_e4m3_decode.restype = i32
         lib.oracle_e4m3_encode.argtypes = [p, i64, f32, p]
@@ -220,3 +223,37 @@ def append_fp8(pool_codes, k_scale, v_scale, page_indptr, page_indices, last_pag
     if rc != 0:
         raise OracleError(f"oracle_append_fp8: {_STATUS.get(rc, rc)}")
     return pool
+
+
+def append_attention(q_bits, pool_bits, dtype, page_indptr, page_indices, last_page_len,
+                     qo_indptr, scale, window_left=-1, sink_tokens=0):
+    """Exact attention of each request's chunk of new query tokens over its cache.
+
+    q_bits    uint16 [nnz_q, Hq, D]; request b's tokens are rows qo_indptr[b]:qo_indptr[b+1]
+    pool_bits uint16 [P, 2, Hkv, ps, D]; the table is the table after the append
+    Query i of request b sits at position L_b - q_len_b + i and sees keys t <= pos
+    (and, with window_left >= 0, t >= pos - window_left unless t < sink_tokens).
+    Returns (out float64 [nnz_q, Hq, D], lse float64 [nnz_q, Hq]).
+    """
+    q_bits, qp = _c(q_bits, np.uint16)
+    pool_bits, pp = _c(pool_bits, np.uint16)
+    P, _, hkv, ps, d = pool_bits.shape
+    nnz, hq, dq = q_bits.shape
+    if dq != d:
+        raise ValueError("q head_dim does not match pool head_dim")
+    B = len(page_indptr) - 1
+    indptr, ip = _c(page_indptr, np.int32)
+    indices, xp = _c(page_indices if len(page_indices) else np.zeros(1, np.int32), np.int32)
+    last, lp = _c(last_page_len if len(last_page_len) else np.zeros(1, np.int32), np.int32)
+    qo, qop = _c(qo_indptr, np.int32)
+    if len(qo) != B + 1 or (B and qo[-1] != nnz):
+        raise ValueError("qo_indptr must have batch + 1 entries ending at nnz_q")
+    out = np.zeros((nnz, hq, d), np.float64)
+    lse = np.zeros((nnz, hq), np.float64)
+    rc = _load().oracle_append_attention(qp, pp, int(dtype), P, ps, hkv, d, B, hq, ip, xp, lp,
+                                         qop, int(window_left), int(sink_tokens), float(scale),
+                                         out.ctypes.data_as(ctypes.c_void_p),
+                                         lse.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise OracleError(f"oracle_append_attention: {_STATUS.get(rc, rc)}")
+    return out, lse

@@ -421,6 +421,121 @@ int oracle_append_fp8(uint8_t* pool, float k_scale, float v_scale, int64_t num_p
 }
 
 /*
+ * Visibility of key position t to a query at position pos in a chunk of new
+ * tokens: causal (t <= pos: the cache holds nothing later), and with a
+ * window (window_left >= 0) also within window_left positions before the
+ * query, or when the key is one of the first sink_tokens positions.  This is
+ * the window-plus-global-tokens mask of "大模型长上下文窗口工程化实战：从RoPE扩展到
+ * 百万Token推理的生产级部署" section 2.3 (half-width window_size / 2 on each
+ * side, global tokens seeing and seen by everything) with its right half cut
+ * off by causality; its rule that global queries see every key adds nothing
+ * then, since every key such a query may see is itself a global token.
+ */
+static int key_visible(int64_t t, int64_t pos, int window_left, int sink_tokens) {
+  if (t > pos) return 0;
+  if (window_left < 0) return 1;
+  return t >= pos - window_left || t < sink_tokens;
+}
+
+/*
+ * oracle_append_attention -- exact attention of a chunk of new query tokens
+ * per request over the paged cache (chunked prefill: a prompt processed a
+ * chunk at a time against the cache that already holds the earlier chunks,
+ * "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署" section 3.1;
+ * also several speculative tokens verified at once).
+ *
+ * q         [nnz_q][num_qo_heads][head_dim] 16-bit; request b's query tokens
+ *           are rows qo_indptr[b] .. qo_indptr[b+1]-1 (qo_indptr[0] = 0,
+ *           nnz_q = qo_indptr[batch])
+ * table     the table after the chunk's K/V were appended: request b holds
+ *           L_b tokens and its q_len_b = qo_indptr[b+1] - qo_indptr[b] query
+ *           tokens are the last q_len_b of them, so query i is at position
+ *           pos = L_b - q_len_b + i
+ * out, lse  [nnz_q][num_qo_heads][head_dim] and [nnz_q][num_qo_heads]
+ *
+ * For each (query row, head h): the single-row attention of the decode over
+ * the keys t with key_visible(t, pos); GQA as in the decode.  Every query
+ * sees at least its own key.
+ */
+int oracle_append_attention(const uint16_t* q, const uint16_t* pool, int dtype,
+                            int64_t num_pages, int page_size, int num_kv_heads, int head_dim,
+                            int batch, int num_qo_heads,
+                            const int32_t* page_indptr, const int32_t* page_indices,
+                            const int32_t* last_page_len, const int32_t* qo_indptr,
+                            int window_left, int sink_tokens, double scale,
+                            double* out, double* lse) {
+  if (batch < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1 ||
+      num_qo_heads < num_kv_heads || num_qo_heads % num_kv_heads != 0 || sink_tokens < 0 ||
+      (dtype != ORACLE_F16 && dtype != ORACLE_BF16))
+    return ORACLE_BAD_ARG;
+  int rc = check_table(num_pages, page_size, batch, page_indptr, page_indices, last_page_len);
+  if (rc != ORACLE_OK) return rc;
+  if (batch > 0 && qo_indptr[0] != 0) return ORACLE_BAD_APPEND;
+  for (int b = 0; b < batch; ++b) {
+    int why = ORACLE_OK;
+    const int64_t len = request_len(b, page_size, page_indptr, last_page_len, &why);
+    const int64_t n_q = (int64_t)qo_indptr[b + 1] - qo_indptr[b];
+    if (n_q < 0 || n_q > len) return ORACLE_BAD_APPEND;
+  }
+  const int64_t nnz = batch > 0 ? (int64_t)qo_indptr[batch] : 0;
+  /* request of every query row */
+  int* req = (int*)malloc(sizeof(int) * (size_t)(nnz > 0 ? nnz : 1));
+  if (!req) return ORACLE_NO_MEMORY;
+  for (int b = 0; b < batch; ++b)
+    for (int64_t r = qo_indptr[b]; r < qo_indptr[b + 1]; ++r) req[r] = b;
+  const int group = num_qo_heads / num_kv_heads;
+  int failed = 0;
+
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t row = 0; row < nnz * num_qo_heads; ++row) {
+    const int64_t r = row / num_qo_heads;    /* query token */
+    const int h = (int)(row % num_qo_heads);
+    const int b = req[r];
+    const int kvh = h / group;
+    int why = ORACLE_OK;
+    const int64_t len = request_len(b, page_size, page_indptr, last_page_len, &why);
+    const int64_t n_q = (int64_t)qo_indptr[b + 1] - qo_indptr[b];
+    const int64_t pos = len - n_q + (r - qo_indptr[b]);
+    double* o = out + (size_t)row * head_dim;
+    double* qd = (double*)malloc(sizeof(double) * (size_t)head_dim);
+    double* s = (double*)malloc(sizeof(double) * (size_t)(pos + 1));
+    if (!qd || !s) {
+      free(qd); free(s);
+#pragma omp atomic write
+      failed = 1;
+      continue;
+    }
+    for (int d = 0; d < head_dim; ++d) qd[d] = widen(q[(size_t)row * head_dim + d], dtype);
+    double m = -INFINITY;
+    for (int64_t t = 0; t <= pos; ++t) {
+      if (!key_visible(t, pos, window_left, sink_tokens)) { s[t] = -INFINITY; continue; }
+      const int64_t page = page_indices[page_indptr[b] + t / page_size];
+      const size_t kk = pool_offset(page, 0, kvh, t % page_size, num_kv_heads, page_size, head_dim);
+      double dot = 0.0;
+      for (int d = 0; d < head_dim; ++d) dot += qd[d] * widen(pool[kk + d], dtype);
+      s[t] = dot * scale;
+      if (s[t] > m) m = s[t];
+    }
+    double l = 0.0;
+    for (int d = 0; d < head_dim; ++d) o[d] = 0.0;
+    for (int64_t t = 0; t <= pos; ++t) {
+      if (s[t] == -INFINITY) continue;          /* invisible: weight exactly 0 */
+      const double wt = exp(s[t] - m);
+      const int64_t page = page_indices[page_indptr[b] + t / page_size];
+      const size_t vv = pool_offset(page, 1, kvh, t % page_size, num_kv_heads, page_size, head_dim);
+      l += wt;
+      for (int d = 0; d < head_dim; ++d) o[d] += wt * widen(pool[vv + d], dtype);
+    }
+    for (int d = 0; d < head_dim; ++d) o[d] /= l;
+    lse[row] = log(l) + m;
+    free(qd);
+    free(s);
+  }
+  free(req);
+  return failed ? ORACLE_NO_MEMORY : ORACLE_OK;
+}
+
+/*
  * oracle_merge -- combine S attention states per (row, head).
  *
  * v [rows][S][H][D] are normalised partial outputs, s [rows][S][H] their

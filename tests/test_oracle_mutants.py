@@ -12,6 +12,7 @@ import subprocess
 import pytest
 
 import oracle
+import test_oracle_append_attn as aapins
 import test_oracle_fp8 as fp8pins
 import test_oracle_pins as pins
 
@@ -44,6 +45,13 @@ MUTANTS = {
                             "(kv_elem(pool, kv_dtype, v + d))"),
     "fp8_append_v_takes_k_scale": ("encode_e4m3((float)widen(vs[d], new_dtype), v_scale)",
                                    "encode_e4m3((float)widen(vs[d], new_dtype), k_scale)"),
+    "chunk_not_causal_on_self": ("if (t > pos) return 0;", "if (t >= pos && pos > 0) return 0;"),
+    "chunk_window_one_short": ("return t >= pos - window_left ||", "return t > pos - window_left ||"),
+    "chunk_head_mapping": ("const int kvh = h / group;", "const int kvh = h % num_kv_heads;"),
+    "chunk_sink_ignored": ("return t >= pos - window_left || t < sink_tokens;",
+                           "return t >= pos - window_left;"),
+    "chunk_positions_from_zero": ("const int64_t pos = len - n_q + (r - qo_indptr[b]);",
+                                  "const int64_t pos = len - n_q + (r - qo_indptr[b]) - 1 + (n_q == 1);"),
 }
 
 PINS = [
@@ -66,6 +74,10 @@ PINS = [
     lambda: [fp8pins.test_fp8_decode_matches_dense_sdpa_on_dequantised_values(c)
              for c in range(len(fp8pins.FP8_CASES))],
     fp8pins.test_fp8_append_positions_and_codes,
+    lambda: [aapins.test_append_attention_matches_masked_sdpa(c) for c in range(len(aapins.CASES))],
+    aapins.test_single_token_chunks_are_the_decode,
+    aapins.test_chunking_invariance,
+    aapins.test_hand_derived_identical_keys_and_windows,
 ]
 
 
@@ -83,7 +95,7 @@ def test_pins_catch_mutant(name, tmp_path, monkeypatch):
     lib = ctypes.CDLL(str(so))
     for fn in ("oracle_decode", "oracle_append", "oracle_merge", "oracle_num_threads",
                "oracle_decode_fp8", "oracle_append_fp8", "oracle_e4m3_decode",
-               "oracle_e4m3_encode"):
+               "oracle_e4m3_encode", "oracle_append_attention"):
         getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         getattr(lib, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", lib)
