@@ -59,6 +59,9 @@ def parse():
     p.add_argument("--kv", choices=["16bit", "fp8"], default="16bit",
                    help="KV pool type: the workload's 16-bit type, or FP8 E4M3 codes with "
                         "per-tensor K/V scales (q and out stay 16-bit)")
+    p.add_argument("--chunk", choices=["prefill", "spec"], default=None,
+                   help="time multi-token append attention instead of the decode: chunked "
+                        "prefill (TFLOP/s) or speculative verification (GB/s)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for cpu_baseline")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="oracle time budget of the reference arm")
     return p.parse_args()
@@ -89,6 +92,16 @@ def max_over_ranks(x, world, device):
 def job_throughput(bytes_per_step_per_rank, world, ms_total, steps):
     """Whole-job GB/s: every rank's bytes over the slowest rank's time."""
     return bytes_per_step_per_rank * world / (ms_total / 1e3 / steps) / 1e9
+
+
+def measured_tensor():
+    """Measured bf16 dense GEMM throughput (burst, TFLOP/s)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def measured_hbm():
@@ -564,8 +577,139 @@ def run_pkv(args):
         torch.distributed.destroy_process_group()
 
 
+def run_chunk(args):
+    """Append K/V of every request's chunk, then the chunk's causal attention."""
+    import paged_kv_cache_479_b200 as pkv
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                             device_id=dev)
+    w, q_lens = wl.named_chunk(args.chunk)
+    qo = wl.chunk_indptr(q_lens)
+    rotation = 2
+    batches = []
+    for r in range(rotation):
+        wv = wl.Workload(**{**w.__dict__, "seed": rank_value_seed(w.seed, rank, r)})
+        _, pool, k_new, v_new = wl.make_tensors(wv, dev)
+        batches.append((wl.make_chunk_queries(wv, q_lens, dev), pool, k_new, v_new))
+    t = lambda a: torch.as_tensor(np.ascontiguousarray(a, np.int32), device=dev)
+    indptr, indices, last = t(w.page_indptr), t(w.page_indices), t(w.last_page_len)
+    app, qo_d = t(w.append_indptr), t(qo)
+    table = pkv.csr_table(indptr, indices, last)
+    plan_h, S = pkv.append_attention_plan(qo, w.kv_lens, w.num_qo_heads, w.num_kv_heads)
+    plan = t(plan_h)
+    need = pkv.append_attention_workspace_bytes(int(qo[-1]), w.num_qo_heads, S)
+    ws = torch.zeros(need // 4 + 64, dtype=torch.int32, device=dev)
+    out = torch.empty_like(batches[0][0])
+    lse = torch.empty(out.shape[:2], dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def append_call(bt):
+        pkv.paged_kv_append(bt[1], indptr, indices, last, bt[2], bt[3], app, error_word=err,
+                            stream=torch.cuda.current_stream(dev))
+
+    def attn_call(bt):
+        pkv.append_attention(bt[0], qo_d, bt[1], table, plan, S, workspace=ws, out=out, lse=lse,
+                             sm_scale=w.sm_scale, error_word=err,
+                             stream=torch.cuda.current_stream(dev))
+
+    def graphed(fn, bt):
+        if args.no_graph:
+            return lambda: fn(bt)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(bt)
+        return g.replay
+    for i in range(args.warmup):
+        append_call(batches[i % rotation])
+        attn_call(batches[i % rotation])
+    torch.cuda.synchronize()
+    if pkv.read_error_word(err) != 0:
+        raise RuntimeError("device error bits set during warm-up")
+    app_g = [graphed(append_call, bt) for bt in batches]
+    att_g = [graphed(attn_call, bt) for bt in batches]
+    clocks = ClockSampler(local)
+    K = args.steps
+    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_host0 = time.time()
+    start.record(stream)
+    for i in range(K):
+        app_g[i % rotation]()
+        d0[i].record(stream)
+        att_g[i % rotation]()
+        d1[i].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    attn_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K, world, dev)
+    if pkv.read_error_word(err) != 0:
+        raise RuntimeError("device error bits set during the timed steps")
+    flops = wl.chunk_flops(w, q_lens)
+    nnz = int(qo[-1])
+    kv = wl.kv_cache_bytes(1, w.num_kv_heads, w.head_dim, int(w.kv_lens.sum()))
+    attn_bytes = kv + 2 * nnz * w.num_qo_heads * w.head_dim * 2 + 4 * nnz * w.num_qo_heads
+    step_bytes = attn_bytes + wl.append_bytes(w)
+    if args.chunk == "prefill":
+        peak, kind = measured_tensor()
+        achieved = flops / (attn_ms / 1e3) / 1e12
+        value = flops * world * K / (ms / 1e3) / 1e12
+        metric, unit, bound, runit = ("append attention, chunked prefill: causal attention TFLOP/s",
+                                      "TFLOP/s", "tensor", "TFLOP/s")
+    else:
+        peak, kind = measured_hbm()
+        achieved = attn_bytes / (attn_ms / 1e3) / 1e9
+        value = job_throughput(step_bytes, world, ms, K)
+        metric, unit, bound, runit = ("append attention, speculative verification: KV HBM GB/s",
+                                      "GB/s", "hbm", "GB/s")
+    if rank == 0:
+        line = {
+            "metric": metric, "value": round(value, 2), "unit": unit, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "query_tokens": nnz,
+                       "kv_tokens_after_append": int(w.kv_lens.sum()), "splits": S,
+                       "row_blocks": int(plan_h.shape[0]), "flops_per_step": flops,
+                       "attention_bytes_per_step": attn_bytes,
+                       "l2": f"2 rotating batch copies of {kv / 1e6:.0f} MB K/V",
+                       "launch": "append and append attention captured as CUDA graphs",
+                       "parallelism": f"dp{world} (independent batches per GPU)"},
+            "us_per_step": round(ms / K * 1e3, 2),
+            "tokens_per_s": round(nnz * world / (ms / K / 1e3), 1),
+            "roofline": {"bound": bound, "kernel": "chunk_kernel" + (" + merge" if S > 1 else ""),
+                         "achieved": round(achieved, 1), "peak": peak, "unit": runit,
+                         "frac": round(achieved / peak, 4),
+                         "peak_kind": f"{kind} (MEASURED_PEAKS.json "
+                                      f"{'bf16_tflops, burst' if bound == 'tensor' else 'hbm_gbs'})",
+                         "traffic": None, "avg_launch_us": round(attn_ms * 1e3, 2)},
+            "gpu_launches": K * (2 + (1 if S > 1 else 0)),
+            "e2e": None,
+            "clocks": clocks.summary(t_host0, t_host1),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     args = parse()
+    if args.chunk and args.impl != "reference":
+        run_chunk(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

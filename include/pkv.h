@@ -260,6 +260,63 @@ PKV_API pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, floa
                                   int32_t* error_word, void* stream);
 
 /*
+ * Multi-token append attention: each request's chunk of new query tokens
+ * attends over its paged cache with a causal mask -- chunked prefill (a long
+ * prompt processed a chunk at a time against the cache that holds the earlier
+ * chunks, "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署"
+ * section 3.1) and the verification of several speculative tokens at once.
+ *
+ * Request b's q_len_b = qo_indptr[b+1] - qo_indptr[b] query tokens are rows
+ * qo_indptr[b] .. of q (qo_indptr[0] = 0, nnz_q = qo_indptr[batch]).  The
+ * table is the table AFTER the chunk's K/V were appended (pkv_append*): the
+ * request holds L_b >= q_len_b tokens and query i sits at position
+ * pos = L_b - q_len_b + i.  Key t is visible to it when t <= pos and, if
+ * window_left >= 0, also t >= pos - window_left or t < sink_tokens (the
+ * sliding window with global tokens of the same article's section 2.3, cut
+ * to its causal half; window_left < 0 = no window).  Query head h reads KV
+ * head h / (Hq / Hkv); out / lse as in pkv_decode, per query token.
+ *
+ * pkv_append_attention_plan (host only) -- the row blocks of the launch:
+ *   qo_indptr_h  host int32 [batch+1]
+ *   kv_len_h     host int32 [batch]: L_b (tokens after the append), or NULL
+ *   plan_h       host int32 [capacity][4] or NULL: {request, first row, rows, 0}
+ *                per block of up to 128 rows (row r = chunk token r / G, query
+ *                head kv_head * G + r % G)
+ *   num_splits   if not NULL, receives a split count for the launch: 1 when
+ *                the row blocks fill num_sms SMs (or kv_len_h is NULL), else
+ *                enough key splits for about two CTAs per SM
+ *   returns the number of row blocks (entries beyond capacity are not
+ *   written), or -1 for invalid arguments.
+ *
+ * pkv_append_attention_workspace_bytes -- fp32 partial states needed with
+ *   num_splits > 1 (0 with one split).
+ *
+ * pkv_append_attention -- the launch:
+ *   q             [nnz_q][num_qo_heads][128], the pool's dtype, 16-byte aligned
+ *   qo_indptr     device int32 [batch+1]
+ *   pool, table   descriptors (16-bit pools, either layout, either table form)
+ *   plan          device int32 [num_row_blocks][4] from the planner, 16-byte aligned
+ *   num_splits    1..1024; the same value the workspace was sized for
+ *   workspace     device, 256-byte aligned (may be NULL with one split)
+ *   out           [nnz_q][num_qo_heads][128] pool dtype;  lse float [nnz_q][Hq] or NULL
+ * Errors as in pkv_decode; a plan entry or request that does not fit the table
+ * sets PKV_DEVERR_APPEND (or the table's bit) and leaves its rows unwritten.
+ */
+PKV_API int64_t pkv_append_attention_plan(const int32_t* qo_indptr_h, const int32_t* kv_len_h,
+                                          int batch, int num_qo_heads, int num_kv_heads,
+                                          int window_left, int sink_tokens, int num_sms,
+                                          int32_t* plan_h, int64_t capacity, int32_t* num_splits);
+PKV_API size_t pkv_append_attention_workspace_bytes(int64_t nnz_q, int num_qo_heads,
+                                                    int num_splits);
+PKV_API pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr, int64_t nnz_q,
+                                        int num_qo_heads, const pkv_pool_desc* pool,
+                                        const pkv_table_desc* table, const int32_t* plan,
+                                        int64_t num_row_blocks, int num_splits, int window_left,
+                                        int sink_tokens, float sm_scale, void* workspace,
+                                        size_t workspace_bytes, void* out, float* lse,
+                                        int32_t* error_word, void* stream);
+
+/*
  * pkv_cascade_decode -- pkv_decode for a batch whose requests all begin with
  * the same shared prefix (a system prompt stored once in shared pages: physical
  * page sharing between requests with a common prefix, "大模型推理极致优化：

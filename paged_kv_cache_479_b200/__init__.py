@@ -21,9 +21,15 @@ Functions (C names in parentheses):
                          NHD pools and dense (vLLM-style) block tables
   paged_decode_attention_fp8 / paged_kv_append_fp8 (pkv_decode_fp8 / pkv_append_fp8)
                          the 8-bit (FP8 E4M3) KV cache with per-tensor K / V scales
+  append_attention       (pkv_append_attention)  a chunk of query tokens per request,
+                         causal over its cache (chunked prefill, speculative tokens)
+  append_attention_plan  (pkv_append_attention_plan)  its host-side row-block plan
 """
 from ._binding import (  # noqa: F401
     BF16,
+    append_attention,
+    append_attention_plan,
+    append_attention_workspace_bytes,
     F16,
     F32,
     FP8_E4M3,
@@ -69,4 +75,5 @@ pkv_cascade_decode = cascade_decode
 pkv_decode_ex = paged_decode_attention_ex
 pkv_append_ex = paged_kv_append_ex
 pkv_decode_fp8 = paged_decode_attention_fp8
+pkv_append_attention = append_attention
 pkv_append_fp8 = paged_kv_append_fp8

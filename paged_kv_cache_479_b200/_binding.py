@@ -70,6 +70,11 @@ _SIGNATURES["pkv_append_ex"] = ([_PP, _TP, _P, _P, _P, _I64, _P, _P], _I32)
 _SIGNATURES["pkv_decode_fp8"] = (
     [_P, _I32, _I32, _PP, _F32, _F32, _TP, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["pkv_append_fp8"] = ([_PP, _F32, _F32, _TP, _P, _P, _I32, _P, _I64, _P, _P], _I32)
+_SIGNATURES["pkv_append_attention_plan"] = (
+    [_P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _I64, _P], _I64)
+_SIGNATURES["pkv_append_attention_workspace_bytes"] = ([_I64, _I32, _I32], _SZ)
+_SIGNATURES["pkv_append_attention"] = (
+    [_P, _P, _I64, _I32, _PP, _TP, _P, _I64, _I32, _I32, _I32, _F32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
 _SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
 _SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
@@ -277,8 +282,10 @@ def csr_table(page_indptr, page_indices, last_page_len) -> TableDesc:
     for name, t in (("page_indptr", page_indptr), ("page_indices", page_indices),
                     ("last_page_len", last_page_len)):
         _dev_tensor(t, name, torch.int32)
-    return TableDesc(TABLE_CSR, last_page_len.numel(), page_indptr.data_ptr(),
-                     page_indices.data_ptr(), last_page_len.data_ptr(), None, None, 0, 0)
+    t = TableDesc(TABLE_CSR, last_page_len.numel(), page_indptr.data_ptr(),
+                  page_indices.data_ptr(), last_page_len.data_ptr(), None, None, 0, 0)
+    t._keep = (page_indptr, page_indices, last_page_len)  # the descriptor holds raw pointers
+    return t
 
 
 def block_table(table, context_lens) -> TableDesc:
@@ -287,8 +294,10 @@ def block_table(table, context_lens) -> TableDesc:
     _dev_tensor(context_lens, "context_lens", torch.int32)
     if table.dim() != 2 or table.shape[0] != context_lens.numel():
         raise ValueError("block_table must be [batch, max_blocks_per_seq]")
-    return TableDesc(TABLE_BLOCK, table.shape[0], None, None, None, table.data_ptr(),
-                     context_lens.data_ptr(), table.shape[1], 0)
+    t = TableDesc(TABLE_BLOCK, table.shape[0], None, None, None, table.data_ptr(),
+                  context_lens.data_ptr(), table.shape[1], 0)
+    t._keep = (table, context_lens)
+    return t
 
 
 def paged_decode_attention_ex(q, pool, table: TableDesc, workspace, layout: str = "HND",
@@ -371,6 +380,62 @@ def paged_kv_append_fp8(pool, table: TableDesc, k_new, v_new, append_indptr, k_s
                               _ptr(append_indptr), k_new.shape[0], _ptr(error_word),
                               _stream(stream, pool.device))
     _check(st, "pkv_append_fp8")
+
+
+def append_attention_plan(qo_indptr_h, kv_len_h, num_qo_heads: int, num_kv_heads: int,
+                          window_left: int = -1, sink_tokens: int = 0, num_sms: int = 0):
+    """pkv_append_attention_plan on host arrays: (plan int32 [n, 4], suggested splits)."""
+    qo = np.ascontiguousarray(qo_indptr_h, np.int32)
+    kl = None if kv_len_h is None else np.ascontiguousarray(kv_len_h, np.int32)
+    B = len(qo) - 1
+    if num_sms == 0 and torch.cuda.is_available():
+        num_sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    splits = ctypes.c_int32(1)
+    kp = None if kl is None else kl.ctypes.data_as(_P)
+    n = lib().pkv_append_attention_plan(qo.ctypes.data_as(_P), kp, B, num_qo_heads, num_kv_heads,
+                                        window_left, sink_tokens, num_sms, None, 0, None)
+    if n < 0:
+        raise ValueError("pkv_append_attention_plan rejected the arguments")
+    plan = np.zeros((max(n, 1), 4), np.int32)
+    n2 = lib().pkv_append_attention_plan(qo.ctypes.data_as(_P), kp, B, num_qo_heads, num_kv_heads,
+                                         window_left, sink_tokens, num_sms,
+                                         plan.ctypes.data_as(_P), n, ctypes.byref(splits))
+    assert n2 == n
+    return plan[:n], int(splits.value)
+
+
+def append_attention_workspace_bytes(nnz_q: int, num_qo_heads: int, num_splits: int) -> int:
+    return int(lib().pkv_append_attention_workspace_bytes(nnz_q, num_qo_heads, num_splits))
+
+
+def append_attention(q, qo_indptr, pool, table: TableDesc, plan, num_splits: int = 1,
+                     layout: str = "HND", window_left: int = -1, sink_tokens: int = 0,
+                     workspace=None, out=None, lse=None, sm_scale=None, error_word=None,
+                     stream=None, return_lse: bool = True):
+    """pkv_append_attention: every request's chunk of query tokens (rows of q,
+    split by the device int32 qo_indptr) over its cache, causal, optional window.
+    plan: device int32 [n, 4] from append_attention_plan."""
+    _dev_tensor(q, "q", pool.dtype)
+    _dev_tensor(qo_indptr, "qo_indptr", torch.int32)
+    _dev_tensor(plan, "plan", torch.int32)
+    pd = pool_desc(pool, layout)
+    nnz, hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((nnz, hq), dtype=torch.float32, device=q.device)
+    need = append_attention_workspace_bytes(nnz, hq, num_splits)
+    if workspace is None and need:
+        workspace = torch.empty(need // 4 + 64, dtype=torch.int32, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_append_attention(_ptr(q), _ptr(qo_indptr), nnz, hq, ctypes.byref(pd),
+                                    ctypes.byref(table), _ptr(plan), plan.shape[0], num_splits,
+                                    window_left, sink_tokens, scale, _ptr(workspace), ws_bytes,
+                                    _ptr(out), _ptr(lse), _ptr(error_word),
+                                    _stream(stream, q.device))
+    _check(st, "pkv_append_attention")
+    return out, lse
 
 
 def merge_states(v, s, out_dtype=torch.float32, v_out=None, s_out=None, stream=None,

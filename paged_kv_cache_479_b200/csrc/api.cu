@@ -731,6 +731,167 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
   return ok();
 }
 
+// ------------------------------------------------------------ append attention
+
+int64_t pkv_append_attention_plan(const int32_t* qo_indptr_h, const int32_t* kv_len_h, int batch,
+                                  int num_qo_heads, int num_kv_heads, int window_left,
+                                  int sink_tokens, int num_sms, int32_t* plan_h,
+                                  int64_t capacity, int32_t* num_splits) {
+  if (batch < 0 || num_kv_heads < 1 || num_qo_heads < num_kv_heads ||
+      num_qo_heads % num_kv_heads != 0 || sink_tokens < 0 || (batch > 0 && !qo_indptr_h) ||
+      capacity < 0 || (batch > 0 && qo_indptr_h[0] != 0))
+    return -1;
+  const int G = num_qo_heads / num_kv_heads;
+  const int R = pkv::chunk_rows_per_cta(), T = pkv::chunk_tile_tokens();
+  int64_t count = 0, ctas = 0;
+  long long max_tiles = 0;
+  for (int b = 0; b < batch; ++b) {
+    const long long q_len = (long long)qo_indptr_h[b + 1] - qo_indptr_h[b];
+    if (q_len < 0) return -1;
+    const long long rows = q_len * G;
+    const long long L = kv_len_h ? kv_len_h[b] : q_len;
+    if (kv_len_h && (L < q_len)) return -1;
+    for (long long r0 = 0; r0 < rows; r0 += R) {
+      const long long n = rows - r0 < R ? rows - r0 : R;
+      if (r0 > 0x7fffffffLL) return -1;
+      if (plan_h && count < capacity) {
+        int32_t* e = plan_h + 4 * count;
+        e[0] = b;
+        e[1] = (int32_t)r0;
+        e[2] = (int32_t)n;
+        e[3] = 0;
+      }
+      ++count;
+      // the kernel's key range for this row block, in tiles (host mirror)
+      const long long base = L - q_len, pf = base + r0 / G, pl = base + (r0 + n - 1) / G;
+      long long lo = window_left >= 0 ? pf - window_left : 0;
+      lo = lo < 0 ? 0 : lo;
+      const long long lo16 = lo & ~15LL;
+      const long long a_end = window_left >= 0 ? (sink_tokens < lo16 ? sink_tokens : lo16) : 0;
+      const long long tiles = (a_end + T - 1) / T + (pl + 1 - lo16 + T - 1) / T;
+      if (tiles > max_tiles) max_tiles = tiles;
+    }
+  }
+  ctas = count * num_kv_heads;
+  if (num_splits) {
+    // cut the key range when there are too few CTAs for the SMs, keeping at
+    // least two tiles per split
+    long long s = 1;
+    if (kv_len_h && num_sms > 0 && ctas > 0 && ctas < num_sms) {
+      s = (2LL * num_sms + ctas - 1) / ctas;
+      const long long cap = max_tiles / 2 > 1 ? max_tiles / 2 : 1;
+      s = s < cap ? s : cap;
+      s = s < 32 ? s : 32;
+    }
+    *num_splits = (int32_t)s;
+  }
+  return count;
+}
+
+size_t pkv_append_attention_workspace_bytes(int64_t nnz_q, int num_qo_heads, int num_splits) {
+  if (nnz_q < 0 || num_qo_heads < 1 || num_splits < 1) return 0;
+  if (num_splits == 1) return 0;
+  const size_t states = (size_t)nnz_q * num_splits * num_qo_heads;
+  return align_up(states * kDecodeHeadDim * 4, 256) + align_up(states * 4, 256);
+}
+
+pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr, int64_t nnz_q,
+                                int num_qo_heads, const pkv_pool_desc* pool,
+                                const pkv_table_desc* table, const int32_t* plan,
+                                int64_t num_row_blocks, int num_splits, int window_left,
+                                int sink_tokens, float sm_scale, void* workspace,
+                                size_t workspace_bytes, void* out, float* lse,
+                                int32_t* error_word, void* stream) {
+  if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
+  pkv::TableView tv;
+  const int32_t* ids = nullptr;
+  pkv_status st = table_view(table, &tv, &ids);
+  if (st != PKV_OK) return st;
+  const int batch = table->batch;
+  if (batch < 0 || nnz_q < 0 || num_row_blocks < 0 || pool->num_pages < 1 ||
+      pool->num_kv_heads < 1 || num_qo_heads < pool->num_kv_heads ||
+      num_qo_heads % pool->num_kv_heads != 0)
+    return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
+  if (pool->dtype != PKV_F16 && pool->dtype != PKV_BF16)
+    return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_F16 or PKV_BF16");
+  if (pool->layout != PKV_LAYOUT_HND && pool->layout != PKV_LAYOUT_NHD)
+    return fail(PKV_ERR_INVALID_ARG, "layout must be PKV_LAYOUT_HND or PKV_LAYOUT_NHD");
+  if (pool->head_dim != kDecodeHeadDim) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (!valid_page_size(pool->page_size))
+    return fail(PKV_ERR_UNSUPPORTED, "page_size must be 16, 32, 64, 128 or 256");
+  if (pool->num_pages > 0x7fffffffLL) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31-1 pages");
+  if (num_splits < 1 || num_splits > 1024)
+    return fail(PKV_ERR_INVALID_ARG, "num_splits must be 1..1024");
+  if (sink_tokens < 0) return fail(PKV_ERR_INVALID_ARG, "sink_tokens < 0");
+  if (!std::isfinite(sm_scale)) return fail(PKV_ERR_INVALID_ARG, "sm_scale is not finite");
+  if (num_row_blocks > 0x7fffffffLL || num_row_blocks * pool->num_kv_heads > 0x7fffffffLL)
+    return fail(PKV_ERR_UNSUPPORTED, "too many row blocks");
+  if (num_row_blocks == 0 || nnz_q == 0 || batch == 0) return ok();
+  if (!q || !qo_indptr || !pool->data || !ids || !plan || !out ||
+      (tv.indptr ? !tv.last_len : (!tv.context_lens || tv.max_blocks < 1)))
+    return fail(PKV_ERR_INVALID_ARG, "null pointer or empty block table");
+  if (!aligned(q, 16) || !aligned(pool->data, 16) || !aligned(out, 16) || !aligned(plan, 16))
+    return fail(PKV_ERR_INVALID_ARG, "q, pool, out and plan must be 16-byte aligned");
+  if (out == q || out == pool->data) return fail(PKV_ERR_INVALID_ARG, "out aliases q or pool");
+  const size_t need = pkv_append_attention_workspace_bytes(nnz_q, num_qo_heads, num_splits);
+  if (need > 0 && (!workspace || !aligned(workspace, 256)))
+    return fail(PKV_ERR_WORKSPACE, "workspace must be non-null and 256-byte aligned");
+  if (workspace_bytes < need)
+    return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+
+  CUtensorMap tmap;
+  int one_box = 0;
+  st = pool_tensor_map(pool->data, pool->num_pages, pool->page_size, pool->num_kv_heads,
+                       pool->dtype, pool->layout, &tmap, &one_box);
+  if (st != PKV_OK) return st;
+  const size_t states = (size_t)nnz_q * num_splits * num_qo_heads;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  pkv::ChunkArgs a;
+  a.q = q;
+  a.qo_indptr = qo_indptr;
+  a.tv = tv;
+  a.indices = ids;
+  a.plan = reinterpret_cast<const int4*>(plan);
+  a.out = out;
+  a.lse = lse;
+  a.state_o = num_splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
+  a.state_lse = num_splits > 1
+                    ? reinterpret_cast<float*>(ws + align_up(states * kDecodeHeadDim * 4, 256))
+                    : nullptr;
+  a.err = reinterpret_cast<int*>(error_word);
+  a.num_pages = pool->num_pages;
+  a.nnz_q = nnz_q;
+  a.batch = batch;
+  a.hq = num_qo_heads;
+  a.hkv = pool->num_kv_heads;
+  a.group = num_qo_heads / pool->num_kv_heads;
+  a.page_size = pool->page_size;
+  a.splits = num_splits;
+  a.window_left = window_left < 0 ? -1 : window_left;
+  a.sink = sink_tokens;
+  a.scale_log2 = sm_scale * 1.4426950408889634f;
+  a.one_box = one_box;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = pkv::launch_chunk(tmap, a, pool->dtype == PKV_BF16, (int)num_row_blocks, s);
+  if (e != cudaSuccess) return cuda_fail(e, "append attention launch");
+  if (num_splits > 1) {
+    pkv::MergeArgs ma;
+    ma.v = a.state_o;
+    ma.s = a.state_lse;
+    ma.v_out = out;
+    ma.s_out = lse;
+    ma.rows = nnz_q;
+    ma.states = num_splits;
+    ma.heads = num_qo_heads;
+    ma.head_dim = kDecodeHeadDim;
+    ma.out_dtype = pool->dtype;
+    ma.vec4 = 1;
+    e = pkv::launch_merge(ma, s);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  return ok();
+}
+
 pkv_status pkv_merge_states(const float* v, const float* s, int64_t num_rows, int num_states,
                             int num_heads, int head_dim, void* v_out, int out_dtype,
                             float* s_out, void* stream) {

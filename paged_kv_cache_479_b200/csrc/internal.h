@@ -68,6 +68,30 @@ int prefix_tile_tokens();
 cudaError_t launch_prefix(const CUtensorMap& tmap, const PrefixArgs& a, bool bf16, int row_blocks,
                           cudaStream_t stream);
 
+// multi-token append attention (chunk.cu)
+struct ChunkArgs {
+  const void* q;               // [nnz_q][Hq][128]
+  const int32_t* qo_indptr;    // [B+1], qo_indptr[0] = 0
+  TableView tv;                // the table after the append
+  const int32_t* indices;
+  const int4* plan;            // row blocks {request, first row, rows, 0}
+  void* out;                   // [nnz_q][Hq][128] (one split)
+  float* lse;                  // [nnz_q][Hq] or null (one split)
+  float* state_o;              // [nnz_q][splits][Hq][128] (several splits)
+  float* state_lse;            // [nnz_q][splits][Hq]
+  int* err;
+  long long num_pages;
+  long long nnz_q;             // rows of q / out
+  int batch, hq, hkv, group, page_size, splits, window_left, sink;
+  float scale_log2;
+  int one_box;
+};
+size_t chunk_smem_bytes();
+int chunk_rows_per_cta();
+int chunk_tile_tokens();
+cudaError_t launch_chunk(const CUtensorMap& tmap, const ChunkArgs& a, bool bf16, int row_blocks,
+                         cudaStream_t stream);
+
 struct AppendArgs {
   void* pool;
   TableView tv;

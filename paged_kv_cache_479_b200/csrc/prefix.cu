@@ -22,6 +22,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include "attn_tile.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "partition.cuh"
@@ -29,14 +30,14 @@
 namespace pkv {
 namespace {
 
-constexpr int kD = 128;
+using tile::kBoxBytes;
+using tile::kBoxes;
+using tile::kD;
+using tile::kHalf;
+using tile::kKVBytes;
+using tile::kTile;
 constexpr int kWarps = 8;                       // consumer warps
 constexpr int kRows = kWarps * 16;              // query rows per CTA
-constexpr int kTile = 64;                       // prefix tokens per stage
-constexpr int kBoxes = kTile / kTileTokens;     // 16-token boxes per K (or V) tile
-constexpr int kBoxBytes = kTileTokens * kD * 2; // 4 KiB
-constexpr int kHalf = kBoxBytes / 2;            // one [16][64] half of a box
-constexpr int kKVBytes = kBoxes * kBoxBytes;    // 16 KiB for K (and for V) of a tile
 constexpr int kStageBytes = 2 * kKVBytes;
 constexpr int kStages = 3;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -49,13 +50,6 @@ struct __align__(16) Ctl {
 };
 
 constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kStageBytes + sizeof(Ctl);
-
-// byte offset of (token t of the tile, 16-byte chunk c of its 128 dims) in a
-// K or V area made of kBoxes 128-byte-swizzled [2][16][64] boxes
-__device__ __forceinline__ uint32_t tile_off(int t, int c) {
-  const int bx = t >> 4, tt = t & 15;
-  return (uint32_t)(bx * kBoxBytes + (c >> 3) * kHalf + tt * 128 + (((c & 7) ^ (tt & 7)) << 4));
-}
 
 template <bool BF16>
 __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
@@ -143,28 +137,20 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
   }
 
   // =========================== consumers ===========================
-  const int g = lane >> 2, cq = lane & 3, mi = lane >> 3, r8 = lane & 7;
+  const int g = lane >> 2, cq = lane & 3;
   const long long nrows = (long long)a.batch * G;
   const long long row0 = (long long)rb * kRows + warp * 16;  // this warp's first row
   // query rows as A fragments: row r -> request r / G, query head kvh * G + r % G
   uint32_t qa[8][4];
   {
     const uint16_t* qp[2];
-    bool qv[2];
     for (int hr = 0; hr < 2; ++hr) {
       const long long r = row0 + g + 8 * hr;
-      qv[hr] = r < nrows;
-      const long long b = qv[hr] ? r / G : 0, hh = qv[hr] ? r % G : 0;
-      qp[hr] = static_cast<const uint16_t*>(a.q) + ((size_t)b * a.hq + (size_t)kvh * G + hh) * kD;
+      qp[hr] = r < nrows ? static_cast<const uint16_t*>(a.q) +
+                               ((size_t)(r / G) * a.hq + (size_t)kvh * G + r % G) * kD
+                         : nullptr;
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int d0 = j * 16 + 2 * cq;
-      qa[j][0] = qv[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + d0) : 0u;
-      qa[j][1] = qv[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + d0) : 0u;
-      qa[j][2] = qv[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + d0 + 8) : 0u;
-      qa[j][3] = qv[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + d0 + 8) : 0u;
-    }
+    tile::load_q(qp[0], qp[1], cq, qa);
   }
   float o[16][4];
 #pragma unroll
@@ -178,24 +164,9 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
     if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kStages) & 1, &ctl.abort, a.err)) return;
     const int valid = ctl.valid[s];
     const uint32_t kb = ring0 + (uint32_t)s * kStageBytes, vb = kb + kKVBytes;
-    // ---- S = Q K^T for 64 tokens (8 n-tiles of 8)
     float sc[8][4];
-#pragma unroll
-    for (int n = 0; n < 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {  // n-tile pair (2np, 2np+1)
-        const int tok = np * 16 + (mi >> 1) * 8 + r8;
-        const int chunk = j * 2 + (mi & 1);
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4(kb + tile_off(tok, chunk), b0, b1, b2, b3);
-        mma_16816<BF16>(sc[2 * np], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b0, b1);
-        mma_16816<BF16>(sc[2 * np + 1], qa[j][0], qa[j][1], qa[j][2], qa[j][3], b2, b3);
-      }
-    }
-    // ---- mask tokens past the prefix, online softmax (log2 units)
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+    tile::qk<BF16>(qa, kb, lane, sc);
+    // tokens past the prefix are not keys
 #pragma unroll
     for (int n = 0; n < 8; ++n) {
       const int t = n * 8 + 2 * cq;
@@ -203,80 +174,10 @@ __global__ void __launch_bounds__((kWarps + 1) * 32, 1)
       sc[n][1] = t + 1 < valid ? sc[n][1] * sl2 : -INFINITY;
       sc[n][2] = t < valid ? sc[n][2] * sl2 : -INFINITY;
       sc[n][3] = t + 1 < valid ? sc[n][3] * sl2 : -INFINITY;
-      mx0 = fmaxf(mx0, fmaxf(sc[n][0], sc[n][1]));
-      mx1 = fmaxf(mx1, fmaxf(sc[n][2], sc[n][3]));
     }
-#pragma unroll
-    for (int off = 1; off < 4; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = mn0 == -INFINITY ? 1.f : ex2(m0 - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : ex2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      sc[n][0] = ex2(sc[n][0] - mn0);
-      sc[n][1] = ex2(sc[n][1] - mn0);
-      sc[n][2] = ex2(sc[n][2] - mn1);
-      sc[n][3] = ex2(sc[n][3] - mn1);
-      ps0 += sc[n][0] + sc[n][1];
-      ps1 += sc[n][2] + sc[n][3];
-    }
-    l0 = l0 * al0 + ps0;
-    l1 = l1 * al1 + ps1;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      o[n][0] *= al0;
-      o[n][1] *= al0;
-      o[n][2] *= al1;
-      o[n][3] *= al1;
-    }
-    // ---- V rows past the prefix may hold anything (even NaN): zero them
-    if (valid < kTile) {
-      uint8_t* vrow = smem + (size_t)s * kStageBytes + kKVBytes;
-      for (int idx = lane; idx < (kTile - valid) * 16; idx += 32) {
-        const int t = valid + (idx >> 4), c = idx & 15;
-        *reinterpret_cast<uint4*>(vrow + tile_off(t, c)) = make_uint4(0, 0, 0, 0);
-      }
-      __syncwarp();
-    }
-    // ---- O += P V  (P of two adjacent n-tiles is the A fragment of one k-step)
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ah[4], al[4];
-      {
-        const float* p0 = sc[2 * kk];
-        const float* p1 = sc[2 * kk + 1];
-        ah[0] = pack2<BF16>(p0[0], p0[1]);
-        ah[1] = pack2<BF16>(p0[2], p0[3]);
-        ah[2] = pack2<BF16>(p1[0], p1[1]);
-        ah[3] = pack2<BF16>(p1[2], p1[3]);
-        if constexpr (BF16) {
-          float2 f;
-          f = unpack2<true>(ah[0]); al[0] = pack2<true>(p0[0] - f.x, p0[1] - f.y);
-          f = unpack2<true>(ah[1]); al[1] = pack2<true>(p0[2] - f.x, p0[3] - f.y);
-          f = unpack2<true>(ah[2]); al[2] = pack2<true>(p1[0] - f.x, p1[1] - f.y);
-          f = unpack2<true>(ah[3]); al[3] = pack2<true>(p1[2] - f.x, p1[3] - f.y);
-        }
-      }
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {  // dim n-tile pair (2np, 2np+1)
-        const int tok = kk * 16 + (mi & 1) * 8 + r8;
-        const int chunk = 2 * np + (mi >> 1);
-        uint32_t b0, b1, b2, b3;
-        ldmatrix_x4_trans(vb + tile_off(tok, chunk), b0, b1, b2, b3);
-        mma_16816<BF16>(o[2 * np], ah[0], ah[1], ah[2], ah[3], b0, b1);
-        mma_16816<BF16>(o[2 * np + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
-        if constexpr (BF16) {
-          mma_16816<BF16>(o[2 * np], al[0], al[1], al[2], al[3], b0, b1);
-          mma_16816<BF16>(o[2 * np + 1], al[0], al[1], al[2], al[3], b2, b3);
-        }
-      }
-    }
+    tile::online_softmax(sc, m0, m1, l0, l1, o);
+    if (valid < kTile) tile::zero_v_rows(smem + (size_t)s * kStageBytes + kKVBytes, valid, lane);
+    tile::pv<BF16>(sc, vb, lane, o);
     if (valid < kTile) fence_proxy_async_smem();
     __syncwarp();
     mbar_arrive(smem_u32(&ctl.empty[s]));

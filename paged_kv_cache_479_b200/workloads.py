@@ -358,6 +358,69 @@ def make_fp8_tensors(w: Workload, device="cpu"):
     return q, pool, k_new, v_new
 
 
+# --------------------------------------------------------------------------
+# multi-token chunks (append attention)
+# --------------------------------------------------------------------------
+
+def chunk_indptr(q_lens) -> np.ndarray:
+    qo = np.zeros(len(q_lens) + 1, np.int32)
+    qo[1:] = np.cumsum(np.asarray(q_lens, np.int64))
+    return qo
+
+
+def make_chunk_queries(w: Workload, q_lens, device="cpu", seed_offset=17):
+    """Query rows [sum(q_lens), Hq, D] of the workload's dtype for chunks of
+    q_lens tokens per request (the last q_lens[b] of request b's tokens)."""
+    device = torch.device(device)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(w.seed) + seed_offset)
+    n = int(np.sum(q_lens))
+    return (torch.randn((n, w.num_qo_heads, w.head_dim), generator=gen, device=device)
+            * w.q_std).to(w.torch_dtype)
+
+
+def named_chunk(kind: str):
+    """Append-attention workloads: (workload, q_lens); the chunk's K/V rows are
+    the workload's appended tokens (append_counts = q_lens).
+
+    "prefill": chunked prefill of a Llama-3-8B-shaped layer -- 4 prompts whose
+      2048-token chunk lands on 6144 cached tokens (8192 after the append),
+      32q/8kv, D128, ps16, bf16.
+    "spec": verification of 4 speculative tokens for the decode batch of the
+      Llama-3-8B-shaped workload -- batch 64, KV U[512,4096] + 4, 32q/8kv, bf16.
+    """
+    seed = SEED_BASE + 100
+    if kind == "prefill":
+        q_lens = np.full(4, 2048, np.int64)
+        w = make_workload("chunked prefill: 4 x (6144 cached + 2048-token chunk), 32q/8kv, D128, ps16, bf16",
+                          [8192] * 4, num_qo_heads=32, num_kv_heads=8, page_size=16,
+                          dtype="bf16", seed=seed, pool_factor=1.1, append_counts=q_lens)
+        return w, q_lens
+    if kind == "spec":
+        rng = np.random.default_rng(seed + 10_000)
+        lens = rng.integers(512, 4096, size=64, endpoint=True) + 4
+        q_lens = np.full(64, 4, np.int64)
+        w = make_workload("speculative verification: batch 64, KV U[512,4096] + 4 draft tokens, 32q/8kv, D128, ps16, bf16",
+                          lens, num_qo_heads=32, num_kv_heads=8, page_size=16, dtype="bf16",
+                          seed=seed + 1, pool_factor=1.25, append_counts=q_lens)
+        return w, q_lens
+    raise ValueError(f"no chunk workload {kind!r}")
+
+
+def chunk_flops(w: Workload, q_lens, window_left: int = -1, sink: int = 0) -> int:
+    """Algorithmic FLOPs of append attention: 2 * D per (query head, visible
+    key) for the scores and as many for P.V."""
+    total = 0
+    for b in range(w.batch):
+        L, n = int(w.kv_lens[b]), int(q_lens[b])
+        pos = np.arange(L - n, L, dtype=np.int64)
+        vis = pos + 1
+        if window_left >= 0:
+            vis = np.minimum(vis, window_left + 1 + np.minimum(sink, np.maximum(pos - window_left, 0)))
+        total += int(vis.sum())
+    return 4 * w.head_dim * w.num_qo_heads * total
+
+
 def bits(t: torch.Tensor) -> np.ndarray:
     """Raw uint16 bit patterns of a 16-bit tensor, on the host."""
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)

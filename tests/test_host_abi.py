@@ -253,3 +253,62 @@ def test_fp8_calls_reject_bad_arguments():
                            ctypes.c_void_p(8192), None, None, None) == 1
     assert L.pkv_append_ex(ctypes.byref(fp8), ctypes.byref(csr), p, p, p, 3, None, None) == 1
     assert b"pkv_append_fp8" in L.pkv_last_error()
+
+
+def test_append_attention_plan_covers_rows_once():
+    rng = np.random.default_rng(9)
+    q_lens = rng.integers(0, 400, size=37)
+    qo = wl.chunk_indptr(q_lens)
+    kv = (q_lens + rng.integers(0, 3000, size=37)).astype(np.int32)
+    for hq, hkv in ((32, 8), (8, 8), (64, 8)):
+        G = hq // hkv
+        plan, S = pkv.append_attention_plan(qo, kv, hq, hkv, num_sms=148)
+        seen = [np.zeros(int(n) * G, int) for n in q_lens]
+        for b, r0, n, pad in plan:
+            assert 1 <= n <= 128 and pad == 0
+            seen[b][r0:r0 + n] += 1
+        assert all((s == 1).all() for s in seen)
+        assert list(plan[:, 0]) == sorted(plan[:, 0])
+        assert 1 <= S <= 32
+
+
+def test_append_attention_plan_splits_and_rejects():
+    L = pkv.lib()
+    qo = np.array([0, 4, 8], np.int32)
+    kv = np.array([4000, 3000], np.int32)
+    _, S = pkv.append_attention_plan(qo, kv, 32, 8, num_sms=148)
+    assert S > 1                                   # 2 blocks x 8 heads on 148 SMs
+    _, S1 = pkv.append_attention_plan(qo, None, 32, 8, num_sms=148)
+    assert S1 == 1                                 # no lengths: no split suggested
+    big = wl.chunk_indptr([2048] * 8)
+    _, S2 = pkv.append_attention_plan(big, np.full(8, 8192, np.int32), 32, 8, num_sms=148)
+    assert S2 == 1                                 # 8 x 64 blocks x 8 heads fill the GPU
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    bad_start = np.array([1, 4, 8], np.int32)
+    assert L.pkv_append_attention_plan(p(bad_start), None, 2, 32, 8, -1, 0, 148, None, 0, None) == -1
+    dec = np.array([0, 4, 2], np.int32)
+    assert L.pkv_append_attention_plan(p(dec), None, 2, 32, 8, -1, 0, 148, None, 0, None) == -1
+    short = np.array([3, 3000], np.int32)           # 4 queries but 3 tokens
+    assert L.pkv_append_attention_plan(p(qo), p(short), 2, 32, 8, -1, 0, 148, None, 0, None) == -1
+    assert L.pkv_append_attention_plan(p(qo), None, 2, 30, 8, -1, 0, 148, None, 0, None) == -1
+    assert pkv.append_attention_workspace_bytes(100, 32, 1) == 0
+    assert pkv.append_attention_workspace_bytes(100, 32, 3) >= 100 * 3 * 32 * 129 * 4
+
+
+def test_append_attention_rejects_bad_arguments():
+    L = pkv.lib()
+    P = ctypes.c_void_p(4096)
+    pool = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.BF16, 0, 0)
+    csr = pkv.TableDesc(0, 4, 4096, 4096, 4096, None, None, 0, 0)
+
+    def call(pool=pool, splits=1, ws_bytes=0, plan=P):
+        return L.pkv_append_attention(P, P, 16, 8, ctypes.byref(pool), ctypes.byref(csr), plan, 3,
+                                      splits, -1, 0, 0.1, None, ws_bytes, ctypes.c_void_p(8192),
+                                      None, None, None)
+
+    assert call(splits=0) == 1
+    assert call(pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.FP8_E4M3, 0, 0)) == 1
+    assert call(pkv.PoolDesc(4096, 64, 16, 2, 64, pkv.BF16, 0, 0)) == 2
+    assert call(pkv.PoolDesc(4096, 64, 8, 2, 128, pkv.BF16, 0, 0)) == 2
+    assert call(splits=4) == 3                       # no workspace for the split states
+    assert call(plan=ctypes.c_void_p(4100)) == 1     # misaligned plan
