@@ -19,6 +19,7 @@ from . import build as _build
 F16 = 0
 BF16 = 1
 FP8_E4M3 = 3
+FP8_E5M2 = 4
 
 _STATUS = {
     0: "ok",
@@ -47,10 +48,10 @@ def _load():
         lib.oracle_merge.argtypes = [p, p, i64, i32, i32, i32, p, p]
         lib.oracle_merge.restype = None
         f32 = ctypes.c_float
-        lib.oracle_decode_fp8.argtypes = [p, i32, p, f32, f32, i64, i32, i32, i32, i32, i32,
-                                          p, p, p, dbl, p, p]
+        lib.oracle_decode_fp8.argtypes = [p, i32, p, i32, f32, f32, i64, i32, i32, i32, i32,
+                                          i32, p, p, p, dbl, p, p]
         lib.oracle_decode_fp8.restype = i32
-        lib.oracle_append_fp8.argtypes = [p, f32, f32, i64, i32, i32, i32, i32, p, p, p,
+        lib.oracle_append_fp8.argtypes = [p, i32, f32, f32, i64, i32, i32, i32, i32, p, p, p,
                                           p, p, i32, p]
         lib.oracle_append_fp8.restype = i32
         lib.oracle_append_attention.argtypes = [p, p, i32, i64, i32, i32, i32, i32, i32,
@@ -60,6 +61,10 @@ def _load():
         lib.oracle_e4m3_decode.restype = i32
         lib.oracle_e4m3_encode.argtypes = [p, i64, f32, p]
         lib.oracle_e4m3_encode.restype = i32
+        lib.oracle_e5m2_decode.argtypes = [p, i64, p]
+        lib.oracle_e5m2_decode.restype = i32
+        lib.oracle_e5m2_encode.argtypes = [p, i64, f32, p]
+        lib.oracle_e5m2_encode.restype = i32
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -152,27 +157,42 @@ def merge(v, s):
     return vo, so
 
 
-def e4m3_values(codes):
-    """Exact value of every E4M3 code (NaN for 0x7f / 0xff), float64."""
+def _fmt(fmt):
+    return {"e4m3": "e4m3", FP8_E4M3: "e4m3", "e5m2": "e5m2", FP8_E5M2: "e5m2"}[fmt]
+
+
+def fp8_values(codes, fmt="e4m3"):
+    """Exact value of every code of the format, float64 (NaN / inf where the format has them)."""
     codes, cp = _c(codes, np.uint8)
     out = np.zeros(codes.shape, np.float64)
-    _load().oracle_e4m3_decode(cp, codes.size, out.ctypes.data_as(ctypes.c_void_p))
+    getattr(_load(), f"oracle_{_fmt(fmt)}_decode")(cp, codes.size,
+                                                   out.ctypes.data_as(ctypes.c_void_p))
     return out
+
+
+def fp8_encode(x, scale=1.0, fmt="e4m3"):
+    """Codes of float32(x) / float32(scale): nearest, ties to even, saturating."""
+    x, xp = _c(x, np.float32)
+    codes = np.zeros(x.shape, np.uint8)
+    rc = getattr(_load(), f"oracle_{_fmt(fmt)}_encode")(xp, x.size, float(scale),
+                                                        codes.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise OracleError(f"oracle_{_fmt(fmt)}_encode: {_STATUS.get(rc, rc)}")
+    return codes
+
+
+def e4m3_values(codes):
+    """Exact value of every E4M3 code (NaN for 0x7f / 0xff), float64."""
+    return fp8_values(codes, "e4m3")
 
 
 def e4m3_encode(x, scale=1.0):
     """E4M3 codes of float32(x) / float32(scale): nearest, ties to even, saturating."""
-    x, xp = _c(x, np.float32)
-    codes = np.zeros(x.shape, np.uint8)
-    rc = _load().oracle_e4m3_encode(xp, x.size, float(scale),
-                                    codes.ctypes.data_as(ctypes.c_void_p))
-    if rc != 0:
-        raise OracleError(f"oracle_e4m3_encode: {_STATUS.get(rc, rc)}")
-    return codes
+    return fp8_encode(x, scale, "e4m3")
 
 
 def decode_fp8(q_bits, q_dtype, pool_codes, k_scale, v_scale, page_indptr, page_indices,
-               last_page_len, scale):
+               last_page_len, scale, fmt="e4m3"):
     """Exact decode attention over an E4M3 pool.
 
     q_bits     uint16 [B, Hq, D]  fp16/bf16 bits (q_dtype)
@@ -192,7 +212,8 @@ def decode_fp8(q_bits, q_dtype, pool_codes, k_scale, v_scale, page_indptr, page_
     last, lp = _c(last_page_len if len(last_page_len) else np.zeros(1, np.int32), np.int32)
     out = np.zeros((B, hq, d), np.float64)
     lse = np.zeros((B, hq), np.float64)
-    rc = _load().oracle_decode_fp8(qp, int(q_dtype), pp, float(k_scale), float(v_scale), P, ps,
+    fp8 = FP8_E4M3 if _fmt(fmt) == "e4m3" else FP8_E5M2
+    rc = _load().oracle_decode_fp8(qp, int(q_dtype), pp, fp8, float(k_scale), float(v_scale), P, ps,
                                    hkv, d, B, hq, ip, xp, lp, float(scale),
                                    out.ctypes.data_as(ctypes.c_void_p),
                                    lse.ctypes.data_as(ctypes.c_void_p))
@@ -202,7 +223,7 @@ def decode_fp8(q_bits, q_dtype, pool_codes, k_scale, v_scale, page_indptr, page_
 
 
 def append_fp8(pool_codes, k_scale, v_scale, page_indptr, page_indices, last_page_len,
-               k_new_bits, v_new_bits, new_dtype, append_indptr):
+               k_new_bits, v_new_bits, new_dtype, append_indptr, fmt="e4m3"):
     """Return a copy of an E4M3 pool with the new 16-bit rows quantised in.
 
     pool_codes uint8 [P, 2, Hkv, ps, D] (not modified); k/v_new uint16 [nnz, Hkv, D]
@@ -217,7 +238,8 @@ def append_fp8(pool_codes, k_scale, v_scale, page_indptr, page_indices, last_pag
     kn, kp = _c(k_new_bits if np.size(k_new_bits) else np.zeros(1, np.uint16), np.uint16)
     vn, vp = _c(v_new_bits if np.size(v_new_bits) else np.zeros(1, np.uint16), np.uint16)
     ap, app = _c(append_indptr, np.int32)
-    rc = _load().oracle_append_fp8(pool.ctypes.data_as(ctypes.c_void_p), float(k_scale),
+    fp8 = FP8_E4M3 if _fmt(fmt) == "e4m3" else FP8_E5M2
+    rc = _load().oracle_append_fp8(pool.ctypes.data_as(ctypes.c_void_p), fp8, float(k_scale),
                                    float(v_scale), P, ps, hkv, d, B, ip, xp, lp, kp, vp,
                                    int(new_dtype), app)
     if rc != 0:

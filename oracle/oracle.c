@@ -66,7 +66,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F16 = 0, ORACLE_BF16 = 1, ORACLE_FP8_E4M3 = 3 };
+enum { ORACLE_F16 = 0, ORACLE_BF16 = 1, ORACLE_FP8_E4M3 = 3, ORACLE_FP8_E5M2 = 4 };
 
 /* Status codes: 0 ok, otherwise the table or arguments break an invariant
  * that the pages state (valid length within a page, page ids inside the
@@ -175,10 +175,60 @@ int oracle_e4m3_encode(const float* x, int64_t n, float scale, uint8_t* codes) {
   return ORACLE_OK;
 }
 
-/* Element idx of a pool of 16-bit (fp16 / bf16) or 8-bit (E4M3) values, widened
- * exactly (E4M3 codes are multiplied by their scale afterwards). */
+/*
+ * FP8 E5M2: sign, 5-bit exponent with bias 15, 2-bit fraction -- the top
+ * byte of an IEEE half, so it keeps infinities (S.11111.00) and NaNs
+ * (S.11111.xx, xx != 0); largest finite magnitude 1.75 * 2^15 = 57344.  The
+ * "fp8_e5m2" KV-cache dtype of "大模型长上下文窗口工程化实战：从RoPE扩展到百万
+ * Token推理的生产级部署" sections 3.1 and 3.2; scales as for E4M3.
+ */
+static double widen_e5m2(uint8_t code) {
+  const int sign = code >> 7, e = (code >> 2) & 0x1f, frac = code & 3;
+  double v;
+  if (e == 31) v = frac ? NAN : INFINITY;
+  else if (e == 0) v = ldexp((double)frac, -16);      /* frac/4 * 2^-14 */
+  else v = ldexp((double)(frac | 4), e - 17);         /* (1 + frac/4) * 2^(e-15) */
+  return sign ? -v : v;
+}
+
+int oracle_e5m2_decode(const uint8_t* codes, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = widen_e5m2(codes[i]);
+  return ORACLE_OK;
+}
+
+/* x / scale as E5M2: nearest finite value, ties to the even code, magnitudes
+ * from 57344 up (infinity included) saturating to +-57344, NaN to 0x7f. */
+static uint8_t encode_e5m2(float x, float scale) {
+  const float q = (float)(x / scale);  /* binary32 quotient */
+  if (isnan(q)) return 0x7f;
+  const int neg = signbit(q) ? 1 : 0;
+  const double a = fabs((double)q);
+  if (a >= 57344.0) return (uint8_t)((neg << 7) | 0x7b);
+  int best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c <= 0x7b; ++c) {          /* non-negative finite codes */
+    const double err = fabs(widen_e5m2((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && !(c & 1))) {     /* tie: even code */
+      best = c;
+      best_err = err;
+    }
+  }
+  return (uint8_t)((neg << 7) | best);
+}
+
+int oracle_e5m2_encode(const float* x, int64_t n, float scale, uint8_t* codes) {
+  if (!(scale > 0.0f) || isinf(scale)) return ORACLE_BAD_ARG;
+  for (int64_t i = 0; i < n; ++i) codes[i] = encode_e5m2(x[i], scale);
+  return ORACLE_OK;
+}
+
+static int is_fp8(int dtype) { return dtype == ORACLE_FP8_E4M3 || dtype == ORACLE_FP8_E5M2; }
+
+/* Element idx of a pool of 16-bit (fp16 / bf16) or 8-bit (E4M3 / E5M2) values,
+ * widened exactly (8-bit codes are multiplied by their scale afterwards). */
 static double kv_elem(const void* pool, int kv_dtype, size_t idx) {
   if (kv_dtype == ORACLE_FP8_E4M3) return widen_e4m3(((const uint8_t*)pool)[idx]);
+  if (kv_dtype == ORACLE_FP8_E5M2) return widen_e5m2(((const uint8_t*)pool)[idx]);
   return widen(((const uint16_t*)pool)[idx], kv_dtype);
 }
 
@@ -241,7 +291,7 @@ static int decode_rows(const uint16_t* q, int q_dtype, const void* pool, int kv_
   if (batch < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1 ||
       num_qo_heads < num_kv_heads || num_qo_heads % num_kv_heads != 0 ||
       (q_dtype != ORACLE_F16 && q_dtype != ORACLE_BF16) ||
-      (kv_dtype != ORACLE_F16 && kv_dtype != ORACLE_BF16 && kv_dtype != ORACLE_FP8_E4M3))
+      (kv_dtype != ORACLE_F16 && kv_dtype != ORACLE_BF16 && !is_fp8(kv_dtype)))
     return ORACLE_BAD_ARG;
   int rc = check_table(num_pages, page_size, batch, page_indptr, page_indices, last_page_len);
   if (rc != ORACLE_OK) return rc;
@@ -308,23 +358,25 @@ int oracle_decode(const uint16_t* q, const uint16_t* pool, int dtype,
                   const int32_t* page_indptr, const int32_t* page_indices,
                   const int32_t* last_page_len, double scale,
                   double* out, double* lse) {
-  if (dtype == ORACLE_FP8_E4M3) return ORACLE_BAD_ARG;
+  if (is_fp8(dtype)) return ORACLE_BAD_ARG;
   return decode_rows(q, dtype, pool, dtype, 1.0, 1.0, num_pages, page_size, num_kv_heads,
                      head_dim, batch, num_qo_heads, page_indptr, page_indices, last_page_len,
                      scale, out, lse);
 }
 
 /*
- * oracle_decode_fp8 -- the same attention over an E4M3 pool: key element =
- * code_value * k_scale, value element = code_value * v_scale (exact in
- * double); q is fp16 or bf16 (q_dtype).
+ * oracle_decode_fp8 -- the same attention over an 8-bit pool (fp8_dtype
+ * ORACLE_FP8_E4M3 or ORACLE_FP8_E5M2): key element = code_value * k_scale,
+ * value element = code_value * v_scale (exact in double); q is fp16 or bf16
+ * (q_dtype).
  */
-int oracle_decode_fp8(const uint16_t* q, int q_dtype, const uint8_t* pool, float k_scale,
-                      float v_scale, int64_t num_pages, int page_size, int num_kv_heads,
-                      int head_dim, int batch, int num_qo_heads,
+int oracle_decode_fp8(const uint16_t* q, int q_dtype, const uint8_t* pool, int fp8_dtype,
+                      float k_scale, float v_scale, int64_t num_pages, int page_size,
+                      int num_kv_heads, int head_dim, int batch, int num_qo_heads,
                       const int32_t* page_indptr, const int32_t* page_indices,
                       const int32_t* last_page_len, double scale, double* out, double* lse) {
-  return decode_rows(q, q_dtype, pool, ORACLE_FP8_E4M3, (double)k_scale, (double)v_scale,
+  if (!is_fp8(fp8_dtype)) return ORACLE_BAD_ARG;
+  return decode_rows(q, q_dtype, pool, fp8_dtype, (double)k_scale, (double)v_scale,
                      num_pages, page_size, num_kv_heads, head_dim, batch, num_qo_heads,
                      page_indptr, page_indices, last_page_len, scale, out, lse);
 }
@@ -349,7 +401,7 @@ static int append_rows(void* pool, int kv_dtype, float k_scale, float v_scale,
                        const uint16_t* k_new, const uint16_t* v_new, int new_dtype,
                        const int32_t* append_indptr) {
   if (batch < 0 || page_size < 1 || num_kv_heads < 1 || head_dim < 1) return ORACLE_BAD_ARG;
-  if (kv_dtype != ORACLE_FP8_E4M3 && kv_dtype != new_dtype) return ORACLE_BAD_ARG;
+  if (!is_fp8(kv_dtype) && kv_dtype != new_dtype) return ORACLE_BAD_ARG;
   int rc = check_table(num_pages, page_size, batch, page_indptr, page_indices, last_page_len);
   if (rc != ORACLE_OK) return rc;
   if (append_indptr[0] < 0) return ORACLE_BAD_APPEND;
@@ -381,6 +433,12 @@ static int append_rows(void* pool, int kv_dtype, float k_scale, float v_scale,
             p8[dk + d] = encode_e4m3((float)widen(ks[d], new_dtype), k_scale);
             p8[dv + d] = encode_e4m3((float)widen(vs[d], new_dtype), v_scale);
           }
+        } else if (kv_dtype == ORACLE_FP8_E5M2) {
+          uint8_t* p8 = (uint8_t*)pool;
+          for (int d = 0; d < head_dim; ++d) {
+            p8[dk + d] = encode_e5m2((float)widen(ks[d], new_dtype), k_scale);
+            p8[dv + d] = encode_e5m2((float)widen(vs[d], new_dtype), v_scale);
+          }
         } else {
           memcpy((uint16_t*)pool + dk, ks, sizeof(uint16_t) * (size_t)head_dim);
           memcpy((uint16_t*)pool + dv, vs, sizeof(uint16_t) * (size_t)head_dim);
@@ -404,18 +462,20 @@ int oracle_append(uint16_t* pool, int64_t num_pages, int page_size, int num_kv_h
 }
 
 /*
- * oracle_append_fp8 -- the same scatter into an E4M3 pool: every new element
- * is quantised as encode(value / scale) (k_scale for K, v_scale for V).
+ * oracle_append_fp8 -- the same scatter into an 8-bit pool (fp8_dtype): every
+ * new element is quantised as encode(value / scale) (k_scale for K, v_scale
+ * for V).
  */
-int oracle_append_fp8(uint8_t* pool, float k_scale, float v_scale, int64_t num_pages,
-                      int page_size, int num_kv_heads, int head_dim, int batch,
+int oracle_append_fp8(uint8_t* pool, int fp8_dtype, float k_scale, float v_scale,
+                      int64_t num_pages, int page_size, int num_kv_heads, int head_dim, int batch,
                       const int32_t* page_indptr, const int32_t* page_indices,
                       const int32_t* last_page_len, const uint16_t* k_new,
                       const uint16_t* v_new, int new_dtype, const int32_t* append_indptr) {
   if (!(k_scale > 0.0f) || !(v_scale > 0.0f) || isinf(k_scale) || isinf(v_scale))
     return ORACLE_BAD_ARG;
   if (new_dtype != ORACLE_F16 && new_dtype != ORACLE_BF16) return ORACLE_BAD_ARG;
-  return append_rows(pool, ORACLE_FP8_E4M3, k_scale, v_scale, num_pages, page_size,
+  if (!is_fp8(fp8_dtype)) return ORACLE_BAD_ARG;
+  return append_rows(pool, fp8_dtype, k_scale, v_scale, num_pages, page_size,
                      num_kv_heads, head_dim, batch, page_indptr, page_indices, last_page_len,
                      k_new, v_new, new_dtype, append_indptr);
 }

@@ -1,8 +1,9 @@
-"""Pins of the oracle's FP8 (E4M3) KV-cache arithmetic against facts fixed
-outside it: the format's definition (bias 7, 3 fraction bits, subnormals,
-NaN code, largest finite 448), torch's own float8_e4m3fn conversions (a
-library routine), round-to-nearest-even at exact midpoints, and exact
-identities of attention under a per-tensor scale.
+"""Pins of the oracle's FP8 (E4M3 and E5M2) KV-cache arithmetic against facts
+fixed outside it: the formats' definitions (E4M3: bias 7, 3 fraction bits,
+NaN code, largest finite 448; E5M2: bias 15, 2 fraction bits, infinities
+and NaNs, largest finite 57344), torch's own float8_e4m3fn / float8_e5m2
+conversions (library routines), round-to-nearest-even at exact midpoints,
+and exact identities of attention under a per-tensor scale.
 
 The 8-bit cache stores one code per K/V element and one binary32 scale for
 all of K and one for all of V ("fp8_e4m3" KV cache of the serving
@@ -21,12 +22,16 @@ from test_oracle_pins import sdpa_reference, to_bits, widen
 E4M3_MAX = 448.0
 
 
-def torch_values(codes):
-    return torch.from_numpy(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+E5M2_MAX = 57344.0
+TORCH_FP8 = {"e4m3": torch.float8_e4m3fn, "e5m2": torch.float8_e5m2}
 
 
-def torch_encode(x):
-    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+def torch_values(codes, fmt="e4m3"):
+    return torch.from_numpy(np.asarray(codes, np.uint8)).view(TORCH_FP8[fmt]).double().numpy()
+
+
+def torch_encode(x, fmt="e4m3"):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(TORCH_FP8[fmt]).view(torch.uint8).numpy()
 
 
 def test_code_values_from_the_format_definition():
@@ -74,6 +79,46 @@ def test_encode_matches_torch_round_to_nearest_even():
     np.testing.assert_array_equal(oracle.e4m3_encode(v.astype(np.float32)), np.arange(0x7f))
 
 
+def test_e5m2_code_values_from_the_format_definition():
+    v = oracle.fp8_values(np.arange(256, dtype=np.uint8), "e5m2")
+    assert v[0x00] == 0.0 and np.signbit(v[0x80])
+    assert v[0x01] == 2.0 ** -16 and v[0x03] == 3 * 2.0 ** -16   # subnormals
+    assert v[0x04] == 2.0 ** -14                                  # smallest normal
+    assert v[0x3c] == 1.0 and v[0x3e] == 1.5 and v[0x40] == 2.0   # exponent field 15 = bias
+    assert v[0x7b] == E5M2_MAX and v[0xfb] == -E5M2_MAX
+    assert v[0x7c] == np.inf and v[0xfc] == -np.inf
+    assert np.isnan(v[[0x7d, 0x7e, 0x7f, 0xfd, 0xfe, 0xff]]).all()
+    np.testing.assert_array_equal(v[0x80:0xfc], -v[0x00:0x7c])
+    assert np.all(np.diff(v[0x00:0x7d]) > 0)
+    # the top byte of an IEEE half: widening is a shift
+    half = torch.from_numpy((np.arange(256, dtype=np.int32) << 8).astype(np.int16)).view(torch.float16)
+    same = (v == half.double().numpy()) | (np.isnan(v) & torch.isnan(half).numpy())
+    assert same.all()
+    t = torch_values(np.arange(256), "e5m2")
+    assert ((v == t) | (np.isnan(v) & np.isnan(t))).all()
+
+
+def test_e5m2_encode_matches_torch_and_saturates():
+    rng = np.random.default_rng(13)
+    n = 60000
+    x = (rng.standard_normal(n) * np.exp(rng.uniform(-18, 11, n))).astype(np.float32)
+    x = x[np.abs(x) < E5M2_MAX]                  # torch overflows to inf past 61440
+    np.testing.assert_array_equal(oracle.fp8_encode(x, 1.0, "e5m2"), torch_encode(x, "e5m2"))
+    v = oracle.fp8_values(np.arange(0x7c, dtype=np.uint8), "e5m2")
+    mids = ((v[:-1] + v[1:]) / 2).astype(np.float32)
+    lo = np.arange(0x7b, dtype=np.uint8)
+    expect = np.where(lo % 2 == 0, lo, lo + 1).astype(np.uint8)
+    np.testing.assert_array_equal(oracle.fp8_encode(mids, 1.0, "e5m2"), expect)
+    np.testing.assert_array_equal(oracle.fp8_encode(v.astype(np.float32), 1.0, "e5m2"),
+                                  np.arange(0x7c))
+    big = np.array([57344, 61439, 61440, 1e9, np.inf, -7e4, -np.inf, np.nan], np.float32)
+    np.testing.assert_array_equal(oracle.fp8_encode(big, 1.0, "e5m2"),
+                                  [0x7b, 0x7b, 0x7b, 0x7b, 0x7b, 0xfb, 0xfb, 0x7f])
+    s32 = np.float32(0.37)
+    np.testing.assert_array_equal(oracle.fp8_encode(x[:5000], s32, "e5m2"),
+                                  oracle.fp8_encode((x[:5000] / s32).astype(np.float32), 1.0, "e5m2"))
+
+
 def test_encode_saturates_and_keeps_nan():
     x = np.array([448, 463.9, 464, 480, 1e6, np.inf, -500, -np.inf, np.nan], np.float32)
     c = oracle.e4m3_encode(x)
@@ -104,13 +149,14 @@ def test_encode_divides_by_the_scale_in_binary32():
 # attention over an 8-bit pool
 # ---------------------------------------------------------------------------
 
-def fp8_case(lens, hq, hkv, ps, seed, q_dtype="bf16", pool_factor=1.5):
+def fp8_case(lens, hq, hkv, ps, seed, q_dtype="bf16", pool_factor=1.5, fmt="e4m3"):
     w = wl.make_workload("fp8pin", lens, num_qo_heads=hq, num_kv_heads=hkv, page_size=ps,
                          dtype=q_dtype, seed=seed, pool_factor=pool_factor, head_dim=128)
     rng = np.random.default_rng(seed)
-    # finite codes only (NaN codes excluded), roughly normal magnitudes
-    finite = np.concatenate([np.arange(0x00, 0x7f), np.arange(0x80, 0xff)]).astype(np.uint8)
-    vals = oracle.e4m3_values(finite)
+    # finite codes only (NaN / inf codes excluded), roughly normal magnitudes
+    top = 0x7f if fmt == "e4m3" else 0x7c
+    finite = np.concatenate([np.arange(0x00, top), np.arange(0x80, 0x80 + top)]).astype(np.uint8)
+    vals = oracle.fp8_values(finite, fmt)
     weight = np.exp(-0.5 * (vals / 2.0) ** 2)
     weight /= weight.sum()
     pool = np.full((w.num_pages, 2, hkv, ps, 128), 0x7f, np.uint8)   # NaN canaries
@@ -130,13 +176,13 @@ def fp8_case(lens, hq, hkv, ps, seed, q_dtype="bf16", pool_factor=1.5):
     return w, q_bits, pool, k_dense, v_dense
 
 
-def dense_sdpa_fp8(w, q_bits, k_codes, v_codes, k_scale, v_scale, scale):
+def dense_sdpa_fp8(w, q_bits, k_codes, v_codes, k_scale, v_scale, scale, fmt="e4m3"):
     """SDPA in float64 on the dequantised dense K/V (code value * scale)."""
     q = widen(q_bits, w.dtype)
     outs, lses = [], []
     for b in range(w.batch):
-        k = torch.from_numpy(torch_values(k_codes[b]) * np.float64(k_scale)).permute(1, 0, 2)[None]
-        v = torch.from_numpy(torch_values(v_codes[b]) * np.float64(v_scale)).permute(1, 0, 2)[None]
+        k = torch.from_numpy(torch_values(k_codes[b], fmt) * np.float64(k_scale)).permute(1, 0, 2)[None]
+        v = torch.from_numpy(torch_values(v_codes[b], fmt) * np.float64(v_scale)).permute(1, 0, 2)[None]
         o = torch.nn.functional.scaled_dot_product_attention(q[b][None, :, None, :], k, v,
                                                              scale=scale, enable_gqa=True)
         outs.append(o[0, :, 0, :])
@@ -146,21 +192,22 @@ def dense_sdpa_fp8(w, q_bits, k_codes, v_codes, k_scale, v_scale, scale):
 
 
 FP8_CASES = [
-    # (lens, hq, hkv, ps, q dtype, k_scale, v_scale)
-    ([17, 64, 130, 1], 8, 2, 16, "bf16", 0.0625, 0.03125),
-    ([200, 33], 32, 8, 16, "f16", 0.1, 0.7),
-    ([65, 3, 100], 8, 1, 64, "bf16", 1.0, 1.0),
+    # (lens, hq, hkv, ps, q dtype, k_scale, v_scale, format)
+    ([17, 64, 130, 1], 8, 2, 16, "bf16", 0.0625, 0.03125, "e4m3"),
+    ([200, 33], 32, 8, 16, "f16", 0.1, 0.7, "e4m3"),
+    ([65, 3, 100], 8, 1, 64, "bf16", 1.0, 1.0, "e4m3"),
+    ([90, 300], 16, 4, 16, "bf16", 0.03, 0.11, "e5m2"),
 ]
 
 
 @pytest.mark.parametrize("case", range(len(FP8_CASES)))
 def test_fp8_decode_matches_dense_sdpa_on_dequantised_values(case):
-    lens, hq, hkv, ps, qd, ks, vs = FP8_CASES[case]
-    w, q_bits, pool, kd, vd = fp8_case(lens, hq, hkv, ps, 300 + case, qd)
+    lens, hq, hkv, ps, qd, ks, vs, fmt = FP8_CASES[case]
+    w, q_bits, pool, kd, vd = fp8_case(lens, hq, hkv, ps, 300 + case, qd, fmt=fmt)
     odt = oracle.BF16 if qd == "bf16" else oracle.F16
     out, lse = oracle.decode_fp8(q_bits, odt, pool, ks, vs, w.page_indptr, w.page_indices,
-                                 w.last_page_len, w.sm_scale)
-    ro, rl = dense_sdpa_fp8(w, q_bits, kd, vd, np.float32(ks), np.float32(vs), w.sm_scale)
+                                 w.last_page_len, w.sm_scale, fmt)
+    ro, rl = dense_sdpa_fp8(w, q_bits, kd, vd, np.float32(ks), np.float32(vs), w.sm_scale, fmt)
     assert np.isfinite(out).all()               # NaN canaries never read
     np.testing.assert_allclose(out, ro, rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-12)
@@ -192,7 +239,8 @@ def test_fp8_pool_equals_16bit_pool_of_the_same_values():
     np.testing.assert_array_equal(l8, l16)
 
 
-def test_fp8_append_positions_and_codes():
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_fp8_append_positions_and_codes(fmt):
     # page_size 4: request 0 owns pages [3, 1] and holds 6 tokens after
     # appending 3 -> positions 3, 4, 5 = page 3 slot 3, page 1 slots 0, 1
     P, ps, hkv, D = 4, 4, 2, 16
@@ -204,20 +252,26 @@ def test_fp8_append_positions_and_codes():
     gen = torch.Generator().manual_seed(5)
     k = torch.randn((3, hkv, D), generator=gen) * 20
     v = torch.randn((3, hkv, D), generator=gen) * 300     # some saturate at scale 0.5
-    ks, vs = np.float32(0.125), np.float32(0.5)
+    if fmt == "e4m3":
+        ks, vs, top, sat = np.float32(0.125), np.float32(0.5), 448.0, 0x7e
+    else:
+        ks, vs, top, sat = np.float32(0.001), np.float32(0.004), E5M2_MAX, 0x7b
     for dt, odt in (("bf16", oracle.BF16), ("f16", oracle.F16)):
         kb, vb = to_bits(k, dt), to_bits(v, dt)
-        out = oracle.append_fp8(pool, ks, vs, indptr, indices, last, kb, vb, odt, app)
+        out = oracle.append_fp8(pool, ks, vs, indptr, indices, last, kb, vb, odt, app, fmt)
         expect = pool.copy()
         kq = widen(kb, dt).float().numpy() / ks
         vq = widen(vb, dt).float().numpy() / vs
-        kc = np.where(np.abs(kq) >= 448, np.where(kq < 0, 0xfe, 0x7e), torch_encode(np.clip(kq, -448, 448)))
-        vc = np.where(np.abs(vq) >= 448, np.where(vq < 0, 0xfe, 0x7e), torch_encode(np.clip(vq, -448, 448)))
+
+        def enc(x):
+            return np.where(np.abs(x) >= top, np.where(x < 0, 0x80 | sat, sat),
+                            torch_encode(np.clip(x, -top, top), fmt))
+        kc, vc = enc(kq), enc(vq)
         for row, (page, slot) in enumerate([(3, 3), (1, 0), (1, 1)]):
             expect[page, 0, :, slot, :] = kc[row]
             expect[page, 1, :, slot, :] = vc[row]
         np.testing.assert_array_equal(out, expect)
-        assert (np.abs(vq) >= 448).any()
+        assert (np.abs(vq) >= top).any()
 
 
 def test_fp8_append_rejects_bad_scales():

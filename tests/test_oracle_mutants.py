@@ -45,6 +45,9 @@ MUTANTS = {
                             "(kv_elem(pool, kv_dtype, v + d))"),
     "fp8_append_v_takes_k_scale": ("encode_e4m3((float)widen(vs[d], new_dtype), v_scale)",
                                    "encode_e4m3((float)widen(vs[d], new_dtype), k_scale)"),
+    "e5m2_exponent_bias": ("ldexp((double)(frac | 4), e - 17)", "ldexp((double)(frac | 4), e - 16)"),
+    "e5m2_ties_to_odd": ("(err == best_err && !(c & 1))", "(err == best_err && (c & 1))"),
+    "e5m2_saturates_to_inf": ("(uint8_t)((neg << 7) | 0x7b)", "(uint8_t)((neg << 7) | 0x7c)"),
     "chunk_not_causal_on_self": ("if (t > pos) return 0;", "if (t >= pos && pos > 0) return 0;"),
     "chunk_window_one_short": ("return t >= pos - window_left ||", "return t > pos - window_left ||"),
     "chunk_head_mapping": ("const int kvh = h / group;", "const int kvh = h % num_kv_heads;"),
@@ -73,7 +76,10 @@ PINS = [
     fp8pins.test_encode_divides_by_the_scale_in_binary32,
     lambda: [fp8pins.test_fp8_decode_matches_dense_sdpa_on_dequantised_values(c)
              for c in range(len(fp8pins.FP8_CASES))],
-    fp8pins.test_fp8_append_positions_and_codes,
+    lambda: fp8pins.test_fp8_append_positions_and_codes("e4m3"),
+    lambda: fp8pins.test_fp8_append_positions_and_codes("e5m2"),
+    fp8pins.test_e5m2_code_values_from_the_format_definition,
+    fp8pins.test_e5m2_encode_matches_torch_and_saturates,
     lambda: [aapins.test_append_attention_matches_masked_sdpa(c) for c in range(len(aapins.CASES))],
     aapins.test_single_token_chunks_are_the_decode,
     aapins.test_chunking_invariance,
@@ -95,7 +101,8 @@ def test_pins_catch_mutant(name, tmp_path, monkeypatch):
     lib = ctypes.CDLL(str(so))
     for fn in ("oracle_decode", "oracle_append", "oracle_merge", "oracle_num_threads",
                "oracle_decode_fp8", "oracle_append_fp8", "oracle_e4m3_decode",
-               "oracle_e4m3_encode", "oracle_append_attention"):
+               "oracle_e4m3_encode", "oracle_append_attention", "oracle_e5m2_decode",
+               "oracle_e5m2_encode"):
         getattr(lib, fn).argtypes = getattr(real, fn).argtypes
         getattr(lib, fn).restype = getattr(real, fn).restype
     monkeypatch.setattr(oracle, "_lib", lib)
