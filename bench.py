@@ -56,9 +56,9 @@ def parse():
                    help="decode a shared-prefix workload with pkv_cascade_decode")
     p.add_argument("--no-graph", action="store_true",
                    help="launch every call from Python instead of replaying CUDA graphs")
-    p.add_argument("--kv", choices=["16bit", "fp8"], default="16bit",
-                   help="KV pool type: the workload's 16-bit type, or FP8 E4M3 codes with "
-                        "per-tensor K/V scales (q and out stay 16-bit)")
+    p.add_argument("--kv", choices=["16bit", "e4m3", "e5m2"], default="16bit",
+                   help="KV pool type: the workload's 16-bit type, or FP8 (E4M3 / E5M2) codes "
+                        "with per-tensor K/V scales (q and out stay 16-bit)")
     p.add_argument("--chunk", choices=["prefill", "spec"], default=None,
                    help="time multi-token append attention instead of the decode: chunked "
                         "prefill (TFLOP/s) or speculative verification (GB/s)")
@@ -199,7 +199,7 @@ FP8_V_SCALE = 0.0071
 
 
 def kv_elem_bytes(args):
-    return 1 if getattr(args, "kv", "16bit") == "fp8" else None
+    return 1 if getattr(args, "kv", "16bit") != "16bit" else None
 
 
 def algorithmic_bytes(w, args=None):
@@ -221,8 +221,8 @@ def workload_config(w, args, rotation, partitions):
            "parallelism": f"dp{args.gpus} (independent batches per GPU)"}
     if w.note:
         cfg["values"] = w.note
-    if getattr(args, "kv", "16bit") == "fp8":
-        cfg["kv_cache"] = (f"FP8 E4M3 codes, k_scale {FP8_K_SCALE}, v_scale {FP8_V_SCALE}; "
+    if getattr(args, "kv", "16bit") != "16bit":
+        cfg["kv_cache"] = (f"FP8 {args.kv.upper()} codes, k_scale {FP8_K_SCALE}, v_scale {FP8_V_SCALE}; "
                            f"q / out {w.dtype}; append quantises the new {w.dtype} rows")
     if getattr(args, "cascade", False):
         cfg["method"] = "shared-prefix cascade: prefix attention once per 128 query rows, own pages by the decode kernel, states merged"
@@ -335,10 +335,12 @@ def pack(tensors, dev):
 class Batch:
     """One copy of the workload's tensors on the device."""
 
-    def __init__(self, w, dev, value_seed, fp8=False):
+    def __init__(self, w, dev, value_seed, fp8=None):
         wv = wl.Workload(**{**w.__dict__, "seed": value_seed})
-        make = wl.make_fp8_tensors if fp8 else wl.make_tensors
-        self.q, self.pool, self.k_new, self.v_new = make(wv, dev)
+        if fp8:
+            self.q, self.pool, self.k_new, self.v_new = wl.make_fp8_tensors(wv, dev, fp8)
+        else:
+            self.q, self.pool, self.k_new, self.v_new = wl.make_tensors(wv, dev)
 
 
 def run_pkv(args):
@@ -359,7 +361,7 @@ def run_pkv(args):
     w = wl.named(args.workload)
     if args.cascade and not w.shared_prefix_pages:
         raise SystemExit("--cascade needs a workload with a shared prefix (workload 5)")
-    fp8 = args.kv == "fp8"
+    fp8 = None if args.kv == "16bit" else args.kv
     if fp8 and args.cascade:
         raise SystemExit("--cascade runs on 16-bit pools only")
     N = args.partitions or pkv.default_partitions(local)
@@ -390,7 +392,7 @@ def run_pkv(args):
         if w.nnz_new and fp8:
             pkv.paged_kv_append_fp8(bt.pool, table, bt.k_new, bt.v_new, app, FP8_K_SCALE,
                                     FP8_V_SCALE, error_word=err,
-                                    stream=torch.cuda.current_stream(dev))
+                                    stream=torch.cuda.current_stream(dev), fp8_format=fp8)
         elif w.nnz_new:
             pkv.paged_kv_append(bt.pool, indptr, indices, last, bt.k_new, bt.v_new, app,
                                 error_word=err, stream=torch.cuda.current_stream(dev))
@@ -400,7 +402,7 @@ def run_pkv(args):
             pkv.paged_decode_attention_fp8(bt.q, bt.pool, table, ws, FP8_K_SCALE, FP8_V_SCALE,
                                            out=out, lse=lse, sm_scale=w.sm_scale,
                                            num_partitions=N, error_word=err,
-                                           stream=torch.cuda.current_stream(dev))
+                                           stream=torch.cuda.current_stream(dev), fp8_format=fp8)
             return
         if args.cascade:
             pkv.cascade_decode(bt.q, bt.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws, out=out,
@@ -494,11 +496,12 @@ def run_pkv(args):
             if fp8:
                 if w.nnz_new:
                     pkv.paged_kv_append_fp8(src.pool, e2e_table, k_d, v_d, ap_d, FP8_K_SCALE,
-                                            FP8_V_SCALE, error_word=err, stream=cur)
+                                            FP8_V_SCALE, error_word=err, stream=cur,
+                                            fp8_format=fp8)
                 pkv.paged_decode_attention_fp8(q_d, src.pool, e2e_table, ws, FP8_K_SCALE,
                                                FP8_V_SCALE, out=out_d, lse=lse_d,
                                                sm_scale=w.sm_scale, num_partitions=N,
-                                               error_word=err, stream=cur)
+                                               error_word=err, stream=cur, fp8_format=fp8)
             else:
                 if w.nnz_new:
                     pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d,
@@ -547,7 +550,7 @@ def run_pkv(args):
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": ("e4m3 KV widened to f16, f32 accumulate" if fp8 else
+            "dtype": (f"{fp8} KV widened to f16, f32 accumulate" if fp8 else
                       ("bf16" if w.dtype == "bf16" else "f16")), "data": "synthetic",
             "config": {**workload_config(w, args, rotation, N),
                        "launch": "direct calls" if args.no_graph else
@@ -559,7 +562,7 @@ def run_pkv(args):
             "roofline": {"bound": "hbm",
                          "kernel": ("pkv_cascade_decode (prefix + own-page decode + merge launches)"
                                     if args.cascade else
-                                    ("decode_kernel (E4M3 pool)" if fp8 else "decode_kernel")),
+                                    (f"decode_kernel ({fp8} pool)" if fp8 else "decode_kernel")),
                          "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"

@@ -71,7 +71,8 @@ typedef enum pkv_dtype {
   PKV_F16 = 0,
   PKV_BF16 = 1,
   PKV_F32 = 2,               /* only as the output type of pkv_merge_states */
-  PKV_FP8_E4M3 = 3           /* only as a pool type, with pkv_decode_fp8 / pkv_append_fp8 */
+  PKV_FP8_E4M3 = 3,          /* only as a pool type, with pkv_decode_fp8 / pkv_append_fp8 */
+  PKV_FP8_E5M2 = 4           /* likewise */
 } pkv_dtype;
 
 /* Pool layouts (the simple calls use HND). */
@@ -224,18 +225,22 @@ PKV_API pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc
                                  int32_t* error_word, void* stream);
 
 /*
- * pkv_decode_fp8 / pkv_append_fp8 -- the 8-bit KV cache: a pool of FP8 E4M3
- * codes ("fp8_e4m3" KV-cache dtype of the serving configurations in
- * "上下文窗口优化实战：如何用PagedAttention+FlashInfer将Llama3-70B的128K上下文
- * 吞吐提升3.8倍？" section 4.1), half the bytes of a 16-bit pool.
+ * pkv_decode_fp8 / pkv_append_fp8 -- the 8-bit KV cache: a pool of FP8 codes
+ * ("fp8_e4m3" KV-cache dtype of the serving configurations in "上下文窗口优化
+ * 实战：如何用PagedAttention+FlashInfer将Llama3-70B的128K上下文吞吐提升3.8倍？"
+ * section 4.1; "fp8_e5m2" in "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token
+ * 推理的生产级部署" sections 3.1 and 3.2), half the bytes of a 16-bit pool.
  *
  * E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits, subnormals,
- * no infinity, codes 0x7f / 0xff are NaN; largest finite magnitude 448.  One
- * binary32 scale for all keys and one for all values: a key element is
- * value(code) * k_scale, a value element value(code) * v_scale.
+ * no infinity, codes 0x7f / 0xff are NaN; largest finite magnitude 448.
+ * E5M2: the top byte of an IEEE half (bias 15, 2 fraction bits, infinities
+ * and NaNs); largest finite magnitude 57344.  One binary32 scale for all keys
+ * and one for all values: a key element is value(code) * k_scale, a value
+ * element value(code) * v_scale.
  *
- *   pool       descriptor with dtype PKV_FP8_E4M3 (either layout; head_dim 128
- *              for the decode, a multiple of 8 for the append); element bytes
+ *   pool       descriptor with dtype PKV_FP8_E4M3 or PKV_FP8_E5M2 (either
+ *              layout; head_dim 128 for the decode, a multiple of 8 for the
+ *              append); element bytes
  *   k_scale, v_scale  finite and > 0, else PKV_ERR_INVALID_ARG
  *   q_dtype    PKV_F16 or PKV_BF16: the type of q and out (decode)
  *   new_dtype  PKV_F16 or PKV_BF16: the type of k_new / v_new (append)
@@ -243,10 +248,11 @@ PKV_API pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc
  * pkv_decode_fp8 computes what pkv_decode_ex computes on the widened keys and
  * values (same table forms, workspace, out / lse and error behaviour).
  * pkv_append_fp8 scatters like pkv_append_ex and stores each new element x
- * as e4m3(float(x) / scale): the quotient rounded to binary32, then to the
- * nearest E4M3 value, ties to even, magnitudes past 448 saturating to +-448.
- * The _ex calls reject E4M3 pools (they carry no scales); pkv_cascade_decode
- * takes 16-bit pools only.
+ * as fp8(float(x) / scale): the quotient rounded to binary32, then to the
+ * nearest finite value of the format, ties to even, larger magnitudes
+ * (infinity included) saturating to +-448 (E4M3) or +-57344 (E5M2).  The _ex
+ * calls reject 8-bit pools (they carry no scales); pkv_cascade_decode and
+ * pkv_append_attention take 16-bit pools only.
  */
 PKV_API pkv_status pkv_decode_fp8(const void* q, int q_dtype, int num_qo_heads,
                                   const pkv_pool_desc* pool, float k_scale, float v_scale,

@@ -20,7 +20,7 @@ Functions (C names in parentheses):
   paged_decode_attention_ex / paged_kv_append_ex (pkv_decode_ex / pkv_append_ex)
                          NHD pools and dense (vLLM-style) block tables
   paged_decode_attention_fp8 / paged_kv_append_fp8 (pkv_decode_fp8 / pkv_append_fp8)
-                         the 8-bit (FP8 E4M3) KV cache with per-tensor K / V scales
+                         the 8-bit (FP8 E4M3 / E5M2) KV cache with per-tensor K / V scales
   append_attention       (pkv_append_attention)  a chunk of query tokens per request,
                          causal over its cache (chunked prefill, speculative tokens)
   append_attention_plan  (pkv_append_attention_plan)  its host-side row-block plan
@@ -33,6 +33,7 @@ from ._binding import (  # noqa: F401
     F16,
     F32,
     FP8_E4M3,
+    FP8_E5M2,
     PkvError,
     PoolDesc,
     TableDesc,

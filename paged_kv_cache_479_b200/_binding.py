@@ -8,7 +8,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-F16, BF16, F32, FP8_E4M3 = 0, 1, 2, 3
+F16, BF16, F32, FP8_E4M3, FP8_E5M2 = 0, 1, 2, 3, 4
 DEVERR_PAGE_ID = 0x01
 DEVERR_INDPTR = 0x02
 DEVERR_LAST_LEN = 0x04
@@ -113,7 +113,7 @@ def _check(status: int, what: str):
 
 
 _DTYPES = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32,
-           torch.uint8: FP8_E4M3, torch.float8_e4m3fn: FP8_E4M3}
+           torch.uint8: FP8_E4M3, torch.float8_e4m3fn: FP8_E4M3, torch.float8_e5m2: FP8_E5M2}
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -334,23 +334,30 @@ def paged_kv_append_ex(pool, table: TableDesc, k_new, v_new, append_indptr, layo
     _check(st, "pkv_append_ex")
 
 
-def _fp8_pool(pool, layout):
-    if pool.dtype not in (torch.uint8, torch.float8_e4m3fn):
-        raise ValueError("an E4M3 pool must be a uint8 or float8_e4m3fn tensor")
-    return pool_desc(pool, layout)
+def _fp8_pool(pool, layout, fmt):
+    """Descriptor of an 8-bit pool: a float8_e4m3fn / float8_e5m2 tensor, or uint8
+    codes of the format `fmt` ("e4m3" or "e5m2")."""
+    if pool.dtype not in (torch.uint8, torch.float8_e4m3fn, torch.float8_e5m2):
+        raise ValueError("an 8-bit pool must be a uint8, float8_e4m3fn or float8_e5m2 tensor")
+    pd = pool_desc(pool, layout)
+    if pool.dtype == torch.uint8:
+        if fmt not in ("e4m3", "e5m2"):
+            raise ValueError("fp8_format must be 'e4m3' or 'e5m2'")
+        pd.dtype = FP8_E4M3 if fmt == "e4m3" else FP8_E5M2
+    return pd
 
 
 def paged_decode_attention_fp8(q, pool, table: TableDesc, workspace, k_scale: float,
                                v_scale: float, layout: str = "HND", out=None, lse=None,
                                sm_scale=None, num_partitions: int = 0, error_word=None,
-                               stream=None, return_lse: bool = True):
-    """pkv_decode_fp8: decode over an E4M3 pool (key = code * k_scale, value = code * v_scale);
+                               stream=None, return_lse: bool = True, fp8_format: str = "e4m3"):
+    """pkv_decode_fp8: decode over an 8-bit pool (key = code * k_scale, value = code * v_scale);
     q and out are fp16 or bf16."""
     _dev_tensor(q, "q")
     if q.dtype not in (torch.float16, torch.bfloat16):
         raise ValueError("q must be fp16 or bf16")
     _dev_tensor(workspace, "workspace")
-    pd = _fp8_pool(pool, layout)
+    pd = _fp8_pool(pool, layout, fp8_format)
     B, hq, d = q.shape
     if out is None:
         out = torch.empty_like(q)
@@ -367,9 +374,9 @@ def paged_decode_attention_fp8(q, pool, table: TableDesc, workspace, k_scale: fl
 
 def paged_kv_append_fp8(pool, table: TableDesc, k_new, v_new, append_indptr, k_scale: float,
                         v_scale: float, layout: str = "HND", error_word=None,
-                        stream=None) -> None:
-    """pkv_append_fp8: quantise fp16/bf16 rows into an E4M3 pool (x -> e4m3(x / scale))."""
-    pd = _fp8_pool(pool, layout)
+                        stream=None, fp8_format: str = "e4m3") -> None:
+    """pkv_append_fp8: quantise fp16/bf16 rows into an 8-bit pool (x -> fp8(x / scale))."""
+    pd = _fp8_pool(pool, layout, fp8_format)
     _dev_tensor(k_new, "k_new")
     _dev_tensor(v_new, "v_new", k_new.dtype)
     if k_new.dtype not in (torch.float16, torch.bfloat16):

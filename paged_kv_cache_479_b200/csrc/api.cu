@@ -39,6 +39,8 @@ pkv_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
 
+bool is_fp8(int dtype) { return dtype == PKV_FP8_E4M3 || dtype == PKV_FP8_E5M2; }
+
 bool valid_page_size(int ps) { return ps == 16 || ps == 32 || ps == 64 || ps == 128 || ps == 256; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -122,8 +124,8 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
   }
   auto encode = get_encode();
   if (!encode) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  if (dtype == PKV_FP8_E4M3) {
-    // E4M3 pool: 4-D view (byte of the row, slot, kv head, 2 page + K/V) with
+  if (is_fp8(dtype)) {
+    // 8-bit pool: 4-D view (byte of the row, slot, kv head, 2 page + K/V) with
     // [2][16 slots][128 bytes] boxes -- one load brings a tile's K and V
     const bool nhd = layout == PKV_LAYOUT_NHD;
     const cuuint64_t row = kDecodeHeadDim;  // one token's K (or V) row: 128 bytes
@@ -138,7 +140,7 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r8 != CUDA_SUCCESS)
-      return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed for the E4M3 pool (%d)", (int)r8);
+      return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed for the 8-bit pool (%d)", (int)r8);
     std::lock_guard<std::mutex> lk(mu);
     keys[next] = key;
     maps[next] = m8;
@@ -206,8 +208,8 @@ pkv_status pkv::set_error(pkv_status s, const char* fmt, ...) {
   return s;
 }
 
-// dtype: type of q and out; kv_dtype: the pool's (dtype, or PKV_FP8_E4M3 with
-// k_scale / v_scale)
+// dtype: type of q and out; kv_dtype: the pool's (dtype, or PKV_FP8_E4M3 /
+// PKV_FP8_E5M2 with k_scale / v_scale)
 static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool, int64_t num_pages,
                       int page_size, int num_kv_heads, int head_dim, int dtype, int layout,
                       const pkv::TableView& tv, const int32_t* page_ids, int batch, float sm_scale,
@@ -220,9 +222,9 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
     return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
   if (dtype != PKV_F16 && dtype != PKV_BF16)
     return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
-  if (kv_dtype != dtype && kv_dtype != PKV_FP8_E4M3)
-    return fail(PKV_ERR_INVALID_ARG, "the pool must hold q's type or PKV_FP8_E4M3 codes");
-  if (kv_dtype == PKV_FP8_E4M3 &&
+  if (kv_dtype != dtype && !is_fp8(kv_dtype))
+    return fail(PKV_ERR_INVALID_ARG, "the pool must hold q's type or 8-bit (E4M3 / E5M2) codes");
+  if (is_fp8(kv_dtype) &&
       !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
     return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
   if (num_qo_heads % num_kv_heads != 0)
@@ -276,7 +278,7 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.hkv = num_kv_heads;
   a.group = group;
   a.page_size = page_size;
-  const bool fp8 = kv_dtype == PKV_FP8_E4M3;
+  const bool fp8 = is_fp8(kv_dtype);
   a.scale_log2 = (float)((double)sm_scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   a.v_scale = fp8 ? v_scale : 1.f;
   a.one_box = one_box;
@@ -284,13 +286,16 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.out_rs = out_rs;
   a.lse_rs = lse_rs;
   cudaError_t e =
-      pkv::launch_decode(tmap, a, dtype == PKV_BF16, fp8, N, static_cast<cudaStream_t>(stream));
+      pkv::launch_decode(tmap, a, dtype == PKV_BF16,
+                         kv_dtype == PKV_FP8_E4M3 ? pkv::kKvE4M3
+                         : kv_dtype == PKV_FP8_E5M2 ? pkv::kKvE5M2 : pkv::kKv16,
+                         N, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }
 
-// dtype: type of k_new / v_new; kv_dtype: the pool's (dtype, or PKV_FP8_E4M3:
-// the rows are quantised with k_scale / v_scale)
+// dtype: type of k_new / v_new; kv_dtype: the pool's (dtype, or an 8-bit
+// type: the rows are quantised with k_scale / v_scale)
 static pkv_status append_impl(void* pool, int64_t num_pages, int page_size, int num_kv_heads,
                               int head_dim, int dtype, int layout, const pkv::TableView& tv,
                               const int32_t* page_ids, int batch, const void* k_new,
@@ -302,9 +307,9 @@ static pkv_status append_impl(void* pool, int64_t num_pages, int page_size, int 
     return fail(PKV_ERR_INVALID_ARG, "negative or zero size");
   if (dtype != PKV_F16 && dtype != PKV_BF16)
     return fail(PKV_ERR_INVALID_ARG, "dtype must be PKV_F16 or PKV_BF16");
-  if (kv_dtype != dtype && kv_dtype != PKV_FP8_E4M3)
-    return fail(PKV_ERR_INVALID_ARG, "the pool must hold the rows' type or PKV_FP8_E4M3 codes");
-  if (kv_dtype == PKV_FP8_E4M3 &&
+  if (kv_dtype != dtype && !is_fp8(kv_dtype))
+    return fail(PKV_ERR_INVALID_ARG, "the pool must hold the rows' type or 8-bit codes");
+  if (is_fp8(kv_dtype) &&
       !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
     return fail(PKV_ERR_INVALID_ARG, "k_scale and v_scale must be finite and positive");
   if (layout != PKV_LAYOUT_HND && layout != PKV_LAYOUT_NHD)
@@ -334,7 +339,7 @@ static pkv_status append_impl(void* pool, int64_t num_pages, int page_size, int 
   a.head_dim = head_dim;
   a.page_size = page_size;
   a.layout = layout;
-  a.fp8 = kv_dtype == PKV_FP8_E4M3;
+  a.fp8 = kv_dtype == PKV_FP8_E4M3 ? pkv::kKvE4M3 : kv_dtype == PKV_FP8_E5M2 ? pkv::kKvE5M2 : 0;
   a.in_bf16 = dtype == PKV_BF16;
   a.k_scale = k_scale;
   a.v_scale = v_scale;
@@ -517,8 +522,8 @@ pkv_status pkv_decode_ex(const void* q, int num_qo_heads, const pkv_pool_desc* p
   const int32_t* ids = nullptr;
   pkv_status st = table_view(table, &tv, &ids);
   if (st != PKV_OK) return st;
-  if (pool->dtype == PKV_FP8_E4M3)
-    return fail(PKV_ERR_INVALID_ARG, "an E4M3 pool needs pkv_decode_fp8 (it carries the scales)");
+  if (is_fp8(pool->dtype))
+    return fail(PKV_ERR_INVALID_ARG, "an 8-bit pool needs pkv_decode_fp8 (it carries the scales)");
   return decode_impl(q, num_qo_heads, pool->data, pool->num_pages, pool->page_size,
                      pool->num_kv_heads, pool->head_dim, pool->dtype, pool->layout, tv, ids,
                      table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
@@ -534,8 +539,8 @@ pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc* table,
   const int32_t* ids = nullptr;
   pkv_status st = table_view(table, &tv, &ids);
   if (st != PKV_OK) return st;
-  if (pool->dtype == PKV_FP8_E4M3)
-    return fail(PKV_ERR_INVALID_ARG, "an E4M3 pool needs pkv_append_fp8 (it carries the scales)");
+  if (is_fp8(pool->dtype))
+    return fail(PKV_ERR_INVALID_ARG, "an 8-bit pool needs pkv_append_fp8 (it carries the scales)");
   return append_impl(pool->data, pool->num_pages, pool->page_size, pool->num_kv_heads,
                      pool->head_dim, pool->dtype, pool->layout, tv, ids, table->batch, k_new,
                      v_new, append_indptr, nnz_new, error_word, stream);
@@ -547,7 +552,8 @@ pkv_status pkv_decode_fp8(const void* q, int q_dtype, int num_qo_heads, const pk
                           size_t workspace_bytes, void* out, float* lse, int32_t* error_word,
                           void* stream) {
   if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
-  if (pool->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_FP8_E4M3");
+  if (!is_fp8(pool->dtype))
+    return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_FP8_E4M3 or PKV_FP8_E5M2");
   pkv::TableView tv;
   const int32_t* ids = nullptr;
   pkv_status st = table_view(table, &tv, &ids);
@@ -556,7 +562,7 @@ pkv_status pkv_decode_fp8(const void* q, int q_dtype, int num_qo_heads, const pk
                      pool->num_kv_heads, pool->head_dim, q_dtype, pool->layout, tv, ids,
                      table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
                      error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
-                     num_qo_heads, PKV_FP8_E4M3, k_scale, v_scale);
+                     num_qo_heads, pool->dtype, k_scale, v_scale);
 }
 
 pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, float v_scale,
@@ -564,14 +570,15 @@ pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, float v_scal
                           int new_dtype, const int32_t* append_indptr, int64_t nnz_new,
                           int32_t* error_word, void* stream) {
   if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
-  if (pool->dtype != PKV_FP8_E4M3) return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_FP8_E4M3");
+  if (!is_fp8(pool->dtype))
+    return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_FP8_E4M3 or PKV_FP8_E5M2");
   pkv::TableView tv;
   const int32_t* ids = nullptr;
   pkv_status st = table_view(table, &tv, &ids);
   if (st != PKV_OK) return st;
   return append_impl(pool->data, pool->num_pages, pool->page_size, pool->num_kv_heads,
                      pool->head_dim, new_dtype, pool->layout, tv, ids, table->batch, k_new, v_new,
-                     append_indptr, nnz_new, error_word, stream, PKV_FP8_E4M3, k_scale, v_scale);
+                     append_indptr, nnz_new, error_word, stream, pool->dtype, k_scale, v_scale);
 }
 
 }  // extern "C"

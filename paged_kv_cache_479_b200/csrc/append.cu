@@ -9,10 +9,10 @@
 // page_indices[indptr[b] + pos / page_size], slot pos % page_size -- the O(1)
 // translation of "Flash Attention与Paged KV Cache优化大模型推理实战" section 3.2.
 // The K row and the V row are copied with 16-byte vector loads and stores;
-// the pool ends up bit-identical to a byte-wise scatter.  Into an E4M3 pool
-// each element x is stored as e4m3(x / scale) instead (binary32 division,
-// then round to nearest even with saturation at +-448): 8 elements per lane,
-// 16 bytes in, 8 bytes out.
+// the pool ends up bit-identical to a byte-wise scatter.  Into an 8-bit pool
+// each element x is stored as fp8(x / scale) instead (binary32 division, then
+// round to nearest even with saturation at the format's largest finite value,
+// 448 for E4M3 and 57344 for E5M2): 8 elements per lane, 16 bytes in, 8 out.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(kWarps * 32) append_kernel(const AppendArgs a)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const float2 f = a.in_bf16 ? unpack2<true>(w[j]) : unpack2<false>(w[j]);
-            c[j] = f32x2_to_e4m3x2(__fdiv_rn(f.x, sc), __fdiv_rn(f.y, sc));
+            const float x0 = __fdiv_rn(f.x, sc), x1 = __fdiv_rn(f.y, sc);
+            c[j] = a.fp8 == kKvE5M2 ? f32x2_to_e5m2x2(x0, x1) : f32x2_to_e4m3x2(x0, x1);
           }
           *reinterpret_cast<uint2*>(pool8 + (is_v ? dv : dk) + x) =
               make_uint2((uint32_t)c[0] | ((uint32_t)c[1] << 16), (uint32_t)c[2] | ((uint32_t)c[3] << 16));

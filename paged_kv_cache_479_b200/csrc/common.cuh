@@ -228,6 +228,14 @@ __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// two fp32 values (lo -> low byte) rounded to nearest even E5M2, saturating
+// at +-57344 (satfinite); NaN stays NaN
+__device__ __forceinline__ uint16_t f32x2_to_e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // 2^x, PTX ex2.approx (relative error about 2^-22); ex2(-inf) = +0
 __device__ __forceinline__ float ex2(float x) {
   float y;

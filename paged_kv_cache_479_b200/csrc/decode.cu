@@ -188,10 +188,26 @@ __device__ __forceinline__ bool cons_sync(Ctl& ctl, uint32_t& phase, int* err) {
   return ok;
 }
 
-template <bool BF16, bool FP8>
+// two 8-bit codes (bytes 0-1, or 2-3, of r) widened exactly to an fp16 pair:
+// E4M3 by conversion, E5M2 (the top byte of a half) by placing each code in
+// the high byte of its lane
+template <int KV>
+__device__ __forceinline__ uint32_t widen_lo(uint32_t r) {
+  if constexpr (KV == kKvE4M3) return e4m3x2_to_f16x2((uint16_t)r);
+  else return prmt(r, 0u, 0x1404u);
+}
+template <int KV>
+__device__ __forceinline__ uint32_t widen_hi(uint32_t r) {
+  if constexpr (KV == kKvE4M3) return e4m3x2_to_f16x2((uint16_t)(r >> 16));
+  else return prmt(r, 0u, 0x3424u);
+}
+
+// KV: the pool's element type -- kKv16 (q's own 16-bit type), kKvE4M3, kKvE5M2
+template <bool BF16, int KV>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
-  // ring geometry of this KV type (16-bit: 16 slots of 8 KiB; E4M3: 32 of 4 KiB)
+  constexpr bool FP8 = KV != kKv16;
+  // ring geometry of this KV type (16-bit: 16 slots of 8 KiB; 8-bit: 32 of 4 KiB)
   constexpr int kSt = FP8 ? 2 * kStages : kStages;
   constexpr int kTileB = FP8 ? kTileBytes / 2 : kTileBytes;
   constexpr int kSlotB = 2 * kTileB;
@@ -586,12 +602,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           const int chunk = 2 * jj + (mi >> 1);
           uint32_t r0, r1, r2, r3;
           ldmatrix_x4(rowb + (uint32_t)(((chunk & 7) ^ r8) << 4), r0, r1, r2, r3);
-          mma_16816<false>(sa, e4m3x2_to_f16x2((uint16_t)r0), e4m3x2_to_f16x2((uint16_t)r1),
-                           e4m3x2_to_f16x2((uint16_t)(r0 >> 16)), e4m3x2_to_f16x2((uint16_t)(r1 >> 16)),
-                           qf[2 * jj][0], qf[2 * jj][1]);
-          mma_16816<false>(sb, e4m3x2_to_f16x2((uint16_t)r2), e4m3x2_to_f16x2((uint16_t)r3),
-                           e4m3x2_to_f16x2((uint16_t)(r2 >> 16)), e4m3x2_to_f16x2((uint16_t)(r3 >> 16)),
-                           qf[2 * jj + 1][0], qf[2 * jj + 1][1]);
+          mma_16816<false>(sa, widen_lo<KV>(r0), widen_lo<KV>(r1), widen_hi<KV>(r0),
+                           widen_hi<KV>(r1), qf[2 * jj][0], qf[2 * jj][1]);
+          mma_16816<false>(sb, widen_lo<KV>(r2), widen_lo<KV>(r3), widen_hi<KV>(r2),
+                           widen_hi<KV>(r3), qf[2 * jj + 1][0], qf[2 * jj + 1][1]);
         }
       } else {
         const int tok = ((mi & 1) << 3) + r8;
@@ -679,15 +693,21 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           const int chunk = 2 * jj + (mi & 1);
           uint32_t r0, r1, r2, r3;
           ldmatrix_x4_trans(rowb + (uint32_t)(((chunk & 7) ^ r8) << 4), r0, r1, r2, r3);
-          r0 = prmt(r0, 0u, 0x3120u);
-          r1 = prmt(r1, 0u, 0x3120u);
-          r2 = prmt(r2, 0u, 0x3120u);
-          r3 = prmt(r3, 0u, 0x3120u);
-          mma_16816<false>(o[2 * jj], e4m3x2_to_f16x2((uint16_t)r0), e4m3x2_to_f16x2((uint16_t)r1),
-                           e4m3x2_to_f16x2((uint16_t)r2), e4m3x2_to_f16x2((uint16_t)r3), bh0, bh1);
-          mma_16816<false>(o[2 * jj + 1], e4m3x2_to_f16x2((uint16_t)(r0 >> 16)),
-                           e4m3x2_to_f16x2((uint16_t)(r1 >> 16)), e4m3x2_to_f16x2((uint16_t)(r2 >> 16)),
-                           e4m3x2_to_f16x2((uint16_t)(r3 >> 16)), bh0, bh1);
+          uint32_t x[4], y[4];  // dim 2g (x) and 2g+1 (y), tokens 2cq and 2cq+1
+          const uint32_t rr[4] = {r0, r1, r2, r3};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (KV == kKvE4M3) {
+              const uint32_t p = prmt(rr[k], 0u, 0x3120u);
+              x[k] = widen_lo<KV>(p);
+              y[k] = widen_hi<KV>(p);
+            } else {  // E5M2: pair and widen in one byte permute each
+              x[k] = prmt(rr[k], 0u, 0x2404u);
+              y[k] = prmt(rr[k], 0u, 0x3414u);
+            }
+          }
+          mma_16816<false>(o[2 * jj], x[0], x[1], x[2], x[3], bh0, bh1);
+          mma_16816<false>(o[2 * jj + 1], y[0], y[1], y[2], y[3], bh0, bh1);
         }
       } else {
         const int tok = ((mi >> 1) << 3) + r8;
@@ -831,14 +851,17 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 
 size_t decode_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, bool fp8,
+cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv,
                           int grid, cudaStream_t stream) {
   static_assert(sizeof(Ctl) % 16 == 0, "Ctl must keep Scratch 16-byte aligned");
-  const int variant = (fp8 ? 2 : 0) + (bf16 ? 1 : 0);
-  auto kern = fp8 ? (bf16 ? decode_kernel<true, true> : decode_kernel<false, true>)
-                  : (bf16 ? decode_kernel<true, false> : decode_kernel<false, false>);
+  if (kv != kKv16 && kv != kKvE4M3 && kv != kKvE5M2) return cudaErrorInvalidValue;
+  const int variant = 2 * kv + (bf16 ? 1 : 0);
+  void (*kern)(const CUtensorMap, const DecodeArgs) =
+      kv == kKvE4M3 ? (bf16 ? decode_kernel<true, kKvE4M3> : decode_kernel<false, kKvE4M3>)
+      : kv == kKvE5M2 ? (bf16 ? decode_kernel<true, kKvE5M2> : decode_kernel<false, kKvE5M2>)
+                      : (bf16 ? decode_kernel<true, kKv16> : decode_kernel<false, kKv16>);
   // the shared-memory opt-in is per function and device; do it once each
-  static bool attr_set[4][64] = {};
+  static bool attr_set[6][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

@@ -26,7 +26,7 @@ struct DecodeArgs {
   long long num_pages;
   int batch, hq, hkv, group, page_size;
   float scale_log2;       // sm_scale * log2(e) (* k_scale for an E4M3 pool)
-  float v_scale;          // E4M3 pool: value of a V code = code value * v_scale
+  float v_scale;          // 8-bit pool: value of a V code = code value * v_scale
   int one_box;            // 1: 5-D tensor map, one box per K/V tile; 0: 4-D map, two boxes
   int out_f32;            // 1: out is fp32 (an attention state for a later merge)
   long long out_rs;       // elements of out between consecutive requests (Hq * 128 when packed)
@@ -44,8 +44,12 @@ constexpr int kDecodeStages = PKV_STAGES;        // K/V ring slots (8 KiB each) 
 constexpr int kDecodeCtasPerSm = PKV_CTAS_PER_SM; // resident decode CTAs per SM
 
 size_t decode_smem_bytes();
-// bf16: q/out type (else fp16); fp8: the pool holds E4M3 codes (else q's type)
-cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, bool fp8,
+// pool element types of the decode kernel
+constexpr int kKv16 = 0;    // q's own 16-bit type
+constexpr int kKvE4M3 = 1;  // FP8 E4M3 codes
+constexpr int kKvE5M2 = 2;  // FP8 E5M2 codes
+// bf16: q/out type (else fp16); kv: one of the pool element types above
+cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv,
                           int grid, cudaStream_t stream);
 
 // attention of every request's queries over one shared prefix (prefix.cu)
@@ -104,7 +108,7 @@ struct AppendArgs {
   long long nnz;
   int batch, hkv, head_dim, page_size;
   int layout;  // PKV_LAYOUT_HND or PKV_LAYOUT_NHD
-  int fp8;     // 1: the pool holds E4M3 codes; rows are quantised as e4m3(x / scale)
+  int fp8;     // kKvE4M3 / kKvE5M2: rows are quantised as fp8(x / scale); 0: 16-bit copy
   int in_bf16; // fp8 only: k_new / v_new are bf16 (else fp16)
   float k_scale, v_scale;
 };

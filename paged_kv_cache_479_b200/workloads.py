@@ -311,8 +311,9 @@ def make_tensors(w: Workload, device="cpu"):
 # 8-bit (E4M3) pools
 # --------------------------------------------------------------------------
 
-FP8_CANARY = 0x7F  # an E4M3 NaN code: fills every slot that holds no token
+FP8_CANARY = 0x7F  # NaN in E4M3 and in E5M2: fills every slot that holds no token
 FP8_EXP_MEAN = 11  # exponent field of a typical code: magnitude 2^(11-7) = 16
+FP8_E5M2_EXP_MEAN = 19  # the same magnitude in E5M2: 2^(19-15) = 16
 
 
 def e4m3_codes(shape, gen, device, exp_mean=FP8_EXP_MEAN, exp_std=1.25):
@@ -329,10 +330,24 @@ def e4m3_codes(shape, gen, device, exp_mean=FP8_EXP_MEAN, exp_std=1.25):
     return code.to(torch.uint8)
 
 
-def make_fp8_tensors(w: Workload, device="cpu"):
+def e5m2_codes(shape, gen, device, exp_mean=FP8_E5M2_EXP_MEAN, exp_std=1.25):
+    """Random E5M2 codes assembled field by field: sign uniform, exponent field
+    round(N(exp_mean, exp_std)) clipped to [0, 23] (0 gives subnormals; the
+    largest magnitude is 448, the E4M3 range, so both formats give values of
+    the same spread -- the far exponents up to 30 stay reachable through the
+    append's quantisation), fraction uniform."""
+    sign = torch.randint(0, 2, shape, generator=gen, device=device, dtype=torch.int32)
+    e = torch.randn(shape, generator=gen, device=device) * exp_std + exp_mean
+    e = e.round().clamp(0, 23).to(torch.int32)
+    m = torch.randint(0, 4, shape, generator=gen, device=device, dtype=torch.int32)
+    return ((sign << 7) | (e << 2) | m).to(torch.uint8)
+
+
+def make_fp8_tensors(w: Workload, device="cpu", fmt="e4m3"):
     """q [B,Hq,D] and new rows [nnz,Hkv,D] in the workload's 16-bit dtype, and
-    an E4M3 pool [P,2,Hkv,ps,D] (uint8 codes; state before the append) whose
-    slots that hold no token carry FP8_CANARY."""
+    an 8-bit pool [P,2,Hkv,ps,D] (uint8 codes of the format; state before the
+    append) whose slots that hold no token carry FP8_CANARY (a NaN code of both
+    formats)."""
     device = torch.device(device)
     gen = torch.Generator(device=device)
     gen.manual_seed(int(w.seed) + 8)
@@ -343,7 +358,8 @@ def make_fp8_tensors(w: Workload, device="cpu"):
     chunk = max(1, (1 << 26) // (2 * w.num_kv_heads * w.page_size * w.head_dim))
     for p0 in range(0, w.num_pages, chunk):
         p1 = min(w.num_pages, p0 + chunk)
-        pool[p0:p1] = e4m3_codes((p1 - p0,) + tuple(w.pool_shape[1:]), gen, device)
+        draw = e4m3_codes if fmt == "e4m3" else e5m2_codes
+        pool[p0:p1] = draw((p1 - p0,) + tuple(w.pool_shape[1:]), gen, device)
     k_new = torch.randn((w.nnz_new, w.num_kv_heads, w.head_dim), generator=gen,
                         device=device).to(dt)
     v_new = torch.randn((w.nnz_new, w.num_kv_heads, w.head_dim), generator=gen,

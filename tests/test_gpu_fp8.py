@@ -1,6 +1,6 @@
-"""GPU parity of the 8-bit (FP8 E4M3) KV cache: pkv_decode_fp8 against the
-oracle's decode over the same codes and scales, and pkv_append_fp8 bit for
-bit against the oracle's quantising scatter."""
+"""GPU parity of the 8-bit (FP8 E4M3 and E5M2) KV cache: pkv_decode_fp8
+against the oracle's decode over the same codes and scales, and
+pkv_append_fp8 bit for bit against the oracle's quantising scatter."""
 import numpy as np
 import pytest
 import torch
@@ -47,20 +47,20 @@ def to_layout(pool, layout):
     return pool.permute(0, 1, 3, 2, 4).contiguous() if layout == "NHD" else pool
 
 
-def fp8_decode(w, q, pool, layout="HND", kind="csr", ks=K_SCALE, vs=V_SCALE, n=0):
+def fp8_decode(w, q, pool, layout="HND", kind="csr", ks=K_SCALE, vs=V_SCALE, n=0, fmt="e4m3"):
     table, keep = table_of(w, kind)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, lse = pkv.paged_decode_attention_fp8(q, to_layout(pool, layout), table, workspace(w, n),
                                               ks, vs, layout=layout, sm_scale=w.sm_scale,
-                                              num_partitions=n, error_word=err)
+                                              num_partitions=n, error_word=err, fp8_format=fmt)
     torch.cuda.synchronize()
     assert pkv.read_error_word(err) == 0
     return out, lse
 
 
-def oracle_fp8(w, q, pool, ks=K_SCALE, vs=V_SCALE):
+def oracle_fp8(w, q, pool, ks=K_SCALE, vs=V_SCALE, fmt="e4m3"):
     return oracle.decode_fp8(wl.bits(q), odtype(w), pool.cpu().numpy(), ks, vs, w.page_indptr,
-                             w.page_indices, w.last_page_len, w.sm_scale)
+                             w.page_indices, w.last_page_len, w.sm_scale, fmt)
 
 
 CASES = [
@@ -73,15 +73,16 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
 @pytest.mark.parametrize("i", range(len(CASES)))
-def test_fp8_decode_matches_oracle(i):
+def test_fp8_decode_matches_oracle(i, fmt):
     lens, hq, hkv, ps, dt = CASES[i]
     w = wl.make_workload("fp8", lens, num_qo_heads=hq, num_kv_heads=hkv, page_size=ps, dtype=dt,
                          seed=900 + i, pool_factor=1.3)
-    q, pool, _, _ = wl.make_fp8_tensors(w, "cpu")
-    out, lse = fp8_decode(w, q.cuda(), pool.cuda())
-    ro, rl = oracle_fp8(w, q, pool)
-    assert_parity(out, lse, ro, rl, what=f"fp8 case {i}")
+    q, pool, _, _ = wl.make_fp8_tensors(w, "cpu", fmt)
+    out, lse = fp8_decode(w, q.cuda(), pool.cuda(), fmt=fmt)
+    ro, rl = oracle_fp8(w, q, pool, fmt=fmt)
+    assert_parity(out, lse, ro, rl, what=f"{fmt} case {i}")
 
 
 @pytest.mark.parametrize("layout,kind", [("HND", "block"), ("NHD", "csr"), ("NHD", "block")])
@@ -106,6 +107,7 @@ def test_fp8_partition_counts(n):
 
 @pytest.mark.parametrize("n", [1, 3, 64])
 def test_fp8_many_short_segments(n):
+    fmt = "e5m2" if n == 3 else "e4m3"
     # hundreds of one-tile (request, kv head) segments per partition: the
     # producer runs many segments ahead of the consumers through the 32-slot
     # ring, so every staged query block and segment record is reused often
@@ -113,10 +115,10 @@ def test_fp8_many_short_segments(n):
     lens = rng.integers(0, 40, size=700)
     w = wl.make_workload("fp8tiny", lens, num_qo_heads=16, num_kv_heads=4, page_size=16,
                          dtype="bf16", seed=914, pool_factor=1.2)
-    q, pool, _, _ = wl.make_fp8_tensors(w, "cpu")
-    out, lse = fp8_decode(w, q.cuda(), pool.cuda(), n=n)
-    ro, rl = oracle_fp8(w, q, pool)
-    assert_parity(out, lse, ro, rl, what=f"fp8 tiny N={n}")
+    q, pool, _, _ = wl.make_fp8_tensors(w, "cpu", fmt)
+    out, lse = fp8_decode(w, q.cuda(), pool.cuda(), n=n, fmt=fmt)
+    ro, rl = oracle_fp8(w, q, pool, fmt=fmt)
+    assert_parity(out, lse, ro, rl, what=f"{fmt} tiny N={n}")
 
 
 def test_fp8_query_scaling_extremes():
@@ -146,47 +148,51 @@ def test_fp8_scales_are_exact_factors_on_the_gpu():
     assert torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
 @pytest.mark.parametrize("layout,kind", [("HND", "csr"), ("HND", "block"), ("NHD", "csr"),
                                          ("NHD", "block")])
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
-def test_fp8_append_bit_exact(layout, kind, dt):
+def test_fp8_append_bit_exact(layout, kind, dt, fmt):
     w = wl.make_workload("fp8a", [1, 15, 16, 17, 33, 300], num_qo_heads=8, num_kv_heads=4,
                          page_size=16, dtype=dt, seed=920, pool_factor=1.5,
                          append_counts=[1, 15, 1, 17, 2, 40])
-    _, pool, k_new, v_new = wl.make_fp8_tensors(w, "cpu")
+    _, pool, k_new, v_new = wl.make_fp8_tensors(w, "cpu", fmt)
     # spread the inputs so the scales reach saturation (K) and subnormals (V)
     k_new = (k_new.float() * 8).to(k_new.dtype)
     v_new = (v_new.float() * 0.002).to(v_new.dtype)
-    ks, vs = 0.015, 0.5
+    ks, vs = (0.015, 0.5) if fmt == "e4m3" else (2e-4, 64.0)
+    sat = 0x7E if fmt == "e4m3" else 0x7B
     expect = oracle.append_fp8(pool.numpy(), ks, vs, w.page_indptr, w.page_indices,
                                w.last_page_len, wl.bits(k_new), wl.bits(v_new), odtype(w),
-                               w.append_indptr)
-    assert (expect == 0x7E).any() and (expect == 0xFE).any()   # saturated codes occur
+                               w.append_indptr, fmt)
+    assert (expect == sat).any() and (expect == 0x80 | sat).any()   # saturated codes occur
     p = to_layout(pool.cuda(), layout)
     table, keep = table_of(w, kind)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     pkv.paged_kv_append_fp8(p, table, k_new.cuda(), v_new.cuda(), i32(w.append_indptr), ks, vs,
-                            layout=layout, error_word=err)
+                            layout=layout, error_word=err, fp8_format=fmt)
     torch.cuda.synchronize()
     assert pkv.read_error_word(err) == 0
     got = (p.permute(0, 1, 3, 2, 4) if layout == "NHD" else p).contiguous().cpu().numpy()
     assert np.array_equal(got, expect)
 
 
-def test_fp8_append_then_decode_step():
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_fp8_append_then_decode_step(fmt):
     w = wl.named(2)
-    q, pool, k_new, v_new = wl.make_fp8_tensors(w, "cpu")
+    q, pool, k_new, v_new = wl.make_fp8_tensors(w, "cpu", fmt)
     ks, vs = K_SCALE, V_SCALE
     after = oracle.append_fp8(pool.numpy(), ks, vs, w.page_indptr, w.page_indices,
                               w.last_page_len, wl.bits(k_new), wl.bits(v_new), odtype(w),
-                              w.append_indptr)
+                              w.append_indptr, fmt)
     p = pool.cuda()
     table, keep = table_of(w, "csr")
-    pkv.paged_kv_append_fp8(p, table, k_new.cuda(), v_new.cuda(), i32(w.append_indptr), ks, vs)
-    out, lse = fp8_decode(w, q.cuda(), p)
+    pkv.paged_kv_append_fp8(p, table, k_new.cuda(), v_new.cuda(), i32(w.append_indptr), ks, vs,
+                            fp8_format=fmt)
+    out, lse = fp8_decode(w, q.cuda(), p, fmt=fmt)
     assert np.array_equal(p.cpu().numpy(), after)
     ro, rl = oracle.decode_fp8(wl.bits(q), odtype(w), after, ks, vs, w.page_indptr,
-                               w.page_indices, w.last_page_len, w.sm_scale)
+                               w.page_indices, w.last_page_len, w.sm_scale, fmt)
     assert_parity(out, lse, ro, rl, what="fp8 append+decode")
 
 
