@@ -286,7 +286,7 @@ PKV_API pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, floa
  *   qo_indptr_h  host int32 [batch+1]
  *   kv_len_h     host int32 [batch]: L_b (tokens after the append), or NULL
  *   plan_h       host int32 [capacity][4] or NULL: {request, first row, rows, 0}
- *                per block of up to 128 rows (row r = chunk token r / G, query
+ *                per block of up to 256 rows (row r = chunk token r / G, query
  *                head kv_head * G + r % G)
  *   num_splits   if not NULL, receives a split count for the launch: 1 when
  *                the row blocks fill num_sms SMs (or kv_len_h is NULL), else

@@ -87,10 +87,10 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 struct MapKey {
   const void* pool;
   long long pages;
-  int ps, hkv, dtype, layout, device;
+  int ps, hkv, dtype, layout, device, halves;
   bool operator==(const MapKey& o) const {
     return pool == o.pool && pages == o.pages && ps == o.ps && hkv == o.hkv && dtype == o.dtype &&
-           layout == o.layout && device == o.device;
+           layout == o.layout && device == o.device && halves == o.halves;
   }
 };
 
@@ -103,8 +103,11 @@ struct MapKey {
 // strides are not increasing), the HND pool falls back to the 4-D form
 // (dim, slot, K/V * Hkv + head, page) with [16][64] boxes: two loads per K or
 // V tile, same shared-memory layout.
+// halves: dim-halves per box of the 16-bit 5-D view -- 2 (the decode and prefix
+// kernels: a [2][16][64] box is one K or V tile) or 1 (the tcgen05 kernel: a
+// [16][64] box per half, so each half of a 64-token tile is contiguous).
 pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, int dtype, int layout,
-                           CUtensorMap* out, int* one_box) {
+                           CUtensorMap* out, int* one_box, int halves = 2) {
   static std::mutex mu;
   static MapKey keys[16];
   static CUtensorMap maps[16];
@@ -112,7 +115,7 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
   static int used = 0, next = 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  const MapKey key{pool, pages, ps, hkv, dtype, layout, dev};
+  const MapKey key{pool, pages, ps, hkv, dtype, layout, dev, is_fp8(dtype) ? 2 : halves};
   {
     std::lock_guard<std::mutex> lk(mu);
     for (int i = 0; i < used; ++i)
@@ -163,7 +166,7 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
     cuuint64_t dims[5] = {64, (cuuint64_t)ps, 2, (cuuint64_t)hkv, (cuuint64_t)2 * pages};
     cuuint64_t strides[4] = {nhd ? (cuuint64_t)hkv * row : row, 128,
                              nhd ? row : (cuuint64_t)ps * row, (cuuint64_t)hkv * ps * row};
-    cuuint32_t box[5] = {64, (cuuint32_t)pkv::kTileTokens, 2, 1, 1};
+    cuuint32_t box[5] = {64, (cuuint32_t)pkv::kTileTokens, (cuuint32_t)halves, 1, 1};
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     r = encode(&m, dt, 5, const_cast<void*>(pool), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -849,7 +852,7 @@ pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr, int64_t
   CUtensorMap tmap;
   int one_box = 0;
   st = pool_tensor_map(pool->data, pool->num_pages, pool->page_size, pool->num_kv_heads,
-                       pool->dtype, pool->layout, &tmap, &one_box);
+                       pool->dtype, pool->layout, &tmap, &one_box, /*halves=*/1);
   if (st != PKV_OK) return st;
   const size_t states = (size_t)nnz_q * num_splits * num_qo_heads;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -879,7 +882,7 @@ pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr, int64_t
   a.scale_log2 = sm_scale * 1.4426950408889634f;
   a.one_box = one_box;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = pkv::launch_chunk(tmap, a, pool->dtype == PKV_BF16, (int)num_row_blocks, s);
+  cudaError_t e = pkv::launch_chunk_tc(tmap, a, pool->dtype == PKV_BF16, (int)num_row_blocks, s);
   if (e != cudaSuccess) return cuda_fail(e, "append attention launch");
   if (num_splits > 1) {
     pkv::MergeArgs ma;

@@ -7,10 +7,8 @@
 //     O[16 x 128] += P[16 x 64] . V_tile     (bf16: P split into high + low parts)
 //
 // This is the blockwise recursive softmax of "大模型推理极致优化：FlashAttention+
-// PageAttention联合调优" section 2.2 for a block of query rows.  Used by the
-// shared-prefix kernel (prefix.cu) and the multi-token append attention
-// (chunk.cu); the callers differ only in which rows they own and which keys
-// each row may see.
+// PageAttention联合调优" section 2.2 for a block of query rows, used by the
+// shared-prefix kernel (prefix.cu).
 //
 // Shared-memory tile: K (then V) of 64 tokens as four 16-token bulk-tensor
 // boxes, each [2][16][64] elements with the 128-byte swizzle.

@@ -1,0 +1,532 @@
+// chunk_tc.cu -- multi-token append attention on the fifth-generation tensor
+// cores (tcgen05, accumulators in tensor memory).
+//
+// Each request's chunk of new query tokens attends over its paged cache with
+// a causal mask and an optional window with sink tokens (chunked prefill,
+// "大模型长上下文窗口工程化实战：从RoPE扩展到百万Token推理的生产级部署" section 3.1;
+// the window of section 2.3 cut to its causal half).  A CTA owns a block of up
+// to 256 rows of one request and KV head -- row r = (chunk token r / G, query
+// head kvh * G + r % G) -- as two 128-row tiles A and B that share every K/V
+// tile their rows may see.  Per 64-token K/V tile and row tile:
+//     S[128 x 64]  = Q[128 x 128] . K_tile^T     tcgen05.mma, A and B in shared memory
+//     online softmax, one thread per row reading S from tensor memory
+//     O[128 x 128] += P[128 x 64] . V_tile        tcgen05.mma, P in tensor memory
+// -- the blockwise recursive softmax of "大模型推理极致优化：FlashAttention+
+// PageAttention联合调优" section 2.2 with a row tile as one MMA.  While one row
+// tile's softmax runs, the tensor core works on the other's products.
+//
+// Warp roles (320 threads): warp 0 issues the bulk-tensor loads of K and V
+// into a 3-stage ring; warp 1 allocates tensor memory and one of its lanes
+// issues every MMA; warps 2..5 own row tile A and warps 6..9 row tile B (one
+// warp per 32-lane quarter of tensor memory): they stage Q, run the softmax
+// and the epilogue.
+//
+// Tensor memory (512 columns x 128 lanes of 32 bits): S of row tile t for
+// tiles of even / odd index in columns [64(2t+b), +64) -- rewritten in place
+// by P (bf16: the high 16 bits of each fp32 probability in the first 32
+// columns, the rounded remainder in the next 32, two MMAs; fp16: one part)
+// -- and O of row tile t in [256 + 128t, +128).
+//
+// The running maximum is only moved (and O, l rescaled) when a tile's
+// maximum exceeds it by more than 8 (log2 units); otherwise exponentials are
+// taken against the stale maximum, which bounds P by 2^8 and changes nothing
+// in o = O / l.
+//
+// Every wait is bounded (common.cuh); on a timeout the kernel sets the
+// timeout bit, lets its own copies and MMAs drain (bounded), frees tensor
+// memory and returns.  Tensor-memory loads and stores are warp-collective, so
+// every branch around them is warp-uniform.  An mbarrier parity wait cannot
+// tell a phase from the one two phases later, so no thread waits for a phase
+// while the phase before it may still be pending: each wait below is
+// preceded, in that thread, by a wait that implies the previous phase.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "partition.cuh"
+#include "umma.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kTileRows = 128;                    // rows of one row tile (the MMA's M)
+constexpr int kRowTiles = 2;
+constexpr int kRows = kRowTiles * kTileRows;      // rows per CTA
+constexpr int kTile = 64;                         // keys per K/V tile
+constexpr int kStages = 3;
+constexpr int kThreads = 64 + kRows;              // producer, MMA, 8 softmax warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256;
+constexpr int kQTileBytes = kTileRows * kD * 2;   // 32 KiB: two 64-dim halves of [128][64]
+constexpr int kQHalf = kTileRows * 128;           // 16 KiB
+constexpr int kKVHalf = kTile * 128;              // 8 KiB: [64 tokens][64 dims]
+constexpr int kKBytes = 2 * kKVHalf;              // 16 KiB
+constexpr int kStageBytes = 2 * kKBytes;          // K then V: 32 KiB
+constexpr int kBoxBytes = kTileTokens * 128;      // one [16][64] box: 2 KiB
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.f;
+constexpr unsigned kAll = 0xffffffffu;
+
+struct __align__(16) Ctl {
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t q_full[kRowTiles];
+  uint64_t s_full[kRowTiles][2];
+  uint64_t p_full[kRowTiles][2];
+  uint64_t o_done[kRowTiles];
+  uint64_t drained;  // one phase: every MMA of the CTA completed
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes =
+    1024 + (size_t)kRowTiles * kQTileBytes + (size_t)kStages * kStageBytes + sizeof(Ctl);
+
+// the visible key range of a row block, as a list of 64-token tiles:
+// sink tiles [0, a_end) then window tiles [lo16, hi)
+struct KeyRange {
+  long long a_end, lo16, hi;
+  int nA, n;
+  __device__ void tile(int j, long long& t0, long long& t1) const {
+    if (j < nA) {
+      t0 = (long long)j * kTile;
+      t1 = t0 + kTile < a_end ? t0 + kTile : a_end;
+    } else {
+      t0 = lo16 + (long long)(j - nA) * kTile;
+      t1 = t0 + kTile < hi ? t0 + kTile : hi;
+    }
+  }
+};
+
+__device__ __forceinline__ int clamp64(long long v) { return v <= 0 ? 0 : (v >= kTile ? kTile : (int)v); }
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* qs = smem;                                        // Q of both row tiles
+  uint8_t* ring = smem + (size_t)kRowTiles * kQTileBytes;    // K/V stages
+  Ctl& ctl = *reinterpret_cast<Ctl*>(ring + (size_t)kStages * kStageBytes);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kvh = blockIdx.y, split = blockIdx.z;
+  const int G = a.group;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&ctl.kv_full[s]), 1);
+      mbar_init(smem_u32(&ctl.kv_empty[s]), 1);
+    }
+    for (int t = 0; t < kRowTiles; ++t) {
+      mbar_init(smem_u32(&ctl.q_full[t]), kTileRows);
+      mbar_init(smem_u32(&ctl.o_done[t]), 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(smem_u32(&ctl.s_full[t][b]), 1);
+        mbar_init(smem_u32(&ctl.p_full[t][b]), kTileRows);
+      }
+    }
+    mbar_init(smem_u32(&ctl.drained), 1);
+    ctl.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    umma::tmem_alloc(smem_u32(&ctl.tmem_base), kTmemCols);
+    umma::tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap);
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tbase = ctl.tmem_base;
+  grid_dependency_wait();
+
+  // ---- this CTA's row block and the keys its rows may see
+  const int4 item = a.plan[blockIdx.x];
+  const int b = item.x, row0 = item.y, nrows = item.z;
+  bool bad = (unsigned)b >= (unsigned)a.batch || nrows < 1 || nrows > kRows || row0 < 0;
+  ReqInfo r{};
+  long long q_len = 0, q_first = 0;
+  if (!bad) {
+    r = request_info(a.tv, b, a.page_size);
+    q_first = a.qo_indptr[b];
+    q_len = (long long)a.qo_indptr[b + 1] - q_first;
+    bad = r.err != 0 || q_len < 0 || q_len > r.len || q_first < 0 ||
+          q_first + q_len > a.nnz_q || (long long)row0 + nrows > q_len * G;
+  }
+  if (bad && tid == 0 && a.err) atomicOr(a.err, r.err ? r.err : kErrAppend);
+  const long long base = r.len - q_len;  // position of chunk token 0
+  const int tiles = nrows > kTileRows ? 2 : 1;  // row tiles with rows
+  KeyRange kr{};
+  int j0 = 0, n = 0;
+  if (!bad) {
+    const long long pos_first = base + row0 / G, pos_last = base + (row0 + nrows - 1) / G;
+    kr.hi = pos_last + 1;
+    long long lo = a.window_left >= 0 ? pos_first - a.window_left : 0;
+    lo = lo < 0 ? 0 : lo;
+    kr.lo16 = lo & ~15LL;
+    kr.a_end = a.window_left >= 0 ? (a.sink < kr.lo16 ? a.sink : kr.lo16) : 0;
+    kr.nA = (int)((kr.a_end + kTile - 1) / kTile);
+    kr.n = kr.nA + (int)((kr.hi - kr.lo16 + kTile - 1) / kTile);
+    const int per = (kr.n + a.splits - 1) / a.splits;
+    j0 = split * per;
+    const int j1 = j0 + per < kr.n ? j0 + per : kr.n;
+    n = j1 > j0 ? j1 - j0 : 0;
+  }
+
+  if (!bad && warp == 0) {
+    // =========================== producer ===========================
+    const uint32_t ring0 = smem_u32(ring);
+    const int* ids = a.indices + r.page_base;
+    bool ok = true;
+    int issued = 0;
+    for (int i = 0; ok && i < n; ++i) {
+      const int s = i % kStages;
+      long long t0, t1;
+      kr.tile(j0 + i, t0, t1);
+      const int valid = (int)(t1 - t0);
+      int page = -1, yoff = 0;
+      if (lane < 4 && lane * kTileTokens < valid) {
+        const long long tok = t0 + lane * kTileTokens;
+        page = ids[tok / a.page_size];
+        if (page < 0 || (long long)page >= a.num_pages) {
+          if (a.err) atomicOr(a.err, kErrPageId);
+          page = -1;
+        }
+        yoff = (int)(tok % a.page_size);
+      }
+      const unsigned have = __ballot_sync(kAll, page >= 0) & 0xfu;
+      // lane L < 16 loads (K / V = L / 8, box = (L / 2) % 4, dim half = L % 2)
+      const int box = (lane >> 1) & 3, half = lane & 1, kv = (lane >> 3) & 1;
+      const int bpage = __shfl_sync(kAll, page, box);
+      const int byoff = __shfl_sync(kAll, yoff, box);
+      int okl = 1;
+      if (lane == 0) {
+        okl = mbar_wait_bounded(smem_u32(&ctl.kv_empty[s]), ((i / kStages) & 1) ^ 1, &ctl.abort,
+                                a.err);
+        if (okl) mbar_arrive_expect_tx(smem_u32(&ctl.kv_full[s]), __popc(have) * 4u * kBoxBytes);
+      }
+      ok = __shfl_sync(kAll, okl, 0) != 0;
+      if (!ok) break;
+      if (lane < 16 && bpage >= 0) {
+        const uint32_t dst = ring0 + (uint32_t)s * kStageBytes + (uint32_t)kv * kKBytes +
+                             (uint32_t)half * kKVHalf + (uint32_t)box * kBoxBytes;
+        const uint32_t full = smem_u32(&ctl.kv_full[s]);
+        if (a.one_box)  // 5-D view (dim % 64, slot, dim / 64, kv head, 2 page + K/V), [16][64] boxes
+          tma_load_5d(dst, &tmap, 0, byoff, half, kvh, 2 * bpage + kv, full);
+        else            // 4-D view of the HND layout (dim, slot, K/V * Hkv + head, page)
+          tma_load_4d(dst, &tmap, 64 * half, byoff, kv * a.hkv + kvh, bpage, full);
+      }
+      issued = i + 1;
+    }
+    if (!ok && lane == 0) {
+      // aborted: let the copies already issued land before the CTA exits
+      const int first = issued > kStages ? issued - kStages : 0;
+      for (int k = first; k < issued; ++k) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(smem_u32(&ctl.kv_full[k % kStages]), (k / kStages) & 1) &&
+               global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (!bad && warp == 1) {
+    // =========================== MMA issuer ===========================
+    if (lane == 0) {
+      const uint32_t ring0 = smem_u32(ring);
+      const uint32_t idesc_s = umma::instr_desc(BF16, kTileRows, kTile, false, false);
+      const uint32_t idesc_pv = umma::instr_desc(BF16, kTileRows, kD, false, true);
+      auto issue_s = [&](int j, int t) {  // S_t(j) into buffer j & 1 of row tile t
+        const uint32_t qb = smem_u32(qs) + (uint32_t)t * kQTileBytes;
+        const uint32_t kbase = ring0 + (uint32_t)(j % kStages) * kStageBytes;
+        const uint32_t d = tbase + (uint32_t)(2 * t + (j & 1)) * kTile;
+#pragma unroll
+        for (int k = 0; k < kD / 16; ++k) {  // 16 dims per MMA: 32 bytes along a swizzled row
+          const uint32_t off = (uint32_t)(k & 3) * 32u;
+          const uint64_t ad = umma::smem_desc(qb + (uint32_t)(k >> 2) * kQHalf + off, 16, 1024);
+          const uint64_t bd = umma::smem_desc(kbase + (uint32_t)(k >> 2) * kKVHalf + off, 16, 1024);
+          umma::mma_ss(d, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+        }
+        umma::commit(smem_u32(&ctl.s_full[t][j & 1]));
+      };
+      auto issue_pv = [&](int j, int t) {  // O_t += P_t(j) . V(j)
+        const uint32_t vbase = ring0 + (uint32_t)(j % kStages) * kStageBytes + kKBytes;
+        const uint32_t p_cols = tbase + (uint32_t)(2 * t + (j & 1)) * kTile;
+        const uint32_t o = tbase + kColO + (uint32_t)t * kD;
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k) {  // 16 keys per MMA: 8 columns of P, 2 KiB of V
+          const uint64_t bd = umma::smem_desc(vbase + (uint32_t)k * 2048u, kKVHalf, 1024);
+          umma::mma_ts(o, p_cols + 8u * k, bd, idesc_pv, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        if constexpr (BF16) {
+#pragma unroll
+          for (int k = 0; k < kTile / 16; ++k) {
+            const uint64_t bd = umma::smem_desc(vbase + (uint32_t)k * 2048u, kKVHalf, 1024);
+            umma::mma_ts(o, p_cols + 32u + 8u * k, bd, idesc_pv, 1u);
+          }
+        }
+        umma::commit(smem_u32(&ctl.o_done[t]));
+      };
+      bool ok = true;
+      for (int t = 0; ok && t < tiles; ++t)
+        ok = mbar_wait_bounded(smem_u32(&ctl.q_full[t]), 0, &ctl.abort, a.err);
+      if (ok && n > 0) {
+        ok = mbar_wait_bounded(smem_u32(&ctl.kv_full[0]), 0, &ctl.abort, a.err);
+        if (ok) {
+          umma::fence_after_sync();
+          for (int t = 0; t < tiles; ++t) issue_s(0, t);
+        }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        // S(j+1) into the other buffers: it overwrites P(j-1), so PV(j-1) must be done
+        if (j + 1 < n) {
+          ok = mbar_wait_bounded(smem_u32(&ctl.kv_full[(j + 1) % kStages]), ((j + 1) / kStages) & 1,
+                                 &ctl.abort, a.err);
+          for (int t = 0; ok && t < tiles && j >= 1; ++t)
+            ok = mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (j - 1) & 1, &ctl.abort, a.err);
+          if (!ok) break;
+          umma::fence_after_sync();
+          for (int t = 0; t < tiles; ++t) issue_s(j + 1, t);
+        }
+        for (int t = 0; ok && t < tiles; ++t) {
+          ok = mbar_wait_bounded(smem_u32(&ctl.p_full[t][j & 1]), (j >> 1) & 1, &ctl.abort, a.err);
+          if (!ok) break;
+          umma::fence_after_sync();
+          issue_pv(j, t);
+        }
+        if (ok) umma::commit(smem_u32(&ctl.kv_empty[j % kStages]));
+      }
+      // let every MMA issued land before tensor memory is freed (a commit
+      // arrives once all MMAs this thread issued before it completed)
+      umma::commit(smem_u32(&ctl.drained));
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(smem_u32(&ctl.drained), 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    __syncwarp();
+  } else if (!bad && warp >= 2 && (warp - 2) / 4 < tiles) {
+    // =========================== softmax warps ===========================
+    const int t = (warp - 2) / 4;                  // row tile
+    const int quarter = warp & 3;                  // tensor-memory lane quarter
+    const int row = quarter * 32 + lane;           // row within the tile
+    const uint32_t trow = tbase + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t t_o = trow + kColO + (uint32_t)t * kD;
+    const int rr = row0 + t * kTileRows + row;     // row within the request's chunk rows
+    const bool has_row = t * kTileRows + row < nrows;
+    const long long pos = has_row ? base + rr / G : -1;
+    uint8_t* qt = qs + (size_t)t * kQTileBytes;
+    // ---- stage this row of Q in the 128-byte-swizzled K-major layout
+    {
+      const uint4* src = has_row ? reinterpret_cast<const uint4*>(
+                                       static_cast<const uint16_t*>(a.q) +
+                                       ((size_t)(q_first + rr / G) * a.hq + (size_t)kvh * G + rr % G) * kD)
+                                 : nullptr;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = src ? src[c] : make_uint4(0, 0, 0, 0);
+        const int half = c >> 3, cc = c & 7;
+        *reinterpret_cast<uint4*>(qt + half * kQHalf + row * 128 + ((cc ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&ctl.q_full[t]));
+    }
+    const float sl2 = a.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int bj = j & 1;
+      const uint32_t t_s = trow + (uint32_t)(2 * t + bj) * kTile;
+      ok = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.s_full[t][bj]), (j >> 1) & 1,
+                                              &ctl.abort, a.err));
+      if (!ok) break;
+      umma::fence_after_sync();
+      uint32_t s0[32], s1[32];
+      umma::ld32(t_s, s0);
+      umma::ld32(t_s + 32u, s1);
+      long long t0, t1;
+      kr.tile(j0 + j, t0, t1);
+      const int valid = (int)(t1 - t0);
+      // visible keys of this row in the tile: k < hk (causal), and k >= lk or k < sk (window)
+      const int hk = pos - t0 + 1 >= valid ? valid : clamp64(pos - t0 + 1);
+      const int lk = a.window_left >= 0 ? clamp64(pos - a.window_left - t0) : 0;
+      const int sk = a.window_left >= 0 ? clamp64((long long)a.sink - t0) : 0;
+      umma::wait_ld();
+      float x[64];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        x[k] = __uint_as_float(s0[k]);
+        x[32 + k] = __uint_as_float(s1[k]);
+      }
+      if (!__all_sync(kAll, hk == kTile && lk == 0)) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          x[k] = ((k < hk) & ((k >= lk) | (k < sk))) ? x[k] : -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx[u] = x[u];
+#pragma unroll
+      for (int k = 8; k < 64; ++k) mx[k & 7] = fmaxf(mx[k & 7], x[k]);
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      const bool move = mt > m_used + kRescaleThreshold;
+      // O (and l) were accumulated against m_used: rescale the rows that move
+      // their maximum, once PV(j-1) is done (the whole warp loads and stores)
+      const bool rescale = move && j > 0 && m_used != -INFINITY;
+      if (__any_sync(kAll, rescale)) {
+        ok = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (j - 1) & 1,
+                                                &ctl.abort, a.err));
+        if (!ok) break;
+        umma::fence_after_sync();
+        const float f = rescale ? ex2(m_used - mt) : 1.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          umma::ld32(t_o + 32u * c, o);
+          umma::wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+          umma::st32(t_o + 32u * c, o);
+        }
+        l *= f;
+      }
+      if (move) m_used = mt;
+      const float mref = m_used == -INFINITY ? 0.f : m_used;
+      // P = 2^(x * scale - m): high part = top 16 bits (bf16 truncation), low
+      // part = the exact remainder rounded to bf16; fp16: one rounding
+      uint32_t hi[32], lo[32];
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const float p0 = ex2(fmaf(x[2 * k], sl2, -mref)), p1 = ex2(fmaf(x[2 * k + 1], sl2, -mref));
+        ps[k & 3] += p0 + p1;
+        if constexpr (BF16) {
+          const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+          hi[k] = prmt(b0, b1, 0x7632u);
+          lo[k] = pack2<true>(p0 - __uint_as_float(b0 & 0xffff0000u),
+                              p1 - __uint_as_float(b1 & 0xffff0000u));
+        } else {
+          hi[k] = pack2<false>(p0, p1);
+        }
+      }
+      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      umma::st32(t_s, hi);
+      if constexpr (BF16) umma::st32(t_s + 32u, lo);
+      // V rows past the tile's keys may hold anything (even NaN): row tile A
+      // zeroes them before the first PV of this tile (B's is issued after A's)
+      if (t == 0 && valid < kTile) {
+        uint8_t* vt = ring + (size_t)(j % kStages) * kStageBytes + kKBytes;
+        const int chunks = (kTile - valid) * 16;  // 16-byte chunks over both dim halves
+        for (int idx = row; idx < chunks; idx += kTileRows) {
+          const int tk = valid + (idx >> 4), half = (idx >> 3) & 1, c = idx & 7;
+          *reinterpret_cast<uint4*>(vt + half * kKVHalf + tk * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      umma::wait_st();
+      umma::fence_before_sync();
+      mbar_arrive(smem_u32(&ctl.p_full[t][bj]));
+    }
+    // ---- epilogue: o = O / l of this row (every lane loads; rows past the block store nothing)
+    if (ok) {
+      // PV(n-2) may still be running when this row's last softmax ends: wait for
+      // its phase first, then PV(n-1)'s
+      bool have_o = n > 0;
+      if (have_o && n >= 2)
+        have_o = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (n - 2) & 1,
+                                                    &ctl.abort, a.err));
+      if (have_o)
+        have_o = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (n - 1) & 1,
+                                                    &ctl.abort, a.err));
+      if (n == 0 || have_o) {
+        umma::fence_after_sync();
+        const size_t tok = has_row ? (size_t)(q_first + rr / G) : 0;
+        const size_t h = has_row ? (size_t)kvh * G + rr % G : 0;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float lse = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          if (have_o) {
+            umma::ld32(t_o + 32u * c, o);
+            umma::wait_ld();
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = 0u;
+          }
+          if (!has_row) continue;
+          if (a.splits == 1) {
+            uint16_t* op = static_cast<uint16_t*>(a.out) + (tok * a.hq + h) * kD + 32 * c;
+#pragma unroll
+            for (int k = 0; k < 32; k += 8) {
+              uint4 w;
+              w.x = pack2<BF16>(__uint_as_float(o[k + 0]) * inv, __uint_as_float(o[k + 1]) * inv);
+              w.y = pack2<BF16>(__uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+              w.z = pack2<BF16>(__uint_as_float(o[k + 4]) * inv, __uint_as_float(o[k + 5]) * inv);
+              w.w = pack2<BF16>(__uint_as_float(o[k + 6]) * inv, __uint_as_float(o[k + 7]) * inv);
+              *reinterpret_cast<uint4*>(op + k) = w;
+            }
+          } else {
+            float* op = a.state_o + ((tok * a.splits + split) * a.hq + h) * kD + 32 * c;
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+              *reinterpret_cast<float4*>(op + k) =
+                  make_float4(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv,
+                              __uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+          }
+        }
+        if (has_row) {
+          if (a.splits == 1) {
+            if (a.lse) a.lse[tok * a.hq + h] = lse;
+          } else {
+            a.state_lse[(tok * a.splits + split) * a.hq + h] = lse;
+          }
+        }
+      }
+    }
+  }
+
+  // ---- free tensor memory once every warp is done with it
+  umma::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    umma::fence_after_sync();
+    umma::tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t chunk_tc_smem_bytes() { return kSmemBytes; }
+int chunk_rows_per_cta() { return kRows; }
+int chunk_tile_tokens() { return kTile; }
+
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const ChunkArgs& a, bool bf16, int row_blocks,
+                            cudaStream_t stream) {
+  auto kern = bf16 ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+  static bool attr_set[2][64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !attr_set[bf16][dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[bf16][dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)row_blocks, (unsigned)a.hkv, (unsigned)a.splits);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tmap, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace pkv

@@ -72,7 +72,7 @@ int prefix_tile_tokens();
 cudaError_t launch_prefix(const CUtensorMap& tmap, const PrefixArgs& a, bool bf16, int row_blocks,
                           cudaStream_t stream);
 
-// multi-token append attention (chunk.cu)
+// multi-token append attention (chunk_tc.cu)
 struct ChunkArgs {
   const void* q;               // [nnz_q][Hq][128]
   const int32_t* qo_indptr;    // [B+1], qo_indptr[0] = 0
@@ -90,11 +90,12 @@ struct ChunkArgs {
   float scale_log2;
   int one_box;
 };
-size_t chunk_smem_bytes();
+// chunk_tc.cu (tcgen05); its tensor map has [16][64] boxes (one dim half each)
 int chunk_rows_per_cta();
 int chunk_tile_tokens();
-cudaError_t launch_chunk(const CUtensorMap& tmap, const ChunkArgs& a, bool bf16, int row_blocks,
-                         cudaStream_t stream);
+size_t chunk_tc_smem_bytes();
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const ChunkArgs& a, bool bf16, int row_blocks,
+                            cudaStream_t stream);
 
 struct AppendArgs {
   void* pool;

@@ -265,7 +265,7 @@ def test_append_attention_plan_covers_rows_once():
         plan, S = pkv.append_attention_plan(qo, kv, hq, hkv, num_sms=148)
         seen = [np.zeros(int(n) * G, int) for n in q_lens]
         for b, r0, n, pad in plan:
-            assert 1 <= n <= 128 and pad == 0
+            assert 1 <= n <= 256 and pad == 0
             seen[b][r0:r0 + n] += 1
         assert all((s == 1).all() for s in seen)
         assert list(plan[:, 0]) == sorted(plan[:, 0])
