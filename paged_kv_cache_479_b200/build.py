@@ -12,7 +12,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libpkv.so")
-SOURCES = ["api.cu", "decode.cu", "prefix.cu", "chunk_tc.cu", "append.cu", "merge.cu", "static_ws.cu"]
+SOURCES = ["api.cu", "decode.cu", "chunk_tc.cu", "append.cu", "merge.cu", "static_ws.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

@@ -588,11 +588,10 @@ pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, float v_scal
 
 namespace {
 
-// Shared-prefix cascade: the prefix kernel's grid (row blocks x splits x kv
-// heads) and the fp32 attention states it and the suffix decode write.
+// Shared-prefix cascade: the prefix step's grid (row blocks x kv heads x key
+// splits) and the fp32 attention states it and the suffix decode write.
 struct CascadePlan {
   int row_blocks, splits, states;
-  long long tokens_per_split;
   size_t state_o, state_lse, decode_ws, total;  // byte offsets / size
 };
 
@@ -600,17 +599,14 @@ CascadePlan cascade_plan(int batch, int hq, int hkv, long long prefix_len, int N
   CascadePlan p;
   const int G = hq / hkv;
   const long long rows = (long long)batch * G;
-  const int R = pkv::prefix_rows_per_cta(), T = pkv::prefix_tile_tokens();
+  const int R = pkv::chunk_rows_per_cta(), T = pkv::chunk_tile_tokens();
   p.row_blocks = (int)((rows + R - 1) / R);
   const long long tiles = (prefix_len + T - 1) / T;
   const long long units = (long long)p.row_blocks * hkv;
-  long long splits = units >= sms ? 1 : sms / units;  // about one wave of CTAs
+  long long splits = units >= sms ? 1 : (sms + units - 1) / units;  // about one wave of CTAs
   if (splits > tiles) splits = tiles;
   if (splits < 1) splits = 1;
-  const long long tiles_per = (tiles + splits - 1) / splits;
-  p.tokens_per_split = tiles_per * T;
-  p.splits = (int)((prefix_len + p.tokens_per_split - 1) / p.tokens_per_split);
-  if (p.splits < 1) p.splits = 1;
+  p.splits = (int)splits;
   p.states = p.splits + 1;
   p.state_o = 0;
   p.state_lse = align_up((size_t)batch * p.states * hq * kDecodeHeadDim * 4, 256);
@@ -686,7 +682,7 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
   CUtensorMap tmap;
   int one_box = 0;
   pkv_status st = pool_tensor_map(pool, num_pages, page_size, num_kv_heads, dtype, PKV_LAYOUT_HND,
-                                  &tmap, &one_box);
+                                  &tmap, &one_box, /*halves=*/1);
   if (st != PKV_OK) return st;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* state_o = reinterpret_cast<float*>(ws + P.state_o);
@@ -694,25 +690,28 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   // 1. the shared prefix, once for every request's queries: state slots 0 .. splits-1
-  pkv::PrefixArgs pa;
+  pkv::ChunkArgs pa = {};
   pa.q = q;
   pa.prefix_pages = prefix_page_indices;
+  pa.prefix_len = prefix_len;
   pa.state_o = state_o;
   pa.state_lse = state_lse;
+  pa.states = P.states;
+  pa.out_states = 1;
   pa.err = reinterpret_cast<int*>(error_word);
   pa.num_pages = num_pages;
-  pa.prefix_len = prefix_len;
-  pa.tokens_per_split = P.tokens_per_split;
+  pa.nnz_q = batch;
   pa.page_size = page_size;
   pa.batch = batch;
   pa.hq = num_qo_heads;
   pa.hkv = num_kv_heads;
   pa.group = group;
-  pa.states = P.states;
   pa.splits = P.splits;
+  pa.window_left = -1;
+  pa.sink = 0;
   pa.scale_log2 = sm_scale * 1.4426950408889634f;
   pa.one_box = one_box;
-  cudaError_t e = pkv::launch_prefix(tmap, pa, dtype == PKV_BF16, P.row_blocks, s);
+  cudaError_t e = pkv::launch_chunk_tc(tmap, pa, dtype == PKV_BF16, P.row_blocks, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
   // 2. each request's own pages: the last state slot, as an fp32 state
   st = decode_impl(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
@@ -864,6 +863,10 @@ pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr, int64_t
   a.plan = reinterpret_cast<const int4*>(plan);
   a.out = out;
   a.lse = lse;
+  a.prefix_pages = nullptr;
+  a.prefix_len = 0;
+  a.states = num_splits;
+  a.out_states = num_splits > 1;
   a.state_o = num_splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
   a.state_lse = num_splits > 1
                     ? reinterpret_cast<float*>(ws + align_up(states * kDecodeHeadDim * 4, 256))

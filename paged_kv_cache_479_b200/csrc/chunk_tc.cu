@@ -15,6 +15,15 @@
 // PageAttention联合调优" section 2.2 with a row tile as one MMA.  While one row
 // tile's softmax runs, the tensor core works on the other's products.
 //
+// The same kernel computes the shared-prefix step of the cascade: for a
+// prefix stored once in shared pages (prefix page sharing, "大模型推理极致优化：
+// FlashAttention+PageAttention联合调优" section 3.2), rows are the (request,
+// query head) pairs of every request for one KV head -- row r = (request
+// r / G, head kvh * G + r % G) -- and the keys are the prefix's, unmasked, so
+// the prefix's K/V is read once per 256 rows instead of once per request.
+// Its result is a fp32 state per row and key split, merged afterwards with
+// the state of the request's own pages.
+//
 // Warp roles (320 threads): warp 0 issues the bulk-tensor loads of K and V
 // into a 3-stage ring; warp 1 allocates tensor memory and one of its lanes
 // issues every MMA; warps 2..5 own row tile A and warps 6..9 row tile B (one
@@ -69,6 +78,7 @@ constexpr int kBoxBytes = kTileTokens * 128;      // one [16][64] box: 2 KiB
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.f;
 constexpr unsigned kAll = 0xffffffffu;
+constexpr long long kNoCausalLimit = 1LL << 60;  // position of a prefix row: sees every key
 
 struct __align__(16) Ctl {
   uint64_t kv_full[kStages];
@@ -144,12 +154,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   grid_dependency_wait();
 
   // ---- this CTA's row block and the keys its rows may see
-  const int4 item = a.plan[blockIdx.x];
-  const int b = item.x, row0 = item.y, nrows = item.z;
-  bool bad = (unsigned)b >= (unsigned)a.batch || nrows < 1 || nrows > kRows || row0 < 0;
+  const bool prefix = a.prefix_pages != nullptr;
+  int b = 0, row0, nrows;
+  if (prefix) {  // rows of every request, in blocks of kRows
+    row0 = (int)blockIdx.x * kRows;
+    const long long left = (long long)a.batch * G - row0;
+    nrows = left < kRows ? (int)left : kRows;
+  } else {
+    const int4 item = a.plan[blockIdx.x];
+    b = item.x;
+    row0 = item.y;
+    nrows = item.z;
+  }
+  bool bad = (!prefix && (unsigned)b >= (unsigned)a.batch) || nrows < 1 || nrows > kRows ||
+             row0 < 0 || (prefix && a.prefix_len < 1);
   ReqInfo r{};
   long long q_len = 0, q_first = 0;
-  if (!bad) {
+  if (!bad && !prefix) {
     r = request_info(a.tv, b, a.page_size);
     q_first = a.qo_indptr[b];
     q_len = (long long)a.qo_indptr[b + 1] - q_first;
@@ -161,7 +182,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles = nrows > kTileRows ? 2 : 1;  // row tiles with rows
   KeyRange kr{};
   int j0 = 0, n = 0;
-  if (!bad) {
+  if (!bad && prefix) {  // every prefix token, unmasked
+    kr.hi = a.prefix_len;
+    kr.n = (int)((kr.hi + kTile - 1) / kTile);
+  } else if (!bad) {
     const long long pos_first = base + row0 / G, pos_last = base + (row0 + nrows - 1) / G;
     kr.hi = pos_last + 1;
     long long lo = a.window_left >= 0 ? pos_first - a.window_left : 0;
@@ -170,6 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     kr.a_end = a.window_left >= 0 ? (a.sink < kr.lo16 ? a.sink : kr.lo16) : 0;
     kr.nA = (int)((kr.a_end + kTile - 1) / kTile);
     kr.n = kr.nA + (int)((kr.hi - kr.lo16 + kTile - 1) / kTile);
+  }
+  if (!bad) {  // this split's share of the key tiles
     const int per = (kr.n + a.splits - 1) / a.splits;
     j0 = split * per;
     const int j1 = j0 + per < kr.n ? j0 + per : kr.n;
@@ -179,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!bad && warp == 0) {
     // =========================== producer ===========================
     const uint32_t ring0 = smem_u32(ring);
-    const int* ids = a.indices + r.page_base;
+    const int* ids = prefix ? a.prefix_pages : a.indices + r.page_base;
     bool ok = true;
     int issued = 0;
     for (int i = 0; ok && i < n; ++i) {
@@ -314,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = trow + kColO + (uint32_t)t * kD;
     const int rr = row0 + t * kTileRows + row;     // row within the request's chunk rows
     const bool has_row = t * kTileRows + row < nrows;
-    const long long pos = has_row ? base + rr / G : -1;
+    const long long pos = has_row ? (prefix ? kNoCausalLimit : base + rr / G) : -1;
     uint8_t* qt = qs + (size_t)t * kQTileBytes;
     // ---- stage this row of Q in the 128-byte-swizzled K-major layout
     {
@@ -456,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 32; ++k) o[k] = 0u;
           }
           if (!has_row) continue;
-          if (a.splits == 1) {
+          if (!a.out_states) {
             uint16_t* op = static_cast<uint16_t*>(a.out) + (tok * a.hq + h) * kD + 32 * c;
 #pragma unroll
             for (int k = 0; k < 32; k += 8) {
@@ -468,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4*>(op + k) = w;
             }
           } else {
-            float* op = a.state_o + ((tok * a.splits + split) * a.hq + h) * kD + 32 * c;
+            float* op = a.state_o + ((tok * a.states + split) * a.hq + h) * kD + 32 * c;
 #pragma unroll
             for (int k = 0; k < 32; k += 4)
               *reinterpret_cast<float4*>(op + k) =
@@ -477,10 +503,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (has_row) {
-          if (a.splits == 1) {
+          if (!a.out_states) {
             if (a.lse) a.lse[tok * a.hq + h] = lse;
           } else {
-            a.state_lse[(tok * a.splits + split) * a.hq + h] = lse;
+            a.state_lse[(tok * a.states + split) * a.hq + h] = lse;
           }
         }
       }

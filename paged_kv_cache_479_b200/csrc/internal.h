@@ -52,27 +52,10 @@ constexpr int kKvE5M2 = 2;  // FP8 E5M2 codes
 cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv,
                           int grid, cudaStream_t stream);
 
-// attention of every request's queries over one shared prefix (prefix.cu)
-struct PrefixArgs {
-  const void* q;               // [B][Hq][128]
-  const int32_t* prefix_pages; // ceil(prefix_len / page_size) page ids
-  float* state_o;              // [B][states][Hq][128] fp32, slot `split` written
-  float* state_lse;            // [B][states][Hq] fp32, natural log
-  int* err;
-  long long num_pages;
-  long long prefix_len;        // tokens
-  long long tokens_per_split;  // multiple of the prefix tile
-  int page_size, batch, hq, hkv, group, states, splits;
-  float scale_log2;
-  int one_box;
-};
-size_t prefix_smem_bytes();
-int prefix_rows_per_cta();
-int prefix_tile_tokens();
-cudaError_t launch_prefix(const CUtensorMap& tmap, const PrefixArgs& a, bool bf16, int row_blocks,
-                          cudaStream_t stream);
-
-// multi-token append attention (chunk_tc.cu)
+// many-row attention on tcgen05 (chunk_tc.cu): multi-token append attention
+// (rows from a host plan, each request's own pages, causal), or the shared
+// prefix of a cascade (prefix_pages set: rows = (request, head) pairs of every
+// request, keys = the prefix, no mask, fp32 states)
 struct ChunkArgs {
   const void* q;               // [nnz_q][Hq][128]
   const int32_t* qo_indptr;    // [B+1], qo_indptr[0] = 0
@@ -81,8 +64,12 @@ struct ChunkArgs {
   const int4* plan;            // row blocks {request, first row, rows, 0}
   void* out;                   // [nnz_q][Hq][128] (one split)
   float* lse;                  // [nnz_q][Hq] or null (one split)
-  float* state_o;              // [nnz_q][splits][Hq][128] (several splits)
-  float* state_lse;            // [nnz_q][splits][Hq]
+  float* state_o;              // [nnz_q][states][Hq][128]: slot `split` written
+  float* state_lse;            // [nnz_q][states][Hq]
+  const int32_t* prefix_pages; // shared prefix: its page ids (null for append attention)
+  long long prefix_len;        // shared prefix: tokens
+  int states;                  // state slots per row
+  int out_states;              // 1: write fp32 states, 0: the final 16-bit output
   int* err;
   long long num_pages;
   long long nnz_q;             // rows of q / out
