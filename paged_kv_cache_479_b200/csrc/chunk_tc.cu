@@ -306,14 +306,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; ok && j < n; ++j) {
         // S(j+1) into the other buffers: it overwrites P(j-1), so PV(j-1) must be done
+        // (per row tile: S_A(j+1) is queued behind PV_B(j-1), so the tensor pipe
+        // does not drain while this thread waits for PV_B(j-1))
         if (j + 1 < n) {
           ok = mbar_wait_bounded(smem_u32(&ctl.kv_full[(j + 1) % kStages]), ((j + 1) / kStages) & 1,
                                  &ctl.abort, a.err);
-          for (int t = 0; ok && t < tiles && j >= 1; ++t)
-            ok = mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (j - 1) & 1, &ctl.abort, a.err);
+          for (int t = 0; ok && t < tiles; ++t) {
+            if (j >= 1)
+              ok = mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (j - 1) & 1, &ctl.abort, a.err);
+            if (!ok) break;
+            umma::fence_after_sync();
+            issue_s(j + 1, t);
+          }
           if (!ok) break;
-          umma::fence_after_sync();
-          for (int t = 0; t < tiles; ++t) issue_s(j + 1, t);
         }
         for (int t = 0; ok && t < tiles; ++t) {
           ok = mbar_wait_bounded(smem_u32(&ctl.p_full[t][j & 1]), (j >> 1) & 1, &ctl.abort, a.err);
@@ -393,9 +398,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx[u] = x[u];
 #pragma unroll
-      for (int k = 8; k < 64; ++k) mx[k & 7] = fmaxf(mx[k & 7], x[k]);
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
+      for (int k = 8; k < 64; k += 16) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = max3(mx[u], x[k + u], x[k + 8 + u < 64 ? k + 8 + u : k + u]);
+      }
+      const float mt = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * sl2;
       const bool move = mt > m_used + kRescaleThreshold;
       // O (and l) were accumulated against m_used: rescale the rows that move
       // their maximum, once PV(j-1) is done (the whole warp loads and stores)
@@ -420,23 +427,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (move) m_used = mt;
       const float mref = m_used == -INFINITY ? 0.f : m_used;
       // P = 2^(x * scale - m): high part = top 16 bits (bf16 truncation), low
-      // part = the exact remainder rounded to bf16; fp16: one rounding
+      // part = the exact remainder rounded to bf16; fp16: one rounding.  Two
+      // keys per paired-fp32 instruction.
       uint32_t hi[32], lo[32];
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint64_t scale2 = f2_pack(sl2, sl2), neg_m2 = f2_pack(-mref, -mref);
+      uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const float p0 = ex2(fmaf(x[2 * k], sl2, -mref)), p1 = ex2(fmaf(x[2 * k + 1], sl2, -mref));
-        ps[k & 3] += p0 + p1;
+        const float2 e = f2_unpack(f2_fma(f2_pack(x[2 * k], x[2 * k + 1]), scale2, neg_m2));
+        const float p0 = ex2(e.x), p1 = ex2(e.y);
+        const uint64_t pp = f2_pack(p0, p1);
+        acc[k & 1] = f2_add(acc[k & 1], pp);
         if constexpr (BF16) {
           const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
           hi[k] = prmt(b0, b1, 0x7632u);
-          lo[k] = pack2<true>(p0 - __uint_as_float(b0 & 0xffff0000u),
-                              p1 - __uint_as_float(b1 & 0xffff0000u));
+          const float2 rem = f2_unpack(f2_sub(pp, f2_pack(__uint_as_float(b0 & 0xffff0000u),
+                                                          __uint_as_float(b1 & 0xffff0000u))));
+          lo[k] = pack2<true>(rem.x, rem.y);
         } else {
           hi[k] = pack2<false>(p0, p1);
         }
       }
-      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      const float2 s2 = f2_unpack(f2_add(acc[0], acc[1]));
+      l += s2.x + s2.y;
       umma::st32(t_s, hi);
       if constexpr (BF16) umma::st32(t_s + 32u, lo);
       // V rows past the tile's keys may hold anything (even NaN): row tile A
