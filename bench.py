@@ -62,6 +62,9 @@ def parse():
     p.add_argument("--chunk", choices=["prefill", "spec"], default=None,
                    help="time multi-token append attention instead of the decode: chunked "
                         "prefill (TFLOP/s) or speculative verification (GB/s)")
+    p.add_argument("--chunk-path", choices=["auto", "tc", "short"], default="auto",
+                   help="append attention kernel: tcgen05 row blocks, the short-chunk decode "
+                        "schedule (q_len * G <= 16), or auto (short when it applies)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget for cpu_baseline")
     p.add_argument("--ref-seconds", type=float, default=150.0, help="oracle time budget of the reference arm")
     return p.parse_args()
@@ -607,6 +610,13 @@ def run_chunk(args):
     plan = t(plan_h)
     need = pkv.append_attention_workspace_bytes(int(qo[-1]), w.num_qo_heads, S)
     ws = torch.zeros(need // 4 + 64, dtype=torch.int32, device=dev)
+    # chunks of at most 16 / G tokens run on the decode schedule (short path)
+    G = w.num_qo_heads // w.num_kv_heads
+    mq = int(q_lens.max())
+    short = args.chunk_path == "short" or (args.chunk_path == "auto" and mq * G <= 16)
+    if short:
+        need_s = pkv.append_attention_short_workspace_bytes(w.num_qo_heads, w.num_kv_heads, mq)
+        ws_s = torch.zeros(need_s // 4 + 64, dtype=torch.int32, device=dev)
     out = torch.empty_like(batches[0][0])
     lse = torch.empty(out.shape[:2], dtype=torch.float32, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -617,9 +627,14 @@ def run_chunk(args):
                             stream=torch.cuda.current_stream(dev))
 
     def attn_call(bt):
-        pkv.append_attention(bt[0], qo_d, bt[1], table, plan, S, workspace=ws, out=out, lse=lse,
-                             sm_scale=w.sm_scale, error_word=err,
-                             stream=torch.cuda.current_stream(dev))
+        if short:
+            pkv.append_attention_short(bt[0], qo_d, bt[1], table, mq, ws_s, out=out, lse=lse,
+                                       sm_scale=w.sm_scale, error_word=err,
+                                       stream=torch.cuda.current_stream(dev))
+        else:
+            pkv.append_attention(bt[0], qo_d, bt[1], table, plan, S, workspace=ws, out=out,
+                                 lse=lse, sm_scale=w.sm_scale, error_word=err,
+                                 stream=torch.cuda.current_stream(dev))
 
     def graphed(fn, bt):
         if args.no_graph:
@@ -685,21 +700,27 @@ def run_chunk(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "query_tokens": nnz,
-                       "kv_tokens_after_append": int(w.kv_lens.sum()), "splits": S,
-                       "row_blocks": int(plan_h.shape[0]), "flops_per_step": flops,
+                       "kv_tokens_after_append": int(w.kv_lens.sum()),
+                       "path": ("short chunks on the decode schedule (pkv_append_attention_short)"
+                                if short else "tcgen05 row blocks (pkv_append_attention)"),
+                       "splits": None if short else S,
+                       "row_blocks": None if short else int(plan_h.shape[0]),
+                       "flops_per_step": flops,
                        "attention_bytes_per_step": attn_bytes,
                        "l2": f"2 rotating batch copies of {kv / 1e6:.0f} MB K/V",
                        "launch": "append and append attention captured as CUDA graphs",
                        "parallelism": f"dp{world} (independent batches per GPU)"},
             "us_per_step": round(ms / K * 1e3, 2),
             "tokens_per_s": round(nnz * world / (ms / K / 1e3), 1),
-            "roofline": {"bound": bound, "kernel": "chunk_kernel" + (" + merge" if S > 1 else ""),
+            "roofline": {"bound": bound,
+                         "kernel": ("decode_kernel (short chunks)" if short
+                                    else "chunk_kernel" + (" + merge" if S > 1 else "")),
                          "achieved": round(achieved, 1), "peak": peak, "unit": runit,
                          "frac": round(achieved / peak, 4),
                          "peak_kind": f"{kind} (MEASURED_PEAKS.json "
                                       f"{'bf16_tflops, burst' if bound == 'tensor' else 'hbm_gbs'})",
                          "traffic": None, "avg_launch_us": round(attn_ms * 1e3, 2)},
-            "gpu_launches": K * (2 + (1 if S > 1 else 0)),
+            "gpu_launches": K * (2 + (1 if S > 1 and not short else 0)),
             "e2e": None,
             "clocks": clocks.summary(t_host0, t_host1),
         }

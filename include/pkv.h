@@ -323,6 +323,34 @@ PKV_API pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr,
                                         int32_t* error_word, void* stream);
 
 /*
+ * pkv_append_attention_short -- pkv_append_attention (no window) for chunks of
+ * at most max_q_len tokens with max_q_len * G <= 16 (G = num_qo_heads /
+ * num_kv_heads), e.g. the verification of a few speculative tokens.  It runs
+ * the decode kernel's split-KV schedule with the chunk's (token, head) pairs
+ * as the columns of its MMAs, so each K/V tile is read once per (request, kv
+ * head) and the work is spread over the SMs by cost whatever the length mix.
+ *   q, qo_indptr, nnz_q, out, lse  as in pkv_append_attention
+ *   max_q_len    host bound on every request's q_len (1 <= max_q_len, max_q_len
+ *                * G <= 16, else PKV_ERR_UNSUPPORTED); a request whose q_len is
+ *                larger, or larger than its cache, sets PKV_DEVERR_APPEND and its
+ *                rows are left unwritten; requests with q_len = 0 write nothing
+ *   pool, table  descriptors (16-bit pools, head_dim 128, either layout and form)
+ *   num_partitions, workspace  as in pkv_decode, the workspace sized by
+ *                pkv_append_attention_short_workspace_bytes (device, zero-filled
+ *                once; the kernel leaves its counters zeroed)
+ * Same results as pkv_append_attention up to rounding order.
+ */
+PKV_API size_t pkv_append_attention_short_workspace_bytes(int num_qo_heads, int num_kv_heads,
+                                                          int max_q_len, int num_partitions);
+PKV_API pkv_status pkv_append_attention_short(const void* q, const int32_t* qo_indptr,
+                                              int64_t nnz_q, int max_q_len, int num_qo_heads,
+                                              const pkv_pool_desc* pool,
+                                              const pkv_table_desc* table, float sm_scale,
+                                              int num_partitions, void* workspace,
+                                              size_t workspace_bytes, void* out, float* lse,
+                                              int32_t* error_word, void* stream);
+
+/*
  * pkv_cascade_decode -- pkv_decode for a batch whose requests all begin with
  * the same shared prefix (a system prompt stored once in shared pages: physical
  * page sharing between requests with a common prefix, "大模型推理极致优化：

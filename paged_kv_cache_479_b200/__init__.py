@@ -24,11 +24,15 @@ Functions (C names in parentheses):
   append_attention       (pkv_append_attention)  a chunk of query tokens per request,
                          causal over its cache (chunked prefill, speculative tokens)
   append_attention_plan  (pkv_append_attention_plan)  its host-side row-block plan
+  append_attention_short (pkv_append_attention_short)  the same for chunks of at most
+                         16 / G tokens (speculative verification) on the decode schedule
 """
 from ._binding import (  # noqa: F401
     BF16,
     append_attention,
     append_attention_plan,
+    append_attention_short,
+    append_attention_short_workspace_bytes,
     append_attention_workspace_bytes,
     F16,
     F32,
@@ -77,4 +81,5 @@ pkv_decode_ex = paged_decode_attention_ex
 pkv_append_ex = paged_kv_append_ex
 pkv_decode_fp8 = paged_decode_attention_fp8
 pkv_append_attention = append_attention
+pkv_append_attention_short = append_attention_short
 pkv_append_fp8 = paged_kv_append_fp8

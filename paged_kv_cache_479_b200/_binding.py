@@ -75,6 +75,9 @@ _SIGNATURES["pkv_append_attention_plan"] = (
 _SIGNATURES["pkv_append_attention_workspace_bytes"] = ([_I64, _I32, _I32], _SZ)
 _SIGNATURES["pkv_append_attention"] = (
     [_P, _P, _I64, _I32, _PP, _TP, _P, _I64, _I32, _I32, _I32, _F32, _P, _SZ, _P, _P, _P, _P], _I32)
+_SIGNATURES["pkv_append_attention_short_workspace_bytes"] = ([_I32, _I32, _I32, _I32], _SZ)
+_SIGNATURES["pkv_append_attention_short"] = (
+    [_P, _P, _I64, _I32, _I32, _PP, _TP, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
 _SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
 _SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
@@ -442,6 +445,37 @@ def append_attention(q, qo_indptr, pool, table: TableDesc, plan, num_splits: int
                                     _ptr(out), _ptr(lse), _ptr(error_word),
                                     _stream(stream, q.device))
     _check(st, "pkv_append_attention")
+    return out, lse
+
+
+def append_attention_short_workspace_bytes(num_qo_heads: int, num_kv_heads: int, max_q_len: int,
+                                           num_partitions: int = 0) -> int:
+    return int(lib().pkv_append_attention_short_workspace_bytes(num_qo_heads, num_kv_heads,
+                                                               max_q_len, num_partitions))
+
+
+def append_attention_short(q, qo_indptr, pool, table: TableDesc, max_q_len: int, workspace,
+                           layout: str = "HND", num_partitions: int = 0, out=None, lse=None,
+                           sm_scale=None, error_word=None, stream=None, return_lse: bool = True):
+    """pkv_append_attention_short: append attention (no window) for chunks of at
+    most max_q_len tokens, max_q_len * (Hq / Hkv) <= 16, on the decode kernel's
+    schedule.  workspace: zero-filled device buffer of
+    append_attention_short_workspace_bytes bytes."""
+    _dev_tensor(q, "q", pool.dtype)
+    _dev_tensor(qo_indptr, "qo_indptr", torch.int32)
+    pd = pool_desc(pool, layout)
+    nnz, hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((nnz, hq), dtype=torch.float32, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_append_attention_short(_ptr(q), _ptr(qo_indptr), nnz, max_q_len, hq,
+                                          ctypes.byref(pd), ctypes.byref(table), scale,
+                                          num_partitions, _ptr(workspace), ws_bytes, _ptr(out),
+                                          _ptr(lse), _ptr(error_word), _stream(stream, q.device))
+    _check(st, "pkv_append_attention_short")
     return out, lse
 
 

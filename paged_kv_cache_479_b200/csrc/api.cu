@@ -47,9 +47,11 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 constexpr int kDecodeHeadDim = 128;
 constexpr int kMaxGroup = 8;
+constexpr int kMaxShortCols = 16;  // short chunks: q_len * G columns per (request, kv head)
 constexpr int kMaxPartitions = 1 << 20;
 
-// workspace layout: counters int32[N] | part_lse float[2N][G] | part_o float[2N][G][128]
+// workspace layout: counters int32[N] | part_lse float[2N][C] | part_o float[2N][C][128],
+// C = state columns per slot (G for the decode, 8 or 16 for short chunks)
 struct WsLayout {
   size_t counters, part_lse, part_o, total;
 };
@@ -219,7 +221,8 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
                       int num_partitions, void* workspace, size_t workspace_bytes, void* out,
                       float* lse, int32_t* error_word, void* stream, int out_f32,
                       long long out_rs, long long lse_rs, int kv_dtype = -1,
-                      float k_scale = 1.f, float v_scale = 1.f) {
+                      float k_scale = 1.f, float v_scale = 1.f,
+                      const int32_t* qo_indptr = nullptr, int64_t nnz_q = 0, int max_q_len = 1) {
   if (kv_dtype < 0) kv_dtype = dtype;
   if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1)
     return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
@@ -234,7 +237,13 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
     return fail(PKV_ERR_INVALID_ARG, "num_qo_heads must be a multiple of num_kv_heads");
   if (head_dim != kDecodeHeadDim) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 128");
   const int group = num_qo_heads / num_kv_heads;
-  if (group > kMaxGroup) return fail(PKV_ERR_UNSUPPORTED, "GQA group must be 1..8");
+  // columns per (request, kv head): G heads of each of up to max_q_len tokens
+  const int64_t cols = (int64_t)group * (qo_indptr ? max_q_len : 1);
+  if (qo_indptr && (max_q_len < 1 || cols > kMaxShortCols))
+    return fail(PKV_ERR_UNSUPPORTED, "short chunks need 1 <= max_q_len and max_q_len * G <= 16");
+  if (!qo_indptr && group > kMaxGroup) return fail(PKV_ERR_UNSUPPORTED, "GQA group must be 1..8");
+  const int nq = cols > kMaxGroup ? 2 : 1;
+  const int pcols = qo_indptr ? kMaxGroup * nq : group;
   if (!valid_page_size(page_size))
     return fail(PKV_ERR_UNSUPPORTED, "page_size must be 16, 32, 64, 128 or 256");
   if (num_pages > 0x7fffffffLL) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31-1 pages");
@@ -253,7 +262,7 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   int N = num_partitions;
   if (N == 0) N = current_device_partitions();
   if (N <= 0) return fail(PKV_ERR_CUDA, "cannot query the SM count");
-  const WsLayout L = ws_layout(group, N);
+  const WsLayout L = ws_layout(pcols, N);
   if (!aligned(workspace, 256)) return fail(PKV_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   if (workspace_bytes < L.total)
     return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes, %zu needed", workspace_bytes, L.total);
@@ -288,11 +297,15 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.out_f32 = out_f32;
   a.out_rs = out_rs;
   a.lse_rs = lse_rs;
+  a.qo_indptr = qo_indptr;
+  a.nnz_q = nnz_q;
+  a.pcols = pcols;
+  a.max_cols = (int)cols;
   cudaError_t e =
       pkv::launch_decode(tmap, a, dtype == PKV_BF16,
                          kv_dtype == PKV_FP8_E4M3 ? pkv::kKvE4M3
                          : kv_dtype == PKV_FP8_E5M2 ? pkv::kKvE5M2 : pkv::kKv16,
-                         N, static_cast<cudaStream_t>(stream));
+                         nq, N, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return ok();
 }
@@ -795,6 +808,41 @@ int64_t pkv_append_attention_plan(const int32_t* qo_indptr_h, const int32_t* kv_
     *num_splits = (int32_t)s;
   }
   return count;
+}
+
+size_t pkv_append_attention_short_workspace_bytes(int num_qo_heads, int num_kv_heads,
+                                                  int max_q_len, int num_partitions) {
+  if (num_kv_heads < 1 || num_qo_heads < num_kv_heads || num_qo_heads % num_kv_heads != 0 ||
+      max_q_len < 1)
+    return 0;
+  const int64_t cols = (int64_t)(num_qo_heads / num_kv_heads) * max_q_len;
+  if (cols > kMaxShortCols) return 0;
+  int N = num_partitions;
+  if (N == 0) N = current_device_partitions();
+  if (N <= 0 || N > kMaxPartitions) return 0;
+  return ws_layout(cols > kMaxGroup ? 2 * kMaxGroup : kMaxGroup, N).total;
+}
+
+pkv_status pkv_append_attention_short(const void* q, const int32_t* qo_indptr, int64_t nnz_q,
+                                      int max_q_len, int num_qo_heads, const pkv_pool_desc* pool,
+                                      const pkv_table_desc* table, float sm_scale,
+                                      int num_partitions, void* workspace, size_t workspace_bytes,
+                                      void* out, float* lse, int32_t* error_word, void* stream) {
+  if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
+  pkv::TableView tv;
+  const int32_t* ids = nullptr;
+  pkv_status st = table_view(table, &tv, &ids);
+  if (st != PKV_OK) return st;
+  if (pool->dtype != PKV_F16 && pool->dtype != PKV_BF16)
+    return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_F16 or PKV_BF16");
+  if (nnz_q < 0) return fail(PKV_ERR_INVALID_ARG, "nnz_q < 0");
+  if (table->batch > 0 && !qo_indptr) return fail(PKV_ERR_INVALID_ARG, "null qo_indptr");
+  if (nnz_q == 0) return ok();
+  return decode_impl(q, num_qo_heads, pool->data, pool->num_pages, pool->page_size,
+                     pool->num_kv_heads, pool->head_dim, pool->dtype, pool->layout, tv, ids,
+                     table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
+                     error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
+                     num_qo_heads, -1, 1.f, 1.f, qo_indptr, nnz_q, max_q_len);
 }
 
 size_t pkv_append_attention_workspace_bytes(int64_t nnz_q, int num_qo_heads, int num_splits) {

@@ -38,6 +38,12 @@
 //                  last partition to arrive (atomic counter, no waiting)
 //                  merges the partial states by their log-sum-exp weights.
 //
+// Short chunks (DecodeArgs::qo_indptr set): a request's q_len chunk tokens
+// (q_len * G <= 16) each attend causally over the cache; the pair's columns
+// are then (chunk token i, head h) at i * G + h, in two n8 column tiles when
+// there are more than 8 (NQ = 2), and the keys of column i end at position
+// L - q_len + i.  Every K/V tile is still read once per (request, kv head).
+//
 // Tokens past a request's length in its last tile are excluded by setting
 // their scores to -inf (a select, never a multiply) and zeroing their V rows
 // in shared memory, so whatever those slots hold (even NaN) never reaches
@@ -72,9 +78,10 @@ constexpr int kSlotBytes = 2 * kTileBytes;        // K + V: 8 KiB
 // same bytes are in flight.
 constexpr int kMaxStages = 2 * kStages;
 constexpr int kSegRecs = 16;                      // segment records in flight
-constexpr int kMaxGroup = 8;
+constexpr int kMaxGroup = 8;                      // columns of one n8 MMA tile
 constexpr int kQBufs = 8;                         // staged query blocks in flight
-constexpr int kQBufBytes = kMaxGroup * 128 * 2;   // G query rows: up to 2 KiB
+// a staged query block: the pair's columns (up to 8 NQ rows of 128 dims)
+constexpr int q_buf_bytes(int nq) { return nq * kMaxGroup * 128 * 2; }
 // The producer refills query buffer (and record) seg % n for segment seg + n
 // only after issuing every tile of segments seg .. seg+n-1 (each a multiple of
 // 8 tiles, at least 8).  With S ring slots that means the tiles up to
@@ -98,8 +105,10 @@ constexpr int kMetaEnd = 1 << 9;
 constexpr int kMetaSegShift = 12;
 
 struct SegRec {
-  int b, kvh, slot, c_first, ncover, pad;
+  int b, kvh, slot, c_first, ncover;
+  int ncol;             // columns with a query row (G, or q_len * G; 0 = none)
   long long pair_start;
+  long long q_row;      // row of q / out of the first column's token
 };
 
 struct __align__(16) Ctl {
@@ -126,8 +135,10 @@ struct Scratch {
 };
 
 constexpr size_t kRingBytes = (size_t)kStages * kSlotBytes;
-constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kRingBytes + (size_t)kQBufs * kQBufBytes +
-                              sizeof(Ctl) + sizeof(Scratch);
+constexpr size_t smem_bytes(int nq) {
+  return 1024 /*alignment slack*/ + kRingBytes + (size_t)kQBufs * q_buf_bytes(nq) + sizeof(Ctl) +
+         sizeof(Scratch);
+}
 
 // output of (request b, query head h): 16-bit final outputs, or fp32 attention
 // states at a caller-chosen request stride (used when the result is merged later)
@@ -202,11 +213,15 @@ __device__ __forceinline__ uint32_t widen_hi(uint32_t r) {
   else return prmt(r, 0u, 0x3424u);
 }
 
-// KV: the pool's element type -- kKv16 (q's own 16-bit type), kKvE4M3, kKvE5M2
-template <bool BF16, int KV>
+// KV: the pool's element type -- kKv16 (q's own 16-bit type), kKvE4M3, kKvE5M2;
+// NQ: n8 column tiles per pair (2 only for short chunks over 16-bit pools)
+template <bool BF16, int KV, int NQ>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   constexpr bool FP8 = KV != kKv16;
+  static_assert(NQ == 1 || (NQ == 2 && !FP8), "two column tiles only for 16-bit pools");
+  constexpr int kCols = NQ * kMaxGroup;
+  constexpr int kQBufBytes = q_buf_bytes(NQ);
   // ring geometry of this KV type (16-bit: 16 slots of 8 KiB; 8-bit: 32 of 4 KiB)
   constexpr int kSt = FP8 ? 2 * kStages : kStages;
   constexpr int kTileB = FP8 ? kTileBytes / 2 : kTileBytes;
@@ -290,14 +305,19 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         const long long t0 = u > kSegmentCost ? u - kSegmentCost : 0;
         const int kvh0 = (int)((f0 - s0) / r.units);
         prefetch_l2(a.indices + r.page_base + (t0 * kTileTokens) / a.page_size);
-        prefetch_l2(static_cast<const uint16_t*>(a.q) + ((size_t)b * a.hq + (size_t)kvh0 * a.group) * kD);
+        const long long qr = a.qo_indptr ? a.qo_indptr[b] : b;
+        prefetch_l2(static_cast<const uint16_t*>(a.q) + ((size_t)qr * a.hq + (size_t)kvh0 * a.group) * kD);
       }
     }
     if (b < B && r.tiles == 0 && (b % (int)gridDim.x) == c) {
-      // a request with no tokens: attention over no keys -> o = 0, lse = -inf
-      for (int h = 0; h < a.hq; ++h) {
-        for (int d = 0; d < kD; d += 4) store_out4<BF16>(a, b, h, d, make_float4(0.f, 0.f, 0.f, 0.f));
-        store_lse(a, b, h, -INFINITY);
+      if (!a.qo_indptr) {
+        // a request with no tokens: attention over no keys -> o = 0, lse = -inf
+        for (int h = 0; h < a.hq; ++h) {
+          for (int d = 0; d < kD; d += 4) store_out4<BF16>(a, b, h, d, make_float4(0.f, 0.f, 0.f, 0.f));
+          store_lse(a, b, h, -INFINITY);
+        }
+      } else if (a.qo_indptr[b + 1] != a.qo_indptr[b] && a.err) {
+        atomicOr(a.err, kErrAppend);  // chunk tokens but no cache: they were never appended
       }
     }
     carry += chunk_total;
@@ -347,15 +367,30 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         r.c_first = pl.c_first;
         r.ncover = pl.ncover;
         r.pair_start = pstart;
-        // stage the segment's G query rows (contiguous in q) for the consumers
+        // the pair's query rows: its G heads of one token (decode) or of each
+        // of the chunk's tokens; a chunk that does not fit gets no columns
+        long long q_row = wk.b;
+        int q_len = 1;
+        if (a.qo_indptr) {
+          q_row = a.qo_indptr[wk.b];
+          const long long ql = (long long)a.qo_indptr[wk.b + 1] - q_row;
+          const bool fits = ql >= 1 && ql * G <= a.max_cols && ql * G <= kCols &&
+                            ql <= wk.ri.len && q_row >= 0 && q_row + ql <= a.nnz_q;
+          if (!fits && ql != 0 && a.err) atomicOr(a.err, kErrAppend);
+          q_len = fits ? (int)ql : 0;
+        }
+        r.ncol = q_len * G;
+        r.q_row = q_row;
+        // stage them (G contiguous rows per token) for the consumers
         const int qb = seg & (kQBufs - 1);
         const uint32_t qbar = smem_u32(&ctl.qfull[qb]);
-        const uint32_t qbytes = (uint32_t)a.group * kD * 2;
-        mbar_arrive_expect_tx(qbar, qbytes);
-        bulk_load(smem_u32(qbuf + (size_t)qb * kQBufBytes),
-                  static_cast<const uint16_t*>(a.q) +
-                      ((size_t)wk.b * a.hq + (size_t)wk.kvh * a.group) * kD,
-                  qbytes, qbar);
+        const uint32_t qbytes = (uint32_t)G * kD * 2;
+        mbar_arrive_expect_tx(qbar, qbytes * (uint32_t)q_len);
+        for (int i = 0; i < q_len; ++i)
+          bulk_load(smem_u32(qbuf + (size_t)qb * kQBufBytes + (size_t)i * qbytes),
+                    static_cast<const uint16_t*>(a.q) +
+                        ((size_t)(q_row + i) * a.hq + (size_t)wk.kvh * G) * kD,
+                    qbytes, qbar);
         // last segment of this request: warm L2 with the next request's table entries
         if (wk.kvh == Hkv - 1 && wk.b + 1 < B) {
           if (a.tv.indptr) {
@@ -386,8 +421,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           }
           const long long tok0 = (t0 + k) * kTileTokens;
           yoff = (int)(tok0 & (ps - 1));
+          // tokens from the tile's first to the request's end, capped at 31: the
+          // tile's valid count, and (for short chunks) each key's distance from
+          // the end, which decides the causal mask
           const long long left = wk.ri.len - tok0;
-          valid = left < kTileTokens ? (int)left : kTileTokens;
+          valid = left < kMetaValid ? (int)left : kMetaValid;
         } else {
           page = -1;
         }
@@ -476,22 +514,33 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   }
 
   // =========================== consumers ===========================
-  const int g = lane >> 2;     // MMA row group: token g / g+8 of the tile, head g of P^T
-  const int cq = lane & 3;     // MMA column pair: heads 2cq, 2cq+1 of S^T
+  const int g = lane >> 2;     // MMA row group: token g / g+8 of the tile, column g of P^T
+  const int cq = lane & 3;     // MMA column pair: columns 2cq, 2cq+1 of S^T (per n8 tile)
   const int mi = lane >> 3;    // ldmatrix: which 8x8 matrix this lane addresses
   const int r8 = lane & 7;     // ldmatrix: row within it
   const float sl2 = a.scale_log2;
   const int ct = warp * 32 + lane;
   const uint32_t ring0 = smem_u32(ring);
 
-  uint32_t qf[8][2];
+  uint32_t qf[NQ][8][2];
   float qsc0 = sl2, qsc1 = sl2;  // score scale of S^T columns 2cq, 2cq+1 (E4M3 pools)
-  float o[8][4];
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float o[NQ][8][4];
+  float m0[NQ], m1[NQ], l0[NQ], l1[NQ];
+  // a key at distance e - r from the request's end is visible to column
+  // (token i, head h) of a chunk of q_len tokens when e - r >= q_len - i;
+  // decode (q_len = 1) and columns without a query row need only e - r >= 1
+  int need0[NQ], need1[NQ];
+#pragma unroll
+  for (int nt = 0; nt < NQ; ++nt) {
+    m0[nt] = m1[nt] = -INFINITY;
+    l0[nt] = l1[nt] = 0.f;
+    need0[nt] = need1[nt] = 1;
+  }
   int cur_seg = -1;
   SegRec rec;
   rec.b = 0;
   rec.kvh = 0;
+  rec.ncol = 0;
   uint32_t cons_phase = 0;
   bool clean = true;
 
@@ -507,7 +556,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     if (sid != cur_seg) {
       cur_seg = sid;
       rec = ctl.seg[sid];
-      if ((unsigned)rec.b >= (unsigned)B || (unsigned)rec.kvh >= (unsigned)Hkv) {
+      if ((unsigned)rec.b >= (unsigned)B || (unsigned)rec.kvh >= (unsigned)Hkv ||
+          (unsigned)rec.ncol > (unsigned)kCols) {
         // never expected: a corrupted record would address out of bounds
         if (lane == 0 && a.err) atomicOr(a.err, kErrTimeout);
         ctl.abort = 1;
@@ -531,7 +581,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         uint2 raw[8];
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) raw[ch] = make_uint2(0u, 0u);
-        if (g < G) {
+        if (g < rec.ncol) {
           const uint8_t* qp = qbuf + (size_t)qb * kQBufBytes + ((size_t)g * kD + 4 * cq) * 2;
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) raw[ch] = *reinterpret_cast<const uint2*>(qp + ch * 32);
@@ -553,14 +603,14 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
             const float2 u = unpack2<true>(raw[ch].x), v = unpack2<true>(raw[ch].y);
-            qf[ch][0] = pack2<false>(u.x * f, u.y * f);
-            qf[ch][1] = pack2<false>(v.x * f, v.y * f);
+            qf[0][ch][0] = pack2<false>(u.x * f, u.y * f);
+            qf[0][ch][1] = pack2<false>(v.x * f, v.y * f);
           }
         } else {
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch) {
-            qf[ch][0] = raw[ch].x;
-            qf[ch][1] = raw[ch].y;
+            qf[0][ch][0] = raw[ch].x;
+            qf[0][ch][1] = raw[ch].y;
           }
         }
         // this lane's S^T columns are heads 2cq and 2cq+1 (held by lanes 8cq and 8cq+4)
@@ -568,30 +618,48 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         const int e1 = __shfl_sync(0xffffffffu, qexp, 8 * cq + 4);
         qsc0 = sl2 * __int_as_float((127 - e0) << 23);
         qsc1 = sl2 * __int_as_float((127 - e1) << 23);
-      } else if (g < G) {
-        const uint16_t* qp =
-            reinterpret_cast<const uint16_t*>(qbuf + (size_t)qb * kQBufBytes) + g * kD + 2 * cq;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          qf[j][0] = ld_u32(qp + j * 16);
-          qf[j][1] = ld_u32(qp + j * 16 + 8);
-        }
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) qf[j][0] = qf[j][1] = 0u;
-      }
+        for (int nt = 0; nt < NQ; ++nt) {
+          const int col = nt * kMaxGroup + g;
+          if (col < rec.ncol) {
+            const uint16_t* qp =
+                reinterpret_cast<const uint16_t*>(qbuf + (size_t)qb * kQBufBytes) + col * kD + 2 * cq;
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-      m0 = m1 = -INFINITY;
-      l0 = l1 = 0.f;
+            for (int j = 0; j < 8; ++j) {
+              qf[nt][j][0] = ld_u32(qp + j * 16);
+              qf[nt][j][1] = ld_u32(qp + j * 16 + 8);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) qf[nt][j][0] = qf[nt][j][1] = 0u;
+          }
+        }
+      }
+      const int q_len = rec.ncol / G;
+#pragma unroll
+      for (int nt = 0; nt < NQ; ++nt) {
+        const int c0 = nt * kMaxGroup + 2 * cq, c1 = c0 + 1;
+        need0[nt] = c0 < rec.ncol ? q_len - c0 / G : 1;
+        need1[nt] = c1 < rec.ncol ? q_len - c1 / G : 1;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+        m0[nt] = m1[nt] = -INFINITY;
+        l0[nt] = l1[nt] = 0.f;
+      }
     }
-    const int valid = (info & kMetaValid) > kTileTokens ? kTileTokens : (info & kMetaValid);
+    const int e_end = info & kMetaValid;  // tokens from the tile's first to the end (<= 31)
+    const int valid = e_end > kTileTokens ? kTileTokens : e_end;
     const uint32_t kb = ring0 + (uint32_t)s * kSlotB;
     const uint32_t vb = kb + kTileB;
     bool wrote_smem = false;
     if (valid > 0) {
-      // ---- S^T = K_tile . Q^T  (tokens on M, heads on N)
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+      // ---- S^T = K_tile . Q^T  (tokens on M, columns on N)
+      float sa[NQ][4], sb[NQ][4];
+#pragma unroll
+      for (int nt = 0; nt < NQ; ++nt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sa[nt][k] = sb[nt][k] = 0.f;
       if constexpr (FP8) {
         // one ldmatrix.x4 = tokens (0-7 | 8-15) x chunks (2jj | 2jj+1) of 16 codes;
         // lane (g, cq) gets codes 4cq .. 4cq+3 of token g's chunk, widened in pairs
@@ -602,10 +670,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           const int chunk = 2 * jj + (mi >> 1);
           uint32_t r0, r1, r2, r3;
           ldmatrix_x4(rowb + (uint32_t)(((chunk & 7) ^ r8) << 4), r0, r1, r2, r3);
-          mma_16816<false>(sa, widen_lo<KV>(r0), widen_lo<KV>(r1), widen_hi<KV>(r0),
-                           widen_hi<KV>(r1), qf[2 * jj][0], qf[2 * jj][1]);
-          mma_16816<false>(sb, widen_lo<KV>(r2), widen_lo<KV>(r3), widen_hi<KV>(r2),
-                           widen_hi<KV>(r3), qf[2 * jj + 1][0], qf[2 * jj + 1][1]);
+          mma_16816<false>(sa[0], widen_lo<KV>(r0), widen_lo<KV>(r1), widen_hi<KV>(r0),
+                           widen_hi<KV>(r1), qf[0][2 * jj][0], qf[0][2 * jj][1]);
+          mma_16816<false>(sb[0], widen_lo<KV>(r2), widen_lo<KV>(r3), widen_hi<KV>(r2),
+                           widen_hi<KV>(r3), qf[0][2 * jj + 1][0], qf[0][2 * jj + 1][1]);
         }
       } else {
         const int tok = ((mi & 1) << 3) + r8;
@@ -617,50 +685,60 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
               rowb + (uint32_t)(j >> 2) * kHalfBytes + (uint32_t)(((chunk & 7) ^ r8) << 4);
           uint32_t a0, a1, a2, a3;
           ldmatrix_x4(addr, a0, a1, a2, a3);
-          if (j & 1)
-            mma_16816<BF16>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-          else
-            mma_16816<BF16>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+#pragma unroll
+          for (int nt = 0; nt < NQ; ++nt) {
+            if (j & 1)
+              mma_16816<BF16>(sb[nt], a0, a1, a2, a3, qf[nt][j][0], qf[nt][j][1]);
+            else
+              mma_16816<BF16>(sa[nt], a0, a1, a2, a3, qf[nt][j][0], qf[nt][j][1]);
+          }
         }
       }
-      // ---- mask tokens past the request's end, online softmax (log2 units)
-      const bool v_lo = g < valid, v_hi = g + 8 < valid;
+      // ---- mask (past the end; causal within a chunk), online softmax (log2 units)
       const float sc0 = FP8 ? qsc0 : sl2, sc1 = FP8 ? qsc1 : sl2;
-      const float x0 = v_lo ? (sa[0] + sb[0]) * sc0 : -INFINITY;  // token g,   head 2cq
-      const float x1 = v_lo ? (sa[1] + sb[1]) * sc1 : -INFINITY;  // token g,   head 2cq+1
-      const float x2 = v_hi ? (sa[2] + sb[2]) * sc0 : -INFINITY;  // token g+8, head 2cq
-      const float x3 = v_hi ? (sa[3] + sb[3]) * sc1 : -INFINITY;  // token g+8, head 2cq+1
-      float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+      const int dlo = e_end - g, dhi = e_end - g - 8;  // distances of tokens g, g+8 from the end
+      uint32_t bh0[NQ], bh1[NQ], bl0[NQ], bl1[NQ];
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-      const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1);
-      const float p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
-      l0 = l0 * al0 + (p0 + p2);
-      l1 = l1 * al1 + (p1 + p3);
-      m0 = mn0;
-      m1 = mn1;
-      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+      for (int nt = 0; nt < NQ; ++nt) {
+        const float x0 = dlo >= need0[nt] ? (sa[nt][0] + sb[nt][0]) * sc0 : -INFINITY;  // token g,   col 2cq
+        const float x1 = dlo >= need1[nt] ? (sa[nt][1] + sb[nt][1]) * sc1 : -INFINITY;  // token g,   col 2cq+1
+        const float x2 = dhi >= need0[nt] ? (sa[nt][2] + sb[nt][2]) * sc0 : -INFINITY;  // token g+8, col 2cq
+        const float x3 = dhi >= need1[nt] ? (sa[nt][3] + sb[nt][3]) * sc1 : -INFINITY;  // token g+8, col 2cq+1
+        float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          o[mt][0] *= al0;
-          o[mt][1] *= al1;
-          o[mt][2] *= al0;
-          o[mt][3] *= al1;
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
         }
-      }
-      // ---- P^T as the B operand of the PV MMA (movmatrix transposes S^T's layout)
-      const uint32_t ph0 = pack2<kMmaBF16>(p0, p1), ph1 = pack2<kMmaBF16>(p2, p3);
-      const uint32_t bh0 = movmatrix_trans(ph0), bh1 = movmatrix_trans(ph1);
-      uint32_t bl0 = 0, bl1 = 0;
-      if constexpr (kMmaBF16) {
-        const float2 f0 = unpack2<true>(ph0), f1 = unpack2<true>(ph1);
-        bl0 = movmatrix_trans(pack2<true>(p0 - f0.x, p1 - f0.y));
-        bl1 = movmatrix_trans(pack2<true>(p2 - f1.x, p3 - f1.y));
+        const float mn0 = fmaxf(m0[nt], mx0), mn1 = fmaxf(m1[nt], mx1);
+        // a column that has seen no visible key yet keeps m = -inf: subtract 0
+        const float ms0 = mn0 == -INFINITY ? 0.f : mn0, ms1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float al0 = ex2(m0[nt] - ms0), al1 = ex2(m1[nt] - ms1);
+        const float p0 = ex2(x0 - ms0), p1 = ex2(x1 - ms1);
+        const float p2 = ex2(x2 - ms0), p3 = ex2(x3 - ms1);
+        l0[nt] = l0[nt] * al0 + (p0 + p2);
+        l1[nt] = l1[nt] * al1 + (p1 + p3);
+        m0[nt] = mn0;
+        m1[nt] = mn1;
+        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            o[nt][mt][0] *= al0;
+            o[nt][mt][1] *= al1;
+            o[nt][mt][2] *= al0;
+            o[nt][mt][3] *= al1;
+          }
+        }
+        // ---- P^T as the B operand of the PV MMA (movmatrix transposes S^T's layout)
+        const uint32_t ph0 = pack2<kMmaBF16>(p0, p1), ph1 = pack2<kMmaBF16>(p2, p3);
+        bh0[nt] = movmatrix_trans(ph0);
+        bh1[nt] = movmatrix_trans(ph1);
+        bl0[nt] = bl1[nt] = 0u;
+        if constexpr (kMmaBF16) {
+          const float2 f0 = unpack2<true>(ph0), f1 = unpack2<true>(ph1);
+          bl0[nt] = movmatrix_trans(pack2<true>(p0 - f0.x, p1 - f0.y));
+          bl1[nt] = movmatrix_trans(pack2<true>(p2 - f1.x, p3 - f1.y));
+        }
       }
       // ---- zero V rows past the end (their slots may hold anything, even NaN)
       if (valid < kTileTokens) {
@@ -680,7 +758,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         wrote_smem = true;
         __syncwarp();
       }
-      // ---- O^T += V_tile^T . P^T   (dims on M, heads on N, tokens on K)
+      // ---- O^T += V_tile^T . P^T   (dims on M, columns on N, tokens on K)
       if constexpr (FP8) {
         // ldmatrix.trans of tokens (0-7 | 8-15) x chunks (2jj | 2jj+1) hands lane
         // (g, cq) codes V[2cq][2g], V[2cq][2g+1], V[2cq+1][2g], V[2cq+1][2g+1];
@@ -706,8 +784,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
               y[k] = prmt(rr[k], 0u, 0x3414u);
             }
           }
-          mma_16816<false>(o[2 * jj], x[0], x[1], x[2], x[3], bh0, bh1);
-          mma_16816<false>(o[2 * jj + 1], y[0], y[1], y[2], y[3], bh0, bh1);
+          mma_16816<false>(o[0][2 * jj], x[0], x[1], x[2], x[3], bh0[0], bh1[0]);
+          mma_16816<false>(o[0][2 * jj + 1], y[0], y[1], y[2], y[3], bh0[0], bh1[0]);
         }
       } else {
         const int tok = ((mi >> 1) << 3) + r8;
@@ -719,8 +797,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
               rowb + (uint32_t)(mt >> 2) * kHalfBytes + (uint32_t)(((chunk & 7) ^ r8) << 4);
           uint32_t a0, a1, a2, a3;
           ldmatrix_x4_trans(addr, a0, a1, a2, a3);
-          mma_16816<BF16>(o[mt], a0, a1, a2, a3, bh0, bh1);
-          if constexpr (BF16) mma_16816<BF16>(o[mt], a0, a1, a2, a3, bl0, bl1);
+#pragma unroll
+          for (int nt = 0; nt < NQ; ++nt) {
+            mma_16816<BF16>(o[nt][mt], a0, a1, a2, a3, bh0[nt], bh1[nt]);
+            if constexpr (BF16) mma_16816<BF16>(o[nt][mt], a0, a1, a2, a3, bl0[nt], bl1[nt]);
+          }
         }
       }
     }
@@ -730,58 +811,68 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 
     if (info & kMetaSegLast) {
       // ================= end of segment: merge the 8 warps' states =================
-      if (!cons_sync(ctl, cons_phase, a.err)) {  // previous merge done with scratch
-        clean = false;
-        break;
-      }
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-      }
-      if (g == 0) {
-        scr.m[warp][2 * cq] = m0;
-        scr.m[warp][2 * cq + 1] = m1;
-        scr.l[warp][2 * cq] = l0;
-        scr.l[warp][2 * cq + 1] = l1;
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        // dims of accumulator rows g and g+8 (see the PV MMA of each KV type)
-        const int d0 = FP8 ? 32 * (mt >> 1) + 2 * g + (mt & 1) : mt * 16 + g;
-        const int d1 = FP8 ? d0 + 16 : d0 + 8;
-        scr.o[warp][2 * cq][d0] = o[mt][0];
-        scr.o[warp][2 * cq + 1][d0] = o[mt][1];
-        scr.o[warp][2 * cq][d1] = o[mt][2];
-        scr.o[warp][2 * cq + 1][d1] = o[mt][3];
-      }
-      if (!cons_sync(ctl, cons_phase, a.err)) {
-        clean = false;
-        break;
-      }
+      // one n8 column tile at a time through the scratch area
       const bool direct = rec.ncover == 1;
-      for (int e = ct; e < G * kD; e += kConsumerThreads) {
-        const int h = e >> 7, d = e & (kD - 1);
-        float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, scr.m[w][h]);
-        float L = 0.f, acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float wt = ex2(scr.m[w][h] - M);
-          L += wt * scr.l[w][h];
-          acc += wt * scr.o[w][h][d];
+      for (int nt = 0; nt < NQ; ++nt) {
+        if (!cons_sync(ctl, cons_phase, a.err)) {  // previous merge done with scratch
+          clean = false;
+          break;
         }
-        const float val = FP8 ? acc * a.v_scale / L : acc / L;
-        if (direct) {
-          const size_t hq = (size_t)rec.kvh * G + h;
-          store_out1<BF16>(a, rec.b, hq, d, val);
-          if (d == 0) store_lse(a, rec.b, hq, (M + log2f(L)) * kLn2);
-        } else {
-          a.part_o[((size_t)rec.slot * G + h) * kD + d] = val;
-          if (d == 0) a.part_lse[(size_t)rec.slot * G + h] = M + log2f(L);
+        float la = l0[nt], lb = l1[nt];
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          la += __shfl_xor_sync(0xffffffffu, la, off);
+          lb += __shfl_xor_sync(0xffffffffu, lb, off);
+        }
+        if (g == 0) {
+          scr.m[warp][2 * cq] = m0[nt];
+          scr.m[warp][2 * cq + 1] = m1[nt];
+          scr.l[warp][2 * cq] = la;
+          scr.l[warp][2 * cq + 1] = lb;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          // dims of accumulator rows g and g+8 (see the PV MMA of each KV type)
+          const int d0 = FP8 ? 32 * (mt >> 1) + 2 * g + (mt & 1) : mt * 16 + g;
+          const int d1 = FP8 ? d0 + 16 : d0 + 8;
+          scr.o[warp][2 * cq][d0] = o[nt][mt][0];
+          scr.o[warp][2 * cq + 1][d0] = o[nt][mt][1];
+          scr.o[warp][2 * cq][d1] = o[nt][mt][2];
+          scr.o[warp][2 * cq + 1][d1] = o[nt][mt][3];
+        }
+        if (!cons_sync(ctl, cons_phase, a.err)) {
+          clean = false;
+          break;
+        }
+        const int ncols = rec.ncol - nt * kMaxGroup;  // columns of this tile with a query row
+        for (int e = ct; e < ncols * kD && e < kMaxGroup * kD; e += kConsumerThreads) {
+          const int h = e >> 7, d = e & (kD - 1);
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, scr.m[w][h]);
+          const float Ms = M == -INFINITY ? 0.f : M;  // no visible key in this share
+          float L = 0.f, acc = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float wt = ex2(scr.m[w][h] - Ms);
+            L += wt * scr.l[w][h];
+            acc += wt * scr.o[w][h][d];
+          }
+          const float val = L > 0.f ? (FP8 ? acc * a.v_scale / L : acc / L) : 0.f;
+          const int col = nt * kMaxGroup + h;
+          if (direct) {
+            const size_t hq = (size_t)rec.kvh * G + col % G;
+            const size_t row = (size_t)rec.q_row + col / G;
+            store_out1<BF16>(a, row, hq, d, val);
+            if (d == 0) store_lse(a, row, hq, (M + log2f(L)) * kLn2);
+          } else {
+            a.part_o[((size_t)rec.slot * a.pcols + col) * kD + d] = val;
+            if (d == 0) a.part_lse[(size_t)rec.slot * a.pcols + col] = M + log2f(L);
+          }
         }
       }
+      if (!clean) break;
       if (!direct && ct == 0 && ctl.npend < kMaxPending) ctl.pend[ctl.npend++] = rec;
     }
   }
@@ -800,17 +891,19 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     }
   if (!cons_sync(ctl, cons_phase, a.err)) return;
   __threadfence();
-  // one warp per (pair, head); lane L owns dims 4L .. 4L+3
-  for (int item = warp; item < npend * G; item += kConsumerWarps) {
-    const int k = item / G, h = item % G;
-    if (!ctl.pend_last[k]) continue;
+  // one warp per (pair, column); lane L owns dims 4L .. 4L+3
+  const int P = a.pcols;  // state columns per slot
+  for (int item = warp; item < npend * kCols; item += kConsumerWarps) {
+    const int k = item / kCols, h = item % kCols;
+    if (!ctl.pend_last[k] || h >= ctl.pend[k].ncol) continue;
     const SegRec pr = ctl.pend[k];
     auto slot_of = [&](int j) { return state_slot(pr.c_first, j); };
     float M = -INFINITY;
     for (int j = lane; j < pr.ncover; j += 32)
-      M = fmaxf(M, __ldcg(a.part_lse + (size_t)slot_of(j) * G + h));
+      M = fmaxf(M, __ldcg(a.part_lse + (size_t)slot_of(j) * P + h));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    M = M == -INFINITY ? 0.f : M;  // (every column of a chunk sees key 0: not expected)
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     constexpr int kBatch = 8;  // partial states loaded together
@@ -822,8 +915,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         const int j = j0 + u;
         if (j < pr.ncover) {
           const int sl = slot_of(j);
-          wt[u] = __ldcg(a.part_lse + (size_t)sl * G + h);
-          v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * G + h) * kD) + lane);
+          wt[u] = __ldcg(a.part_lse + (size_t)sl * P + h);
+          v[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((size_t)sl * P + h) * kD) + lane);
         } else {
           wt[u] = -INFINITY;
           v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -839,34 +932,41 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         acc.w += w * v[u].w;
       }
     }
-    const float inv = 1.f / L;
-    const size_t hq = (size_t)pr.kvh * G + h;
-    store_out4<BF16>(a, pr.b, hq, 4 * lane,
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const size_t hq = (size_t)pr.kvh * G + h % G;
+    const size_t row = (size_t)pr.q_row + h / G;
+    store_out4<BF16>(a, row, hq, 4 * lane,
                      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
-    if (lane == 0) store_lse(a, pr.b, hq, (M + log2f(L)) * kLn2);
+    if (lane == 0) store_lse(a, row, hq, L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY);
   }
 }
 
 }  // namespace
 
-size_t decode_smem_bytes() { return kSmemBytes; }
+size_t decode_smem_bytes(int nq) { return smem_bytes(nq); }
 
-cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv,
+cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv, int nq,
                           int grid, cudaStream_t stream) {
   static_assert(sizeof(Ctl) % 16 == 0, "Ctl must keep Scratch 16-byte aligned");
   if (kv != kKv16 && kv != kKvE4M3 && kv != kKvE5M2) return cudaErrorInvalidValue;
-  const int variant = 2 * kv + (bf16 ? 1 : 0);
-  void (*kern)(const CUtensorMap, const DecodeArgs) =
-      kv == kKvE4M3 ? (bf16 ? decode_kernel<true, kKvE4M3> : decode_kernel<false, kKvE4M3>)
-      : kv == kKvE5M2 ? (bf16 ? decode_kernel<true, kKvE5M2> : decode_kernel<false, kKvE5M2>)
-                      : (bf16 ? decode_kernel<true, kKv16> : decode_kernel<false, kKv16>);
+  if (nq != 1 && (nq != 2 || kv != kKv16)) return cudaErrorInvalidValue;
+  using Kern = void (*)(const CUtensorMap, const DecodeArgs);
+  // variants: 16-bit (fp16, bf16), E4M3 (fp16, bf16), E5M2 (fp16, bf16), 16-bit NQ=2 (fp16, bf16)
+  static const Kern kKerns[8] = {
+      decode_kernel<false, kKv16, 1>,   decode_kernel<true, kKv16, 1>,
+      decode_kernel<false, kKvE4M3, 1>, decode_kernel<true, kKvE4M3, 1>,
+      decode_kernel<false, kKvE5M2, 1>, decode_kernel<true, kKvE5M2, 1>,
+      decode_kernel<false, kKv16, 2>,   decode_kernel<true, kKv16, 2>};
+  const int variant = (nq == 2 ? 6 : 2 * kv) + (bf16 ? 1 : 0);
+  const Kern kern = kKerns[variant];
+  const size_t smem = smem_bytes(nq);
   // the shared-memory opt-in is per function and device; do it once each
-  static bool attr_set[6][64] = {};
+  static bool attr_set[8][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !attr_set[variant][dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[variant][dev] = true;
   }
@@ -875,7 +975,7 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kDecodeThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -20,8 +20,8 @@ struct DecodeArgs {
   TableView tv;           // page table (CSR or dense block table)
   const int32_t* indices; // page ids: CSR indices, or the [B][max_blocks] block table
   int* counters;          // [N] arrival counters (zero between launches)
-  float* part_lse;        // [2N][G], log2 domain
-  float* part_o;          // [2N][G][128]
+  float* part_lse;        // [2N][pcols], log2 domain
+  float* part_o;          // [2N][pcols][128]
   int* err;               // device error word or null
   long long num_pages;
   int batch, hq, hkv, group, page_size;
@@ -31,6 +31,12 @@ struct DecodeArgs {
   int out_f32;            // 1: out is fp32 (an attention state for a later merge)
   long long out_rs;       // elements of out between consecutive requests (Hq * 128 when packed)
   long long lse_rs;       // elements of lse between consecutive requests (Hq when packed)
+  // short chunks: request b's query tokens are rows qo_indptr[b] .. of q / out
+  // (null for decode: one token, row b)
+  const int32_t* qo_indptr;
+  long long nnz_q;        // rows of q (short chunks)
+  int pcols;              // columns per partial-state slot (G for decode)
+  int max_cols;           // short chunks: the caller's bound on q_len * G
 };
 
 constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp
@@ -43,13 +49,14 @@ constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp
 constexpr int kDecodeStages = PKV_STAGES;        // K/V ring slots (8 KiB each) per CTA
 constexpr int kDecodeCtasPerSm = PKV_CTAS_PER_SM; // resident decode CTAs per SM
 
-size_t decode_smem_bytes();
+size_t decode_smem_bytes(int nq);
 // pool element types of the decode kernel
 constexpr int kKv16 = 0;    // q's own 16-bit type
 constexpr int kKvE4M3 = 1;  // FP8 E4M3 codes
 constexpr int kKvE5M2 = 2;  // FP8 E5M2 codes
 // bf16: q/out type (else fp16); kv: one of the pool element types above
-cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv,
+// nq: n8 column tiles per (request, kv head) -- 1, or 2 (16-bit pools only)
+cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv, int nq,
                           int grid, cudaStream_t stream);
 
 // many-row attention on tcgen05 (chunk_tc.cu): multi-token append attention

@@ -58,6 +58,30 @@ class ChunkCase:
         assert pkv.read_error_word(err) == 0
         return out, lse
 
+    def run_short(self, max_q_len, layout="HND", kind="csr", parts=0, out=None):
+        w = self.w
+        pool = self.pool.cuda()
+        if layout == "NHD":
+            pool = pool.permute(0, 1, 3, 2, 4).contiguous()
+        if kind == "csr":
+            keep = (i32(w.page_indptr), i32(w.page_indices), i32(w.last_page_len))
+            table = pkv.csr_table(*keep)
+        else:
+            bt, ctx = dense_block_table(w)
+            keep = (i32(bt), i32(ctx))
+            table = pkv.block_table(*keep)
+        nb = pkv.append_attention_short_workspace_bytes(w.num_qo_heads, w.num_kv_heads, max_q_len,
+                                                        parts)
+        assert nb > 0
+        ws = torch.zeros(nb // 4 + 64, dtype=torch.int32, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out, lse = pkv.append_attention_short(self.q.cuda(), i32(self.qo), pool, table, max_q_len,
+                                              ws, layout=layout, num_partitions=parts, out=out,
+                                              sm_scale=w.sm_scale, error_word=err)
+        torch.cuda.synchronize()
+        self.err = pkv.read_error_word(err)
+        return out, lse
+
     def oracle(self, window_left=-1, sink=0):
         w = self.w
         return oracle.append_attention(wl.bits(self.q), wl.bits(self.pool), odtype(w),
@@ -161,6 +185,104 @@ def test_chunked_prefill_shape_sampled():
             row = int(qo[b]) + i
             ro, rl = oracle.decode(wl.bits(q[row:row + 1]), sub, odtype(w), ip,
                                    inv.astype(np.int32), ll, w.sm_scale)
+            assert_parity(out[row:row + 1], lse[row:row + 1], ro, rl, what=f"b{b} i{i}")
+
+
+@pytest.mark.parametrize("big", [65280.0, 65536.0, 1e30, 2e-6])
+def test_bf16_values_outside_fp16_range(big):
+    # V entries at and beyond fp16's range (65280 is the largest bf16 value
+    # fp16 holds) and below its normal range: the bf16 P.V must stay exact
+    c = ChunkCase([300, 130, 70], [70, 130, 1], 16, 4, 16, "bf16", 725)
+    w = c.w
+    rng = np.random.default_rng(9)
+    for b in range(w.batch):
+        pages = w.pages_of(b)
+        for tok in rng.choice(int(w.kv_lens[b]), size=4, replace=False):
+            pg, slot = int(pages[tok // w.page_size]), int(tok % w.page_size)
+            dims = torch.as_tensor(rng.choice(128, size=3, replace=False))
+            signs = torch.as_tensor(rng.choice([-1.0, 1.0], size=3), dtype=torch.float32)
+            c.pool[pg, 1, :, slot, dims] = (signs * big).to(c.pool.dtype)
+    out, lse = c.run(splits=1)
+    ro, rl = c.oracle()
+    o = out.float().cpu().numpy().reshape(ro.shape)
+    assert np.isfinite(o).all()
+    # large outputs: the bf16 store rounds by up to 2^-8 relative (half an ulp
+    # at the bottom of a binade)
+    assert np.all(np.abs(o - ro) <= 1e-2 + 6e-3 * np.abs(ro))
+    assert np.abs(lse.cpu().numpy().reshape(rl.shape) - rl).max() <= 1e-3
+
+
+SHORT_CASES = [
+    # lens, q_lens, hq, hkv, ps, dtype, max_q_len  (columns = max_q_len * hq / hkv)
+    ([40, 100, 17, 64, 300, 1000], [4, 3, 1, 4, 2, 4], 32, 8, 16, "bf16", 4),   # 16 columns
+    ([33, 700, 16, 129], [2, 2, 1, 2], 16, 2, 32, "f16", 2),                    # G = 8
+    ([300, 18, 65], [16, 16, 5], 8, 8, 16, "bf16", 16),                         # G = 1
+    ([90, 513, 2000], [1, 2, 2], 16, 4, 64, "bf16", 2),                         # 8 columns
+    ([1, 5, 3000], [1, 0, 3], 8, 2, 16, "f16", 4),                              # q_len 0
+    ([33, 20], [4, 4], 16, 4, 16, "bf16", 4),                                   # chunk across tiles
+]
+
+
+@pytest.mark.parametrize("parts", [0, 3, 148])
+@pytest.mark.parametrize("i", range(len(SHORT_CASES)))
+def test_short_chunks_match_oracle(i, parts):
+    lens, q_lens, hq, hkv, ps, dt, mq = SHORT_CASES[i]
+    c = ChunkCase(lens, q_lens, hq, hkv, ps, dt, 740 + i)
+    out, lse = c.run_short(mq, parts=parts)
+    assert c.err == 0
+    ro, rl = c.oracle()
+    assert_parity(out, lse, ro, rl, what=f"short case {i} parts {parts}")
+
+
+@pytest.mark.parametrize("layout,kind", [("HND", "block"), ("NHD", "csr")])
+def test_short_chunks_layouts_and_tables_bitwise(layout, kind):
+    c = ChunkCase([400, 17, 1000], [4, 2, 3], 32, 8, 16, "bf16", 746)
+    ref = c.run_short(4)
+    out, lse = c.run_short(4, layout=layout, kind=kind)
+    assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
+
+
+def test_short_chunk_longer_than_bound_sets_error_bit():
+    c = ChunkCase([100, 100, 60], [2, 5, 3], 32, 8, 16, "bf16", 747)
+    sentinel = torch.full_like(c.q, 7.0, device="cuda")
+    out, lse = c.run_short(4, out=sentinel)
+    assert c.err & pkv.DEVERR_APPEND
+    ro, rl = c.oracle()
+    qo = c.qo
+    keep = np.r_[qo[0]:qo[1], qo[2]:qo[3]]
+    assert_parity(out[keep], lse[keep], ro[keep], rl[keep], what="in-bound requests")
+    assert bool((out[qo[1]:qo[2]] == 7.0).all())    # the long chunk's rows are left alone
+
+
+def test_speculative_verification_shape_sampled():
+    # the speculative-verification workload at full size through the short
+    # path, checked on sampled query rows against the truncated-request decode
+    w, q_lens = wl.named_chunk("spec")
+    _, pool, k_new, v_new = wl.make_tensors(w, "cuda")
+    qo = wl.chunk_indptr(q_lens)
+    q = wl.make_chunk_queries(w, q_lens, "cuda")
+    ip, ix, ll = i32(w.page_indptr), i32(w.page_indices), i32(w.last_page_len)
+    table = pkv.csr_table(ip, ix, ll)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.paged_kv_append(pool, ip, ix, ll, k_new, v_new, i32(w.append_indptr), error_word=err)
+    mq = int(q_lens.max())
+    nb = pkv.append_attention_short_workspace_bytes(w.num_qo_heads, w.num_kv_heads, mq)
+    ws = torch.zeros(nb // 4 + 64, dtype=torch.int32, device="cuda")
+    out, lse = pkv.append_attention_short(q, i32(qo), pool, table, mq, ws, sm_scale=w.sm_scale,
+                                          error_word=err)
+    torch.cuda.synchronize()
+    assert pkv.read_error_word(err) == 0
+    rng = np.random.default_rng(5)
+    for b in sorted(rng.choice(w.batch, size=12, replace=False).tolist()):
+        L, n = int(w.kv_lens[b]), int(q_lens[b])
+        for i in range(n):
+            pos = L - n + i
+            ip_, ix_, ll_ = truncated_request(w, b, pos)
+            uniq, inv = np.unique(ix_, return_inverse=True)
+            sub = wl.bits(pool[torch.as_tensor(uniq, device="cuda", dtype=torch.long)])
+            row = int(qo[b]) + i
+            ro, rl = oracle.decode(wl.bits(q[row:row + 1]), sub, odtype(w), ip_,
+                                   inv.astype(np.int32), ll_, w.sm_scale)
             assert_parity(out[row:row + 1], lse[row:row + 1], ro, rl, what=f"b{b} i{i}")
 
 

@@ -312,3 +312,31 @@ def test_append_attention_rejects_bad_arguments():
     assert call(pkv.PoolDesc(4096, 64, 8, 2, 128, pkv.BF16, 0, 0)) == 2
     assert call(splits=4) == 3                       # no workspace for the split states
     assert call(plan=ctypes.c_void_p(4100)) == 1     # misaligned plan
+
+
+def test_append_attention_short_rejects_bad_arguments():
+    L = pkv.lib()
+    P = ctypes.c_void_p(4096)
+    WS = ctypes.c_void_p(1 << 20)
+    pool = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.BF16, 0, 0)      # 2 kv heads: G = 4 with hq 8
+    csr = pkv.TableDesc(0, 4, 4096, 4096, 4096, None, None, 0, 0)
+    need = pkv.append_attention_short_workspace_bytes(8, 2, 4, 4)
+
+    def call(pool=pool, max_q_len=4, hq=8, ws_bytes=need, qo=P):
+        return L.pkv_append_attention_short(P, qo, 16, max_q_len, hq, ctypes.byref(pool),
+                                            ctypes.byref(csr), 0.1, 4, WS, ws_bytes,
+                                            ctypes.c_void_p(8192), None, None, None)
+
+    assert call(max_q_len=5) == 2                     # 5 tokens x 4 heads > 16 columns
+    assert call(max_q_len=0) == 2
+    assert call(hq=7) == 1                            # not a multiple of the kv heads
+    assert call(pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.FP8_E4M3, 0, 0)) == 1
+    assert call(pkv.PoolDesc(4096, 64, 16, 2, 64, pkv.BF16, 0, 0)) == 2
+    assert call(ws_bytes=need - 1) == 3
+    assert call(qo=None) == 1
+    # 8 or 16 state columns per slot
+    assert pkv.append_attention_short_workspace_bytes(32, 8, 5, 4) == 0
+    assert pkv.append_attention_short_workspace_bytes(32, 8, 0, 4) == 0
+    w2 = pkv.append_attention_short_workspace_bytes(32, 8, 2, 148)
+    w4 = pkv.append_attention_short_workspace_bytes(32, 8, 4, 148)
+    assert w2 >= 2 * 148 * 8 * 129 * 4 and w4 >= 2 * 148 * 16 * 129 * 4 and w4 > w2
