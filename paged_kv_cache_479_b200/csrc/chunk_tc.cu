@@ -111,6 +111,37 @@ struct KeyRange {
   }
 };
 
+// mbar_wait_bounded with a suspend-time hint on the try-wait: a waiting
+// thread sleeps until the phase completes (or 10 ms pass) instead of spinning,
+// which leaves the issue slots to the warps that have work (the softmax warps
+// of one row tile wait while the other's compute).  Same bound, abort and
+// error behaviour.
+__device__ __forceinline__ bool try_wait_sleeping(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(10000000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool wait_sleeping(uint32_t bar, uint32_t parity, volatile int* abort,
+                                              int* err) {
+  if (try_wait_sleeping(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (*abort) return false;
+    if (try_wait_sleeping(bar, parity)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      if (err) atomicOr(err, kErrTimeout);
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ int clamp64(long long v) { return v <= 0 ? 0 : (v >= kTile ? kTile : (int)v); }
 
 template <bool BF16>
@@ -230,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int byoff = __shfl_sync(kAll, yoff, box);
       int okl = 1;
       if (lane == 0) {
-        okl = mbar_wait_bounded(smem_u32(&ctl.kv_empty[s]), ((i / kStages) & 1) ^ 1, &ctl.abort,
+        okl = wait_sleeping(smem_u32(&ctl.kv_empty[s]), ((i / kStages) & 1) ^ 1, &ctl.abort,
                                 a.err);
         if (okl) mbar_arrive_expect_tx(smem_u32(&ctl.kv_full[s]), __popc(have) * 4u * kBoxBytes);
       }
@@ -296,9 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = true;
       for (int t = 0; ok && t < tiles; ++t)
-        ok = mbar_wait_bounded(smem_u32(&ctl.q_full[t]), 0, &ctl.abort, a.err);
+        ok = wait_sleeping(smem_u32(&ctl.q_full[t]), 0, &ctl.abort, a.err);
       if (ok && n > 0) {
-        ok = mbar_wait_bounded(smem_u32(&ctl.kv_full[0]), 0, &ctl.abort, a.err);
+        ok = wait_sleeping(smem_u32(&ctl.kv_full[0]), 0, &ctl.abort, a.err);
         if (ok) {
           umma::fence_after_sync();
           for (int t = 0; t < tiles; ++t) issue_s(0, t);
@@ -309,11 +340,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (per row tile: S_A(j+1) is queued behind PV_B(j-1), so the tensor pipe
         // does not drain while this thread waits for PV_B(j-1))
         if (j + 1 < n) {
-          ok = mbar_wait_bounded(smem_u32(&ctl.kv_full[(j + 1) % kStages]), ((j + 1) / kStages) & 1,
+          ok = wait_sleeping(smem_u32(&ctl.kv_full[(j + 1) % kStages]), ((j + 1) / kStages) & 1,
                                  &ctl.abort, a.err);
           for (int t = 0; ok && t < tiles; ++t) {
             if (j >= 1)
-              ok = mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (j - 1) & 1, &ctl.abort, a.err);
+              ok = wait_sleeping(smem_u32(&ctl.o_done[t]), (j - 1) & 1, &ctl.abort, a.err);
             if (!ok) break;
             umma::fence_after_sync();
             issue_s(j + 1, t);
@@ -321,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
         }
         for (int t = 0; ok && t < tiles; ++t) {
-          ok = mbar_wait_bounded(smem_u32(&ctl.p_full[t][j & 1]), (j >> 1) & 1, &ctl.abort, a.err);
+          ok = wait_sleeping(smem_u32(&ctl.p_full[t][j & 1]), (j >> 1) & 1, &ctl.abort, a.err);
           if (!ok) break;
           umma::fence_after_sync();
           issue_pv(j, t);
@@ -368,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n; ++j) {
       const int bj = j & 1;
       const uint32_t t_s = trow + (uint32_t)(2 * t + bj) * kTile;
-      ok = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.s_full[t][bj]), (j >> 1) & 1,
+      ok = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.s_full[t][bj]), (j >> 1) & 1,
                                               &ctl.abort, a.err));
       if (!ok) break;
       umma::fence_after_sync();
@@ -408,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // their maximum, once PV(j-1) is done (the whole warp loads and stores)
       const bool rescale = move && j > 0 && m_used != -INFINITY;
       if (__any_sync(kAll, rescale)) {
-        ok = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (j - 1) & 1,
+        ok = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.o_done[t]), (j - 1) & 1,
                                                 &ctl.abort, a.err));
         if (!ok) break;
         umma::fence_after_sync();
@@ -473,10 +504,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // its phase first, then PV(n-1)'s
       bool have_o = n > 0;
       if (have_o && n >= 2)
-        have_o = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (n - 2) & 1,
+        have_o = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.o_done[t]), (n - 2) & 1,
                                                     &ctl.abort, a.err));
       if (have_o)
-        have_o = __all_sync(kAll, mbar_wait_bounded(smem_u32(&ctl.o_done[t]), (n - 1) & 1,
+        have_o = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.o_done[t]), (n - 1) & 1,
                                                     &ctl.abort, a.err));
       if (n == 0 || have_o) {
         umma::fence_after_sync();
