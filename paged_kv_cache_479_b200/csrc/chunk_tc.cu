@@ -7,10 +7,13 @@
 // the window of section 2.3 cut to its causal half).  A CTA owns a block of up
 // to 256 rows of one request and KV head -- row r = (chunk token r / G, query
 // head kvh * G + r % G) -- as two 128-row tiles A and B that share every K/V
-// tile their rows may see.  Per 64-token K/V tile and row tile:
-//     S[128 x 64]  = Q[128 x 128] . K_tile^T     tcgen05.mma, A and B in shared memory
-//     online softmax, one thread per row reading S from tensor memory
+// tile their rows may see.  Keys come in pairs of 64-token tiles; per pair,
+// tile and row tile:
+//     S[128 x 128] = Q[128 x 128] . K_pair^T     tcgen05.mma, A and B in shared memory
+//     online softmax per 64-key tile, one thread per row reading S from tensor memory
 //     O[128 x 128] += P[128 x 64] . V_tile        tcgen05.mma, P in tensor memory
+// (An MMA costs about the same issue time at N = 64 as at N = 128 -- ~95
+// cycles for M = 128, K = 16 -- so S is taken 128 keys at a time.)
 // -- the blockwise recursive softmax of "大模型推理极致优化：FlashAttention+
 // PageAttention联合调优" section 2.2 with a row tile as one MMA.  While one row
 // tile's softmax runs, the tensor core works on the other's products.
@@ -25,13 +28,13 @@
 // the state of the request's own pages.
 //
 // Warp roles (320 threads): warp 0 issues the bulk-tensor loads of K and V
-// into a 3-stage ring; warp 1 allocates tensor memory and one of its lanes
+// into a 2-stage ring of 128-key pairs; warp 1 allocates tensor memory and one of its lanes
 // issues every MMA; warps 2..5 own row tile A and warps 6..9 row tile B (one
 // warp per 32-lane quarter of tensor memory): they stage Q, run the softmax
 // and the epilogue.
 //
 // Tensor memory (512 columns x 128 lanes of 32 bits): S of row tile t for
-// tiles of even / odd index in columns [64(2t+b), +64) -- rewritten in place
+// the first / second tile of a pair in columns [64(2t+b), +64) -- rewritten in place
 // by P (bf16: the high 16 bits of each fp32 probability in the first 32
 // columns, the rounded remainder in the next 32, two MMAs; fp16: one part)
 // -- and O of row tile t in [256 + 128t, +128).
@@ -45,9 +48,11 @@
 // timeout bit, lets its own copies and MMAs drain (bounded), frees tensor
 // memory and returns.  Tensor-memory loads and stores are warp-collective, so
 // every branch around them is warp-uniform.  An mbarrier parity wait cannot
-// tell a phase from the one two phases later, so no thread waits for a phase
-// while the phase before it may still be pending: each wait below is
-// preceded, in that thread, by a wait that implies the previous phase.
+// tell a phase from the one two phases later or earlier, so a thread waits for
+// a phase only when the phase before it is known complete and the phase after
+// it cannot have completed yet (it needs something this thread does first);
+// where that cannot be arranged (the end of a row tile) the barrier has one
+// phase.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -64,16 +69,17 @@ constexpr int kD = 128;
 constexpr int kTileRows = 128;                    // rows of one row tile (the MMA's M)
 constexpr int kRowTiles = 2;
 constexpr int kRows = kRowTiles * kTileRows;      // rows per CTA
-constexpr int kTile = 64;                         // keys per K/V tile
-constexpr int kStages = 3;
+constexpr int kTile = 64;                         // keys per softmax / P.V tile
+constexpr int kPairKeys = 2 * kTile;              // keys per S product and ring stage
+constexpr int kStages = 2;                        // ring stages (pairs)
 constexpr int kThreads = 64 + kRows;              // producer, MMA, 8 softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
 constexpr int kQTileBytes = kTileRows * kD * 2;   // 32 KiB: two 64-dim halves of [128][64]
 constexpr int kQHalf = kTileRows * 128;           // 16 KiB
-constexpr int kKVHalf = kTile * 128;              // 8 KiB: [64 tokens][64 dims]
-constexpr int kKBytes = 2 * kKVHalf;              // 16 KiB
-constexpr int kStageBytes = 2 * kKBytes;          // K then V: 32 KiB
+constexpr int kKVHalf = kPairKeys * 128;          // 16 KiB: [128 tokens][64 dims]
+constexpr int kKBytes = 2 * kKVHalf;              // 32 KiB
+constexpr int kStageBytes = 2 * kKBytes;          // K then V: 64 KiB
 constexpr int kBoxBytes = kTileTokens * 128;      // one [16][64] box: 2 KiB
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.f;
@@ -84,9 +90,10 @@ struct __align__(16) Ctl {
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t q_full[kRowTiles];
-  uint64_t s_full[kRowTiles][2];
+  uint64_t s_full[kRowTiles];      // S of a pair
   uint64_t p_full[kRowTiles][2];
-  uint64_t o_done[kRowTiles];
+  uint64_t o_done[kRowTiles];   // one phase per P.V tile (the softmax's rescale waits)
+  uint64_t o_final[kRowTiles];  // one phase: the row tile's last P.V done
   uint64_t drained;  // one phase: every MMA of the CTA completed
   uint32_t tmem_base;
   int abort;
@@ -164,10 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < kRowTiles; ++t) {
       mbar_init(smem_u32(&ctl.q_full[t]), kTileRows);
       mbar_init(smem_u32(&ctl.o_done[t]), 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(smem_u32(&ctl.s_full[t][b]), 1);
-        mbar_init(smem_u32(&ctl.p_full[t][b]), kTileRows);
-      }
+      mbar_init(smem_u32(&ctl.o_final[t]), 1);
+      mbar_init(smem_u32(&ctl.s_full[t]), 1);
+      for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&ctl.p_full[t][b]), kTileRows);
     }
     mbar_init(smem_u32(&ctl.drained), 1);
     ctl.abort = 0;
@@ -239,24 +245,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int* ids = prefix ? a.prefix_pages : a.indices + r.page_base;
     bool ok = true;
     int issued = 0;
-    for (int i = 0; ok && i < n; ++i) {
+    const int np = (n + 1) / 2;  // pairs of tiles
+    for (int i = 0; ok && i < np; ++i) {
       const int s = i % kStages;
-      long long t0, t1;
-      kr.tile(j0 + i, t0, t1);
-      const int valid = (int)(t1 - t0);
+      // lane L < 8 looks up box L: tokens 16 (L % 4) .. of tile 2i + L / 4
       int page = -1, yoff = 0;
-      if (lane < 4 && lane * kTileTokens < valid) {
-        const long long tok = t0 + lane * kTileTokens;
-        page = ids[tok / a.page_size];
-        if (page < 0 || (long long)page >= a.num_pages) {
-          if (a.err) atomicOr(a.err, kErrPageId);
-          page = -1;
+      if (lane < 8 && 2 * i + (lane >> 2) < n) {
+        long long t0, t1;
+        kr.tile(j0 + 2 * i + (lane >> 2), t0, t1);
+        const int sub = lane & 3;
+        if (sub * kTileTokens < (int)(t1 - t0)) {
+          const long long tok = t0 + sub * kTileTokens;
+          page = ids[tok / a.page_size];
+          if (page < 0 || (long long)page >= a.num_pages) {
+            if (a.err) atomicOr(a.err, kErrPageId);
+            page = -1;
+          }
+          yoff = (int)(tok % a.page_size);
         }
-        yoff = (int)(tok % a.page_size);
       }
-      const unsigned have = __ballot_sync(kAll, page >= 0) & 0xfu;
-      // lane L < 16 loads (K / V = L / 8, box = (L / 2) % 4, dim half = L % 2)
-      const int box = (lane >> 1) & 3, half = lane & 1, kv = (lane >> 3) & 1;
+      const unsigned have = __ballot_sync(kAll, page >= 0) & 0xffu;
+      // every lane loads one box (K / V = L / 16, dim half = L / 8 % 2, box = L % 8)
+      const int box = lane & 7, half = (lane >> 3) & 1, kv = lane >> 4;
       const int bpage = __shfl_sync(kAll, page, box);
       const int byoff = __shfl_sync(kAll, yoff, box);
       int okl = 1;
@@ -267,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = __shfl_sync(kAll, okl, 0) != 0;
       if (!ok) break;
-      if (lane < 16 && bpage >= 0) {
+      if (bpage >= 0) {
         const uint32_t dst = ring0 + (uint32_t)s * kStageBytes + (uint32_t)kv * kKBytes +
                              (uint32_t)half * kKVHalf + (uint32_t)box * kBoxBytes;
         const uint32_t full = smem_u32(&ctl.kv_full[s]);
@@ -292,12 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // =========================== MMA issuer ===========================
     if (lane == 0) {
       const uint32_t ring0 = smem_u32(ring);
-      const uint32_t idesc_s = umma::instr_desc(BF16, kTileRows, kTile, false, false);
+      const uint32_t idesc_s = umma::instr_desc(BF16, kTileRows, kPairKeys, false, false);
       const uint32_t idesc_pv = umma::instr_desc(BF16, kTileRows, kD, false, true);
-      auto issue_s = [&](int j, int t) {  // S_t(j) into buffer j & 1 of row tile t
+      auto issue_s = [&](int p, int t) {  // S_t of pair p into both buffers of row tile t
         const uint32_t qb = smem_u32(qs) + (uint32_t)t * kQTileBytes;
-        const uint32_t kbase = ring0 + (uint32_t)(j % kStages) * kStageBytes;
-        const uint32_t d = tbase + (uint32_t)(2 * t + (j & 1)) * kTile;
+        const uint32_t kbase = ring0 + (uint32_t)(p % kStages) * kStageBytes;
+        const uint32_t d = tbase + (uint32_t)(2 * t) * kTile;
 #pragma unroll
         for (int k = 0; k < kD / 16; ++k) {  // 16 dims per MMA: 32 bytes along a swizzled row
           const uint32_t off = (uint32_t)(k & 3) * 32u;
@@ -305,10 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = umma::smem_desc(kbase + (uint32_t)(k >> 2) * kKVHalf + off, 16, 1024);
           umma::mma_ss(d, ad, bd, idesc_s, k > 0 ? 1u : 0u);
         }
-        umma::commit(smem_u32(&ctl.s_full[t][j & 1]));
+        umma::commit(smem_u32(&ctl.s_full[t]));
       };
       auto issue_pv = [&](int j, int t) {  // O_t += P_t(j) . V(j)
-        const uint32_t vbase = ring0 + (uint32_t)(j % kStages) * kStageBytes + kKBytes;
+        const uint32_t vbase = ring0 + (uint32_t)((j >> 1) % kStages) * kStageBytes + kKBytes +
+                               (uint32_t)(j & 1) * (kTile * 128);
         const uint32_t p_cols = tbase + (uint32_t)(2 * t + (j & 1)) * kTile;
         const uint32_t o = tbase + kColO + (uint32_t)t * kD;
 #pragma unroll
@@ -335,29 +346,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < tiles; ++t) issue_s(0, t);
         }
       }
-      for (int j = 0; ok && j < n; ++j) {
-        // S(j+1) into the other buffers: it overwrites P(j-1), so PV(j-1) must be done
-        // (per row tile: S_A(j+1) is queued behind PV_B(j-1), so the tensor pipe
-        // does not drain while this thread waits for PV_B(j-1))
-        if (j + 1 < n) {
-          ok = wait_sleeping(smem_u32(&ctl.kv_full[(j + 1) % kStages]), ((j + 1) / kStages) & 1,
-                                 &ctl.abort, a.err);
-          for (int t = 0; ok && t < tiles; ++t) {
-            if (j >= 1)
-              ok = wait_sleeping(smem_u32(&ctl.o_done[t]), (j - 1) & 1, &ctl.abort, a.err);
-            if (!ok) break;
-            umma::fence_after_sync();
-            issue_s(j + 1, t);
-          }
-          if (!ok) break;
-        }
+      const int np = (n + 1) / 2;
+      // per pair: PV of its first tile for A and B; then, per row tile, PV of
+      // its second tile followed at once by S of the next pair, so the tensor
+      // core alternates between the row tiles (A's next S runs while B's
+      // softmax still works on its second tile)
+      for (int p = 0; ok && p < np; ++p) {
+        const int ja = 2 * p, jb = 2 * p + 1;
         for (int t = 0; ok && t < tiles; ++t) {
-          ok = wait_sleeping(smem_u32(&ctl.p_full[t][j & 1]), (j >> 1) & 1, &ctl.abort, a.err);
+          ok = wait_sleeping(smem_u32(&ctl.p_full[t][0]), p & 1, &ctl.abort, a.err);
           if (!ok) break;
           umma::fence_after_sync();
-          issue_pv(j, t);
+          issue_pv(ja, t);
+          if (ja == n - 1) umma::commit(smem_u32(&ctl.o_final[t]));
         }
-        if (ok) umma::commit(smem_u32(&ctl.kv_empty[j % kStages]));
+        if (ok && jb < n) {
+          const bool next = p + 1 < np;
+          if (next)
+            ok = wait_sleeping(smem_u32(&ctl.kv_full[(p + 1) % kStages]), ((p + 1) / kStages) & 1,
+                               &ctl.abort, a.err);
+          for (int t = 0; ok && t < tiles; ++t) {
+            ok = wait_sleeping(smem_u32(&ctl.p_full[t][1]), p & 1, &ctl.abort, a.err);
+            if (!ok) break;
+            umma::fence_after_sync();
+            issue_pv(jb, t);
+            if (jb == n - 1) umma::commit(smem_u32(&ctl.o_final[t]));
+            // S of the next pair overwrites both P buffers of this row tile: no
+            // wait, the MMAs of one thread run in issue order, so both PVs
+            // have read P before it writes (and the softmax wrote P before
+            // its p_full arrival)
+            if (next) issue_s(p + 1, t);
+          }
+        }
+        if (ok) umma::commit(smem_u32(&ctl.kv_empty[p % kStages]));
       }
       // let every MMA issued land before tensor memory is freed (a commit
       // arrives once all MMAs this thread issued before it completed)
@@ -397,11 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const int bj = j & 1;
+      const int bj = j & 1;  // tile within its pair: the S / P buffer
       const uint32_t t_s = trow + (uint32_t)(2 * t + bj) * kTile;
-      ok = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.s_full[t][bj]), (j >> 1) & 1,
-                                              &ctl.abort, a.err));
-      if (!ok) break;
+      if (bj == 0) {  // one S product covers both tiles of the pair
+        ok = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.s_full[t]), (j >> 1) & 1, &ctl.abort,
+                                            a.err));
+        if (!ok) break;
+      }
       umma::fence_after_sync();
       uint32_t s0[32], s1[32];
       umma::ld32(t_s, s0);
@@ -486,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // V rows past the tile's keys may hold anything (even NaN): row tile A
       // zeroes them before the first PV of this tile (B's is issued after A's)
       if (t == 0 && valid < kTile) {
-        uint8_t* vt = ring + (size_t)(j % kStages) * kStageBytes + kKBytes;
+        uint8_t* vt = ring + (size_t)((j >> 1) % kStages) * kStageBytes + kKBytes + bj * (kTile * 128);
         const int chunks = (kTile - valid) * 16;  // 16-byte chunks over both dim halves
         for (int idx = row; idx < chunks; idx += kTileRows) {
           const int tk = valid + (idx >> 4), half = (idx >> 3) & 1, c = idx & 7;
@@ -500,15 +523,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // ---- epilogue: o = O / l of this row (every lane loads; rows past the block store nothing)
     if (ok) {
-      // PV(n-2) may still be running when this row's last softmax ends: wait for
-      // its phase first, then PV(n-1)'s
+      // the row tile's last P.V (and every MMA before it): a one-phase barrier,
+      // so the wait cannot alias however far the P.V phases have run
       bool have_o = n > 0;
-      if (have_o && n >= 2)
-        have_o = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.o_done[t]), (n - 2) & 1,
-                                                    &ctl.abort, a.err));
       if (have_o)
-        have_o = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.o_done[t]), (n - 1) & 1,
-                                                    &ctl.abort, a.err));
+        have_o = __all_sync(kAll, wait_sleeping(smem_u32(&ctl.o_final[t]), 0, &ctl.abort, a.err));
       if (n == 0 || have_o) {
         umma::fence_after_sync();
         const size_t tok = has_row ? (size_t)(q_first + rr / G) : 0;
