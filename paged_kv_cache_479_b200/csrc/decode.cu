@@ -81,7 +81,7 @@ constexpr int kSegRecs = 16;                      // segment records in flight
 constexpr int kMaxGroup = 8;                      // columns of one n8 MMA tile
 constexpr int kQBufs = 8;                         // staged query blocks in flight
 // a staged query block: the pair's columns (up to 8 NQ rows of 128 dims)
-constexpr int q_buf_bytes(int nq) { return nq * kMaxGroup * 128 * 2; }
+__host__ __device__ constexpr int q_buf_bytes(int nq) { return nq * kMaxGroup * 128 * 2; }
 // The producer refills query buffer (and record) seg % n for segment seg + n
 // only after issuing every tile of segments seg .. seg+n-1 (each a multiple of
 // 8 tiles, at least 8).  With S ring slots that means the tiles up to
@@ -214,12 +214,15 @@ __device__ __forceinline__ uint32_t widen_hi(uint32_t r) {
 }
 
 // KV: the pool's element type -- kKv16 (q's own 16-bit type), kKvE4M3, kKvE5M2;
-// NQ: n8 column tiles per pair (2 only for short chunks over 16-bit pools)
-template <bool BF16, int KV, int NQ>
+// NQ: n8 column tiles per pair (2 only for short chunks over 16-bit pools);
+// CHUNK: short chunks (causal limits per column), else decode (one token per request)
+template <bool BF16, int KV, int NQ, bool CHUNK>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   constexpr bool FP8 = KV != kKv16;
   static_assert(NQ == 1 || (NQ == 2 && !FP8), "two column tiles only for 16-bit pools");
+  static_assert(!CHUNK || !FP8, "short chunks only for 16-bit pools");
+  static_assert(CHUNK || NQ == 1, "the decode has one column tile");
   constexpr int kCols = NQ * kMaxGroup;
   constexpr int kQBufBytes = q_buf_bytes(NQ);
   // ring geometry of this KV type (16-bit: 16 slots of 8 KiB; 8-bit: 32 of 4 KiB)
@@ -371,7 +374,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         // of the chunk's tokens; a chunk that does not fit gets no columns
         long long q_row = wk.b;
         int q_len = 1;
-        if (a.qo_indptr) {
+        if (CHUNK) {
           q_row = a.qo_indptr[wk.b];
           const long long ql = (long long)a.qo_indptr[wk.b + 1] - q_row;
           const bool fits = ql >= 1 && ql * G <= a.max_cols && ql * G <= kCols &&
@@ -636,12 +639,12 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           }
         }
       }
-      const int q_len = rec.ncol / G;
+      const int q_len = CHUNK ? rec.ncol / G : 1;
 #pragma unroll
       for (int nt = 0; nt < NQ; ++nt) {
         const int c0 = nt * kMaxGroup + 2 * cq, c1 = c0 + 1;
-        need0[nt] = c0 < rec.ncol ? q_len - c0 / G : 1;
-        need1[nt] = c1 < rec.ncol ? q_len - c1 / G : 1;
+        need0[nt] = CHUNK && c0 < rec.ncol ? q_len - c0 / G : 1;
+        need1[nt] = CHUNK && c1 < rec.ncol ? q_len - c1 / G : 1;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
         m0[nt] = m1[nt] = -INFINITY;
@@ -700,10 +703,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       uint32_t bh0[NQ], bh1[NQ], bl0[NQ], bl1[NQ];
 #pragma unroll
       for (int nt = 0; nt < NQ; ++nt) {
-        const float x0 = dlo >= need0[nt] ? (sa[nt][0] + sb[nt][0]) * sc0 : -INFINITY;  // token g,   col 2cq
-        const float x1 = dlo >= need1[nt] ? (sa[nt][1] + sb[nt][1]) * sc1 : -INFINITY;  // token g,   col 2cq+1
-        const float x2 = dhi >= need0[nt] ? (sa[nt][2] + sb[nt][2]) * sc0 : -INFINITY;  // token g+8, col 2cq
-        const float x3 = dhi >= need1[nt] ? (sa[nt][3] + sb[nt][3]) * sc1 : -INFINITY;  // token g+8, col 2cq+1
+        const int nd0 = CHUNK ? need0[nt] : 1, nd1 = CHUNK ? need1[nt] : 1;
+        const float x0 = dlo >= nd0 ? (sa[nt][0] + sb[nt][0]) * sc0 : -INFINITY;  // token g,   col 2cq
+        const float x1 = dlo >= nd1 ? (sa[nt][1] + sb[nt][1]) * sc1 : -INFINITY;  // token g,   col 2cq+1
+        const float x2 = dhi >= nd0 ? (sa[nt][2] + sb[nt][2]) * sc0 : -INFINITY;  // token g+8, col 2cq
+        const float x3 = dhi >= nd1 ? (sa[nt][3] + sb[nt][3]) * sc1 : -INFINITY;  // token g+8, col 2cq+1
         float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
@@ -711,8 +715,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
         }
         const float mn0 = fmaxf(m0[nt], mx0), mn1 = fmaxf(m1[nt], mx1);
-        // a column that has seen no visible key yet keeps m = -inf: subtract 0
-        const float ms0 = mn0 == -INFINITY ? 0.f : mn0, ms1 = mn1 == -INFINITY ? 0.f : mn1;
+        // a chunk column that has seen no visible key yet keeps m = -inf:
+        // subtract 0 (every decode tile has a visible key for every column)
+        const float ms0 = CHUNK && mn0 == -INFINITY ? 0.f : mn0;
+        const float ms1 = CHUNK && mn1 == -INFINITY ? 0.f : mn1;
         const float al0 = ex2(m0[nt] - ms0), al1 = ex2(m1[nt] - ms1);
         const float p0 = ex2(x0 - ms0), p1 = ex2(x1 - ms1);
         const float p2 = ex2(x2 - ms0), p3 = ex2(x3 - ms1);
@@ -851,7 +857,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           float M = -INFINITY;
 #pragma unroll
           for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, scr.m[w][h]);
-          const float Ms = M == -INFINITY ? 0.f : M;  // no visible key in this share
+          const float Ms = CHUNK && M == -INFINITY ? 0.f : M;  // no visible key in this share
           float L = 0.f, acc = 0.f;
 #pragma unroll
           for (int w = 0; w < kConsumerWarps; ++w) {
@@ -859,7 +865,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
             L += wt * scr.l[w][h];
             acc += wt * scr.o[w][h][d];
           }
-          const float val = L > 0.f ? (FP8 ? acc * a.v_scale / L : acc / L) : 0.f;
+          const float val = !CHUNK || L > 0.f ? (FP8 ? acc * a.v_scale / L : acc / L) : 0.f;
           const int col = nt * kMaxGroup + h;
           if (direct) {
             const size_t hq = (size_t)rec.kvh * G + col % G;
@@ -903,7 +909,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       M = fmaxf(M, __ldcg(a.part_lse + (size_t)slot_of(j) * P + h));
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    M = M == -INFINITY ? 0.f : M;  // (every column of a chunk sees key 0: not expected)
+    if (CHUNK) M = M == -INFINITY ? 0.f : M;  // (every column of a chunk sees key 0: not expected)
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     constexpr int kBatch = 8;  // partial states loaded together
@@ -932,12 +938,12 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         acc.w += w * v[u].w;
       }
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const float inv = !CHUNK || L > 0.f ? 1.f / L : 0.f;
     const size_t hq = (size_t)pr.kvh * G + h % G;
     const size_t row = (size_t)pr.q_row + h / G;
     store_out4<BF16>(a, row, hq, 4 * lane,
                      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
-    if (lane == 0) store_lse(a, row, hq, L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY);
+    if (lane == 0) store_lse(a, row, hq, !CHUNK || L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY);
   }
 }
 
@@ -949,19 +955,23 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
                           int grid, cudaStream_t stream) {
   static_assert(sizeof(Ctl) % 16 == 0, "Ctl must keep Scratch 16-byte aligned");
   if (kv != kKv16 && kv != kKvE4M3 && kv != kKvE5M2) return cudaErrorInvalidValue;
-  if (nq != 1 && (nq != 2 || kv != kKv16)) return cudaErrorInvalidValue;
+  const bool chunk = a.qo_indptr != nullptr;
+  if ((nq != 1 && nq != 2) || (chunk && kv != kKv16) || (!chunk && nq != 1))
+    return cudaErrorInvalidValue;
   using Kern = void (*)(const CUtensorMap, const DecodeArgs);
-  // variants: 16-bit (fp16, bf16), E4M3 (fp16, bf16), E5M2 (fp16, bf16), 16-bit NQ=2 (fp16, bf16)
-  static const Kern kKerns[8] = {
-      decode_kernel<false, kKv16, 1>,   decode_kernel<true, kKv16, 1>,
-      decode_kernel<false, kKvE4M3, 1>, decode_kernel<true, kKvE4M3, 1>,
-      decode_kernel<false, kKvE5M2, 1>, decode_kernel<true, kKvE5M2, 1>,
-      decode_kernel<false, kKv16, 2>,   decode_kernel<true, kKv16, 2>};
-  const int variant = (nq == 2 ? 6 : 2 * kv) + (bf16 ? 1 : 0);
+  // decode: 16-bit, E4M3, E5M2 pools (fp16, bf16 each); short chunks: one or
+  // two column tiles over 16-bit pools (fp16, bf16 each)
+  static const Kern kKerns[10] = {
+      decode_kernel<false, kKv16, 1, false>,   decode_kernel<true, kKv16, 1, false>,
+      decode_kernel<false, kKvE4M3, 1, false>, decode_kernel<true, kKvE4M3, 1, false>,
+      decode_kernel<false, kKvE5M2, 1, false>, decode_kernel<true, kKvE5M2, 1, false>,
+      decode_kernel<false, kKv16, 1, true>,    decode_kernel<true, kKv16, 1, true>,
+      decode_kernel<false, kKv16, 2, true>,    decode_kernel<true, kKv16, 2, true>};
+  const int variant = (chunk ? 4 + 2 * nq : 2 * kv) + (bf16 ? 1 : 0);
   const Kern kern = kKerns[variant];
   const size_t smem = smem_bytes(nq);
   // the shared-memory opt-in is per function and device; do it once each
-  static bool attr_set[8][64] = {};
+  static bool attr_set[10][64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
