@@ -51,6 +51,9 @@ def parse():
     p.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
     p.add_argument("--partitions", type=int, default=0, help="split-KV partitions (0 = one per SM)")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--separate-append", action="store_true",
+                   help="launch the append on its own instead of fusing it into the decode "
+                        "(pkv_decode_append; 16-bit pools, plain decode)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cascade", action="store_true",
                    help="decode a shared-prefix workload with pkv_cascade_decode")
@@ -387,11 +390,16 @@ def run_pkv(args):
     out = torch.empty_like(batches[0].q)
     lse = torch.empty((w.batch, w.num_qo_heads), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = (3 if args.cascade else 1) + (1 if w.nnz_new else 0)
+    # the step's append runs inside the decode launch (pkv_decode_append) unless
+    # it cannot (8-bit pool, cascade) or --separate-append asks otherwise
+    fused = bool(w.nnz_new) and not fp8 and not args.cascade and not args.separate_append
+    launches_per_step = (3 if args.cascade else 1) + (1 if w.nnz_new and not fused else 0)
 
     table = pkv.csr_table(indptr, indices, last)
 
     def append_call(bt):
+        if fused:
+            return
         if w.nnz_new and fp8:
             pkv.paged_kv_append_fp8(bt.pool, table, bt.k_new, bt.v_new, app, FP8_K_SCALE,
                                     FP8_V_SCALE, error_word=err,
@@ -411,6 +419,11 @@ def run_pkv(args):
             pkv.cascade_decode(bt.q, bt.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws, out=out,
                                lse=lse, sm_scale=w.sm_scale, num_partitions=N, error_word=err,
                                stream=torch.cuda.current_stream(dev))
+            return
+        if fused:
+            pkv.paged_decode_append(bt.q, bt.pool, table, bt.k_new, bt.v_new, app, ws, out=out,
+                                    lse=lse, sm_scale=w.sm_scale, num_partitions=N,
+                                    error_word=err, stream=torch.cuda.current_stream(dev))
             return
         pkv.paged_decode_attention(bt.q, bt.pool, indptr, indices, last, ws, out=out, lse=lse,
                                    sm_scale=w.sm_scale, num_partitions=N, error_word=err,
@@ -433,7 +446,8 @@ def run_pkv(args):
         with torch.cuda.graph(g):
             fn(bt)
         return g.replay
-    app_g = [graphed(append_call, bt) if w.nnz_new else (lambda: None) for bt in batches]
+    app_g = [graphed(append_call, bt) if w.nnz_new and not fused else (lambda: None)
+             for bt in batches]
     dec_g = [graphed(decode_call, bt) for bt in batches]
     for i in range(2 * rotation):
         app_g[i % rotation]()
@@ -472,7 +486,8 @@ def run_pkv(args):
     step_bytes = algorithmic_bytes(w, args)
     s_per_step = ms / 1e3 / K
     value = job_throughput(step_bytes, world, ms, K)
-    dec_bytes = wl.decode_bytes(w, kv_elem_bytes(args))
+    # the timed launch's algorithmic bytes (with the append when it is fused in)
+    dec_bytes = wl.decode_bytes(w, kv_elem_bytes(args)) + (wl.append_bytes(w) if fused else 0)
     peak, peak_kind = measured_hbm()
     achieved = dec_bytes / (decode_ms_max / 1e3) / 1e9
 
@@ -505,6 +520,10 @@ def run_pkv(args):
                                                FP8_V_SCALE, out=out_d, lse=lse_d,
                                                sm_scale=w.sm_scale, num_partitions=N,
                                                error_word=err, stream=cur, fp8_format=fp8)
+            elif fused:
+                pkv.paged_decode_append(q_d, src.pool, e2e_table, k_d, v_d, ap_d, ws, out=out_d,
+                                        lse=lse_d, sm_scale=w.sm_scale, num_partitions=N,
+                                        error_word=err, stream=cur)
             else:
                 if w.nnz_new:
                     pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d,
@@ -542,8 +561,9 @@ def run_pkv(args):
         e2e = {"value": round(job_throughput(step_bytes, world, e_ms, K), 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "us_per_step": round(e_ms / K * 1e3, 2),
-               "path": "pinned host -> device (1 copy), append + decode, device -> pinned host "
-                       "(1 copy), stream sync every step" +
+               "path": "pinned host -> device (1 copy), " +
+                       ("append fused into the decode launch" if fused else "append + decode") +
+                       ", device -> pinned host (1 copy), stream sync every step" +
                        ("" if args.no_graph else "; the step's calls replayed as one CUDA graph")}
     clocks.stop()
 
@@ -556,8 +576,10 @@ def run_pkv(args):
             "dtype": (f"{fp8} KV widened to f16, f32 accumulate" if fp8 else
                       ("bf16" if w.dtype == "bf16" else "f16")), "data": "synthetic",
             "config": {**workload_config(w, args, rotation, N),
-                       "launch": "direct calls" if args.no_graph else
-                       "append and decode each captured once per batch copy as a CUDA graph, replayed"},
+                       "launch": ("direct calls" if args.no_graph else
+                                  ("the fused append + decode launch (pkv_decode_append)" if fused
+                                   else "append and decode each") +
+                                  " captured once per batch copy as a CUDA graph, replayed")},
             "us_per_step": round(ms / K * 1e3, 2),
             "tokens_per_s": round(w.batch * world / s_per_step, 1),
             "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
@@ -565,7 +587,8 @@ def run_pkv(args):
             "roofline": {"bound": "hbm",
                          "kernel": ("pkv_cascade_decode (prefix + own-page decode + merge launches)"
                                     if args.cascade else
-                                    (f"decode_kernel ({fp8} pool)" if fp8 else "decode_kernel")),
+                                    (f"decode_kernel ({fp8} pool)" if fp8 else
+                                     ("decode_kernel (append fused)" if fused else "decode_kernel"))),
                          "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"

@@ -225,6 +225,28 @@ PKV_API pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc
                                  int32_t* error_word, void* stream);
 
 /*
+ * pkv_decode_append -- one decode step in one launch: pkv_append_ex of the
+ * step's new rows followed by pkv_decode_ex, fused.  The decode kernel writes
+ * each new row into its page just before it loads the tile that holds it (the
+ * one CTA that reads that tile), so the append costs no launch of its own.
+ *   q, pool, table, sm_scale, num_partitions, workspace, out, lse, error_word,
+ *   stream   as in pkv_decode_ex (the table is the one after the append)
+ *   k_new, v_new, append_indptr, nnz_new   as in pkv_append_ex; the pool must be
+ *            16-bit (PKV_F16 / PKV_BF16, as k_new / v_new; 8-bit pools:
+ *            pkv_append_fp8 then pkv_decode_fp8); nnz_new = 0 is a plain decode
+ * On return (stream order) the pool holds exactly what pkv_append_ex would have
+ * written and out / lse what pkv_decode_ex would have computed on it.  Bad
+ * append_indptr entries set PKV_DEVERR_APPEND and leave that request's rows
+ * unwritten.  k_new / v_new must not alias the pool or out.
+ */
+PKV_API pkv_status pkv_decode_append(const void* q, int num_qo_heads, const pkv_pool_desc* pool,
+                                     const pkv_table_desc* table, const void* k_new,
+                                     const void* v_new, const int32_t* append_indptr,
+                                     int64_t nnz_new, float sm_scale, int num_partitions,
+                                     void* workspace, size_t workspace_bytes, void* out,
+                                     float* lse, int32_t* error_word, void* stream);
+
+/*
  * pkv_decode_fp8 / pkv_append_fp8 -- the 8-bit KV cache: a pool of FP8 codes
  * ("fp8_e4m3" KV-cache dtype of the serving configurations in "上下文窗口优化
  * 实战：如何用PagedAttention+FlashInfer将Llama3-70B的128K上下文吞吐提升3.8倍？"

@@ -19,6 +19,7 @@ Functions (C names in parentheses):
   cascade_decode         (pkv_cascade_decode)  decode for a batch sharing one prefix
   paged_decode_attention_ex / paged_kv_append_ex (pkv_decode_ex / pkv_append_ex)
                          NHD pools and dense (vLLM-style) block tables
+  paged_decode_append    (pkv_decode_append)   append + decode of a step in one launch
   paged_decode_attention_fp8 / paged_kv_append_fp8 (pkv_decode_fp8 / pkv_append_fp8)
                          the 8-bit (FP8 E4M3 / E5M2) KV cache with per-tensor K / V scales
   append_attention       (pkv_append_attention)  a chunk of query tokens per request,
@@ -52,6 +53,7 @@ from ._binding import (  # noqa: F401
     lib,
     merge_states,
     paged_decode_attention,
+    paged_decode_append,
     paged_decode_attention_ex,
     paged_decode_attention_fp8,
     paged_kv_append,
@@ -78,6 +80,7 @@ pkv_decode_static_workspace = decode_static_workspace
 pkv_merge_states = merge_states
 pkv_cascade_decode = cascade_decode
 pkv_decode_ex = paged_decode_attention_ex
+pkv_decode_append = paged_decode_append
 pkv_append_ex = paged_kv_append_ex
 pkv_decode_fp8 = paged_decode_attention_fp8
 pkv_append_attention = append_attention

@@ -78,6 +78,8 @@ _SIGNATURES["pkv_append_attention"] = (
 _SIGNATURES["pkv_append_attention_short_workspace_bytes"] = ([_I32, _I32, _I32, _I32], _SZ)
 _SIGNATURES["pkv_append_attention_short"] = (
     [_P, _P, _I64, _I32, _I32, _PP, _TP, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
+_SIGNATURES["pkv_decode_append"] = (
+    [_P, _I32, _PP, _TP, _P, _P, _P, _I64, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
 _SIGNATURES["paged_decode_attention"] = _SIGNATURES["pkv_decode"]
 _SIGNATURES["merge_states"] = _SIGNATURES["pkv_merge_states"]
@@ -335,6 +337,33 @@ def paged_kv_append_ex(pool, table: TableDesc, k_new, v_new, append_indptr, layo
                              _ptr(append_indptr), k_new.shape[0], _ptr(error_word),
                              _stream(stream, pool.device))
     _check(st, "pkv_append_ex")
+
+
+def paged_decode_append(q, pool, table: TableDesc, k_new, v_new, append_indptr, workspace,
+                        layout: str = "HND", out=None, lse=None, sm_scale=None,
+                        num_partitions: int = 0, error_word=None, stream=None,
+                        return_lse: bool = True):
+    """pkv_decode_append: the step's append (k_new / v_new rows by the int32
+    append_indptr) and the decode in one launch; table = the table after the append."""
+    _dev_tensor(q, "q", pool.dtype)
+    _dev_tensor(workspace, "workspace")
+    _dev_tensor(k_new, "k_new", pool.dtype)
+    _dev_tensor(v_new, "v_new", pool.dtype)
+    _dev_tensor(append_indptr, "append_indptr", torch.int32)
+    pd = pool_desc(pool, layout)
+    B, hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
+    st = lib().pkv_decode_append(_ptr(q), hq, ctypes.byref(pd), ctypes.byref(table), _ptr(k_new),
+                                 _ptr(v_new), _ptr(append_indptr), k_new.shape[0], scale,
+                                 num_partitions, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _ptr(out),
+                                 _ptr(lse), _ptr(error_word), _stream(stream, q.device))
+    _check(st, "pkv_decode_append")
+    return out, lse
 
 
 def _fp8_pool(pool, layout, fmt):

@@ -222,7 +222,9 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
                       float* lse, int32_t* error_word, void* stream, int out_f32,
                       long long out_rs, long long lse_rs, int kv_dtype = -1,
                       float k_scale = 1.f, float v_scale = 1.f,
-                      const int32_t* qo_indptr = nullptr, int64_t nnz_q = 0, int max_q_len = 1) {
+                      const int32_t* qo_indptr = nullptr, int64_t nnz_q = 0, int max_q_len = 1,
+                      const void* k_new = nullptr, const void* v_new = nullptr,
+                      const int32_t* append_indptr = nullptr, int64_t nnz_new = 0) {
   if (kv_dtype < 0) kv_dtype = dtype;
   if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1)
     return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
@@ -259,6 +261,17 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   if (!aligned(q, 16) || !aligned(pool, 16) || !aligned(out, 16))
     return fail(PKV_ERR_INVALID_ARG, "q, pool and out must be 16-byte aligned");
   if (out == q || out == pool) return fail(PKV_ERR_INVALID_ARG, "out aliases q or pool");
+  const bool fused = nnz_new > 0;
+  if (nnz_new < 0) return fail(PKV_ERR_INVALID_ARG, "nnz_new < 0");
+  if (fused) {
+    if (kv_dtype != dtype) return fail(PKV_ERR_INVALID_ARG, "a fused append needs a 16-bit pool");
+    if (!k_new || !v_new || !append_indptr)
+      return fail(PKV_ERR_INVALID_ARG, "null k_new, v_new or append_indptr");
+    if (!aligned(k_new, 16) || !aligned(v_new, 16))
+      return fail(PKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+    if (nnz_new * (int64_t)num_kv_heads > (int64_t)1 << 40)
+      return fail(PKV_ERR_UNSUPPORTED, "too many new rows");
+  }
   int N = num_partitions;
   if (N == 0) N = current_device_partitions();
   if (N <= 0) return fail(PKV_ERR_CUDA, "cannot query the SM count");
@@ -301,6 +314,12 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.nnz_q = nnz_q;
   a.pcols = pcols;
   a.max_cols = (int)cols;
+  a.pool = const_cast<void*>(pool);
+  a.layout = layout;
+  a.k_new = fused ? k_new : nullptr;
+  a.v_new = fused ? v_new : nullptr;
+  a.append_indptr = fused ? append_indptr : nullptr;
+  a.nnz_new = fused ? nnz_new : 0;
   cudaError_t e =
       pkv::launch_decode(tmap, a, dtype == PKV_BF16,
                          kv_dtype == PKV_FP8_E4M3 ? pkv::kKvE4M3
@@ -527,6 +546,29 @@ pkv_status pkv_decode(const void* q, int num_qo_heads, const void* pool, int64_t
                      batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
                      error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
                      num_qo_heads);
+}
+
+pkv_status pkv_decode_append(const void* q, int num_qo_heads, const pkv_pool_desc* pool,
+                             const pkv_table_desc* table, const void* k_new, const void* v_new,
+                             const int32_t* append_indptr, int64_t nnz_new, float sm_scale,
+                             int num_partitions, void* workspace, size_t workspace_bytes,
+                             void* out, float* lse, int32_t* error_word, void* stream) {
+  if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
+  pkv::TableView tv;
+  const int32_t* ids = nullptr;
+  pkv_status st = table_view(table, &tv, &ids);
+  if (st != PKV_OK) return st;
+  if (is_fp8(pool->dtype))
+    return fail(PKV_ERR_INVALID_ARG, "the fused append takes 16-bit pools (8-bit: pkv_append_fp8)");
+  if (nnz_new < 0) return fail(PKV_ERR_INVALID_ARG, "nnz_new < 0");
+  if (nnz_new > 0 && (pool->data == k_new || pool->data == v_new || out == k_new || out == v_new))
+    return fail(PKV_ERR_INVALID_ARG, "k_new / v_new alias the pool or out");
+  return decode_impl(q, num_qo_heads, pool->data, pool->num_pages, pool->page_size,
+                     pool->num_kv_heads, pool->head_dim, pool->dtype, pool->layout, tv, ids,
+                     table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
+                     error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
+                     num_qo_heads, -1, 1.f, 1.f, nullptr, 0, 1, k_new, v_new, append_indptr,
+                     nnz_new);
 }
 
 pkv_status pkv_decode_ex(const void* q, int num_qo_heads, const pkv_pool_desc* pool,

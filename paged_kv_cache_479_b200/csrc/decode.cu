@@ -213,6 +213,50 @@ __device__ __forceinline__ uint32_t widen_hi(uint32_t r) {
   else return prmt(r, 0u, 0x3424u);
 }
 
+// Fused append: the new rows of (request b, kv head kvh) at positions in
+// [tok_lo, tok_hi) are copied from k_new / v_new into their pages (16-byte
+// pieces spread over the warp's lanes), then each lane orders its stores
+// before the async-proxy (bulk-tensor) loads the warp issues next.  Each
+// position lies in exactly one tile, and only the CTA that owns that tile
+// reads it in this launch.
+__device__ __forceinline__ void write_new_rows(const DecodeArgs& a, const ReqInfo& ri, int b,
+                                               int kvh, long long tok_lo, long long tok_hi,
+                                               int lane) {
+  const long long a0 = a.append_indptr[b], a1 = a.append_indptr[b + 1];
+  const long long n_new = a1 - a0;
+  if (n_new <= 0) return;
+  if (a0 < 0 || a1 > a.nnz_new || n_new > ri.len) {
+    if (lane == 0 && a.err) atomicOr(a.err, kErrAppend);
+    return;
+  }
+  const long long first = ri.len - n_new;  // position of the first new row
+  const long long lo = tok_lo > first ? tok_lo : first;
+  const long long hi = tok_hi < ri.len ? tok_hi : ri.len;
+  if (lo >= hi) return;
+  const int ps = a.page_size;
+  const long long pieces = (hi - lo) * 2 * (kD / 8);  // rows x (K, V) x 16-byte pieces
+  for (long long e = lane; e < pieces; e += 32) {
+    const long long pos = lo + e / (2 * (kD / 8));
+    const int kv = (int)((e / (kD / 8)) & 1), c = (int)(e % (kD / 8));
+    const int page = a.indices[ri.page_base + pos / ps];
+    if (page < 0 || (long long)page >= a.num_pages) {
+      if (a.err) atomicOr(a.err, kErrPageId);
+      continue;
+    }
+    const long long slot = pos % ps;
+    const size_t src = ((size_t)(a0 + pos - first) * a.hkv + kvh) * kD + (size_t)c * 8;
+    const size_t dst =
+        (a.layout == PKV_LAYOUT_NHD
+             ? ((((size_t)page * 2 + kv) * ps + slot) * a.hkv + kvh) * kD
+             : ((((size_t)page * 2 + kv) * a.hkv + kvh) * ps + slot) * kD) +
+        (size_t)c * 8;
+    const uint16_t* from = static_cast<const uint16_t*>(kv ? a.v_new : a.k_new);
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.pool) + dst) =
+        *reinterpret_cast<const uint4*>(from + src);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // KV: the pool's element type -- kKv16 (q's own 16-bit type), kKvE4M3, kKvE5M2;
 // NQ: n8 column tiles per pair (2 only for short chunks over 16-bit pools);
 // CHUNK: short chunks (causal limits per column), else decode (one token per request)
@@ -431,6 +475,14 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           valid = left < kMetaValid ? (int)left : kMetaValid;
         } else {
           page = -1;
+        }
+        if constexpr (!FP8) {
+          if (a.k_new) {  // fused append: this batch's tiles' new rows, before their loads
+            const long long tiles_here = (n - k0) < 32 ? (n - k0) : 32;
+            write_new_rows(a, wk.ri, wk.b, wk.kvh, (t0 + k0) * kTileTokens,
+                           (t0 + k0 + (tiles_here > 0 ? tiles_here : 0)) * kTileTokens, lane);
+            __syncwarp();
+          }
         }
         const int flags = ((k >= n_pad - kConsumerWarps) ? kMetaSegLast : 0) |
                           ((seg & (kSegRecs - 1)) << kMetaSegShift);

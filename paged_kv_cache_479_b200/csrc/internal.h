@@ -37,6 +37,16 @@ struct DecodeArgs {
   long long nnz_q;        // rows of q (short chunks)
   int pcols;              // columns per partial-state slot (G for decode)
   int max_cols;           // short chunks: the caller's bound on q_len * G
+  // fused append (16-bit pools; k_new null = none): the step's new rows
+  // k_new / v_new [nnz_new][Hkv][128], request b's at append_indptr[b] ..,
+  // written into the pool (layout: PKV_LAYOUT_*) before the tiles holding them
+  // are loaded
+  void* pool;
+  int layout;
+  const void* k_new;
+  const void* v_new;
+  const int32_t* append_indptr;
+  long long nnz_new;
 };
 
 constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp

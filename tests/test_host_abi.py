@@ -340,3 +340,22 @@ def test_append_attention_short_rejects_bad_arguments():
     w2 = pkv.append_attention_short_workspace_bytes(32, 8, 2, 148)
     w4 = pkv.append_attention_short_workspace_bytes(32, 8, 4, 148)
     assert w2 >= 2 * 148 * 8 * 129 * 4 and w4 >= 2 * 148 * 16 * 129 * 4 and w4 > w2
+
+
+def test_decode_append_rejects_bad_arguments():
+    L = pkv.lib()
+    P = ctypes.c_void_p(4096)
+    K, V = ctypes.c_void_p(12288), ctypes.c_void_p(16384)
+    WS = ctypes.c_void_p(1 << 20)
+    pool = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.BF16, 0, 0)
+    csr = pkv.TableDesc(0, 4, 4096, 4096, 4096, None, None, 0, 0)
+
+    def call(pool=pool, k=K, v=V, nnz=4):
+        return L.pkv_decode_append(P, 8, ctypes.byref(pool), ctypes.byref(csr), k, v, P, nnz, 0.1,
+                                   4, WS, 1 << 20, ctypes.c_void_p(8192), None, None, None)
+
+    assert call(pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.FP8_E4M3, 0, 0)) == 1  # 8-bit pool
+    assert call(k=None) == 1
+    assert call(v=ctypes.c_void_p(16388)) == 1        # misaligned
+    assert call(nnz=-1) == 1
+    assert call(k=ctypes.c_void_p(4096)) == 1         # k_new aliases the pool
