@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--separate-append", action="store_true",
                    help="launch the append on its own instead of fusing it into the decode "
                         "(pkv_decode_append; 16-bit pools, plain decode)")
+    p.add_argument("--fused-chunk-append", action="store_true",
+                   help="--chunk spec: append the chunk's K/V inside the short-chunk launch "
+                        "(slower than a separate append at 4 rows per request)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cascade", action="store_true",
                    help="decode a shared-prefix workload with pkv_cascade_decode")
@@ -645,15 +648,23 @@ def run_chunk(args):
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # the short path can append the chunk's K/V inside its own launch; with 4 rows
+    # per (request, kv head) the producer-side writes delay the loads more than a
+    # separate append costs, so it is opt-in
+    fuse_short = short and args.fused_chunk_append
+
     def append_call(bt):
+        if fuse_short:
+            return
         pkv.paged_kv_append(bt[1], indptr, indices, last, bt[2], bt[3], app, error_word=err,
                             stream=torch.cuda.current_stream(dev))
 
     def attn_call(bt):
         if short:
+            fused_rows = dict(k_new=bt[2], v_new=bt[3], append_indptr=app) if fuse_short else {}
             pkv.append_attention_short(bt[0], qo_d, bt[1], table, mq, ws_s, out=out, lse=lse,
                                        sm_scale=w.sm_scale, error_word=err,
-                                       stream=torch.cuda.current_stream(dev))
+                                       stream=torch.cuda.current_stream(dev), **fused_rows)
         else:
             pkv.append_attention(bt[0], qo_d, bt[1], table, plan, S, workspace=ws, out=out,
                                  lse=lse, sm_scale=w.sm_scale, error_word=err,
@@ -672,7 +683,7 @@ def run_chunk(args):
     torch.cuda.synchronize()
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during warm-up")
-    app_g = [graphed(append_call, bt) for bt in batches]
+    app_g = [(lambda: None) if fuse_short else graphed(append_call, bt) for bt in batches]
     att_g = [graphed(attn_call, bt) for bt in batches]
     clocks = ClockSampler(local)
     K = args.steps
@@ -712,7 +723,8 @@ def run_chunk(args):
                                       "TFLOP/s", "tensor", "TFLOP/s")
     else:
         peak, kind = measured_hbm()
-        achieved = attn_bytes / (attn_ms / 1e3) / 1e9
+        launch_bytes = attn_bytes + (wl.append_bytes(w) if fuse_short else 0)
+        achieved = launch_bytes / (attn_ms / 1e3) / 1e9
         value = job_throughput(step_bytes, world, ms, K)
         metric, unit, bound, runit = ("append attention, speculative verification: KV HBM GB/s",
                                       "GB/s", "hbm", "GB/s")
@@ -731,19 +743,21 @@ def run_chunk(args):
                        "flops_per_step": flops,
                        "attention_bytes_per_step": attn_bytes,
                        "l2": f"2 rotating batch copies of {kv / 1e6:.0f} MB K/V",
-                       "launch": "append and append attention captured as CUDA graphs",
+                       "launch": ("append fused into the attention launch, captured as a CUDA "
+                                  "graph" if fuse_short else
+                                  "append and append attention captured as CUDA graphs"),
                        "parallelism": f"dp{world} (independent batches per GPU)"},
             "us_per_step": round(ms / K * 1e3, 2),
             "tokens_per_s": round(nnz * world / (ms / K / 1e3), 1),
             "roofline": {"bound": bound,
-                         "kernel": ("decode_kernel (short chunks)" if short
+                         "kernel": ("decode_kernel (short chunks" + (", append fused)" if fuse_short else ")") if short
                                     else "chunk_kernel" + (" + merge" if S > 1 else "")),
                          "achieved": round(achieved, 1), "peak": peak, "unit": runit,
                          "frac": round(achieved / peak, 4),
                          "peak_kind": f"{kind} (MEASURED_PEAKS.json "
                                       f"{'bf16_tflops, burst' if bound == 'tensor' else 'hbm_gbs'})",
                          "traffic": None, "avg_launch_us": round(attn_ms * 1e3, 2)},
-            "gpu_launches": K * (2 + (1 if S > 1 and not short else 0)),
+            "gpu_launches": K * ((1 if fuse_short else 2) + (1 if S > 1 and not short else 0)),
             "e2e": None,
             "clocks": clocks.summary(t_host0, t_host1),
         }

@@ -357,6 +357,10 @@ PKV_API pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr,
  *                larger, or larger than its cache, sets PKV_DEVERR_APPEND and its
  *                rows are left unwritten; requests with q_len = 0 write nothing
  *   pool, table  descriptors (16-bit pools, head_dim 128, either layout and form)
+ *   k_new, v_new, append_indptr, nnz_new   optional (nnz_new = 0: none): the
+ *                chunk's own K/V rows as in pkv_append_ex, written into the pool
+ *                by the same launch before the tiles that hold them are loaded
+ *                (the pool ends bitwise as after pkv_append_ex; 16-bit rows)
  *   num_partitions, workspace  as in pkv_decode, the workspace sized by
  *                pkv_append_attention_short_workspace_bytes (device, zero-filled
  *                once; the kernel leaves its counters zeroed)
@@ -367,7 +371,9 @@ PKV_API size_t pkv_append_attention_short_workspace_bytes(int num_qo_heads, int 
 PKV_API pkv_status pkv_append_attention_short(const void* q, const int32_t* qo_indptr,
                                               int64_t nnz_q, int max_q_len, int num_qo_heads,
                                               const pkv_pool_desc* pool,
-                                              const pkv_table_desc* table, float sm_scale,
+                                              const pkv_table_desc* table, const void* k_new,
+                                              const void* v_new, const int32_t* append_indptr,
+                                              int64_t nnz_new, float sm_scale,
                                               int num_partitions, void* workspace,
                                               size_t workspace_bytes, void* out, float* lse,
                                               int32_t* error_word, void* stream);

@@ -77,7 +77,7 @@ _SIGNATURES["pkv_append_attention"] = (
     [_P, _P, _I64, _I32, _PP, _TP, _P, _I64, _I32, _I32, _I32, _F32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["pkv_append_attention_short_workspace_bytes"] = ([_I32, _I32, _I32, _I32], _SZ)
 _SIGNATURES["pkv_append_attention_short"] = (
-    [_P, _P, _I64, _I32, _I32, _PP, _TP, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
+    [_P, _P, _I64, _I32, _I32, _PP, _TP, _P, _P, _P, _I64, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["pkv_decode_append"] = (
     [_P, _I32, _PP, _TP, _P, _P, _P, _I64, _F32, _I32, _P, _SZ, _P, _P, _P, _P], _I32)
 _SIGNATURES["paged_kv_append"] = _SIGNATURES["pkv_append"]
@@ -485,13 +485,21 @@ def append_attention_short_workspace_bytes(num_qo_heads: int, num_kv_heads: int,
 
 def append_attention_short(q, qo_indptr, pool, table: TableDesc, max_q_len: int, workspace,
                            layout: str = "HND", num_partitions: int = 0, out=None, lse=None,
-                           sm_scale=None, error_word=None, stream=None, return_lse: bool = True):
+                           sm_scale=None, error_word=None, stream=None, return_lse: bool = True,
+                           k_new=None, v_new=None, append_indptr=None):
     """pkv_append_attention_short: append attention (no window) for chunks of at
     most max_q_len tokens, max_q_len * (Hq / Hkv) <= 16, on the decode kernel's
     schedule.  workspace: zero-filled device buffer of
-    append_attention_short_workspace_bytes bytes."""
+    append_attention_short_workspace_bytes bytes.  With k_new / v_new /
+    append_indptr the chunk's K/V rows are appended by the same launch."""
     _dev_tensor(q, "q", pool.dtype)
     _dev_tensor(qo_indptr, "qo_indptr", torch.int32)
+    nnz_new = 0
+    if k_new is not None:
+        _dev_tensor(k_new, "k_new", pool.dtype)
+        _dev_tensor(v_new, "v_new", pool.dtype)
+        _dev_tensor(append_indptr, "append_indptr", torch.int32)
+        nnz_new = k_new.shape[0]
     pd = pool_desc(pool, layout)
     nnz, hq, d = q.shape
     if out is None:
@@ -501,7 +509,8 @@ def append_attention_short(q, qo_indptr, pool, table: TableDesc, max_q_len: int,
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     scale = float(sm_scale) if sm_scale is not None else 1.0 / float(d) ** 0.5
     st = lib().pkv_append_attention_short(_ptr(q), _ptr(qo_indptr), nnz, max_q_len, hq,
-                                          ctypes.byref(pd), ctypes.byref(table), scale,
+                                          ctypes.byref(pd), ctypes.byref(table), _ptr(k_new),
+                                          _ptr(v_new), _ptr(append_indptr), nnz_new, scale,
                                           num_partitions, _ptr(workspace), ws_bytes, _ptr(out),
                                           _ptr(lse), _ptr(error_word), _stream(stream, q.device))
     _check(st, "pkv_append_attention_short")

@@ -867,9 +867,11 @@ size_t pkv_append_attention_short_workspace_bytes(int num_qo_heads, int num_kv_h
 
 pkv_status pkv_append_attention_short(const void* q, const int32_t* qo_indptr, int64_t nnz_q,
                                       int max_q_len, int num_qo_heads, const pkv_pool_desc* pool,
-                                      const pkv_table_desc* table, float sm_scale,
-                                      int num_partitions, void* workspace, size_t workspace_bytes,
-                                      void* out, float* lse, int32_t* error_word, void* stream) {
+                                      const pkv_table_desc* table, const void* k_new,
+                                      const void* v_new, const int32_t* append_indptr,
+                                      int64_t nnz_new, float sm_scale, int num_partitions,
+                                      void* workspace, size_t workspace_bytes, void* out,
+                                      float* lse, int32_t* error_word, void* stream) {
   if (!pool) return fail(PKV_ERR_INVALID_ARG, "null pool descriptor");
   pkv::TableView tv;
   const int32_t* ids = nullptr;
@@ -879,12 +881,18 @@ pkv_status pkv_append_attention_short(const void* q, const int32_t* qo_indptr, i
     return fail(PKV_ERR_INVALID_ARG, "pool dtype must be PKV_F16 or PKV_BF16");
   if (nnz_q < 0) return fail(PKV_ERR_INVALID_ARG, "nnz_q < 0");
   if (table->batch > 0 && !qo_indptr) return fail(PKV_ERR_INVALID_ARG, "null qo_indptr");
+  if (nnz_new < 0) return fail(PKV_ERR_INVALID_ARG, "nnz_new < 0");
+  if (nnz_new > 0 && (pool->data == k_new || pool->data == v_new || out == k_new || out == v_new))
+    return fail(PKV_ERR_INVALID_ARG, "k_new / v_new alias the pool or out");
+  if (nnz_q == 0 && nnz_new > 0)
+    return pkv_append_ex(pool, table, k_new, v_new, append_indptr, nnz_new, error_word, stream);
   if (nnz_q == 0) return ok();
   return decode_impl(q, num_qo_heads, pool->data, pool->num_pages, pool->page_size,
                      pool->num_kv_heads, pool->head_dim, pool->dtype, pool->layout, tv, ids,
                      table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
                      error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
-                     num_qo_heads, -1, 1.f, 1.f, qo_indptr, nnz_q, max_q_len);
+                     num_qo_heads, -1, 1.f, 1.f, qo_indptr, nnz_q, max_q_len, k_new, v_new,
+                     append_indptr, nnz_new);
 }
 
 size_t pkv_append_attention_workspace_bytes(int64_t nnz_q, int num_qo_heads, int num_splits) {

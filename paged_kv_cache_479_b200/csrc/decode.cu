@@ -235,24 +235,40 @@ __device__ __forceinline__ void write_new_rows(const DecodeArgs& a, const ReqInf
   if (lo >= hi) return;
   const int ps = a.page_size;
   const long long pieces = (hi - lo) * 2 * (kD / 8);  // rows x (K, V) x 16-byte pieces
-  for (long long e = lane; e < pieces; e += 32) {
-    const long long pos = lo + e / (2 * (kD / 8));
-    const int kv = (int)((e / (kD / 8)) & 1), c = (int)(e % (kD / 8));
-    const int page = a.indices[ri.page_base + pos / ps];
-    if (page < 0 || (long long)page >= a.num_pages) {
-      if (a.err) atomicOr(a.err, kErrPageId);
-      continue;
+  // up to 4 pieces per lane per round: every load of the round is issued
+  // before its stores, so a round costs one load latency, not four
+  constexpr int kU = 4;
+  for (long long e0 = 0; e0 < pieces; e0 += 32 * kU) {
+    uint4 val[kU];
+    size_t dst[kU];
+    bool put[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const long long e = e0 + u * 32 + lane;
+      put[u] = false;
+      dst[u] = 0;
+      if (e < pieces) {
+        const long long pos = lo + e / (2 * (kD / 8));
+        const int kv = (int)((e / (kD / 8)) & 1), c = (int)(e % (kD / 8));
+        const int page = __ldg(a.indices + ri.page_base + pos / ps);
+        const long long slot = pos % ps;
+        const size_t src = ((size_t)(a0 + pos - first) * a.hkv + kvh) * kD + (size_t)c * 8;
+        const uint16_t* from = static_cast<const uint16_t*>(kv ? a.v_new : a.k_new);
+        val[u] = __ldg(reinterpret_cast<const uint4*>(from + src));
+        if (page < 0 || (long long)page >= a.num_pages) {
+          if (a.err) atomicOr(a.err, kErrPageId);
+        } else {
+          put[u] = true;
+          dst[u] = (a.layout == PKV_LAYOUT_NHD
+                        ? ((((size_t)page * 2 + kv) * ps + slot) * a.hkv + kvh) * kD
+                        : ((((size_t)page * 2 + kv) * a.hkv + kvh) * ps + slot) * kD) +
+                   (size_t)c * 8;
+        }
+      }
     }
-    const long long slot = pos % ps;
-    const size_t src = ((size_t)(a0 + pos - first) * a.hkv + kvh) * kD + (size_t)c * 8;
-    const size_t dst =
-        (a.layout == PKV_LAYOUT_NHD
-             ? ((((size_t)page * 2 + kv) * ps + slot) * a.hkv + kvh) * kD
-             : ((((size_t)page * 2 + kv) * a.hkv + kvh) * ps + slot) * kD) +
-        (size_t)c * 8;
-    const uint16_t* from = static_cast<const uint16_t*>(kv ? a.v_new : a.k_new);
-    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.pool) + dst) =
-        *reinterpret_cast<const uint4*>(from + src);
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (put[u]) *reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.pool) + dst[u]) = val[u];
   }
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }

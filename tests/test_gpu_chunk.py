@@ -242,6 +242,41 @@ def test_short_chunks_layouts_and_tables_bitwise(layout, kind):
     assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
 
 
+@pytest.mark.parametrize("parts", [0, 5])
+def test_short_chunks_fused_append_matches_separate(parts):
+    # the chunk's K/V rows appended by the attention launch itself: the pool and
+    # the outputs are bitwise those of the separate append and attention
+    q_lens = np.array([4, 3, 1, 4, 2, 4], np.int64)
+    w = wl.make_workload("short-fused", [40, 100, 17, 300, 33, 2000], num_qo_heads=32,
+                         num_kv_heads=8, page_size=16, dtype="bf16", seed=760, pool_factor=1.3,
+                         append_counts=q_lens)
+    _, pool, k_new, v_new = wl.make_tensors(w, "cuda")
+    qo = wl.chunk_indptr(q_lens)
+    q = wl.make_chunk_queries(w, q_lens, "cuda")
+    ip, ix, ll = i32(w.page_indptr), i32(w.page_indices), i32(w.last_page_len)
+    table = pkv.csr_table(ip, ix, ll)
+    app, qoi = i32(w.append_indptr), i32(qo)
+    nb = pkv.append_attention_short_workspace_bytes(w.num_qo_heads, w.num_kv_heads, 4, parts)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    p_sep = pool.clone()
+    pkv.paged_kv_append(p_sep, ip, ix, ll, k_new, v_new, app, error_word=err)
+    ws = torch.zeros(nb // 4 + 64, dtype=torch.int32, device="cuda")
+    o_sep, l_sep = pkv.append_attention_short(q, qoi, p_sep, table, 4, ws, num_partitions=parts,
+                                              sm_scale=w.sm_scale, error_word=err)
+    p_fus = pool.clone()
+    ws = torch.zeros(nb // 4 + 64, dtype=torch.int32, device="cuda")
+    o_fus, l_fus = pkv.append_attention_short(q, qoi, p_fus, table, 4, ws, num_partitions=parts,
+                                              sm_scale=w.sm_scale, error_word=err,
+                                              k_new=k_new, v_new=v_new, append_indptr=app)
+    torch.cuda.synchronize()
+    assert pkv.read_error_word(err) == 0
+    assert torch.equal(p_fus.view(torch.int16), p_sep.view(torch.int16))
+    assert torch.equal(o_fus, o_sep) and torch.equal(l_fus, l_sep)
+    ro, rl = oracle.append_attention(wl.bits(q), wl.bits(p_fus), odtype(w), w.page_indptr,
+                                     w.page_indices, w.last_page_len, qo, w.sm_scale)
+    assert_parity(o_fus, l_fus, ro, rl, what="fused short")
+
+
 def test_short_chunk_longer_than_bound_sets_error_bit():
     c = ChunkCase([100, 100, 60], [2, 5, 3], 32, 8, 16, "bf16", 747)
     sentinel = torch.full_like(c.q, 7.0, device="cuda")

@@ -324,8 +324,8 @@ def test_append_attention_short_rejects_bad_arguments():
 
     def call(pool=pool, max_q_len=4, hq=8, ws_bytes=need, qo=P):
         return L.pkv_append_attention_short(P, qo, 16, max_q_len, hq, ctypes.byref(pool),
-                                            ctypes.byref(csr), 0.1, 4, WS, ws_bytes,
-                                            ctypes.c_void_p(8192), None, None, None)
+                                            ctypes.byref(csr), None, None, None, 0, 0.1, 4, WS,
+                                            ws_bytes, ctypes.c_void_p(8192), None, None, None)
 
     assert call(max_q_len=5) == 2                     # 5 tokens x 4 heads > 16 columns
     assert call(max_q_len=0) == 2
@@ -334,6 +334,13 @@ def test_append_attention_short_rejects_bad_arguments():
     assert call(pkv.PoolDesc(4096, 64, 16, 2, 64, pkv.BF16, 0, 0)) == 2
     assert call(ws_bytes=need - 1) == 3
     assert call(qo=None) == 1
+    # the optional fused append: negative count, rows aliasing the pool
+    assert L.pkv_append_attention_short(P, P, 16, 4, 8, ctypes.byref(pool), ctypes.byref(csr),
+                                        None, None, None, -1, 0.1, 4, WS, need,
+                                        ctypes.c_void_p(8192), None, None, None) == 1
+    assert L.pkv_append_attention_short(P, P, 16, 4, 8, ctypes.byref(pool), ctypes.byref(csr),
+                                        ctypes.c_void_p(4096), ctypes.c_void_p(12288), P, 4, 0.1,
+                                        4, WS, need, ctypes.c_void_p(8192), None, None, None) == 1
     # 8 or 16 state columns per slot
     assert pkv.append_attention_short_workspace_bytes(32, 8, 5, 4) == 0
     assert pkv.append_attention_short_workspace_bytes(32, 8, 0, 4) == 0
