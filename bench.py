@@ -4,7 +4,9 @@
 One step = one pass of the whole decode hot path over one batch: append the
 step's new K/V token(s) into their pages (when the workload appends), then
 decode attention for every request with the split-KV partition and the
-in-kernel merge.  Default workload: the Llama-3-8B-shaped decode layer
+in-kernel merge.  On 16-bit pools the append runs inside the decode launch
+(pkv_decode_append; --separate-append launches it on its own).  Default
+workload: the Llama-3-8B-shaped decode layer
 (batch 64, KV lengths U[512,4096] + 1 appended token, 32 q / 8 kv heads,
 head_dim 128, page size 16, bf16, pool 1.25x the pages needed).
 
