@@ -235,9 +235,11 @@ PKV_API pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc
  *            16-bit (PKV_F16 / PKV_BF16, as k_new / v_new; 8-bit pools:
  *            pkv_append_fp8 then pkv_decode_fp8); nnz_new = 0 is a plain decode
  * On return (stream order) the pool holds exactly what pkv_append_ex would have
- * written and out / lse what pkv_decode_ex would have computed on it.  Bad
- * append_indptr entries set PKV_DEVERR_APPEND and leave that request's rows
- * unwritten.  k_new / v_new must not alias the pool or out.
+ * written and out / lse what pkv_decode_ex would have computed on it.  A
+ * request whose append_indptr entries start below 0, end past nnz_new or claim
+ * more rows than the request holds sets PKV_DEVERR_APPEND and gets no rows
+ * written (a decreasing pair appends nothing).  k_new / v_new must not alias
+ * the pool or out.
  */
 PKV_API pkv_status pkv_decode_append(const void* q, int num_qo_heads, const pkv_pool_desc* pool,
                                      const pkv_table_desc* table, const void* k_new,
