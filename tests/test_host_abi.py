@@ -366,3 +366,26 @@ def test_decode_append_rejects_bad_arguments():
     assert call(v=ctypes.c_void_p(16388)) == 1        # misaligned
     assert call(nnz=-1) == 1
     assert call(k=ctypes.c_void_p(4096)) == 1         # k_new aliases the pool
+
+
+@pytest.mark.parametrize("N", [1, 3, 7, 148, 600])
+def test_fused_append_writes_every_new_row_once(N):
+    # the fused append writes a new row from the segment that owns its tile, in
+    # the 32-tile batch that holds it; over the host mirror of the partition
+    # every (request, kv head, new position) comes out exactly once
+    lens = [1, 15, 16, 17, 33, 300, 700, 0, 4097, 2]
+    counts = [1, 15, 1, 17, 2, 40, 600, 0, 513, 2]
+    w = wl.make_workload("fa", lens, num_qo_heads=8, num_kv_heads=4, page_size=16,
+                         dtype="bf16", seed=5, append_counts=counts)
+    seg = pkv.plan_segments(w.page_indptr, w.last_page_len, 16, 4, N)
+    written = []
+    for c, b, g, t0, t1, slot, ncov in seg.tolist():
+        L, n_new = int(w.kv_lens[b]), int(counts[b])
+        n = t1 - t0
+        for k0 in range(0, max(n, 0), 32):
+            lo = max((t0 + k0) * 16, L - n_new)
+            hi = min((t0 + min(k0 + 32, n)) * 16, L)
+            written += [(b, g, p) for p in range(lo, hi)]
+    expect = [(b, g, p) for b in range(w.batch) for g in range(4)
+              for p in range(int(w.kv_lens[b]) - counts[b], int(w.kv_lens[b]))]
+    assert sorted(written) == sorted(expect)
