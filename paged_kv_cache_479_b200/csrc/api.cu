@@ -658,9 +658,22 @@ CascadePlan cascade_plan(int batch, int hq, int hkv, long long prefix_len, int N
   p.row_blocks = (int)((rows + R - 1) / R);
   const long long tiles = (prefix_len + T - 1) / T;
   const long long units = (long long)p.row_blocks * hkv;
-  long long splits = units >= sms ? 1 : (sms + units - 1) / units;  // about one wave of CTAs
-  if (splits > tiles) splits = tiles;
-  if (splits < 1) splits = 1;
+  // key splits: the count that minimises (waves of CTAs) x (tiles per CTA), one
+  // CTA per SM being resident, plus half a tile per split for its state's share
+  // of the merge -- ceil(sms / units) splits can spill a few CTAs into a second
+  // wave that doubles the step (32 units on 148 SMs: 5 splits = 160 CTAs)
+  long long splits = 1;
+  if (units < sms && tiles > 1) {
+    double best = 1e300;
+    for (long long sp = 1; sp <= tiles && sp <= 64; ++sp) {
+      const long long waves = (units * sp + sms - 1) / sms;
+      const double cost = (double)(waves * ((tiles + sp - 1) / sp)) + 0.5 * (double)sp;
+      if (cost < best) {
+        best = cost;
+        splits = sp;
+      }
+    }
+  }
   p.splits = (int)splits;
   p.states = p.splits + 1;
   p.state_o = 0;
