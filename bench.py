@@ -236,7 +236,7 @@ def workload_config(w, args, rotation, partitions):
         cfg["kv_cache"] = (f"FP8 {args.kv.upper()} codes, k_scale {FP8_K_SCALE}, v_scale {FP8_V_SCALE}; "
                            f"q / out {w.dtype}; append quantises the new {w.dtype} rows")
     if getattr(args, "cascade", False):
-        cfg["method"] = "shared-prefix cascade: prefix attention once per 128 query rows, own pages by the decode kernel, states merged"
+        cfg["method"] = "shared-prefix cascade: prefix attention once per 256 query rows (tcgen05), own pages by the decode kernel, states merged"
     return cfg
 
 
