@@ -6,9 +6,13 @@ step's new K/V token(s) into their pages (when the workload appends), then
 decode attention for every request with the split-KV partition and the
 in-kernel merge.  On 16-bit pools the append runs inside the decode launch
 (pkv_decode_append; --separate-append launches it on its own).  Default
-workload: the Llama-3-8B-shaped decode layer
-(batch 64, KV lengths U[512,4096] + 1 appended token, 32 q / 8 kv heads,
-head_dim 128, page size 16, bf16, pool 1.25x the pages needed).
+workload: the Llama3-70B-shaped 128K long context (batch 8, every KV length
+131072, 64 q / 8 kv heads, head_dim 128, page size 16, bf16, 4 GiB of K/V,
+random page placement, split-KV on).  Its line also carries `per_config`:
+the same measurement, same steps, for the tiny case, the Llama-3-8B-shaped
+decode layer (with its append), the single 200K sequence and the shared-
+prefix batch (plain decode and the cascade), each with its own oracle
+cpu_baseline.
 
 Metric: KV HBM GB/s (algorithmic bytes: unique K/V once + q + out + page
 table + lse, plus the append's rows), with us/step and decoded tokens/s.
@@ -50,7 +54,7 @@ def parse():
     p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["pkv", "reference"], default="pkv")
-    p.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    p.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
     p.add_argument("--partitions", type=int, default=0, help="split-KV partitions (0 = one per SM)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--separate-append", action="store_true",
@@ -60,6 +64,11 @@ def parse():
                    help="--chunk spec: append the chunk's K/V inside the short-chunk launch "
                         "(slower than a separate append at 4 rows per request)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="headline workload only (by default the 128K headline line also "
+                        "carries per_config numbers of workloads 1, 2, 4, 5 and the 5 cascade)")
+    p.add_argument("--per-config-cpu-seconds", type=float, default=4.0,
+                   help="oracle time budget of each per_config cpu_baseline")
     p.add_argument("--cascade", action="store_true",
                    help="decode a shared-prefix workload with pkv_cascade_decode")
     p.add_argument("--no-graph", action="store_true",
@@ -148,31 +157,68 @@ def recorded_traffic(workload_id):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
-              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
-              "clocks_event_reasons.sw_power_cap"]
+    """SM clock, power and throttle reasons of one GPU, read through NVML
+    every 2 ms from a background thread (read-only queries; no setting is
+    touched), so that even a timed region of a few milliseconds holds
+    samples.  Falls back to `nvidia-smi -lms 100` when NVML is unavailable."""
     REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    PERIOD_S = 0.002
 
     def __init__(self, device_index):
         self.samples = []
+        self.source = None
+        self._stop = threading.Event()
         self.proc = None
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        self.ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
         try:
-            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
-            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(self.ident)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.bits = [pynvml.nvmlClocksEventReasonHwSlowdown,
+                         pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                         pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                         pynvml.nvmlClocksEventReasonSwPowerCap]
+            self.source = f"NVML every {self.PERIOD_S * 1e3:.0f} ms"
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+        except Exception:
+            self._start_smi()
+
+    def _poll_nvml(self):
+        nv, h = self.nvml, self.handle
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                r = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                self.samples.append((time.time(), mhz, self.max_mhz, pw,
+                                     [bool(r & b) for b in self.bits]))
+            except Exception:
+                pass
+            self._stop.wait(self.PERIOD_S)
+
+    def _start_smi(self):
+        fields = ["clocks.sm", "clocks.max.sm", "power.draw",
+                  "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                  "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", ident, f"--query-gpu={','.join(self.FIELDS)}",
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={','.join(fields)}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi every 100 ms"
+            self.thread = threading.Thread(target=self._read_smi, args=(len(fields),), daemon=True)
             self.thread.start()
         except Exception:
             self.proc = None
 
-    def _read(self):
+    def _read_smi(self, nf):
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) != len(self.FIELDS):
+            if len(parts) != nf:
                 continue
             try:
                 self.samples.append((time.time(), float(parts[0]), float(parts[1]),
@@ -182,6 +228,7 @@ class ClockSampler:
                 continue
 
     def stop(self):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -194,14 +241,15 @@ class ClockSampler:
         window = "timed region"
         if not inside:
             inside = self.samples
-            window = "whole run (timed region shorter than the 100 ms sampling period)"
+            window = "whole run (timed region shorter than the sampling period)"
         if not inside:
             return None
         mhz = [s[1] for s in inside]
         reasons = sorted({self.REASONS[i] for s in inside for i, a in enumerate(s[4]) if a})
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(s[2] for s in inside),
-                "reasons": reasons, "samples": len(inside), "window": window,
-                "power_w_max": max(s[3] for s in inside)}
+        return {"sm_mhz": statistics.median(mhz), "sm_mhz_min": min(mhz),
+                "sm_max_mhz": max(s[2] for s in inside), "reasons": reasons,
+                "samples": len(inside), "window": window, "source": self.source,
+                "power_w_max": round(max(s[3] for s in inside), 1)}
 
 
 # scales of the E4M3 pools (typical codes have magnitude ~16: keys ~1, values ~0.1)
@@ -354,36 +402,28 @@ class Batch:
             self.q, self.pool, self.k_new, self.v_new = wl.make_tensors(wv, dev)
 
 
-def run_pkv(args):
+def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=False,
+                   clocks=None):
+    """Time args.steps decode steps of workload w (after args.warmup untimed
+    ones); returns a dict of the measurement.  A step is the append (fused into
+    the decode launch on 16-bit pools) and the decode, or the three launches of
+    the shared-prefix cascade."""
     import paged_kv_cache_479_b200 as pkv
-
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
-                                             device_id=dev)
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    w = wl.named(args.workload)
-    if args.cascade and not w.shared_prefix_pages:
-        raise SystemExit("--cascade needs a workload with a shared prefix (workload 5)")
-    fp8 = None if args.kv == "16bit" else args.kv
-    if fp8 and args.cascade:
-        raise SystemExit("--cascade runs on 16-bit pools only")
-    N = args.partitions or pkv.default_partitions(local)
-    kv_bytes = wl.logical_kv_bytes(w, kv_elem_bytes(args))
+    N = args.partitions or pkv.default_partitions(dev.index)
+    kvb = 1 if fp8 else None
+    kv_bytes = wl.logical_kv_bytes(w, kvb)
     rotation = 2 if kv_bytes < (2 << 30) else 1
     batches = [Batch(w, dev, rank_value_seed(w.seed, rank, r), fp8) for r in range(rotation)]
     t = lambda a: torch.as_tensor(a, device=dev)
     indptr, indices, last = t(w.page_indptr), t(w.page_indices), t(w.last_page_len)
     app = t(w.append_indptr)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    if args.cascade:
+    if cascade:
         c_prefix, c_len, c_ip, c_ix, c_ll = wl.cascade_view(w)
         c_prefix, c_ip, c_ix, c_ll = (t(np.ascontiguousarray(x, np.int32)) for x in
                                       (c_prefix, c_ip, c_ix, c_ll))
@@ -397,9 +437,8 @@ def run_pkv(args):
     stream = torch.cuda.current_stream(dev)
     # the step's append runs inside the decode launch (pkv_decode_append) unless
     # it cannot (8-bit pool, cascade) or --separate-append asks otherwise
-    fused = bool(w.nnz_new) and not fp8 and not args.cascade and not args.separate_append
-    launches_per_step = (3 if args.cascade else 1) + (1 if w.nnz_new and not fused else 0)
-
+    fused = bool(w.nnz_new) and not fp8 and not cascade and not args.separate_append
+    launches_per_step = (3 if cascade else 1) + (1 if w.nnz_new and not fused else 0)
     table = pkv.csr_table(indptr, indices, last)
 
     def append_call(bt):
@@ -414,27 +453,25 @@ def run_pkv(args):
                                 error_word=err, stream=torch.cuda.current_stream(dev))
 
     def decode_call(bt):
+        cur = torch.cuda.current_stream(dev)
         if fp8:
             pkv.paged_decode_attention_fp8(bt.q, bt.pool, table, ws, FP8_K_SCALE, FP8_V_SCALE,
                                            out=out, lse=lse, sm_scale=w.sm_scale,
-                                           num_partitions=N, error_word=err,
-                                           stream=torch.cuda.current_stream(dev), fp8_format=fp8)
-            return
-        if args.cascade:
+                                           num_partitions=N, error_word=err, stream=cur,
+                                           fp8_format=fp8)
+        elif cascade:
             pkv.cascade_decode(bt.q, bt.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws, out=out,
                                lse=lse, sm_scale=w.sm_scale, num_partitions=N, error_word=err,
-                               stream=torch.cuda.current_stream(dev))
-            return
-        if fused:
+                               stream=cur)
+        elif fused:
             pkv.paged_decode_append(bt.q, bt.pool, table, bt.k_new, bt.v_new, app, ws, out=out,
                                     lse=lse, sm_scale=w.sm_scale, num_partitions=N,
-                                    error_word=err, stream=torch.cuda.current_stream(dev))
-            return
-        pkv.paged_decode_attention(bt.q, bt.pool, indptr, indices, last, ws, out=out, lse=lse,
-                                   sm_scale=w.sm_scale, num_partitions=N, error_word=err,
-                                   stream=torch.cuda.current_stream(dev))
+                                    error_word=err, stream=cur)
+        else:
+            pkv.paged_decode_attention(bt.q, bt.pool, indptr, indices, last, ws, out=out, lse=lse,
+                                       sm_scale=w.sm_scale, num_partitions=N, error_word=err,
+                                       stream=cur)
 
-    clocks = ClockSampler(local)
     for i in range(args.warmup):
         append_call(batches[i % rotation])
         decode_call(batches[i % rotation])
@@ -444,12 +481,15 @@ def run_pkv(args):
 
     # the same calls captured once per batch copy and replayed (no Python on the
     # launch path); each library call is capturable: no allocation, no sync
+    graphs = []
+
     def graphed(fn, bt):
         if args.no_graph:
             return lambda: fn(bt)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             fn(bt)
+        graphs.append(g)
         return g.replay
     app_g = [graphed(append_call, bt) if w.nnz_new and not fused else (lambda: None)
              for bt in batches]
@@ -458,14 +498,6 @@ def run_pkv(args):
         app_g[i % rotation]()
         dec_g[i % rotation]()
     torch.cuda.synchronize()
-
-    def step(r, ev0=None, ev1=None):
-        app_g[r]()
-        if ev0 is not None:
-            ev0.record(stream)
-        dec_g[r]()
-        if ev1 is not None:
-            ev1.record(stream)
 
     K = args.steps
     d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -476,31 +508,30 @@ def run_pkv(args):
     t_host0 = time.time()
     start.record(stream)
     for i in range(K):
-        step(i % rotation, d0[i], d1[i])
+        app_g[i % rotation]()
+        d0[i].record(stream)
+        dec_g[i % rotation]()
+        d1[i].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.time()
     barrier()
-    ms_local = start.elapsed_time(end)
-    decode_ms = sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K
-    ms = max_over_ranks(ms_local, world, dev)
-    decode_ms_max = max_over_ranks(decode_ms, world, dev)
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    decode_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K, world, dev)
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during the timed steps")
 
-    step_bytes = algorithmic_bytes(w, args)
-    s_per_step = ms / 1e3 / K
-    value = job_throughput(step_bytes, world, ms, K)
+    step_bytes = algorithmic_bytes(w, args if fp8 else None)
     # the timed launch's algorithmic bytes (with the append when it is fused in)
-    dec_bytes = wl.decode_bytes(w, kv_elem_bytes(args)) + (wl.append_bytes(w) if fused else 0)
-    peak, peak_kind = measured_hbm()
-    achieved = dec_bytes / (decode_ms_max / 1e3) / 1e9
+    dec_bytes = wl.decode_bytes(w, kvb) + (wl.append_bytes(w) if fused else 0)
+    res = {"ms": ms, "K": K, "decode_ms": decode_ms, "step_bytes": step_bytes,
+           "dec_bytes": dec_bytes, "fused": fused, "launches_per_step": launches_per_step,
+           "rotation": rotation, "N": N, "t_host0": t_host0, "t_host1": t_host1, "e2e": None}
 
     # ---- end to end through the public API with host buffers: every step copies
     # its inputs (q, new K/V rows, the page table) from pinned host memory in one
     # transfer, runs append + decode, and reads out + lse back in one transfer
-    e2e = None
-    if not args.no_e2e:
+    if e2e:
         src = batches[0]
         inputs = [src.q.cpu(), src.k_new.cpu(), src.v_new.cpu()] + [
             torch.from_numpy(np.ascontiguousarray(x)) for x in
@@ -510,7 +541,6 @@ def run_pkv(args):
         h_out, d_out = pack([out.cpu(), lse.cpu()], dev)
         out_d, lse_d = d_out
         h2d, d2h = h_in[0].numel(), h_out[0].numel()
-
         e2e_table = pkv.csr_table(ip_d, ix_d, ll_d)
 
         def e2e_calls(_):
@@ -533,7 +563,7 @@ def run_pkv(args):
                 if w.nnz_new:
                     pkv.paged_kv_append(src.pool, ip_d, ix_d, ll_d, k_d, v_d, ap_d,
                                         error_word=err, stream=cur)
-                if args.cascade:
+                if cascade:
                     pkv.cascade_decode(q_d, src.pool, c_prefix, c_len, c_ip, c_ix, c_ll, ws,
                                        out=out_d, lse=lse_d, sm_scale=w.sm_scale,
                                        num_partitions=N, error_word=err, stream=cur)
@@ -563,13 +593,91 @@ def run_pkv(args):
         torch.cuda.synchronize()
         barrier()
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        e2e = {"value": round(job_throughput(step_bytes, world, e_ms, K), 2), "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "us_per_step": round(e_ms / K * 1e3, 2),
-               "path": "pinned host -> device (1 copy), " +
-                       ("append fused into the decode launch" if fused else "append + decode") +
-                       ", device -> pinned host (1 copy), stream sync every step" +
-                       ("" if args.no_graph else "; the step's calls replayed as one CUDA graph")}
+        if pkv.read_error_word(err) != 0:
+            raise RuntimeError("device error bits set during the end-to-end steps")
+        res["e2e"] = {"value": round(job_throughput(step_bytes, world, e_ms, K), 2), "unit": "GB/s",
+                      "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                      "us_per_step": round(e_ms / K * 1e3, 2),
+                      "path": "pinned host -> device (1 copy), " +
+                              ("append fused into the decode launch" if fused else
+                               ("append + " if w.nnz_new else "") +
+                               ("cascade decode" if cascade else "decode")) +
+                              ", device -> pinned host (1 copy), stream sync every step" +
+                              ("" if args.no_graph else "; the step's calls replayed as one CUDA graph")}
+    del graphs
+    return res
+
+
+def kernel_name(fused, cascade, fp8):
+    if cascade:
+        return "pkv_cascade_decode (prefix + own-page decode + merge launches)"
+    if fp8:
+        return f"decode_kernel ({fp8} pool)"
+    return "decode_kernel (append fused)" if fused else "decode_kernel"
+
+
+def per_config_entry(w, args, r, world, peak, cascade, with_cpu):
+    """One workload's numbers for the line's per_config object."""
+    us = r["ms"] / r["K"] * 1e3
+    value = job_throughput(r["step_bytes"], world, r["ms"], r["K"])
+    achieved = r["dec_bytes"] / (r["decode_ms"] / 1e3) / 1e9
+    e = {"workload": w.name, "method": ("shared-prefix cascade (pkv_cascade_decode)" if cascade
+                                        else ("fused append + decode" if r["fused"] else "decode")),
+         "us_per_step": round(us, 2), "decode_us": round(r["decode_ms"] * 1e3, 2),
+         "kv_gb_s": round(value, 2), "tokens_per_s": round(w.batch * world / (us / 1e6), 1),
+         "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+         "frac_of_measured_hbm": round(value / world / peak, 4),
+         "decode_launch_gb_s": round(achieved, 1),
+         "decode_launch_frac_of_measured_hbm": round(achieved / peak, 4),
+         "algorithmic_bytes_per_step": r["step_bytes"],
+         "unique_kv_bytes": wl.kv_cache_bytes(1, w.num_kv_heads, w.head_dim,
+                                              wl.unique_kv_tokens(w), w.elem_bytes),
+         "gpu_launches_per_step": r["launches_per_step"]}
+    if with_cpu:
+        e["cpu_baseline"] = cpu_baseline(w, args.per_config_cpu_seconds)
+    return e
+
+
+def run_pkv(args):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                             device_id=dev)
+
+    w = wl.named(args.workload)
+    if args.cascade and not w.shared_prefix_pages:
+        raise SystemExit("--cascade needs a workload with a shared prefix (workload 5)")
+    fp8 = None if args.kv == "16bit" else args.kv
+    if fp8 and args.cascade:
+        raise SystemExit("--cascade runs on 16-bit pools only")
+    peak, peak_kind = measured_hbm()
+
+    clocks = ClockSampler(local)
+    r = measure_decode(w, args, dev, rank, world, cascade=args.cascade, fp8=fp8,
+                       e2e=not args.no_e2e)
+    clock_summary = clocks.summary(r["t_host0"], r["t_host1"])
+    K, ms = r["K"], r["ms"]
+    value = job_throughput(r["step_bytes"], world, ms, K)
+    achieved = r["dec_bytes"] / (r["decode_ms"] / 1e3) / 1e9
+    fused = r["fused"]
+
+    # the other named workloads, each the same number of steps, one at a time
+    per_config = None
+    if not args.no_per_config and not fp8 and not args.cascade and args.workload == 3:
+        per_config = {}
+        plan = [(1, False), (2, False), (4, False), (5, False), (5, True)]
+        for wid, casc in plan:
+            wk = wl.named(wid)
+            torch.cuda.empty_cache()
+            rk = measure_decode(wk, args, dev, rank, world, cascade=casc)
+            key = f"{wid}{'_cascade' if casc else ''}"
+            per_config[key] = per_config_entry(
+                wk, args, rk, world, peak, casc,
+                with_cpu=(world == 1 and not args.no_cpu_baseline and not casc))
+        torch.cuda.empty_cache()
     clocks.stop()
 
     if rank == 0:
@@ -580,32 +688,32 @@ def run_pkv(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": (f"{fp8} KV widened to f16, f32 accumulate" if fp8 else
                       ("bf16" if w.dtype == "bf16" else "f16")), "data": "synthetic",
-            "config": {**workload_config(w, args, rotation, N),
+            "config": {**workload_config(w, args, r["rotation"], r["N"]),
                        "launch": ("direct calls" if args.no_graph else
                                   ("the fused append + decode launch (pkv_decode_append)" if fused
-                                   else "append and decode each") +
+                                   else ("the cascade's launches" if args.cascade else
+                                         ("append and decode each" if w.nnz_new else "decode"))) +
                                   " captured once per batch copy as a CUDA graph, replayed")},
             "us_per_step": round(ms / K * 1e3, 2),
-            "tokens_per_s": round(w.batch * world / s_per_step, 1),
+            "tokens_per_s": round(w.batch * world / (ms / 1e3 / K), 1),
             "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
             "roofline": {"bound": "hbm",
-                         "kernel": ("pkv_cascade_decode (prefix + own-page decode + merge launches)"
-                                    if args.cascade else
-                                    (f"decode_kernel ({fp8} pool)" if fp8 else
-                                     ("decode_kernel (append fused)" if fused else "decode_kernel"))),
+                         "kernel": kernel_name(fused, args.cascade, fp8),
                          "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",
-                         "traffic": traffic, "algorithmic_bytes_per_launch": dec_bytes,
-                         "avg_launch_us": round(decode_ms_max * 1e3, 2)},
-            "gpu_launches": K * launches_per_step,
-            "e2e": e2e,
-            "clocks": clocks.summary(t_host0, t_host1),
+                         "traffic": traffic, "algorithmic_bytes_per_launch": r["dec_bytes"],
+                         "avg_launch_us": round(r["decode_ms"] * 1e3, 2)},
+            "gpu_launches": K * r["launches_per_step"],
+            "e2e": r["e2e"],
+            "clocks": clock_summary,
         }
         if world == 1 and not args.no_cpu_baseline and not fp8:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        if per_config is not None:
+            line["per_config"] = per_config
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

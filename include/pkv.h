@@ -133,6 +133,22 @@ PKV_API const char* pkv_status_string(int status);
 /* Detail of the last non-OK status returned on this host thread ("" if none). */
 PKV_API const char* pkv_last_error(void);
 
+/*
+ * Time limit, in nanoseconds, of every wait inside the decode kernel
+ * (pkv_decode and the calls built on it) for launches made after this call;
+ * 0 restores the default of one second.  Returns the previous limit.  A wait
+ * that runs past it sets PKV_DEVERR_TIMEOUT and the CTA gives up: it still
+ * lets its own copies in flight land (with the full one-second limit) and
+ * counts itself in on the split pairs it shares, so the launch completes,
+ * the CUDA context stays usable and the workspace can be reused as it is by
+ * the next call; only that launch's outputs are invalid.  The library never
+ * needs a limit below the default; a short one exists so that tests can make
+ * a wait run out and check this error path.  Process-wide; safe to call from
+ * any host thread.  (No counterpart in the pages: it is part of the failure
+ * handling of this library.)
+ */
+PKV_API uint64_t pkv_set_wait_limit_ns(uint64_t nanoseconds);
+
 /* Number of split-KV partitions pkv_decode uses when num_partitions = 0 on
  * `device`: one persistent CTA per SM.  Returns a value < 0 on error. */
 PKV_API int pkv_default_partitions(int device);
@@ -142,9 +158,11 @@ PKV_API int pkv_default_partitions(int device);
  * count (num_partitions = 0 means pkv_default_partitions(current device)).
  * The workspace holds one arrival counter per partition and at most two
  * partial (o, lse) states per partition.  It must be 256-byte aligned and
- * ZERO-FILLED before its first use; pkv_decode leaves the counters at zero
- * when it returns, so the same workspace can be reused by later calls on
- * the same stream without clearing.  Returns 0 for invalid shapes.
+ * ZERO-FILLED before its first use; every launch leaves the counters at zero
+ * when it completes -- also a launch that set a PKV_DEVERR_* bit -- so the
+ * same workspace can be reused by later calls on the same stream without
+ * clearing.  Calls that overlap on the GPU must not share a workspace.
+ * Returns 0 for invalid shapes.
  */
 PKV_API size_t pkv_decode_workspace_bytes(int batch, int num_qo_heads, int num_kv_heads,
                                   int head_dim, int num_partitions);

@@ -13,6 +13,7 @@ Functions (C names in parentheses):
   decode_workspace_bytes (pkv_decode_workspace_bytes)
   default_partitions     (pkv_default_partitions)
   read_error_word        (pkv_read_error_word)
+  set_wait_limit_ns      (pkv_set_wait_limit_ns)  time limit of the decode's internal waits
   check_table            (pkv_check_table)     host-side table check
   plan_segments          (pkv_plan_segments)   host mirror of the split-KV partition
   decode_static_workspace (pkv_decode_static_workspace)  decode on the library's own scratch
@@ -58,6 +59,7 @@ from ._binding import (  # noqa: F401
     paged_decode_attention_fp8,
     paged_kv_append,
     paged_kv_append_ex,
+    set_wait_limit_ns,
     paged_kv_append_fp8,
     pool_desc,
     plan_segments,

@@ -39,6 +39,7 @@ _SIGNATURES = {
     "pkv_read_error_word": ([_P, _P, _I32, _P], _I32),
     "pkv_check_table": ([_P, _P, _P, _I32, _I64, _I32], _I32),
     "pkv_plan_segments": ([_P, _P, _I32, _I32, _I32, _I32, _P, _I64], _I64),
+    "pkv_set_wait_limit_ns": ([ctypes.c_uint64], ctypes.c_uint64),
 }
 _SIGNATURES["pkv_decode_static_workspace"] = (
     [_P, _I32, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P, _I32, _F32, _I32, _P, _P, _P, _P], _I32)
@@ -138,6 +139,12 @@ def _dev_tensor(t: torch.Tensor, name: str, dtype=None):
 def _stream(stream, device) -> ctypes.c_void_p:
     s = stream if stream is not None else torch.cuda.current_stream(device)
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def set_wait_limit_ns(nanoseconds: int) -> int:
+    """Time limit of the decode kernel's internal waits for later launches
+    (0 = the default, one second); returns the previous limit."""
+    return int(lib().pkv_set_wait_limit_ns(int(nanoseconds)))
 
 
 def default_partitions(device=None) -> int:

@@ -6,12 +6,16 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 
+#include "common.cuh"
 #include "internal.h"
 #include "partition.cuh"
 #include "pkv.h"
@@ -205,6 +209,36 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
 
 }  // namespace
 
+namespace {
+// the decode kernel's wait limit (pkv_set_wait_limit_ns); 0 selects the default
+std::atomic<unsigned long long> g_wait_ns{0};
+}  // namespace
+
+size_t pkv::decode_counter_bytes(int group, int num_partitions) {
+  const int N = num_partitions ? num_partitions : current_device_partitions();
+  if (N <= 0 || N > kMaxPartitions || group < 1) return 0;
+  return ws_layout(group, N).part_lse;
+}
+
+unsigned long long pkv::decode_wait_limit_ns() {
+  const unsigned long long v = g_wait_ns.load(std::memory_order_relaxed);
+  return v ? v : (unsigned long long)pkv::kWaitLimitNs;
+}
+
+cudaError_t pkv::ensure_smem_opt_in(const void* func, size_t bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({func, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  done.insert({func, dev});
+  return cudaSuccess;
+}
+
 pkv_status pkv::set_error(pkv_status s, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -320,6 +354,7 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.v_new = fused ? v_new : nullptr;
   a.append_indptr = fused ? append_indptr : nullptr;
   a.nnz_new = fused ? nnz_new : 0;
+  a.wait_ns = pkv::decode_wait_limit_ns();
   cudaError_t e =
       pkv::launch_decode(tmap, a, dtype == PKV_BF16,
                          kv_dtype == PKV_FP8_E4M3 ? pkv::kKvE4M3
@@ -418,6 +453,12 @@ const char* pkv_status_string(int status) {
 }
 
 const char* pkv_last_error(void) { return g_err; }
+
+uint64_t pkv_set_wait_limit_ns(uint64_t nanoseconds) {
+  const unsigned long long prev = pkv::decode_wait_limit_ns();
+  g_wait_ns.store(nanoseconds, std::memory_order_relaxed);
+  return prev;
+}
 
 int pkv_default_partitions(int device) {
   int sms = 0;

@@ -288,8 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       issued = i + 1;
     }
-    if (!ok && lane == 0) {
-      // aborted: let the copies already issued land before the CTA exits
+    if (lane == 0) {
+      // never leave with copies in flight, whoever gave up (the MMA or softmax
+      // warps may have stopped waiting while this warp finished cleanly)
       const int first = issued > kStages ? issued - kStages : 0;
       for (int k = first; k < issued; ++k) {
         const uint64_t t0 = global_timer_ns();
@@ -594,15 +595,8 @@ int chunk_tile_tokens() { return kTile; }
 cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const ChunkArgs& a, bool bf16, int row_blocks,
                             cudaStream_t stream) {
   auto kern = bf16 ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
-  static bool attr_set[2][64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = ensure_smem_opt_in(reinterpret_cast<const void*>(kern), kSmemBytes);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !attr_set[bf16][dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set[bf16][dev] = true;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)row_blocks, (unsigned)a.hkv, (unsigned)a.splits);
   cfg.blockDim = dim3(kThreads);

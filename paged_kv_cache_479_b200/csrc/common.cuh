@@ -57,18 +57,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // Wait for the phase of `bar` with the given parity to complete, for at most
-// kWaitLimitNs.  Returns false on timeout or when *abort is already set; on
+// limit_ns (default kWaitLimitNs).  Returns false on timeout or when *abort is already set; on
 // timeout it sets *abort and the PKV timeout bit in *err (if any).
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort, int* err) {
+                                                  volatile int* abort, int* err,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (*abort) return false;
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort = 1;
       if (err) atomicOr(err, 0x10);
       return false;

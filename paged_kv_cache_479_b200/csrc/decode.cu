@@ -111,21 +111,30 @@ struct SegRec {
   long long q_row;      // row of q / out of the first column's token
 };
 
+// A (request, kv head) pair this partition shares with others: the partition
+// holding its first tile owns counters[c_first]; ncover partitions hold its
+// tiles (ncover = 0: no such pair).
+struct SplitPair {
+  int c_first, ncover;
+};
+
 struct __align__(16) Ctl {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t cons;                      // consumer-only barrier (256 arrivals)
   uint64_t qfull[kQBufs];             // a segment's query rows landed in qbuf[i]
   int meta[kMaxStages];
+  int last_it[kMaxStages];            // ring position of the last hand-over of each slot (-1: none)
   SegRec seg[kSegRecs];
   long long warp_tot[kDecodeThreads / 32];
   long long Cb0;
   SegRec pend[kMaxPending];   // split pairs this CTA wrote partial states for
   int pend_last[kMaxPending]; // 1 when this CTA arrived last for that pair
+  SplitPair split[kMaxPending];  // the pairs holding this share's first and last unit
   int npend;
   int b0;
   int abort;
-  int pad_;
+  int counted;                // 1 once this CTA has counted itself in on its split pairs
 };
 
 struct Scratch {
@@ -192,11 +201,48 @@ __device__ __forceinline__ uint32_t ld_u32(const void* p) {
 }
 
 // all 256 consumer threads meet; bounded
-__device__ __forceinline__ bool cons_sync(Ctl& ctl, uint32_t& phase, int* err) {
+__device__ __forceinline__ bool cons_sync(Ctl& ctl, uint32_t& phase, int* err, uint64_t limit) {
   mbar_arrive(smem_u32(&ctl.cons));
-  const bool ok = mbar_wait_bounded(smem_u32(&ctl.cons), phase, &ctl.abort, err);
+  const bool ok = mbar_wait_bounded(smem_u32(&ctl.cons), phase, &ctl.abort, err, limit);
   phase ^= 1u;
   return ok;
+}
+
+// The pair holding unit `off` of request r (whose units start at flat unit
+// Hkv * Cb), if partition c holds one of its tiles and shares it with others.
+__device__ __forceinline__ SplitPair split_pair_at(long long W, int N, int c, int Hkv,
+                                                   long long Cb, const ReqInfo& r, long long off) {
+  SplitPair sp;
+  sp.c_first = 0;
+  sp.ncover = 0;
+  const long long kvh = off / r.units;
+  const SegPlace pl = seg_place(W, N, (long long)Hkv * Cb + kvh * r.units, r.units, c);
+  if (pl.ncover > 1 && c >= pl.c_first && c < pl.c_first + pl.ncover) {
+    sp.c_first = pl.c_first;
+    sp.ncover = pl.ncover;
+  }
+  return sp;
+}
+
+// Count this partition in on each pair it shares (at most two: the ones
+// holding its first and its last unit; every pair in between lies wholly
+// inside its share).  The last arrival resets the pair's counter and, when
+// this partition finished cleanly, merges the pair (pend_last).  Called once
+// per CTA on every path out of the kernel, so the counters are back at zero
+// when the launch ends, even after a wait ran out.
+__device__ void count_in(const DecodeArgs& a, Ctl& ctl, bool clean) {
+#pragma unroll
+  for (int k = 0; k < kMaxPending; ++k) {
+    const SplitPair sp = ctl.split[k];
+    if (sp.ncover <= 1) continue;
+    if (k == 1 && ctl.split[0].ncover > 1 && ctl.split[0].c_first == sp.c_first) continue;
+    const int old = atomicAdd(&a.counters[sp.c_first], 1);
+    if (old != sp.ncover - 1) continue;
+    a.counters[sp.c_first] = 0;  // the last arrival is the counter's only remaining user
+    if (!clean) continue;
+    for (int j = 0; j < ctl.npend && j < kMaxPending; ++j)
+      if (ctl.pend[j].c_first == sp.c_first) ctl.pend_last[j] = 1;
+  }
 }
 
 // two 8-bit codes (bytes 0-1, or 2-3, of r) widened exactly to an fp16 pair:
@@ -317,7 +363,14 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     }
     mbar_init(smem_u32(&ctl.cons), kConsumerThreads);
     for (int i = 0; i < kQBufs; ++i) mbar_init(smem_u32(&ctl.qfull[i]), 1);
+    for (int s = 0; s < kSt; ++s) ctl.last_it[s] = -1;
+    for (int k = 0; k < kMaxPending; ++k) {
+      ctl.pend_last[k] = 0;
+      ctl.split[k].c_first = 0;
+      ctl.split[k].ncover = 0;
+    }
     ctl.abort = 0;
+    ctl.counted = 0;
     ctl.b0 = -1;
     ctl.npend = 0;
     fence_barrier_init();
@@ -359,9 +412,13 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     const long long excl = incl - r.units;
     if (b < B && r.units > 0 && f0 < f1) {
       const long long s0 = (long long)Hkv * (carry + excl), s1 = (long long)Hkv * (carry + incl);
+      // the pair holding this share's last unit, if it is shared with others
+      if (s0 <= f1 - 1 && f1 - 1 < s1)
+        ctl.split[1] = split_pair_at(W, N, c, Hkv, carry + excl, r, f1 - 1 - s0);
       if (s0 <= f0 && f0 < s1) {
         ctl.b0 = b;
         ctl.Cb0 = carry + excl;
+        ctl.split[0] = split_pair_at(W, N, c, Hkv, carry + excl, r, f0 - s0);
         // warm L2 with the first page ids and query rows this partition needs,
         // while the rest of the prologue runs
         const long long u = (f0 - s0) % r.units;
@@ -510,9 +567,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
             const uint32_t it = i + (uint32_t)(lane - jb);
             const int s = (int)(it % kSt);
             okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kSt) & 1u) ^ 1u,
-                                    &ctl.abort, a.err);
+                                    &ctl.abort, a.err, a.wait_ns);
             if (okl) {
               const uint32_t full = smem_u32(&ctl.full[s]);
+              ctl.last_it[s] = (int)it;
               if (page >= 0 && valid > 0) {
                 ctl.meta[s] = valid | flags;
                 mbar_arrive_expect_tx(full, kSlotB);
@@ -553,8 +611,9 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         const uint32_t it = i + lane;
         const int s = (int)(it % kSt);
         okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kSt) & 1u) ^ 1u, &ctl.abort,
-                                a.err);
+                                a.err, a.wait_ns);
         if (okl) {
+          ctl.last_it[s] = (int)it;
           ctl.meta[s] = kMetaEnd;
           mbar_arrive(smem_u32(&ctl.full[s]));
         }
@@ -562,13 +621,17 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       ok = __all_sync(0xffffffffu, okl) != 0;
       i += kConsumerWarps;
     }
-    if (!ok && lane == 0) {
-      // aborted: let the copies already issued land before the CTA exits
-      const uint32_t first = i > (uint32_t)kSt ? i - kSt : 0;
-      for (uint32_t k = first; k < i; ++k) {
-        const uint32_t bar = smem_u32(&ctl.full[k % kSt]);
+    __syncwarp();
+    if (lane == 0) {
+      // Never leave with copies in flight, whoever gave up (the consumers may
+      // have stopped waiting while this warp finished cleanly): wait for the
+      // last hand-over of every slot to land, and for every staged query block.
+      for (int s = 0; s < kSt; ++s) {
+        const int it = ctl.last_it[s];
+        if (it < 0) continue;
+        const uint32_t bar = smem_u32(&ctl.full[s]);
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bar, (k / kSt) & 1u) &&
+        while (!mbar_try_wait(bar, ((uint32_t)it / kSt) & 1u) &&
                global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
@@ -617,7 +680,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 
   for (uint32_t i = warp;; i += kConsumerWarps) {
     const int s = (int)(i % kSt);
-    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kSt) & 1u, &ctl.abort, a.err)) {
+    if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kSt) & 1u, &ctl.abort, a.err, a.wait_ns)) {
       clean = false;
       break;
     }
@@ -638,7 +701,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       // the segment's query rows, staged by the producer
       const int qb = sid & (kQBufs - 1);
       if (!mbar_wait_bounded(smem_u32(&ctl.qfull[qb]), (uint32_t)(sid / kQBufs) & 1u, &ctl.abort,
-                             a.err)) {
+                             a.err, a.wait_ns)) {
         clean = false;
         break;
       }
@@ -889,7 +952,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       const bool direct = rec.ncover == 1;
 #pragma unroll
       for (int nt = 0; nt < NQ; ++nt) {
-        if (!cons_sync(ctl, cons_phase, a.err)) {  // previous merge done with scratch
+        if (!cons_sync(ctl, cons_phase, a.err, a.wait_ns)) {  // previous merge done with scratch
           clean = false;
           break;
         }
@@ -915,7 +978,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           scr.o[warp][2 * cq][d1] = o[nt][mt][2];
           scr.o[warp][2 * cq + 1][d1] = o[nt][mt][3];
         }
-        if (!cons_sync(ctl, cons_phase, a.err)) {
+        if (!cons_sync(ctl, cons_phase, a.err, a.wait_ns)) {
           clean = false;
           break;
         }
@@ -950,20 +1013,21 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       if (!direct && ct == 0 && ctl.npend < kMaxPending) ctl.pend[ctl.npend++] = rec;
     }
   }
-  if (!clean || ctl.abort) return;
-
   // ============ end of the partition: split pairs, last arrival merges ============
-  __threadfence();  // this CTA's partial states are visible before it counts itself in
-  if (!cons_sync(ctl, cons_phase, a.err)) return;
+  // On the clean path thread 0 counts the CTA in after every consumer has
+  // written its partial states; on a failed path (a wait ran out, a bad
+  // record) the first thread out counts it in and nothing is merged -- the
+  // launch's outputs are invalid then (PKV_DEVERR_TIMEOUT or _INDPTR), but
+  // the workspace stays reusable.
+  bool synced = clean && !ctl.abort;
+  if (synced) {
+    __threadfence();  // this CTA's partial states are visible before it counts itself in
+    synced = cons_sync(ctl, cons_phase, a.err, a.wait_ns);
+  }
+  if ((!synced || ct == 0) && atomicCAS(&ctl.counted, 0, 1) == 0) count_in(a, ctl, synced);
+  if (!synced) return;
   const int npend = ctl.npend;
-  if (ct == 0)
-    for (int k = 0; k < npend; ++k) {
-      const int old = atomicAdd(&a.counters[ctl.pend[k].c_first], 1);
-      ctl.pend_last[k] = (old == ctl.pend[k].ncover - 1);
-      // the last arrival is the pair's only remaining user of the counter
-      if (ctl.pend_last[k]) a.counters[ctl.pend[k].c_first] = 0;
-    }
-  if (!cons_sync(ctl, cons_phase, a.err)) return;
+  if (!cons_sync(ctl, cons_phase, a.err, a.wait_ns)) return;
   __threadfence();
   // one warp per (pair, column); lane L owns dims 4L .. 4L+3
   const int P = a.pcols;  // state columns per slot
@@ -1038,16 +1102,8 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
   const int variant = (chunk ? 4 + 2 * nq : 2 * kv) + (bf16 ? 1 : 0);
   const Kern kern = kKerns[variant];
   const size_t smem = smem_bytes(nq);
-  // the shared-memory opt-in is per function and device; do it once each
-  static bool attr_set[10][64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = ensure_smem_opt_in(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !attr_set[variant][dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set[variant][dev] = true;
-  }
   // programmatic dependent launch: CTAs may become resident while the previous
   // kernel drains; the kernel waits for it before reading any input
   cudaLaunchConfig_t cfg = {};

@@ -47,7 +47,22 @@ struct DecodeArgs {
   const void* v_new;
   const int32_t* append_indptr;
   long long nnz_new;
+  // time limit of every pipeline wait (ns); the drain of a CTA's own copies
+  // before it exits always uses the full kWaitLimitNs
+  unsigned long long wait_ns;
 };
+
+// wait limit of the decode kernel's pipeline waits (pkv_set_wait_limit_ns)
+unsigned long long decode_wait_limit_ns();
+
+// Bytes at the start of pkv_decode's workspace that hold its arrival
+// counters (the only part that must be zero before a launch), for the GQA
+// group and partition count given (0 = the current device's default).
+size_t decode_counter_bytes(int group, int num_partitions);
+
+// Raise `func`'s dynamic shared-memory limit to `bytes` on the current device,
+// once per (function, device); safe to call from several host threads.
+cudaError_t ensure_smem_opt_in(const void* func, size_t bytes);
 
 constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp
 #ifndef PKV_STAGES

@@ -75,9 +75,14 @@ pkv_status pkv_decode_static_workspace(const void* q, int num_qo_heads, const vo
   cudaError_t e = scratch_address(&scratch);
   if (e != cudaSuccess)
     return pkv::set_error(PKV_ERR_CUDA, "locating the static scratch: %s", cudaGetErrorString(e));
-  // The scratch keeps whatever the previous call left; the arrival counters
-  // it holds must start at zero, so clear the part this call uses.
-  e = cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream));
+  // The scratch keeps whatever the previous call left.  Only its arrival
+  // counters must start at zero (every partial state is written before it is
+  // read), so clear the counters of this call's partition count.
+  const size_t counters =
+      pkv::decode_counter_bytes(num_qo_heads / num_kv_heads, num_partitions);
+  if (counters == 0 || counters > need)
+    return pkv::set_error(PKV_ERR_CUDA, "cannot size the static scratch's counters");
+  e = cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess)
     return pkv::set_error(PKV_ERR_CUDA, "clearing the static scratch: %s", cudaGetErrorString(e));
   return pkv_decode(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,

@@ -30,6 +30,18 @@ def test_library_exports_every_declared_symbol():
             "paged_kv_append", "paged_decode_attention", "merge_states"} <= set(names)
 
 
+def test_wait_limit_setting_round_trips():
+    """pkv_set_wait_limit_ns returns the previous limit; 0 selects the
+    default of one second (host-only state, no launch)."""
+    prev = pkv.set_wait_limit_ns(0)
+    try:
+        assert pkv.set_wait_limit_ns(5000) == 1_000_000_000
+        assert pkv.set_wait_limit_ns(0) == 5000
+        assert pkv.set_wait_limit_ns(0) == 1_000_000_000
+    finally:
+        pkv.set_wait_limit_ns(prev)
+
+
 def test_status_strings():
     L = pkv.lib()
     assert L.pkv_status_string(0) == b"PKV_OK"
@@ -389,3 +401,57 @@ def test_fused_append_writes_every_new_row_once(N):
     expect = [(b, g, p) for b in range(w.batch) for g in range(4)
               for p in range(int(w.kv_lens[b]) - counts[b], int(w.kv_lens[b]))]
     assert sorted(written) == sorted(expect)
+
+
+def _shared_pairs_by_first_and_last_unit(lens, ps, hkv, N, seg_cost=16):
+    """For every partition, the (request, kv head) pairs holding its first and
+    its last flat unit, kept when the partition holds a tile of the pair and
+    the pair's tiles span several partitions -- written from the partition's
+    definition (fixed cost first, then the pair's 16-token tiles)."""
+    units = [(-(-L // 16) + seg_cost) if L > 0 else 0 for L in lens]
+    W = hkv * sum(units)
+    Np = min(N, W)
+    part_of = lambda f: ((f + 1) * Np - 1) // W
+    starts = np.concatenate([[0], np.cumsum(units)])
+
+    def pair_at(f):
+        b = int(np.searchsorted(starts, f // hkv, side="right")) - 1
+        while units[b] == 0 or not (hkv * starts[b] <= f < hkv * (starts[b] + units[b])):
+            b += 1 if f >= hkv * (starts[b] + units[b]) else -1
+        kvh = (f - hkv * starts[b]) // units[b]
+        ps0 = hkv * starts[b] + kvh * units[b]
+        return b, kvh, part_of(ps0 + seg_cost), part_of(ps0 + units[b] - 1)
+
+    out = {}
+    for c in range(Np):
+        f0, f1 = W * c // Np, W * (c + 1) // Np
+        got = set()
+        for f in (f0, f1 - 1):
+            b, kvh, c_first, c_last = pair_at(f)
+            if c_last > c_first and c_first <= c <= c_last:
+                got.add((b, kvh))
+        out[c] = got
+    return out
+
+
+@pytest.mark.parametrize("lens,ps,hkv,N", [
+    ([3000, 500, 17, 8000, 1, 2049], 16, 8, 148),
+    ([3000, 500, 17, 8000, 1, 2049], 16, 8, 7),
+    ([1, 2, 3, 0, 4, 5], 16, 2, 300),
+    ([200000], 256, 8, 148),
+    ([131072] * 8, 16, 8, 148),
+    ([100, 4096, 0, 33, 77, 5000, 1, 16], 32, 4, 37),
+])
+def test_shared_pairs_are_those_of_the_first_and_last_unit(lens, ps, hkv, N):
+    """The decode kernel counts each partition in on the pairs holding its
+    first and last unit (also when it gives up part-way); that must be exactly
+    the set of split pairs whose partial states the partition writes, as the
+    host mirror of the partition lists them."""
+    w = wl.make_workload("pairs", lens, num_qo_heads=hkv, num_kv_heads=hkv, page_size=ps,
+                         dtype="bf16", seed=3)
+    seg = pkv.plan_segments(w.page_indptr, w.last_page_len, ps, hkv, N)
+    expect = _shared_pairs_by_first_and_last_unit(list(w.kv_lens), ps, hkv, N)
+    for c, pairs in expect.items():
+        rows = seg[(seg[:, 0] == c) & (seg[:, 6] > 1)]
+        assert {(int(r[1]), int(r[2])) for r in rows} == pairs, f"partition {c}"
+        assert len(pairs) <= 2
