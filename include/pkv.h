@@ -408,7 +408,7 @@ PKV_API pkv_status pkv_append_attention_short(const void* q, const int32_t* qo_i
  * Request b attends over the prefix's prefix_len tokens followed by its own
  * tokens; the result equals pkv_decode on the concatenated page lists up to
  * fp32 rounding.  Instead of reading the prefix once per request, the prefix's
- * K/V are read once per block of 128 (request, query head) rows and multiplied
+ * K/V are read once per block of 256 (request, query head) rows and multiplied
  * on tensor cores against all requests' queries; each request's own pages go
  * through the decode kernel; the two attention states are merged by their
  * log-sum-exp weights.

@@ -547,7 +547,8 @@ int64_t pkv_plan_segments(const int32_t* page_indptr_h, const int32_t* last_page
     while (!wk.done()) {
       const long long t0 = wk.t0(), t1 = wk.t1();
       if (t1 > t0) {
-        const pkv::SegPlace pl = pkv::seg_place(W, N, wk.pair_start(), wk.ri.units, c);
+        // the kernel's form (no division for pair ends inside the share)
+        const pkv::SegPlace pl = pkv::seg_place_in(W, N, wk.pair_start(), wk.ri.units, c, f0, f1);
         if (segments && count < max_segments) {
           int64_t* row = segments + 7 * count;
           row[0] = c;

@@ -461,6 +461,11 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     uint32_t i = 0;  // tiles handed to the ring so far
     int seg = 0;
     bool ok = true;
+    // page ids of the previous segment's first 32 tiles: the kv heads of one
+    // request share its pages, so the next head's segment over the same
+    // tiles reuses them instead of loading them again
+    long long ids_base = -1, ids_t0 = -1, ids_n = 0;
+    int ids_first = -1;
     while (ok && !wk.done()) {
       if (wk.seg_units() <= 0) {  // only possible if the table changed under the kernel
         if (lane == 0) {
@@ -479,7 +484,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       const long long n_pad = (n + kConsumerWarps - 1) / kConsumerWarps * kConsumerWarps;
       const long long pstart = wk.pair_start();
       if (lane == 0) {
-        const SegPlace pl = seg_place(W, N, pstart, wk.ri.units, c);
+        const SegPlace pl = seg_place_in(W, N, pstart, wk.ri.units, c, f0, f1);
         SegRec& r = ctl.seg[seg & (kSegRecs - 1)];
         r.b = wk.b;
         r.kvh = wk.kvh;
@@ -527,7 +532,15 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       // page ids, one tile per lane, loaded one 32-tile batch ahead of their use
       const int* idx = a.indices + wk.ri.page_base;
       int page_next = -1;
-      if (lane < n) page_next = idx[((t0 + lane) * kTileTokens) >> ps_shift];
+      if (wk.ri.page_base == ids_base && t0 == ids_t0 && (n < 32 ? n : 32) <= ids_n) {
+        page_next = lane < n ? ids_first : -1;
+      } else if (lane < n) {
+        page_next = idx[((t0 + lane) * kTileTokens) >> ps_shift];
+      }
+      ids_base = wk.ri.page_base;
+      ids_t0 = t0;
+      ids_n = n < 32 ? n : 32;
+      ids_first = page_next;
       for (long long k0 = 0; ok && k0 < n_pad; k0 += 32) {
         int page = page_next;
         if (k0 + 32 + lane < n)

@@ -138,6 +138,21 @@ PKV_HD SegPlace seg_place(int64_t W, int N, int64_t pair_start, int64_t pair_uni
   return p;
 }
 
+// seg_place for partition c whose share is [f0, f1) (f0 = part_start(c),
+// f1 = part_start(c + 1)) and which holds at least one tile of the pair: a
+// pair end inside the share belongs to c, so the divisions of part_of are only
+// needed for an end outside it (the share's first and last pair).
+PKV_HD SegPlace seg_place_in(int64_t W, int N, int64_t pair_start, int64_t pair_units, int c,
+                             int64_t f0, int64_t f1) {
+  SegPlace p;
+  const int64_t first = pair_start + kSegmentCost, last = pair_start + pair_units - 1;
+  p.c_first = first >= f0 ? c : part_of(W, N, first);
+  const int c_last = last < f1 ? c : part_of(W, N, last);
+  p.ncover = c_last - p.c_first + 1;
+  p.slot = p.ncover == 1 ? -1 : state_slot(p.c_first, c - p.c_first);
+  return p;
+}
+
 // Sequential walk over the segments of one partition.  Table pointers may be
 // host or device memory (whichever side runs the walk).  A segment whose
 // share of the pair holds only fixed-cost units has no tiles (t0 == t1).

@@ -88,6 +88,25 @@ def test_cascade_matches_oracle_small(case):
     assert_parity(out, lse, ref_o, ref_l, what=str(case))
 
 
+@pytest.mark.parametrize("N", [1, 3])
+def test_cascade_requests_without_own_tokens(N):
+    """Requests that hold only the prefix get the prefix's attention alone; with
+    one or three partitions a CTA finalises more of them than it lists, so both
+    the warps' path and the per-thread path run."""
+    batch = 45
+    own = np.zeros(batch, np.int64)
+    own[[3, 20, 44]] = [17, 300, 1]
+    full = 6 * 16
+    w = wl.make_workload("cascade-empty", full + own, num_qo_heads=32, num_kv_heads=8,
+                         page_size=16, dtype="bf16", seed=61, shared_prefix_len=full,
+                         pool_factor=1.2)
+    prefix, _, ip, ix, ll = wl.cascade_view(w)
+    q, pool, _, _ = wl.make_tensors(w, "cpu")
+    out, lse = run_cascade(w, q.cuda(), pool.cuda(), prefix, full, ip, ix, ll, num_partitions=N)
+    ref_o, ref_l = repacked_oracle(w, wl.bits(q), wl.bits(pool), prefix, full, ip, ix, ll)
+    assert_parity(out, lse, ref_o, ref_l, what=f"empty own, N={N}")
+
+
 def test_cascade_equals_decode_on_shared_prefix_workload():
     w = wl.named(5)
     q, pool, _, _ = wl.make_tensors(w, "cuda")
