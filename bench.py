@@ -64,6 +64,9 @@ def parse():
                    help="--chunk spec: append the chunk's K/V inside the short-chunk launch "
                         "(slower than a separate append at 4 rows per request)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-early-table", action="store_true",
+                   help="do not mark the page table ready at launch (the decode then waits for "
+                        "the previous kernel before it reads the table)")
     p.add_argument("--no-per-config", action="store_true",
                    help="headline workload only (by default the 128K headline line also "
                         "carries per_config numbers of workloads 1, 2, 4, 5 and the 5 cascade)")
@@ -439,7 +442,10 @@ def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=Fa
     # it cannot (8-bit pool, cascade) or --separate-append asks otherwise
     fused = bool(w.nnz_new) and not fp8 and not cascade and not args.separate_append
     launches_per_step = (3 if cascade else 1) + (1 if w.nnz_new and not fused else 0)
-    table = pkv.csr_table(indptr, indices, last)
+    # nothing in a step writes the page table, so the decode may read it while
+    # the previous step's kernel drains (PKV_TABLE_READY_AT_LAUNCH)
+    early = not getattr(args, "no_early_table", False)
+    table = pkv.csr_table(indptr, indices, last, ready_at_launch=early)
 
     def append_call(bt):
         if fused:
@@ -468,9 +474,9 @@ def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=Fa
                                     lse=lse, sm_scale=w.sm_scale, num_partitions=N,
                                     error_word=err, stream=cur)
         else:
-            pkv.paged_decode_attention(bt.q, bt.pool, indptr, indices, last, ws, out=out, lse=lse,
-                                       sm_scale=w.sm_scale, num_partitions=N, error_word=err,
-                                       stream=cur)
+            pkv.paged_decode_attention_ex(bt.q, bt.pool, table, ws, out=out, lse=lse,
+                                          sm_scale=w.sm_scale, num_partitions=N, error_word=err,
+                                          stream=cur)
 
     for i in range(args.warmup):
         append_call(batches[i % rotation])
@@ -526,7 +532,8 @@ def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=Fa
     dec_bytes = wl.decode_bytes(w, kvb) + (wl.append_bytes(w) if fused else 0)
     res = {"ms": ms, "K": K, "decode_ms": decode_ms, "step_bytes": step_bytes,
            "dec_bytes": dec_bytes, "fused": fused, "launches_per_step": launches_per_step,
-           "rotation": rotation, "N": N, "t_host0": t_host0, "t_host1": t_host1, "e2e": None}
+           "rotation": rotation, "N": N, "t_host0": t_host0, "t_host1": t_host1, "e2e": None,
+           "early_table": early}
 
     # ---- end to end through the public API with host buffers: every step copies
     # its inputs (q, new K/V rows, the page table) from pinned host memory in one
@@ -541,7 +548,7 @@ def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=Fa
         h_out, d_out = pack([out.cpu(), lse.cpu()], dev)
         out_d, lse_d = d_out
         h2d, d2h = h_in[0].numel(), h_out[0].numel()
-        e2e_table = pkv.csr_table(ip_d, ix_d, ll_d)
+        e2e_table = pkv.csr_table(ip_d, ix_d, ll_d, ready_at_launch=early)
 
         def e2e_calls(_):
             cur = torch.cuda.current_stream(dev)
@@ -568,9 +575,9 @@ def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=Fa
                                        out=out_d, lse=lse_d, sm_scale=w.sm_scale,
                                        num_partitions=N, error_word=err, stream=cur)
                 else:
-                    pkv.paged_decode_attention(q_d, src.pool, ip_d, ix_d, ll_d, ws, out=out_d,
-                                               lse=lse_d, sm_scale=w.sm_scale, num_partitions=N,
-                                               error_word=err, stream=cur)
+                    pkv.paged_decode_attention_ex(q_d, src.pool, e2e_table, ws, out=out_d,
+                                                  lse=lse_d, sm_scale=w.sm_scale,
+                                                  num_partitions=N, error_word=err, stream=cur)
             h_out[0].copy_(h_out[1], non_blocking=True)
 
         e2e_calls(None)
@@ -693,7 +700,10 @@ def run_pkv(args):
                                   ("the fused append + decode launch (pkv_decode_append)" if fused
                                    else ("the cascade's launches" if args.cascade else
                                          ("append and decode each" if w.nnz_new else "decode"))) +
-                                  " captured once per batch copy as a CUDA graph, replayed")},
+                                  " captured once per batch copy as a CUDA graph, replayed") +
+                                 ("; page table marked ready at launch (read while the previous "
+                                  "step's kernel drains)" if r["early_table"] and not args.cascade
+                                  else "")},
             "us_per_step": round(ms / K * 1e3, 2),
             "tokens_per_s": round(w.batch * world / (ms / 1e3 / K), 1),
             "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),

@@ -116,8 +116,20 @@ typedef struct pkv_table_desc {
   const int32_t* block_table;
   const int32_t* context_lens;
   int32_t max_blocks_per_seq;
-  int32_t reserved;
+  int32_t flags;  /* PKV_TABLE_* bits, 0 for none */
 } pkv_table_desc;
+
+/*
+ * PKV_TABLE_READY_AT_LAUNCH: the caller promises that the page table (indptr /
+ * indices / last_page_len, or block_table / context_lens) is not written by
+ * the kernel that runs just before this call in the stream.  The decode then
+ * reads the table and plans its split-KV partition while that kernel is still
+ * finishing (programmatic dependent launch), and waits for it only before it
+ * reads q, the pool or new rows and before it writes anything.  Host-to-device
+ * copies of the table before the call are fine: a copy is not a kernel and
+ * the decode starts after it.  Without the flag the decode waits first.
+ */
+#define PKV_TABLE_READY_AT_LAUNCH 0x1
 
 /* Bits the kernels OR into *error_word. */
 #define PKV_DEVERR_PAGE_ID   0x01  /* page id outside [0, num_pages): page skipped */

@@ -17,6 +17,7 @@ DEVERR_TIMEOUT = 0x10
 DEVERR_CONTEXT_LEN = 0x20
 LAYOUT_HND, LAYOUT_NHD = 0, 1
 TABLE_CSR, TABLE_BLOCK = 0, 1
+TABLE_READY_AT_LAUNCH = 0x1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpkv.so")
@@ -61,7 +62,7 @@ class TableDesc(ctypes.Structure):
                 ("page_indptr", ctypes.c_void_p), ("page_indices", ctypes.c_void_p),
                 ("last_page_len", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
                 ("context_lens", ctypes.c_void_p), ("max_blocks_per_seq", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("flags", ctypes.c_int32)]
 
 
 _PP = ctypes.POINTER(PoolDesc)
@@ -290,24 +291,30 @@ def pool_desc(pool, layout: str = "HND") -> PoolDesc:
                     LAYOUT_HND if layout == "HND" else LAYOUT_NHD, 0)
 
 
-def csr_table(page_indptr, page_indices, last_page_len) -> TableDesc:
+def csr_table(page_indptr, page_indices, last_page_len, ready_at_launch: bool = False) -> TableDesc:
+    """CSR page table.  ready_at_launch: no kernel right before the call in the
+    stream writes the table (PKV_TABLE_READY_AT_LAUNCH), so the decode may read
+    it while that kernel finishes."""
     for name, t in (("page_indptr", page_indptr), ("page_indices", page_indices),
                     ("last_page_len", last_page_len)):
         _dev_tensor(t, name, torch.int32)
     t = TableDesc(TABLE_CSR, last_page_len.numel(), page_indptr.data_ptr(),
-                  page_indices.data_ptr(), last_page_len.data_ptr(), None, None, 0, 0)
+                  page_indices.data_ptr(), last_page_len.data_ptr(), None, None, 0,
+                  TABLE_READY_AT_LAUNCH if ready_at_launch else 0)
     t._keep = (page_indptr, page_indices, last_page_len)  # the descriptor holds raw pointers
     return t
 
 
-def block_table(table, context_lens) -> TableDesc:
-    """Dense [batch, max_blocks_per_seq] block table + context lengths (tokens)."""
+def block_table(table, context_lens, ready_at_launch: bool = False) -> TableDesc:
+    """Dense [batch, max_blocks_per_seq] block table + context lengths (tokens);
+    ready_at_launch as for csr_table."""
     _dev_tensor(table, "block_table", torch.int32)
     _dev_tensor(context_lens, "context_lens", torch.int32)
     if table.dim() != 2 or table.shape[0] != context_lens.numel():
         raise ValueError("block_table must be [batch, max_blocks_per_seq]")
     t = TableDesc(TABLE_BLOCK, table.shape[0], None, None, None, table.data_ptr(),
-                  context_lens.data_ptr(), table.shape[1], 0)
+                  context_lens.data_ptr(), table.shape[1],
+                  TABLE_READY_AT_LAUNCH if ready_at_launch else 0)
     t._keep = (table, context_lens)
     return t
 

@@ -258,7 +258,8 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
                       float k_scale = 1.f, float v_scale = 1.f,
                       const int32_t* qo_indptr = nullptr, int64_t nnz_q = 0, int max_q_len = 1,
                       const void* k_new = nullptr, const void* v_new = nullptr,
-                      const int32_t* append_indptr = nullptr, int64_t nnz_new = 0) {
+                      const int32_t* append_indptr = nullptr, int64_t nnz_new = 0,
+                      int early_table = 0) {
   if (kv_dtype < 0) kv_dtype = dtype;
   if (batch < 0 || num_pages < 1 || num_kv_heads < 1 || num_qo_heads < 1)
     return fail(PKV_ERR_INVALID_ARG, "sizes out of range");
@@ -355,6 +356,7 @@ static pkv_status decode_impl(const void* q, int num_qo_heads, const void* pool,
   a.append_indptr = fused ? append_indptr : nullptr;
   a.nnz_new = fused ? nnz_new : 0;
   a.wait_ns = pkv::decode_wait_limit_ns();
+  a.early_table = early_table;
   cudaError_t e =
       pkv::launch_decode(tmap, a, dtype == PKV_BF16,
                          kv_dtype == PKV_FP8_E4M3 ? pkv::kKvE4M3
@@ -421,6 +423,8 @@ static pkv_status append_impl(void* pool, int64_t num_pages, int page_size, int 
 // unpack the descriptors of the _ex calls
 static pkv_status table_view(const pkv_table_desc* t, pkv::TableView* tv, const int32_t** ids) {
   if (!t) return fail(PKV_ERR_INVALID_ARG, "null table descriptor");
+  if (t->flags & ~PKV_TABLE_READY_AT_LAUNCH)
+    return fail(PKV_ERR_INVALID_ARG, "unknown table flags 0x%x", (unsigned)t->flags);
   if (t->kind == PKV_TABLE_CSR) {
     *tv = pkv::csr_view(t->page_indptr, t->last_page_len);
     *ids = t->page_indices;
@@ -610,7 +614,7 @@ pkv_status pkv_decode_append(const void* q, int num_qo_heads, const pkv_pool_des
                      table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
                      error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
                      num_qo_heads, -1, 1.f, 1.f, nullptr, 0, 1, k_new, v_new, append_indptr,
-                     nnz_new);
+                     nnz_new, table->flags & PKV_TABLE_READY_AT_LAUNCH);
 }
 
 pkv_status pkv_decode_ex(const void* q, int num_qo_heads, const pkv_pool_desc* pool,
@@ -628,7 +632,8 @@ pkv_status pkv_decode_ex(const void* q, int num_qo_heads, const pkv_pool_desc* p
                      pool->num_kv_heads, pool->head_dim, pool->dtype, pool->layout, tv, ids,
                      table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
                      error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
-                     num_qo_heads);
+                     num_qo_heads, -1, 1.f, 1.f, nullptr, 0, 1, nullptr, nullptr, nullptr, 0,
+                     table->flags & PKV_TABLE_READY_AT_LAUNCH);
 }
 
 pkv_status pkv_append_ex(const pkv_pool_desc* pool, const pkv_table_desc* table,
@@ -662,7 +667,8 @@ pkv_status pkv_decode_fp8(const void* q, int q_dtype, int num_qo_heads, const pk
                      pool->num_kv_heads, pool->head_dim, q_dtype, pool->layout, tv, ids,
                      table->batch, sm_scale, num_partitions, workspace, workspace_bytes, out, lse,
                      error_word, stream, 0, (long long)num_qo_heads * kDecodeHeadDim,
-                     num_qo_heads, pool->dtype, k_scale, v_scale);
+                     num_qo_heads, pool->dtype, k_scale, v_scale, nullptr, 0, 1, nullptr, nullptr,
+                     nullptr, 0, table->flags & PKV_TABLE_READY_AT_LAUNCH);
 }
 
 pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, float v_scale,

@@ -377,8 +377,13 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   }
   if (warp == kConsumerWarps && lane == 0) prefetch_tensormap(&tmap);
   // With programmatic dependent launch this CTA may start while the previous
-  // kernel in the stream still runs; everything above touched no input.
-  grid_dependency_wait();
+  // kernel in the stream still runs; everything above touched no input.  When
+  // the caller promises that kernel does not write the page table
+  // (early_table), the prologue and the producer's first page-id loads run
+  // before the wait; every thread waits before it reads q, the pool or new
+  // rows, and before it writes anything.
+  const bool early = a.early_table != 0;
+  if (!early) grid_dependency_wait();
   grid_dependents_launch();
 
   // ---- prologue: total work W, this partition's share [f0, f1), its first request
@@ -389,7 +394,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     mine += r.units;
     errs |= r.err;
   }
-  if (errs && c == 0 && a.err) atomicOr(a.err, errs);
+  if (errs && c == 0 && a.err) {
+    if (early) grid_dependency_wait();
+    atomicOr(a.err, errs);
+  }
   long long total_units;
   (void)block_incl_scan(mine, ctl.warp_tot, &total_units);
   const long long W = (long long)Hkv * total_units;
@@ -430,6 +438,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       }
     }
     if (b < B && r.tiles == 0 && (b % (int)gridDim.x) == c) {
+      if (early) grid_dependency_wait();
       if (!a.qo_indptr) {
         // a request with no tokens: attention over no keys -> o = 0, lse = -inf
         for (int h = 0; h < a.hq; ++h) {
@@ -483,6 +492,19 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       }
       const long long n_pad = (n + kConsumerWarps - 1) / kConsumerWarps * kConsumerWarps;
       const long long pstart = wk.pair_start();
+      // page ids, one tile per lane, loaded one 32-tile batch ahead of their use
+      const int* idx = a.indices + wk.ri.page_base;
+      int page_next = -1;
+      if (wk.ri.page_base == ids_base && t0 == ids_t0 && (n < 32 ? n : 32) <= ids_n) {
+        page_next = lane < n ? ids_first : -1;
+      } else if (lane < n) {
+        page_next = idx[((t0 + lane) * kTileTokens) >> ps_shift];
+      }
+      ids_base = wk.ri.page_base;
+      ids_t0 = t0;
+      ids_n = n < 32 ? n : 32;
+      ids_first = page_next;
+      if (early && seg == 0) grid_dependency_wait();  // before q, the pool or new rows
       if (lane == 0) {
         const SegPlace pl = seg_place_in(W, N, pstart, wk.ri.units, c, f0, f1);
         SegRec& r = ctl.seg[seg & (kSegRecs - 1)];
@@ -529,18 +551,6 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         }
       }
       __syncwarp();  // the record is written before any lane publishes a tile of it
-      // page ids, one tile per lane, loaded one 32-tile batch ahead of their use
-      const int* idx = a.indices + wk.ri.page_base;
-      int page_next = -1;
-      if (wk.ri.page_base == ids_base && t0 == ids_t0 && (n < 32 ? n : 32) <= ids_n) {
-        page_next = lane < n ? ids_first : -1;
-      } else if (lane < n) {
-        page_next = idx[((t0 + lane) * kTileTokens) >> ps_shift];
-      }
-      ids_base = wk.ri.page_base;
-      ids_t0 = t0;
-      ids_n = n < 32 ? n : 32;
-      ids_first = page_next;
       for (long long k0 = 0; ok && k0 < n_pad; k0 += 32) {
         int page = page_next;
         if (k0 + 32 + lane < n)
@@ -661,6 +671,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   }
 
   // =========================== consumers ===========================
+  if (early) grid_dependency_wait();  // before any output is written
   const int g = lane >> 2;     // MMA row group: token g / g+8 of the tile, column g of P^T
   const int cq = lane & 3;     // MMA column pair: columns 2cq, 2cq+1 of S^T (per n8 tile)
   const int mi = lane >> 3;    // ldmatrix: which 8x8 matrix this lane addresses

@@ -50,6 +50,9 @@ struct DecodeArgs {
   // time limit of every pipeline wait (ns); the drain of a CTA's own copies
   // before it exits always uses the full kWaitLimitNs
   unsigned long long wait_ns;
+  // 1: the table is not written by the preceding kernel in the stream, so it
+  // is read (and the partition planned) before waiting for that kernel
+  int early_table;
 };
 
 // wait limit of the decode kernel's pipeline waits (pkv_set_wait_limit_ns)

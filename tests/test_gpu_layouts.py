@@ -101,3 +101,49 @@ def test_block_table_context_len_beyond_row_sets_error():
     torch.cuda.synchronize()
     assert pkv.read_error_word(err) & pkv.DEVERR_CONTEXT_LEN
     assert torch.all(out[1] == 0)
+
+
+@pytest.mark.parametrize("kind", ["csr", "block"])
+def test_table_ready_at_launch(kind):
+    """PKV_TABLE_READY_AT_LAUNCH lets the decode read the table before the
+    preceding kernel finishes.  That kernel may still write q and the pool:
+    here each decode runs right after a kernel that rewrites q (and one that
+    rewrites a page), and must see the new values -- bitwise the result of
+    the same decode without the flag, and within the oracle's bounds."""
+    w = wl.make_workload("early", [3000, 17, 0, 900, 1, 4096], num_qo_heads=32, num_kv_heads=8,
+                         page_size=16, dtype="bf16", seed=82, pool_factor=1.3)
+    q, pool, _, _ = wl.make_tensors(w, "cpu")
+    q, pool = q.cuda(), pool.cuda()
+    t = lambda a: torch.as_tensor(np.ascontiguousarray(a, np.int32), device="cuda")
+    ip, ix, ll = t(w.page_indptr), t(w.page_indices), t(w.last_page_len)
+    if kind == "csr":
+        keep = (ip, ix, ll)
+        table_f = pkv.csr_table(ip, ix, ll, ready_at_launch=True)
+        table_0 = pkv.csr_table(ip, ix, ll)
+    else:
+        bt, ctx = dense_block_table(w)
+        keep = (t(bt), t(ctx))
+        table_f = pkv.block_table(*keep, ready_at_launch=True)
+        table_0 = pkv.block_table(*keep)
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    qs = [torch.randn(q.shape, generator=gen, device="cuda").to(q.dtype) for _ in range(4)]
+    page = int(w.pages_of(0)[3])
+    vals = [torch.randn(pool[page].shape, generator=gen, device="cuda").to(pool.dtype) for _ in range(4)]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ws_f, ws_0 = workspace(w), workspace(w)
+    outs = []
+    for i in range(4):
+        q.copy_(qs[i])            # a kernel right before the decode writes q ...
+        pool[page].copy_(vals[i])  # ... and a page the decode reads
+        outs.append(pkv.paged_decode_attention_ex(q, pool, table_f, ws_f, sm_scale=w.sm_scale,
+                                                  error_word=err))
+    torch.cuda.synchronize()
+    assert pkv.read_error_word(err) == 0
+    for i in range(4):
+        q.copy_(qs[i])
+        pool[page].copy_(vals[i])
+        ref = pkv.paged_decode_attention_ex(q, pool, table_0, ws_0, sm_scale=w.sm_scale)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i][0], ref[0]) and torch.equal(outs[i][1], ref[1]), i
+    ro, rl = oracle_decode(w, wl.bits(q), wl.bits(pool))
+    assert_parity(outs[3][0], outs[3][1], ro, rl, what=f"ready at launch, {kind}")

@@ -42,6 +42,17 @@ def test_wait_limit_setting_round_trips():
         pkv.set_wait_limit_ns(prev)
 
 
+def test_unknown_table_flags_rejected():
+    L = pkv.lib()
+    p = ctypes.c_void_p(4096)
+    pool = pkv.PoolDesc(4096, 64, 16, 2, 128, pkv.BF16, 0, 0)
+    for flags, status in ((2, 1), (0x80000000, 1)):
+        table = pkv.TableDesc(0, 4, 4096, 4096, 4096, None, None, 0, flags)
+        assert L.pkv_decode_ex(p, 8, ctypes.byref(pool), ctypes.byref(table), 0.1, 8, p, 1 << 30,
+                               ctypes.c_void_p(8192), None, None, None) == status
+    assert b"table flags" in L.pkv_last_error()
+
+
 def test_status_strings():
     L = pkv.lib()
     assert L.pkv_status_string(0) == b"PKV_OK"
