@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace pkv {
@@ -34,7 +35,13 @@ __device__ __forceinline__ void store_val(const MergeArgs& a, size_t i, float v)
   }
 }
 
+constexpr int kBatch = 8;  // states whose values are loaded together (head_dim 128)
+
 __global__ void __launch_bounds__(kWarps * 32) merge_kernel(const MergeArgs a) {
+  // programmatic dependent launch: the CTAs may be resident before the kernel
+  // that writes the states has finished; wait for it before reading them
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int lane = threadIdx.x & 31;
   const long long gw = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (gw >= a.rows * a.heads) return;
@@ -55,6 +62,39 @@ __global__ void __launch_bounds__(kWarps * 32) merge_kernel(const MergeArgs a) {
     return;
   }
   const bool vec = a.vec4 != 0;
+  if (vec) {
+    // head_dim 128: each lane owns dims 4L .. 4L+3; the values of kBatch states
+    // are loaded together, one round trip per batch, then weighted in state order
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    for (int j0 = 0; j0 < S; j0 += kBatch) {
+      float sj[kBatch];
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        sj[u] = j0 + u < S ? s_row[(size_t)(j0 + u) * H] : -INFINITY;
+        v[u] = j0 + u < S ? *reinterpret_cast<const float4*>(v_row + (size_t)(j0 + u) * H * D + 4 * lane)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (sj[u] == -INFINITY) continue;  // (uniform) no keys: its values may be anything, even NaN
+        const float wk = expf(sj[u] - M);
+        wsum += wk;
+        acc.x += wk * v[u].x;
+        acc.y += wk * v[u].y;
+        acc.z += wk * v[u].z;
+        acc.w += wk * v[u].w;
+      }
+    }
+    const float inv = 1.f / wsum;
+    store_val(a, orow + 4 * lane + 0, acc.x * inv);
+    store_val(a, orow + 4 * lane + 1, acc.y * inv);
+    store_val(a, orow + 4 * lane + 2, acc.z * inv);
+    store_val(a, orow + 4 * lane + 3, acc.w * inv);
+    if (lane == 0 && a.s_out) a.s_out[(size_t)r * H + h] = M + logf(wsum);
+    return;
+  }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);  // vec: dims 4L..4L+3
   float accs[4] = {0.f, 0.f, 0.f, 0.f};          // otherwise: dims L, L+32, L+64, L+96
   float wsum = 0.f;
@@ -109,7 +149,18 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream) {
   const long long warps = a.rows * a.heads;
   if (warps == 0) return cudaSuccess;
   const long long blocks = (warps + kWarps - 1) / kWarps;
-  merge_kernel<<<(unsigned)blocks, kWarps * 32, 0, stream>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, merge_kernel, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
