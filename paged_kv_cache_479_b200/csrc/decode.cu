@@ -63,6 +63,10 @@ constexpr int kD = 128;
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kStages = kDecodeStages;
+// GQA groups of at most 4 need half the query-block and merge-scratch room, which
+// buys a 24-slot ring (192 KiB in flight instead of 128 KiB); wider groups and
+// short chunks keep kStages slots
+constexpr int kStagesNarrow = kStages + kStages / 2;
 constexpr int kIssueLanes = kStages < 16 ? kStages : 16;  // producer lanes issuing at once
 // Consumer warp w takes ring positions w, w+8, w+16, ...  With the slot count
 // a multiple of the warp count, every slot has ONE consumer warp, so a warp
@@ -76,12 +80,12 @@ constexpr int kTileBytes = 2 * kHalfBytes;        // K or V of one 16-bit tile: 
 constexpr int kSlotBytes = 2 * kTileBytes;        // K + V: 8 KiB
 // An 8-bit (E4M3) tile is half the bytes; its ring has twice the slots, so the
 // same bytes are in flight.
-constexpr int kMaxStages = 2 * kStages;
+constexpr int kMaxStages = 2 * kStagesNarrow;
 constexpr int kSegRecs = 16;                      // segment records in flight
 constexpr int kMaxGroup = 8;                      // columns of one n8 MMA tile
 constexpr int kQBufs = 8;                         // staged query blocks in flight
-// a staged query block: the pair's columns (up to 8 NQ rows of 128 dims)
-__host__ __device__ constexpr int q_buf_bytes(int nq) { return nq * kMaxGroup * 128 * 2; }
+// a staged query block: the pair's columns (up to gc NQ rows of 128 dims)
+__host__ __device__ constexpr int q_buf_bytes(int nq, int gc) { return nq * gc * 128 * 2; }
 // The producer refills query buffer (and record) seg % n for segment seg + n
 // only after issuing every tile of segments seg .. seg+n-1 (each a multiple of
 // 8 tiles, at least 8).  With S ring slots that means the tiles up to
@@ -137,17 +141,23 @@ struct __align__(16) Ctl {
   int counted;                // 1 once this CTA has counted itself in on its split pairs
 };
 
+// the 8 consumer warps' states of up to GC columns, merged at a segment end
+template <int GC>
 struct Scratch {
-  float m[kConsumerWarps][kMaxGroup];
-  float l[kConsumerWarps][kMaxGroup];
-  float o[kConsumerWarps][kMaxGroup][kScratchStride];
+  float m[kConsumerWarps][GC];
+  float l[kConsumerWarps][GC];
+  float o[kConsumerWarps][GC][kScratchStride];
 };
 
-constexpr size_t kRingBytes = (size_t)kStages * kSlotBytes;
-constexpr size_t smem_bytes(int nq) {
-  return 1024 /*alignment slack*/ + kRingBytes + (size_t)kQBufs * q_buf_bytes(nq) + sizeof(Ctl) +
-         sizeof(Scratch);
+__host__ __device__ constexpr int ring_stages(int gc) { return gc <= 4 ? kStagesNarrow : kStages; }
+constexpr size_t smem_bytes(int nq, int gc) {
+  return 1024 /*alignment slack*/ + (size_t)ring_stages(gc) * kSlotBytes +
+         (size_t)kQBufs * q_buf_bytes(nq, gc) + sizeof(Ctl) +
+         (gc <= 4 ? sizeof(Scratch<4>) : sizeof(Scratch<kMaxGroup>));
 }
+static_assert(smem_bytes(1, 4) <= 227 * 1024 && smem_bytes(1, kMaxGroup) <= 227 * 1024 &&
+                  smem_bytes(2, kMaxGroup) <= 227 * 1024,
+              "shared memory per CTA");
 
 // output of (request b, query head h): 16-bit final outputs, or fp32 attention
 // states at a caller-chosen request stride (used when the result is merged later)
@@ -322,17 +332,20 @@ __device__ __forceinline__ void write_new_rows(const DecodeArgs& a, const ReqInf
 // KV: the pool's element type -- kKv16 (q's own 16-bit type), kKvE4M3, kKvE5M2;
 // NQ: n8 column tiles per pair (2 only for short chunks over 16-bit pools);
 // CHUNK: short chunks (causal limits per column), else decode (one token per request)
-template <bool BF16, int KV, int NQ, bool CHUNK>
+// GC: the GQA groups the variant takes, 8 (any) or 4 (a deeper ring)
+template <bool BF16, int KV, int NQ, bool CHUNK, int GC>
 __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   constexpr bool FP8 = KV != kKv16;
   static_assert(NQ == 1 || (NQ == 2 && !FP8), "two column tiles only for 16-bit pools");
   static_assert(!CHUNK || !FP8, "short chunks only for 16-bit pools");
   static_assert(CHUNK || NQ == 1, "the decode has one column tile");
-  constexpr int kCols = NQ * kMaxGroup;
-  constexpr int kQBufBytes = q_buf_bytes(NQ);
+  static_assert(GC == kMaxGroup || (GC == 4 && NQ == 1 && !CHUNK), "narrow groups: decode only");
+  constexpr int kCols = NQ * GC;  // columns with a query row at most
+  constexpr int kQBufBytes = q_buf_bytes(NQ, GC);
+  constexpr int kRingBytes = ring_stages(GC) * kSlotBytes;
   // ring geometry of this KV type (16-bit: 16 slots of 8 KiB; 8-bit: 32 of 4 KiB)
-  constexpr int kSt = FP8 ? 2 * kStages : kStages;
+  constexpr int kSt = FP8 ? 2 * ring_stages(GC) : ring_stages(GC);
   constexpr int kTileB = FP8 ? kTileBytes / 2 : kTileBytes;
   constexpr int kSlotB = 2 * kTileB;
   constexpr int kIssue = kSt < 16 ? kSt : 16;
@@ -347,7 +360,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   uint8_t* ring = smem;
   uint8_t* qbuf = smem + kRingBytes;
   Ctl& ctl = *reinterpret_cast<Ctl*>(qbuf + (size_t)kQBufs * kQBufBytes);
-  Scratch& scr = *reinterpret_cast<Scratch*>(reinterpret_cast<uint8_t*>(&ctl) + sizeof(Ctl));
+  Scratch<GC>& scr = *reinterpret_cast<Scratch<GC>*>(reinterpret_cast<uint8_t*>(&ctl) + sizeof(Ctl));
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -986,28 +999,31 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           la += __shfl_xor_sync(0xffffffffu, la, off);
           lb += __shfl_xor_sync(0xffffffffu, lb, off);
         }
-        if (g == 0) {
-          scr.m[warp][2 * cq] = m0[nt];
-          scr.m[warp][2 * cq + 1] = m1[nt];
-          scr.l[warp][2 * cq] = la;
-          scr.l[warp][2 * cq + 1] = lb;
-        }
+        // this lane's columns 2cq, 2cq + 1 (a narrow variant keeps the first GC)
+        if (2 * cq < GC) {
+          if (g == 0) {
+            scr.m[warp][2 * cq] = m0[nt];
+            scr.m[warp][2 * cq + 1] = m1[nt];
+            scr.l[warp][2 * cq] = la;
+            scr.l[warp][2 * cq + 1] = lb;
+          }
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          // dims of accumulator rows g and g+8 (see the PV MMA of each KV type)
-          const int d0 = FP8 ? 32 * (mt >> 1) + 2 * g + (mt & 1) : mt * 16 + g;
-          const int d1 = FP8 ? d0 + 16 : d0 + 8;
-          scr.o[warp][2 * cq][d0] = o[nt][mt][0];
-          scr.o[warp][2 * cq + 1][d0] = o[nt][mt][1];
-          scr.o[warp][2 * cq][d1] = o[nt][mt][2];
-          scr.o[warp][2 * cq + 1][d1] = o[nt][mt][3];
+          for (int mt = 0; mt < 8; ++mt) {
+            // dims of accumulator rows g and g+8 (see the PV MMA of each KV type)
+            const int d0 = FP8 ? 32 * (mt >> 1) + 2 * g + (mt & 1) : mt * 16 + g;
+            const int d1 = FP8 ? d0 + 16 : d0 + 8;
+            scr.o[warp][2 * cq][d0] = o[nt][mt][0];
+            scr.o[warp][2 * cq + 1][d0] = o[nt][mt][1];
+            scr.o[warp][2 * cq][d1] = o[nt][mt][2];
+            scr.o[warp][2 * cq + 1][d1] = o[nt][mt][3];
+          }
         }
         if (!cons_sync(ctl, cons_phase, a.err, a.wait_ns)) {
           clean = false;
           break;
         }
         const int ncols = rec.ncol - nt * kMaxGroup;  // columns of this tile with a query row
-        for (int e = ct; e < ncols * kD && e < kMaxGroup * kD; e += kConsumerThreads) {
+        for (int e = ct; e < ncols * kD && e < GC * kD; e += kConsumerThreads) {
           const int h = e >> 7, d = e & (kD - 1);
           float M = -INFINITY;
 #pragma unroll
@@ -1105,7 +1121,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 
 }  // namespace
 
-size_t decode_smem_bytes(int nq) { return smem_bytes(nq); }
+size_t decode_smem_bytes(int nq) { return smem_bytes(nq, kMaxGroup); }
 
 cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf16, int kv, int nq,
                           int grid, cudaStream_t stream) {
@@ -1115,17 +1131,25 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
   if ((nq != 1 && nq != 2) || (chunk && kv != kKv16) || (!chunk && nq != 1))
     return cudaErrorInvalidValue;
   using Kern = void (*)(const CUtensorMap, const DecodeArgs);
-  // decode: 16-bit, E4M3, E5M2 pools (fp16, bf16 each); short chunks: one or
-  // two column tiles over 16-bit pools (fp16, bf16 each)
-  static const Kern kKerns[10] = {
-      decode_kernel<false, kKv16, 1, false>,   decode_kernel<true, kKv16, 1, false>,
-      decode_kernel<false, kKvE4M3, 1, false>, decode_kernel<true, kKvE4M3, 1, false>,
-      decode_kernel<false, kKvE5M2, 1, false>, decode_kernel<true, kKvE5M2, 1, false>,
-      decode_kernel<false, kKv16, 1, true>,    decode_kernel<true, kKv16, 1, true>,
-      decode_kernel<false, kKv16, 2, true>,    decode_kernel<true, kKv16, 2, true>};
-  const int variant = (chunk ? 4 + 2 * nq : 2 * kv) + (bf16 ? 1 : 0);
+  // decode: 16-bit, E4M3, E5M2 pools (fp16, bf16 each), for any GQA group and
+  // for groups of at most 4 (the deeper ring); short chunks: one or two column
+  // tiles over 16-bit pools (fp16, bf16 each)
+  static const Kern kKerns[16] = {
+      decode_kernel<false, kKv16, 1, false, 8>,   decode_kernel<true, kKv16, 1, false, 8>,
+      decode_kernel<false, kKvE4M3, 1, false, 8>, decode_kernel<true, kKvE4M3, 1, false, 8>,
+      decode_kernel<false, kKvE5M2, 1, false, 8>, decode_kernel<true, kKvE5M2, 1, false, 8>,
+      decode_kernel<false, kKv16, 1, true, 8>,    decode_kernel<true, kKv16, 1, true, 8>,
+      decode_kernel<false, kKv16, 2, true, 8>,    decode_kernel<true, kKv16, 2, true, 8>,
+      decode_kernel<false, kKv16, 1, false, 4>,   decode_kernel<true, kKv16, 1, false, 4>,
+      decode_kernel<false, kKvE4M3, 1, false, 4>, decode_kernel<true, kKvE4M3, 1, false, 4>,
+      decode_kernel<false, kKvE5M2, 1, false, 4>, decode_kernel<true, kKvE5M2, 1, false, 4>};
+  // the deeper ring pays where many (request, kv head) pairs (at least one per
+  // CTA) each stream a short run of tiles; a few long pairs split across
+  // many CTAs stream as fast with 16 slots and slow down with 24
+  const bool narrow = !chunk && a.group <= 4 && (long long)a.batch * a.hkv >= grid;
+  const int variant = (chunk ? 4 + 2 * nq : 2 * kv + (narrow ? 10 : 0)) + (bf16 ? 1 : 0);
   const Kern kern = kKerns[variant];
-  const size_t smem = smem_bytes(nq);
+  const size_t smem = smem_bytes(nq, narrow ? 4 : kMaxGroup);
   cudaError_t e = ensure_smem_opt_in(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   // programmatic dependent launch: CTAs may become resident while the previous
