@@ -209,6 +209,46 @@ pkv_status pool_tensor_map(const void* pool, long long pages, int ps, int hkv, i
 
 }  // namespace
 
+namespace pkv {
+
+// q [nnz_q][hq][128] (16-bit) as (dim % 64, dim / 64, head, token): a box of
+// [128 / G tokens][G heads][64 dims] is one dim half of a 128-row tile of the
+// tcgen05 kernel, rows (token, head) in order, 128-byte swizzled
+bool chunk_q_map(const void* q, long long nnz_q, int hq, int group, bool bf16, CUtensorMap* m) {
+  auto encode = get_encode();
+  if (!encode || group < 1 || 128 % group != 0 || hq < group || nnz_q < 1 ||
+      nnz_q > 0x7fffffffLL || !aligned(q, 16))
+    return false;
+  cuuint64_t dims[4] = {64, 2, (cuuint64_t)hq, (cuuint64_t)nnz_q};
+  cuuint64_t strides[3] = {128, 256, (cuuint64_t)hq * 256};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)group, (cuuint32_t)(128 / group)};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return encode(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 states [nnz_q][states][hq][128] as (dim % 32, dim / 32, head, slot,
+// token): a box of [128 / G tokens][G heads][32 dims] is a quarter of a
+// 128-row tile's states in one slot, 128-byte swizzled
+bool chunk_state_map(float* state_o, long long nnz_q, int states, int hq, int group,
+                     CUtensorMap* m) {
+  auto encode = get_encode();
+  if (!encode || !state_o || group < 1 || 128 % group != 0 || hq < group || states < 1 ||
+      nnz_q < 1 || nnz_q > 0x7fffffffLL || !aligned(state_o, 16))
+    return false;
+  cuuint64_t dims[5] = {32, 4, (cuuint64_t)hq, (cuuint64_t)states, (cuuint64_t)nnz_q};
+  cuuint64_t strides[4] = {128, 512, (cuuint64_t)hq * 512, (cuuint64_t)states * hq * 512};
+  cuuint32_t box[5] = {32, 1, (cuuint32_t)group, 1, (cuuint32_t)(128 / group)};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, state_o, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace pkv
+
 namespace {
 // the decode kernel's wait limit (pkv_set_wait_limit_ns); 0 selects the default
 std::atomic<unsigned long long> g_wait_ns{0};
@@ -827,7 +867,10 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
   pa.sink = 0;
   pa.scale_log2 = sm_scale * 1.4426950408889634f;
   pa.one_box = one_box;
-  cudaError_t e = pkv::launch_chunk_tc(tmap, pa, dtype == PKV_BF16, P.row_blocks, s);
+  CUtensorMap qmap = {}, omap = {};
+  pa.q_tma = pkv::chunk_q_map(q, batch, num_qo_heads, group, dtype == PKV_BF16, &qmap) ? 1 : 0;
+  pa.o_tma = pkv::chunk_state_map(state_o, batch, P.states, num_qo_heads, group, &omap) ? 1 : 0;
+  cudaError_t e = pkv::launch_chunk_tc(tmap, qmap, omap, pa, dtype == PKV_BF16, P.row_blocks, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
   // 2. each request's own pages: the last state slot, as an fp32 state
   st = decode_impl(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
@@ -1043,8 +1086,15 @@ pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr, int64_t
   a.sink = sink_tokens;
   a.scale_log2 = sm_scale * 1.4426950408889634f;
   a.one_box = one_box;
+  CUtensorMap qmap = {}, omap = {};
+  a.q_tma = pkv::chunk_q_map(q, nnz_q, num_qo_heads, a.group, pool->dtype == PKV_BF16, &qmap) ? 1 : 0;
+  a.o_tma = num_splits > 1 && pkv::chunk_state_map(a.state_o, nnz_q, num_splits, num_qo_heads,
+                                                   a.group, &omap)
+                ? 1
+                : 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = pkv::launch_chunk_tc(tmap, a, pool->dtype == PKV_BF16, (int)num_row_blocks, s);
+  cudaError_t e = pkv::launch_chunk_tc(tmap, qmap, omap, a, pool->dtype == PKV_BF16,
+                                       (int)num_row_blocks, s);
   if (e != cudaSuccess) return cuda_fail(e, "append attention launch");
   if (num_splits > 1) {
     pkv::MergeArgs ma;

@@ -95,6 +95,7 @@ struct __align__(16) Ctl {
   uint64_t o_done[kRowTiles];   // one phase per P.V tile (the softmax's rescale waits)
   uint64_t o_final[kRowTiles];  // one phase: the row tile's last P.V done
   uint64_t drained;  // one phase: every MMA of the CTA completed
+  uint64_t staged[kRowTiles];  // one phase: the row tile's states are in shared memory
   uint32_t tmem_base;
   int abort;
 };
@@ -149,11 +150,22 @@ __device__ __forceinline__ bool wait_sleeping(uint32_t bar, uint32_t parity, vol
   }
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, float x, float y, float z, float w) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(x), "f"(y), "f"(z),
+               "f"(w)
+               : "memory");
+}
+
 __device__ __forceinline__ int clamp64(long long v) { return v <= 0 ? 0 : (v >= kTile ? kTile : (int)v); }
 
+// qmap (when a.q_tma): q as (dim % 64, dim / 64, head, token) with boxes of
+// [128 / G tokens][G heads][64 dims] -- one row tile's half, 128-byte swizzled.
+// omap (when a.o_tma): the fp32 states as (dim % 32, dim / 32, head, slot,
+// token) with boxes of [128 / G tokens][G heads][32 dims].
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const ChunkArgs a) {
+    chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap qmap,
+                    const __grid_constant__ CUtensorMap omap, const ChunkArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* qs = smem;                                        // Q of both row tiles
@@ -172,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&ctl.q_full[t]), kTileRows);
       mbar_init(smem_u32(&ctl.o_done[t]), 1);
       mbar_init(smem_u32(&ctl.o_final[t]), 1);
+      mbar_init(smem_u32(&ctl.staged[t]), kTileRows);
       mbar_init(smem_u32(&ctl.s_full[t]), 1);
       for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&ctl.p_full[t][b]), kTileRows);
     }
@@ -183,7 +196,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma::tmem_alloc(smem_u32(&ctl.tmem_base), kTmemCols);
     umma::tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap);
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap);
+    if (a.q_tma) prefetch_tensormap(&qmap);
+    if (a.o_tma) prefetch_tensormap(&omap);
+  }
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
@@ -398,10 +415,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = trow + kColO + (uint32_t)t * kD;
     const int rr = row0 + t * kTileRows + row;     // row within the request's chunk rows
     const bool has_row = t * kTileRows + row < nrows;
+    const bool full_tile = t * kTileRows + kTileRows <= nrows;
     const long long pos = has_row ? (prefix ? kNoCausalLimit : base + rr / G) : -1;
     uint8_t* qt = qs + (size_t)t * kQTileBytes;
-    // ---- stage this row of Q in the 128-byte-swizzled K-major layout
-    {
+    // the row tile's first row is (token q_first + (row0 + 128 t) / G, head
+    // kvh * G) when G divides its start
+    if (a.q_tma && (row0 + t * kTileRows) % G == 0) {
+      // ---- Q by two bulk-tensor loads (rows past the tensor read as zeros;
+      // rows past the block, another request's, are masked like any such row:
+      // the rows of a tile never mix in its products)
+      if (warp == 2 + 4 * t && lane == 0) {
+        const uint32_t bar = smem_u32(&ctl.q_full[t]);
+        mbar_arrive_expect_tx(bar, kQTileBytes);
+        for (int half = 0; half < 2; ++half)
+          tma_load_4d(smem_u32(qt) + (uint32_t)half * kQHalf, &qmap, 0, half, kvh * G,
+                      (int)(q_first + (row0 + t * kTileRows) / G), bar);
+      } else {
+        mbar_arrive(smem_u32(&ctl.q_full[t]));
+      }
+    } else {
+      // ---- stage this row of Q in the 128-byte-swizzled K-major layout
       const uint4* src = has_row ? reinterpret_cast<const uint4*>(
                                        static_cast<const uint16_t*>(a.q) +
                                        ((size_t)(q_first + rr / G) * a.hq + (size_t)kvh * G + rr % G) * kD)
@@ -535,35 +568,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t h = has_row ? (size_t)kvh * G + rr % G : 0;
         const float inv = l > 0.f ? 1.f / l : 0.f;
         const float lse = l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+        // fp32 states of a row tile whose rows are all its own (or past the
+        // tensor: the prefix's last block) go out as four bulk-tensor stores
+        // of [128 rows][32 dims], staged 128-byte swizzled in a ring stage no
+        // MMA reads any more: A takes the stage of the pair before the last (its
+        // last P.V completed every MMA issued before it, B's of that pair
+        // included), B the last pair's (its last P.V is the CTA's last MMA)
+        const bool st_tma = a.out_states && a.o_tma && (row0 + t * kTileRows) % G == 0 &&
+                            (a.prefix_pages != nullptr || full_tile);
+        if (st_tma) {
+          const uint32_t stg = smem_u32(ring) + (uint32_t)((((n + 1) >> 1) + t) & 1) * kStageBytes;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          if (have_o) {
-            umma::ld32(t_o + 32u * c, o);
-            umma::wait_ld();
-          } else {
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            if (have_o) {
+              umma::ld32(t_o + 32u * c, o);
+              umma::wait_ld();
+            } else {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = 0u;
-          }
-          if (!has_row) continue;
-          if (!a.out_states) {
-            uint16_t* op = static_cast<uint16_t*>(a.out) + (tok * a.hq + h) * kD + 32 * c;
-#pragma unroll
-            for (int k = 0; k < 32; k += 8) {
-              uint4 w;
-              w.x = pack2<BF16>(__uint_as_float(o[k + 0]) * inv, __uint_as_float(o[k + 1]) * inv);
-              w.y = pack2<BF16>(__uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
-              w.z = pack2<BF16>(__uint_as_float(o[k + 4]) * inv, __uint_as_float(o[k + 5]) * inv);
-              w.w = pack2<BF16>(__uint_as_float(o[k + 6]) * inv, __uint_as_float(o[k + 7]) * inv);
-              *reinterpret_cast<uint4*>(op + k) = w;
+              for (int k = 0; k < 32; ++k) o[k] = 0u;
             }
-          } else {
-            float* op = a.state_o + ((tok * a.states + split) * a.hq + h) * kD + 32 * c;
+            const uint32_t box = stg + (uint32_t)(c * kTileRows * 128 + row * 128);
 #pragma unroll
-            for (int k = 0; k < 32; k += 4)
-              *reinterpret_cast<float4*>(op + k) =
-                  make_float4(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv,
-                              __uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+            for (int k = 0; k < 8; ++k)
+              st_shared_v4(box + (uint32_t)((k ^ (row & 7)) << 4),
+                           __uint_as_float(o[4 * k]) * inv, __uint_as_float(o[4 * k + 1]) * inv,
+                           __uint_as_float(o[4 * k + 2]) * inv, __uint_as_float(o[4 * k + 3]) * inv);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(smem_u32(&ctl.staged[t]));
+          if (warp == 2 + 4 * t && lane == 0 &&
+              wait_sleeping(smem_u32(&ctl.staged[t]), 0, &ctl.abort, a.err)) {
+            for (int c = 0; c < 4; ++c)
+              tma_store_5d(&omap, stg + (uint32_t)(c * kTileRows * 128), 0, c, kvh * G,
+                           split, (int)(q_first + (row0 + t * kTileRows) / G));
+            bulk_store_commit_and_wait_read();
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            if (have_o) {
+              umma::ld32(t_o + 32u * c, o);
+              umma::wait_ld();
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = 0u;
+            }
+            if (!has_row) continue;
+            if (!a.out_states) {
+              uint16_t* op = static_cast<uint16_t*>(a.out) + (tok * a.hq + h) * kD + 32 * c;
+#pragma unroll
+              for (int k = 0; k < 32; k += 8) {
+                uint4 w;
+                w.x = pack2<BF16>(__uint_as_float(o[k + 0]) * inv, __uint_as_float(o[k + 1]) * inv);
+                w.y = pack2<BF16>(__uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+                w.z = pack2<BF16>(__uint_as_float(o[k + 4]) * inv, __uint_as_float(o[k + 5]) * inv);
+                w.w = pack2<BF16>(__uint_as_float(o[k + 6]) * inv, __uint_as_float(o[k + 7]) * inv);
+                *reinterpret_cast<uint4*>(op + k) = w;
+              }
+            } else {
+              float* op = a.state_o + ((tok * a.states + split) * a.hq + h) * kD + 32 * c;
+#pragma unroll
+              for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<float4*>(op + k) =
+                    make_float4(__uint_as_float(o[k]) * inv, __uint_as_float(o[k + 1]) * inv,
+                                __uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+            }
           }
         }
         if (has_row) {
@@ -592,7 +663,8 @@ size_t chunk_tc_smem_bytes() { return kSmemBytes; }
 int chunk_rows_per_cta() { return kRows; }
 int chunk_tile_tokens() { return kTile; }
 
-cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const ChunkArgs& a, bool bf16, int row_blocks,
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& qmap,
+                            const CUtensorMap& omap, const ChunkArgs& a, bool bf16, int row_blocks,
                             cudaStream_t stream) {
   auto kern = bf16 ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
   cudaError_t e = ensure_smem_opt_in(reinterpret_cast<const void*>(kern), kSmemBytes);
@@ -607,7 +679,7 @@ cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const ChunkArgs& a, bool bf
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, tmap, a);
+  e = cudaLaunchKernelEx(&cfg, kern, tmap, qmap, omap, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -125,6 +125,22 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// 5-D tiled bulk-tensor store shared -> global in the calling thread's bulk
+// group; the parts of the box outside the tensor are not written
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap* m, uint32_t src, int x, int y,
+                                             int z, int w, int v) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v)
+      : "memory");
+}
+// close the calling thread's bulk group and wait until its stores have read
+// their shared-memory source (the memory may then be reused)
+__device__ __forceinline__ void bulk_store_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
 }

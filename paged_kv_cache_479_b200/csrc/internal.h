@@ -111,12 +111,19 @@ struct ChunkArgs {
   int batch, hq, hkv, group, page_size, splits, window_left, sink;
   float scale_log2;
   int one_box;
+  int q_tma;                   // 1: qmap describes q (G divides 128), Q comes in by bulk-tensor loads
+  int o_tma;                   // 1: omap describes state_o, full row tiles' states go out by bulk-tensor stores
 };
 // chunk_tc.cu (tcgen05); its tensor map has [16][64] boxes (one dim half each)
 int chunk_rows_per_cta();
 int chunk_tile_tokens();
 size_t chunk_tc_smem_bytes();
-cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const ChunkArgs& a, bool bf16, int row_blocks,
+// q / state tensor maps for ChunkArgs::q_tma / o_tma; false when the shapes do
+// not allow them (the kernel then stages Q and writes states per thread)
+bool chunk_q_map(const void* q, long long nnz_q, int hq, int group, bool bf16, CUtensorMap* m);
+bool chunk_state_map(float* state_o, long long nnz_q, int states, int hq, int group, CUtensorMap* m);
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& qmap,
+                            const CUtensorMap& omap, const ChunkArgs& a, bool bf16, int row_blocks,
                             cudaStream_t stream);
 
 struct AppendArgs {

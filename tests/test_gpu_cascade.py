@@ -71,6 +71,7 @@ def repacked_oracle(w, q_bits, pool_bits, prefix, prefix_len, indptr, indices, l
     (5, "rand", 16, 2, 32, "f16", 5, 31),
     (3, "zero", 32, 8, 16, "bf16", 4, 7),
     (70, "rand", 8, 1, 256, "bf16", 2, 200),
+    (50, "rand", 24, 8, 16, "bf16", 6, 3),    # G = 3: Q staged and states written per thread
 ])
 def test_cascade_matches_oracle_small(case):
     batch, mode, hq, hkv, ps, dt, prefix_pages, cut = case

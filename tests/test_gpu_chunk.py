@@ -97,6 +97,7 @@ CASES = [
     ([260, 90, 513], [120, 90, 3], 8, 1, 64, "f16", 50, 7),
     ([1000, 600], [300, 600], 32, 8, 256, "bf16", 100, 4),
     ([77], [77], 8, 2, 16, "bf16", 0, 0),
+    ([300, 45, 129], [70, 45, 100], 12, 4, 16, "bf16", -1, 0),   # G = 3: Q staged per thread
 ]
 
 
@@ -118,6 +119,17 @@ def test_append_attention_key_splits(S):
     out, lse = c.run(splits=S, window_left=300, sink=16)
     ro, rl = c.oracle(300, 16)
     assert_parity(out, lse, ro, rl, what=f"splits={S} window")
+
+
+@pytest.mark.parametrize("hq,hkv", [(12, 4), (8, 8)])
+def test_append_attention_key_splits_other_groups(hq, hkv):
+    """Key splits write fp32 states: by bulk-tensor stores for whole 128-row
+    tiles when G divides 128 (G = 1 here), per thread otherwise (G = 3) and
+    for the partial tiles of every block."""
+    c = ChunkCase([1500, 700, 90], [100, 43, 90], hq, hkv, 16, "bf16", 725)
+    out, lse = c.run(splits=3)
+    ro, rl = c.oracle()
+    assert_parity(out, lse, ro, rl, what=f"G={hq // hkv} splits=3")
 
 
 def test_append_attention_planner_splits():
