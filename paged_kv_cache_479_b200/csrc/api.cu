@@ -894,6 +894,7 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
   ma.head_dim = kDecodeHeadDim;
   ma.out_dtype = dtype;
   ma.vec4 = 1;
+  ma.rows_ok = 1;
   e = pkv::launch_merge(ma, s);
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();
@@ -1108,6 +1109,7 @@ pkv_status pkv_append_attention(const void* q, const int32_t* qo_indptr, int64_t
     ma.head_dim = kDecodeHeadDim;
     ma.out_dtype = pool->dtype;
     ma.vec4 = 1;
+    ma.rows_ok = 1;
     e = pkv::launch_merge(ma, s);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
@@ -1133,7 +1135,8 @@ pkv_status pkv_merge_states(const float* v, const float* s, int64_t num_rows, in
   a.heads = num_heads;
   a.head_dim = head_dim;
   a.out_dtype = out_dtype;
-  a.vec4 = head_dim == 128 && aligned(v, 16);
+  a.vec4 = head_dim == 128 && aligned(v, 16) && aligned(v_out, 16);
+  a.rows_ok = aligned(s, 16);
   cudaError_t e = pkv::launch_merge(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return ok();

@@ -151,7 +151,8 @@ struct MergeArgs {
   float* s_out;
   long long rows;
   int states, heads, head_dim, out_dtype;
-  int vec4;  // 1: head_dim 128 and v 16-byte aligned (float4 loads)
+  int vec4;  // 1: head_dim 128, v and v_out 16-byte aligned (16-byte loads, 8- or 16-byte stores)
+  int rows_ok;  // 1: s 16-byte aligned too (whole rows may be bulk-copied to shared memory)
 };
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream);
 

@@ -197,12 +197,16 @@ def test_append_overflow_sets_error_bit():
 
 # ------------------------------------------------------------------ merge
 
-@pytest.mark.parametrize("out_dtype,S,D", [(torch.float32, 5, 128), (torch.bfloat16, 5, 128),
-                                           (torch.float16, 5, 128), (torch.float32, 40, 128),
-                                           (torch.float32, 3, 64), (torch.float32, 7, 200)])
-def test_merge_states_matches_oracle(out_dtype, S, D):
+# whole rows through shared memory (S * H a multiple of 4, rows up to 112 KiB),
+# one warp per (row, head) with 16-byte loads (40 states: five batches of 8;
+# 3 x 3 heads), per-dim loads (head_dim 64, 200)
+@pytest.mark.parametrize("out_dtype,S,D,H", [(torch.float32, 5, 128, 8), (torch.bfloat16, 5, 128, 8),
+                                             (torch.float16, 5, 128, 8), (torch.float32, 40, 128, 8),
+                                             (torch.bfloat16, 3, 128, 3), (torch.float32, 3, 64, 8),
+                                             (torch.float32, 7, 200, 8)])
+def test_merge_states_matches_oracle(out_dtype, S, D, H):
     g = torch.Generator().manual_seed(9)
-    N, H = 37, 8
+    N = 37
     v = torch.randn((N, S, H, D), generator=g)
     s = torch.randn((N, S, H), generator=g) * 4
     s[3, 2] = -float("inf")
@@ -218,6 +222,30 @@ def test_merge_states_matches_oracle(out_dtype, S, D):
     assert np.all(np.isneginf(so[5])) and np.all(vo[5] == 0)
     fin = np.isfinite(ref_s)
     np.testing.assert_allclose(so[fin], ref_s[fin], rtol=0, atol=1e-5)
+
+
+def test_merge_paths_bitwise_equal():
+    """Up to 8 states the shared-memory row path and the per-warp path take the
+    same maximum and add in the same order: bitwise equal results.  A lse array
+    one float off 16-byte alignment sends the call down the per-warp path."""
+    g = torch.Generator().manual_seed(11)
+    N, S, H, D = 29, 5, 8, 128
+    v = torch.randn((N, S, H, D), generator=g).cuda()
+    s = torch.randn((N, S, H), generator=g) * 4
+    s[2, 1] = -float("inf")
+    s[4] = -float("inf")
+    s_aligned = s.cuda()
+    buf = torch.empty(N * S * H + 1, device="cuda")
+    s_offset = buf[1:].view(N, S, H)
+    s_offset.copy_(s_aligned)
+    assert s_aligned.data_ptr() % 16 == 0 and s_offset.data_ptr() % 16 != 0
+    for dt, iv in ((torch.bfloat16, torch.int16), (torch.float16, torch.int16),
+                   (torch.float32, torch.int32)):
+        o1, l1 = pkv.merge_states(v, s_aligned, out_dtype=dt)
+        o2, l2 = pkv.merge_states(v, s_offset, out_dtype=dt)
+        torch.cuda.synchronize()
+        assert torch.equal(o1.view(iv), o2.view(iv)), dt
+        assert torch.equal(l1.view(torch.int32), l2.view(torch.int32)), dt
 
 
 def test_merge_of_gpu_splits_equals_whole():
