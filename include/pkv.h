@@ -341,7 +341,9 @@ PKV_API pkv_status pkv_append_fp8(const pkv_pool_desc* pool, float k_scale, floa
  *   kv_len_h     host int32 [batch]: L_b (tokens after the append), or NULL
  *   plan_h       host int32 [capacity][4] or NULL: {request, first row, rows, 0}
  *                per block of up to 256 rows (row r = chunk token r / G, query
- *                head kv_head * G + r % G)
+ *                head kv_head * G + r % G), the blocks with the most key tiles
+ *                first (the launch runs them in plan order, every kv head of a
+ *                block before the next block, so it ends on short ones)
  *   num_splits   if not NULL, receives a split count for the launch: 1 when
  *                the row blocks fill num_sms SMs (or kv_len_h is NULL), else
  *                enough key splits for about two CTAs per SM

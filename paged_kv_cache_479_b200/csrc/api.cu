@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -14,6 +15,7 @@
 #include <mutex>
 #include <set>
 #include <utility>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -912,7 +914,12 @@ int64_t pkv_append_attention_plan(const int32_t* qo_indptr_h, const int32_t* kv_
     return -1;
   const int G = num_qo_heads / num_kv_heads;
   const int R = pkv::chunk_rows_per_cta(), T = pkv::chunk_tile_tokens();
-  int64_t count = 0, ctas = 0;
+  struct Block {
+    long long tiles;
+    int32_t b, r0, n;
+  };
+  std::vector<Block> blocks;
+  int64_t ctas = 0;
   long long max_tiles = 0;
   for (int b = 0; b < batch; ++b) {
     const long long q_len = (long long)qo_indptr_h[b + 1] - qo_indptr_h[b];
@@ -923,14 +930,6 @@ int64_t pkv_append_attention_plan(const int32_t* qo_indptr_h, const int32_t* kv_
     for (long long r0 = 0; r0 < rows; r0 += R) {
       const long long n = rows - r0 < R ? rows - r0 : R;
       if (r0 > 0x7fffffffLL) return -1;
-      if (plan_h && count < capacity) {
-        int32_t* e = plan_h + 4 * count;
-        e[0] = b;
-        e[1] = (int32_t)r0;
-        e[2] = (int32_t)n;
-        e[3] = 0;
-      }
-      ++count;
       // the kernel's key range for this row block, in tiles (host mirror)
       const long long base = L - q_len, pf = base + r0 / G, pl = base + (r0 + n - 1) / G;
       long long lo = window_left >= 0 ? pf - window_left : 0;
@@ -939,6 +938,21 @@ int64_t pkv_append_attention_plan(const int32_t* qo_indptr_h, const int32_t* kv_
       const long long a_end = window_left >= 0 ? (sink_tokens < lo16 ? sink_tokens : lo16) : 0;
       const long long tiles = (a_end + T - 1) / T + (pl + 1 - lo16 + T - 1) / T;
       if (tiles > max_tiles) max_tiles = tiles;
+      blocks.push_back({tiles, b, (int32_t)r0, (int32_t)n});
+    }
+  }
+  // longest first: CTAs are dispatched in block order as SMs free up, so the
+  // launch ends on short blocks (ties keep request and row order)
+  std::stable_sort(blocks.begin(), blocks.end(),
+                   [](const Block& x, const Block& y) { return x.tiles > y.tiles; });
+  const int64_t count = (int64_t)blocks.size();
+  if (plan_h) {
+    for (int64_t i = 0; i < count && i < capacity; ++i) {
+      int32_t* e = plan_h + 4 * i;
+      e[0] = blocks[i].b;
+      e[1] = blocks[i].r0;
+      e[2] = blocks[i].n;
+      e[3] = 0;
     }
   }
   ctas = count * num_kv_heads;

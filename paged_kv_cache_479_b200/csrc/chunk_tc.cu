@@ -172,7 +172,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ring = smem + (size_t)kRowTiles * kQTileBytes;    // K/V stages
   Ctl& ctl = *reinterpret_cast<Ctl*>(ring + (size_t)kStages * kStageBytes);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int kvh = blockIdx.y, split = blockIdx.z;
+  // blocks in launch order: the kv heads of a row block, then the next row
+  // block (the planner lists the row blocks longest first); key splits on y
+  const int kvh = (int)(blockIdx.x % (unsigned)a.hkv), split = blockIdx.y;
+  const int rblock = (int)(blockIdx.x / (unsigned)a.hkv);
   const int G = a.group;
 
   if (tid == 0) {
@@ -211,11 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool prefix = a.prefix_pages != nullptr;
   int b = 0, row0, nrows;
   if (prefix) {  // rows of every request, in blocks of kRows
-    row0 = (int)blockIdx.x * kRows;
+    row0 = rblock * kRows;
     const long long left = (long long)a.batch * G - row0;
     nrows = left < kRows ? (int)left : kRows;
   } else {
-    const int4 item = a.plan[blockIdx.x];
+    const int4 item = a.plan[rblock];
     b = item.x;
     row0 = item.y;
     nrows = item.z;
@@ -670,7 +673,7 @@ cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& qmap,
   cudaError_t e = ensure_smem_opt_in(reinterpret_cast<const void*>(kern), kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)row_blocks, (unsigned)a.hkv, (unsigned)a.splits);
+  cfg.gridDim = dim3((unsigned)row_blocks * (unsigned)a.hkv, (unsigned)a.splits);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;

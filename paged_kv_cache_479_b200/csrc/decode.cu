@@ -1076,18 +1076,10 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     if (!ctl.pend_last[k] || h >= ctl.pend[k].ncol) continue;
     const SegRec pr = ctl.pend[k];
     auto slot_of = [&](int j) { return state_slot(pr.c_first, j); };
-    float M = -INFINITY;
-    for (int j = lane; j < pr.ncover; j += 32)
-      M = fmaxf(M, __ldcg(a.part_lse + (size_t)slot_of(j) * P + h));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (CHUNK) M = M == -INFINITY ? 0.f : M;  // (every column of a chunk sees key 0: not expected)
-    float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     constexpr int kBatch = 8;  // partial states loaded together
-    for (int j0 = 0; j0 < pr.ncover; j0 += kBatch) {
-      float wt[kBatch];
-      float4 v[kBatch];
+    float wt[kBatch];
+    float4 v[kBatch];
+    auto load_batch = [&](int j0) {
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int j = j0 + u;
@@ -1100,6 +1092,20 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+    };
+    // the first batch's loads go out with the maximum's: up to kBatch states,
+    // one round trip
+    load_batch(0);
+    float M = -INFINITY;
+    for (int j = lane; j < pr.ncover; j += 32)
+      M = fmaxf(M, __ldcg(a.part_lse + (size_t)slot_of(j) * P + h));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (CHUNK) M = M == -INFINITY ? 0.f : M;  // (every column of a chunk sees key 0: not expected)
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < pr.ncover; j0 += kBatch) {
+      if (j0 > 0) load_batch(j0);
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const float w = ex2(wt[u] - M);

@@ -338,7 +338,8 @@ def test_bad_plan_entry_sets_error_bit():
     w = c.w
     plan, _ = pkv.append_attention_plan(c.qo, w.kv_lens, 8, 2)
     bad = plan.copy()
-    bad[0, 2] = 10 * 4 + 1                          # more rows than the chunk has
+    k = int(np.flatnonzero(plan[:, 0] == 0)[0])     # request 0's (only) block
+    bad[k, 2] = 10 * 4 + 1                          # more rows than the chunk has
     keep = (i32(w.page_indptr), i32(w.page_indices), i32(w.last_page_len))
     table = pkv.csr_table(*keep)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -291,7 +291,14 @@ def test_append_attention_plan_covers_rows_once():
             assert 1 <= n <= 256 and pad == 0
             seen[b][r0:r0 + n] += 1
         assert all((s == 1).all() for s in seen)
-        assert list(plan[:, 0]) == sorted(plan[:, 0])
+        # longest first: key tiles of 64 up to the block's last row (no window),
+        # non-increasing, ties in request and row order
+        base = kv.astype(np.int64) - q_lens
+        tiles = [(int(base[b]) + (int(r0) + int(n) - 1) // G + 1 + 63) // 64 for b, r0, n, _ in plan]
+        assert all(x >= y for x, y in zip(tiles, tiles[1:]))
+        for i in range(len(plan) - 1):
+            if tiles[i] == tiles[i + 1]:
+                assert tuple(plan[i, :2]) < tuple(plan[i + 1, :2])
         assert 1 <= S <= 32
 
 
