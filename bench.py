@@ -17,6 +17,13 @@ cpu_baseline.
 Metric: KV HBM GB/s (algorithmic bytes: unique K/V once + q + out + page
 table + lse, plus the append's rows), with us/step and decoded tokens/s.
 
+Timing: W untimed steps, then the K steps captured back to back in one CUDA
+graph and replayed once between two CUDA events on the launching stream
+(barrier and synchronize on both sides, max over ranks).  Nothing sits
+between two launches, so each may start while the previous one drains
+(programmatic dependent launch), as in a serving loop; the per-launch time
+in `roofline` is the timed region divided by its launches.
+
   python bench.py [--gpus N --steps K --warmup W] [--workload 1..5] [--impl reference]
 
 N > 1 (launched by torch.distributed.run, one rank per GPU): every rank runs
@@ -75,7 +82,7 @@ def parse():
     p.add_argument("--cascade", action="store_true",
                    help="decode a shared-prefix workload with pkv_cascade_decode")
     p.add_argument("--no-graph", action="store_true",
-                   help="launch every call from Python instead of replaying CUDA graphs")
+                   help="launch every call from Python instead of replaying one CUDA graph")
     p.add_argument("--kv", choices=["16bit", "e4m3", "e5m2"], default="16bit",
                    help="KV pool type: the workload's 16-bit type, or FP8 (E4M3 / E5M2) codes "
                         "with per-tensor K/V scales (q and out stay 16-bit)")
@@ -485,45 +492,48 @@ def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=Fa
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during warm-up")
 
-    # the same calls captured once per batch copy and replayed (no Python on the
-    # launch path); each library call is capturable: no allocation, no sync
+    # The K timed steps go back to back into one CUDA graph (each library call
+    # is capturable: no allocation, no sync) replayed once between two events:
+    # no event or host work sits between launches, so each launch may start
+    # (programmatic dependent launch) while the previous one drains, as in a
+    # serving loop.  Per-launch time = the timed region / its launches.
     graphs = []
+    K = args.steps
 
-    def graphed(fn, bt):
+    def steps_fn(n, with_append=True):
+        def run():
+            for i in range(n):
+                if with_append:
+                    append_call(batches[i % rotation])
+                decode_call(batches[i % rotation])
         if args.no_graph:
-            return lambda: fn(bt)
+            return run
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            fn(bt)
+            run()
         graphs.append(g)
         return g.replay
-    app_g = [graphed(append_call, bt) if w.nnz_new and not fused else (lambda: None)
-             for bt in batches]
-    dec_g = [graphed(decode_call, bt) for bt in batches]
-    for i in range(2 * rotation):
-        app_g[i % rotation]()
-        dec_g[i % rotation]()
-    torch.cuda.synchronize()
 
-    K = args.steps
-    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    t_host0 = time.time()
-    start.record(stream)
-    for i in range(K):
-        app_g[i % rotation]()
-        d0[i].record(stream)
-        dec_g[i % rotation]()
-        d1[i].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize()
-    t_host1 = time.time()
-    barrier()
-    ms = max_over_ranks(start.elapsed_time(end), world, dev)
-    decode_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K, world, dev)
+    def timed(fn):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        h0 = time.time()
+        start.record(stream)
+        fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+        h1 = time.time()
+        barrier()
+        return max_over_ranks(start.elapsed_time(end), world, dev), h0, h1
+
+    steps_g = steps_fn(K)
+    ms, t_host0, t_host1 = timed(steps_g)
+    if launches_per_step == 1 or cascade:
+        decode_ms = ms / K   # the decode launch (with the fused append), or the cascade's step
+    else:
+        # the append runs as its own launch: time the decode launches alone too
+        decode_ms = timed(steps_fn(K, with_append=False))[0] / K
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during the timed steps")
 
@@ -582,7 +592,14 @@ def measure_decode(w, args, dev, rank, world, *, cascade=False, fp8=None, e2e=Fa
 
         e2e_calls(None)
         torch.cuda.synchronize()
-        e2e_replay = graphed(e2e_calls, None)
+        if args.no_graph:
+            e2e_replay = lambda: e2e_calls(None)
+        else:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                e2e_calls(None)
+            graphs.append(g)
+            e2e_replay = g.replay
 
         def e2e_step():
             e2e_replay()
@@ -696,14 +713,18 @@ def run_pkv(args):
             "dtype": (f"{fp8} KV widened to f16, f32 accumulate" if fp8 else
                       ("bf16" if w.dtype == "bf16" else "f16")), "data": "synthetic",
             "config": {**workload_config(w, args, r["rotation"], r["N"]),
-                       "launch": ("direct calls" if args.no_graph else
-                                  ("the fused append + decode launch (pkv_decode_append)" if fused
+                       "launch": (("the fused append + decode launch (pkv_decode_append)" if fused
                                    else ("the cascade's launches" if args.cascade else
-                                         ("append and decode each" if w.nnz_new else "decode"))) +
-                                  " captured once per batch copy as a CUDA graph, replayed") +
-                                 ("; page table marked ready at launch (read while the previous "
-                                  "step's kernel drains)" if r["early_table"] and not args.cascade
-                                  else "")},
+                                         ("append and decode" if w.nnz_new else "decode"))) +
+                                  (" of the K steps called back to back" if args.no_graph else
+                                   " of the K steps captured back to back in one CUDA graph, "
+                                   "replayed once") +
+                                  " between two events (nothing between launches: each may "
+                                  "start while the previous drains); per launch = the region / "
+                                  "its launches" +
+                                  ("; page table marked ready at launch (read while the previous "
+                                   "step's kernel drains)" if r["early_table"] and not args.cascade
+                                   else ""))},
             "us_per_step": round(ms / K * 1e3, 2),
             "tokens_per_s": round(w.batch * world / (ms / 1e3 / K), 1),
             "pct_of_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
@@ -790,44 +811,52 @@ def run_chunk(args):
                                  lse=lse, sm_scale=w.sm_scale, error_word=err,
                                  stream=torch.cuda.current_stream(dev))
 
-    def graphed(fn, bt):
-        if args.no_graph:
-            return lambda: fn(bt)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn(bt)
-        return g.replay
     for i in range(args.warmup):
         append_call(batches[i % rotation])
         attn_call(batches[i % rotation])
     torch.cuda.synchronize()
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during warm-up")
-    app_g = [(lambda: None) if fuse_short else graphed(append_call, bt) for bt in batches]
-    att_g = [graphed(attn_call, bt) for bt in batches]
-    clocks = ClockSampler(local)
     K = args.steps
-    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    t_host0 = time.time()
-    start.record(stream)
-    for i in range(K):
-        app_g[i % rotation]()
-        d0[i].record(stream)
-        att_g[i % rotation]()
-        d1[i].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize()
-    t_host1 = time.time()
-    if world > 1:
-        torch.distributed.barrier()
+    graphs = []
+
+    # the K steps back to back in one CUDA graph, replayed once between two
+    # events (as in the decode bench); the attention launches alone are timed
+    # the same way when the append is a launch of its own
+    def steps_fn(n, with_append=True):
+        def run():
+            for i in range(n):
+                if with_append:
+                    append_call(batches[i % rotation])
+                attn_call(batches[i % rotation])
+        if args.no_graph:
+            return run
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        graphs.append(g)
+        return g.replay
+
+    def timed(fn):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        h0 = time.time()
+        start.record(stream)
+        fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+        h1 = time.time()
+        if world > 1:
+            torch.distributed.barrier()
+        return max_over_ranks(start.elapsed_time(end), world, dev), h0, h1
+
+    clocks = ClockSampler(local)
+    ms, t_host0, t_host1 = timed(steps_fn(K))
+    attn_ms = ms / K if fuse_short else timed(steps_fn(K, with_append=False))[0] / K
     clocks.stop()
-    ms = max_over_ranks(start.elapsed_time(end), world, dev)
-    attn_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K, world, dev)
+    del graphs
     if pkv.read_error_word(err) != 0:
         raise RuntimeError("device error bits set during the timed steps")
     flops = wl.chunk_flops(w, q_lens)
@@ -863,9 +892,11 @@ def run_chunk(args):
                        "flops_per_step": flops,
                        "attention_bytes_per_step": attn_bytes,
                        "l2": f"2 rotating batch copies of {kv / 1e6:.0f} MB K/V",
-                       "launch": ("append fused into the attention launch, captured as a CUDA "
-                                  "graph" if fuse_short else
-                                  "append and append attention captured as CUDA graphs"),
+                       "launch": ("append fused into the attention launch" if fuse_short else
+                                  "append and append attention") +
+                                 " of the K steps captured back to back in one CUDA graph, "
+                                 "replayed once between two events; the attention launches "
+                                 "alone timed the same way",
                        "parallelism": f"dp{world} (independent batches per GPU)"},
             "us_per_step": round(ms / K * 1e3, 2),
             "tokens_per_s": round(nnz * world / (ms / K / 1e3), 1),
