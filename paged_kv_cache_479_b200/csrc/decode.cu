@@ -60,8 +60,8 @@ namespace pkv {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kConsumerWarps = 8;    // consumer warps of every variant but one (below)
+constexpr int kMaxWarps = 16;        // consumer warps + the producer, at most
 constexpr int kStages = kDecodeStages;
 // GQA groups of at most 4 need half the query-block and merge-scratch room, which
 // buys a 24-slot ring (192 KiB in flight instead of 128 KiB); wider groups and
@@ -96,6 +96,18 @@ __host__ __device__ constexpr int q_buf_bytes(int nq, int gc) { return nq * gc *
 static_assert(kMaxStages <= kConsumerWarps * (kQBufs - 1) &&
                   kMaxStages <= kConsumerWarps * (kSegRecs - 1) && kSegRecs % (2 * kQBufs) == 0,
               "a query buffer or segment record could be refilled before every warp read it");
+// 8-bit pools with GQA groups of at most 4: their tiles carry half the bytes
+// of a 16-bit tile for the same MMA work, so the consumers, not the loads, set
+// the pace; 12 consumer warps on a 36-slot ring (144 KiB in flight) keep more
+// tiles in work per SM than 8 on 48 (the 12 warps' merge scratch leaves no room
+// for 48 slots)
+constexpr int kFp8Warps = 12;
+constexpr int kFp8WarpsStages = 36;
+// ring slots of a variant: 16-bit tiles (8 KiB), 8-bit tiles (4 KiB)
+__host__ __device__ constexpr int ring_slots(int gc, bool fp8, int cw) {
+  return !fp8 ? (gc <= 4 ? kStagesNarrow : kStages)
+              : (cw == kFp8Warps ? kFp8WarpsStages : 2 * (gc <= 4 ? kStagesNarrow : kStages));
+}
 constexpr int kScratchStride = kD + 4;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -125,12 +137,12 @@ struct SplitPair {
 struct __align__(16) Ctl {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t cons;                      // consumer-only barrier (256 arrivals)
+  uint64_t cons;                      // consumer-only barrier (every consumer thread)
   uint64_t qfull[kQBufs];             // a segment's query rows landed in qbuf[i]
   int meta[kMaxStages];
   int last_it[kMaxStages];            // ring position of the last hand-over of each slot (-1: none)
   SegRec seg[kSegRecs];
-  long long warp_tot[kDecodeThreads / 32];
+  long long warp_tot[kMaxWarps];
   long long Cb0;
   SegRec pend[kMaxPending];   // split pairs this CTA wrote partial states for
   int pend_last[kMaxPending]; // 1 when this CTA arrived last for that pair
@@ -141,22 +153,24 @@ struct __align__(16) Ctl {
   int counted;                // 1 once this CTA has counted itself in on its split pairs
 };
 
-// the 8 consumer warps' states of up to GC columns, merged at a segment end
-template <int GC>
+// the CW consumer warps' states of up to GC columns, merged at a segment end
+template <int GC, int CW>
 struct Scratch {
-  float m[kConsumerWarps][GC];
-  float l[kConsumerWarps][GC];
-  float o[kConsumerWarps][GC][kScratchStride];
+  float m[CW][GC];
+  float l[CW][GC];
+  float o[CW][GC][kScratchStride];
 };
 
-__host__ __device__ constexpr int ring_stages(int gc) { return gc <= 4 ? kStagesNarrow : kStages; }
-constexpr size_t smem_bytes(int nq, int gc) {
-  return 1024 /*alignment slack*/ + (size_t)ring_stages(gc) * kSlotBytes +
-         (size_t)kQBufs * q_buf_bytes(nq, gc) + sizeof(Ctl) +
-         (gc <= 4 ? sizeof(Scratch<4>) : sizeof(Scratch<kMaxGroup>));
+constexpr size_t scratch_bytes(int gc, int cw) {
+  return (size_t)cw * gc * (2 + kScratchStride) * sizeof(float);
+}
+constexpr size_t smem_bytes(int nq, int gc, bool fp8 = false, int cw = kConsumerWarps) {
+  return 1024 /*alignment slack*/ + (size_t)ring_slots(gc, fp8, cw) * (fp8 ? kSlotBytes / 2 : kSlotBytes) +
+         (size_t)kQBufs * q_buf_bytes(nq, gc) + sizeof(Ctl) + scratch_bytes(gc <= 4 ? 4 : kMaxGroup, cw);
 }
 static_assert(smem_bytes(1, 4) <= 227 * 1024 && smem_bytes(1, kMaxGroup) <= 227 * 1024 &&
-                  smem_bytes(2, kMaxGroup) <= 227 * 1024,
+                  smem_bytes(2, kMaxGroup) <= 227 * 1024 &&
+                  smem_bytes(1, 4, true, kFp8Warps) <= 227 * 1024,
               "shared memory per CTA");
 
 // output of (request b, query head h): 16-bit final outputs, or fp32 attention
@@ -182,8 +196,9 @@ __device__ __forceinline__ void store_lse(const DecodeArgs& a, size_t b, size_t 
   if (a.lse) a.lse[b * (size_t)a.lse_rs + h] = v;
 }
 
-// inclusive scan over the whole block (kDecodeThreads threads); returns the
-// prefix for this thread and the block total in *total
+// inclusive scan over the whole block (NW warps); returns the prefix for this
+// thread and the block total in *total
+template <int NW>
 __device__ long long block_incl_scan(long long v, long long* warp_tot, long long* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   long long x = v;
@@ -196,7 +211,7 @@ __device__ long long block_incl_scan(long long v, long long* warp_tot, long long
   __syncthreads();
   long long before = 0, all = 0;
 #pragma unroll
-  for (int w = 0; w < kDecodeThreads / 32; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const long long t = warp_tot[w];
     if (w < warp) before += t;
     all += t;
@@ -210,7 +225,7 @@ __device__ __forceinline__ uint32_t ld_u32(const void* p) {
   return *reinterpret_cast<const uint32_t*>(p);
 }
 
-// all 256 consumer threads meet; bounded
+// all consumer threads meet; bounded
 __device__ __forceinline__ bool cons_sync(Ctl& ctl, uint32_t& phase, int* err, uint64_t limit) {
   mbar_arrive(smem_u32(&ctl.cons));
   const bool ok = mbar_wait_bounded(smem_u32(&ctl.cons), phase, &ctl.abort, err, limit);
@@ -333,24 +348,31 @@ __device__ __forceinline__ void write_new_rows(const DecodeArgs& a, const ReqInf
 // NQ: n8 column tiles per pair (2 only for short chunks over 16-bit pools);
 // CHUNK: short chunks (causal limits per column), else decode (one token per request)
 // GC: the GQA groups the variant takes, 8 (any) or 4 (a deeper ring)
-template <bool BF16, int KV, int NQ, bool CHUNK, int GC>
-__global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
+template <bool BF16, int KV, int NQ, bool CHUNK, int GC, int CW = kConsumerWarps>
+__global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   constexpr bool FP8 = KV != kKv16;
+  constexpr int kThreads = (CW + 1) * 32;  // CW consumer warps, then the producer warp
+  static_assert(CW == kConsumerWarps || (CW == kFp8Warps && FP8 && GC == 4),
+                "12 consumer warps: 8-bit pools, narrow groups");
+  static_assert(CW + 1 <= kMaxWarps, "warp count");
   static_assert(NQ == 1 || (NQ == 2 && !FP8), "two column tiles only for 16-bit pools");
   static_assert(!CHUNK || !FP8, "short chunks only for 16-bit pools");
   static_assert(CHUNK || NQ == 1, "the decode has one column tile");
   static_assert(GC == kMaxGroup || (GC == 4 && NQ == 1 && !CHUNK), "narrow groups: decode only");
   constexpr int kCols = NQ * GC;  // columns with a query row at most
   constexpr int kQBufBytes = q_buf_bytes(NQ, GC);
-  constexpr int kRingBytes = ring_stages(GC) * kSlotBytes;
-  // ring geometry of this KV type (16-bit: 16 slots of 8 KiB; 8-bit: 32 of 4 KiB)
-  constexpr int kSt = FP8 ? 2 * ring_stages(GC) : ring_stages(GC);
+  // ring geometry of this variant (16-bit: 16 or 24 slots of 8 KiB; 8-bit: 32,
+  // 36 or 48 of 4 KiB)
+  constexpr int kSt = ring_slots(GC, FP8, CW);
   constexpr int kTileB = FP8 ? kTileBytes / 2 : kTileBytes;
   constexpr int kSlotB = 2 * kTileB;
+  constexpr int kRingBytes = kSt * kSlotB;
   constexpr int kIssue = kSt < 16 ? kSt : 16;
-  static_assert(kSt % kConsumerWarps == 0 && 32 % kIssue == 0 && kSt <= kMaxStages,
+  static_assert(kSt % CW == 0 && 32 % kIssue == 0 && kSt <= kMaxStages,
                 "each ring slot must have a single consumer warp");
+  static_assert(kSt <= CW * (kQBufs - 1) && kSt <= CW * (kSegRecs - 1),
+                "a query buffer or segment record could be refilled before every warp read it");
   // MMA operand type: 16-bit pools use their own type; E4M3 codes are widened
   // to fp16 (exact), so those tiles run the fp16 MMA
   constexpr bool kMmaBF16 = BF16 && !FP8;
@@ -360,7 +382,8 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   uint8_t* ring = smem;
   uint8_t* qbuf = smem + kRingBytes;
   Ctl& ctl = *reinterpret_cast<Ctl*>(qbuf + (size_t)kQBufs * kQBufBytes);
-  Scratch<GC>& scr = *reinterpret_cast<Scratch<GC>*>(reinterpret_cast<uint8_t*>(&ctl) + sizeof(Ctl));
+  Scratch<GC, CW>& scr =
+      *reinterpret_cast<Scratch<GC, CW>*>(reinterpret_cast<uint8_t*>(&ctl) + sizeof(Ctl));
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -374,7 +397,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
       mbar_init(smem_u32(&ctl.full[s]), 1);
       mbar_init(smem_u32(&ctl.empty[s]), 32);
     }
-    mbar_init(smem_u32(&ctl.cons), kConsumerThreads);
+    mbar_init(smem_u32(&ctl.cons), CW * 32);
     for (int i = 0; i < kQBufs; ++i) mbar_init(smem_u32(&ctl.qfull[i]), 1);
     for (int s = 0; s < kSt; ++s) ctl.last_it[s] = -1;
     for (int k = 0; k < kMaxPending; ++k) {
@@ -388,7 +411,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     ctl.npend = 0;
     fence_barrier_init();
   }
-  if (warp == kConsumerWarps && lane == 0) prefetch_tensormap(&tmap);
+  if (warp == CW && lane == 0) prefetch_tensormap(&tmap);
   // With programmatic dependent launch this CTA may start while the previous
   // kernel in the stream still runs; everything above touched no input.  When
   // the caller promises that kernel does not write the page table
@@ -402,7 +425,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   // ---- prologue: total work W, this partition's share [f0, f1), its first request
   long long mine = 0;
   int errs = 0;
-  for (int b = tid; b < B; b += kDecodeThreads) {
+  for (int b = tid; b < B; b += kThreads) {
     const ReqInfo r = request_info(a.tv, b, a.page_size);
     mine += r.units;
     errs |= r.err;
@@ -412,7 +435,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     atomicOr(a.err, errs);
   }
   long long total_units;
-  (void)block_incl_scan(mine, ctl.warp_tot, &total_units);
+  (void)block_incl_scan<CW + 1>(mine, ctl.warp_tot, &total_units);
   const long long W = (long long)Hkv * total_units;
   // with fewer units than CTAs only the first W partitions get work, so that
   // every partition that covers a (request, kv head) pair is non-empty
@@ -421,7 +444,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   const long long f1 = c < N ? part_start(W, N, c + 1) : 0;
 
   long long carry = 0;
-  for (int base = 0; base < B; base += kDecodeThreads) {
+  for (int base = 0; base < B; base += kThreads) {
     const int b = base + tid;
     ReqInfo r;
     r.tiles = 0;
@@ -429,7 +452,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     r.len = 0;
     if (b < B) r = request_info(a.tv, b, a.page_size);
     long long chunk_total;
-    const long long incl = block_incl_scan(r.units, ctl.warp_tot, &chunk_total);
+    const long long incl = block_incl_scan<CW + 1>(r.units, ctl.warp_tot, &chunk_total);
     const long long excl = incl - r.units;
     if (b < B && r.units > 0 && f0 < f1) {
       const long long s0 = (long long)Hkv * (carry + excl), s1 = (long long)Hkv * (carry + incl);
@@ -469,7 +492,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
 
   const int G = a.group;
 
-  if (warp == kConsumerWarps) {
+  if (warp == CW) {
     // =========================== producer ===========================
     Walk wk;
     wk.tv = a.tv;
@@ -503,7 +526,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         wk.advance();
         continue;
       }
-      const long long n_pad = (n + kConsumerWarps - 1) / kConsumerWarps * kConsumerWarps;
+      const long long n_pad = (n + CW - 1) / CW * CW;
       const long long pstart = wk.pair_start();
       // page ids, one tile per lane, loaded one 32-tile batch ahead of their use
       const int* idx = a.indices + wk.ri.page_base;
@@ -593,7 +616,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
             __syncwarp();
           }
         }
-        const int flags = ((k >= n_pad - kConsumerWarps) ? kMetaSegLast : 0) |
+        const int flags = ((k >= n_pad - CW) ? kMetaSegLast : 0) |
                           ((seg & (kSegRecs - 1)) << kMetaSegShift);
         const int cnt = (int)((n_pad - k0) < 32 ? (n_pad - k0) : 32);
         // lanes [jb, jb + kIssue) publish their tiles concurrently (distinct ring slots)
@@ -643,7 +666,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     // one end marker per consumer warp
     if (ok) {
       int okl = 1;
-      if (lane < kConsumerWarps) {
+      if (lane < CW) {
         const uint32_t it = i + lane;
         const int s = (int)(it % kSt);
         okl = mbar_wait_bounded(smem_u32(&ctl.empty[s]), ((it / kSt) & 1u) ^ 1u, &ctl.abort,
@@ -655,7 +678,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
         }
       }
       ok = __all_sync(0xffffffffu, okl) != 0;
-      i += kConsumerWarps;
+      i += CW;
     }
     __syncwarp();
     if (lane == 0) {
@@ -715,7 +738,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   uint32_t cons_phase = 0;
   bool clean = true;
 
-  for (uint32_t i = warp;; i += kConsumerWarps) {
+  for (uint32_t i = warp;; i += CW) {
     const int s = (int)(i % kSt);
     if (!mbar_wait_bounded(smem_u32(&ctl.full[s]), (i / kSt) & 1u, &ctl.abort, a.err, a.wait_ns)) {
       clean = false;
@@ -984,7 +1007,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
     mbar_arrive(smem_u32(&ctl.empty[s]));
 
     if (info & kMetaSegLast) {
-      // ================= end of segment: merge the 8 warps' states =================
+      // ================= end of segment: merge the CW warps' states =================
       // one n8 column tile at a time through the scratch area
       const bool direct = rec.ncover == 1;
 #pragma unroll
@@ -1023,15 +1046,15 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
           break;
         }
         const int ncols = rec.ncol - nt * kMaxGroup;  // columns of this tile with a query row
-        for (int e = ct; e < ncols * kD && e < GC * kD; e += kConsumerThreads) {
+        for (int e = ct; e < ncols * kD && e < GC * kD; e += CW * 32) {
           const int h = e >> 7, d = e & (kD - 1);
           float M = -INFINITY;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, scr.m[w][h]);
+          for (int w = 0; w < CW; ++w) M = fmaxf(M, scr.m[w][h]);
           const float Ms = CHUNK && M == -INFINITY ? 0.f : M;  // no visible key in this share
           float L = 0.f, acc = 0.f;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) {
+          for (int w = 0; w < CW; ++w) {
             const float wt = ex2(scr.m[w][h] - Ms);
             L += wt * scr.l[w][h];
             acc += wt * scr.o[w][h][d];
@@ -1071,7 +1094,7 @@ __global__ void __launch_bounds__(kDecodeThreads, kDecodeCtasPerSm)
   __threadfence();
   // one warp per (pair, column); lane L owns dims 4L .. 4L+3
   const int P = a.pcols;  // state columns per slot
-  for (int item = warp; item < npend * kCols; item += kConsumerWarps) {
+  for (int item = warp; item < npend * kCols; item += CW) {
     const int k = item / kCols, h = item % kCols;
     if (!ctl.pend_last[k] || h >= ctl.pend[k].ncol) continue;
     const SegRec pr = ctl.pend[k];
@@ -1138,8 +1161,9 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
     return cudaErrorInvalidValue;
   using Kern = void (*)(const CUtensorMap, const DecodeArgs);
   // decode: 16-bit, E4M3, E5M2 pools (fp16, bf16 each), for any GQA group and
-  // for groups of at most 4 (the deeper ring); short chunks: one or two column
-  // tiles over 16-bit pools (fp16, bf16 each)
+  // for groups of at most 4 (16-bit: the deeper ring; 8-bit: 12 consumer
+  // warps); short chunks: one or two column tiles over 16-bit pools (fp16,
+  // bf16 each)
   static const Kern kKerns[16] = {
       decode_kernel<false, kKv16, 1, false, 8>,   decode_kernel<true, kKv16, 1, false, 8>,
       decode_kernel<false, kKvE4M3, 1, false, 8>, decode_kernel<true, kKvE4M3, 1, false, 8>,
@@ -1147,22 +1171,26 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
       decode_kernel<false, kKv16, 1, true, 8>,    decode_kernel<true, kKv16, 1, true, 8>,
       decode_kernel<false, kKv16, 2, true, 8>,    decode_kernel<true, kKv16, 2, true, 8>,
       decode_kernel<false, kKv16, 1, false, 4>,   decode_kernel<true, kKv16, 1, false, 4>,
-      decode_kernel<false, kKvE4M3, 1, false, 4>, decode_kernel<true, kKvE4M3, 1, false, 4>,
-      decode_kernel<false, kKvE5M2, 1, false, 4>, decode_kernel<true, kKvE5M2, 1, false, 4>};
-  // the deeper ring pays where many (request, kv head) pairs (at least one per
-  // CTA) each stream a short run of tiles; a few long pairs split across
-  // many CTAs stream as fast with 16 slots and slow down with 24
+      decode_kernel<false, kKvE4M3, 1, false, 4, kFp8Warps>,
+      decode_kernel<true, kKvE4M3, 1, false, 4, kFp8Warps>,
+      decode_kernel<false, kKvE5M2, 1, false, 4, kFp8Warps>,
+      decode_kernel<true, kKvE5M2, 1, false, 4, kFp8Warps>};
+  // the narrow variants pay where many (request, kv head) pairs (at least one
+  // per CTA) each stream a short run of tiles; a few long pairs split across
+  // many CTAs stream as fast with the default ring and slow down with 24 slots
   const bool narrow = !chunk && a.group <= 4 && (long long)a.batch * a.hkv >= grid;
   const int variant = (chunk ? 4 + 2 * nq : 2 * kv + (narrow ? 10 : 0)) + (bf16 ? 1 : 0);
   const Kern kern = kKerns[variant];
-  const size_t smem = smem_bytes(nq, narrow ? 4 : kMaxGroup);
+  const bool fp8 = kv != kKv16;
+  const int cw = narrow && fp8 ? kFp8Warps : kConsumerWarps;
+  const size_t smem = smem_bytes(nq, narrow ? 4 : kMaxGroup, fp8, cw);
   cudaError_t e = ensure_smem_opt_in(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   // programmatic dependent launch: CTAs may become resident while the previous
   // kernel drains; the kernel waits for it before reading any input
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.blockDim = dim3((unsigned)(cw + 1) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

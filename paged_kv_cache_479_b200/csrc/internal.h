@@ -67,7 +67,6 @@ size_t decode_counter_bytes(int group, int num_partitions);
 // once per (function, device); safe to call from several host threads.
 cudaError_t ensure_smem_opt_in(const void* func, size_t bytes);
 
-constexpr int kDecodeThreads = 288;  // 8 consumer warps + 1 producer warp
 #ifndef PKV_STAGES
 #define PKV_STAGES 16
 #endif
