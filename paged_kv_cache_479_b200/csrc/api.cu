@@ -874,7 +874,11 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
   pa.o_tma = pkv::chunk_state_map(state_o, batch, P.states, num_qo_heads, group, &omap) ? 1 : 0;
   cudaError_t e = pkv::launch_chunk_tc(tmap, qmap, omap, pa, dtype == PKV_BF16, P.row_blocks, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefix launch");
-  // 2. each request's own pages: the last state slot, as an fp32 state
+  // 2. each request's own pages: the last state slot, as an fp32 state.  The
+  // prefix launch lets it start once the prefix has waited for the kernels
+  // before the cascade, and nothing in the cascade writes the own-page table:
+  // it is read before this launch's dependency wait (its CTAs fill the SMs
+  // the prefix leaves idle); q, the pool and the state slot only after it.
   st = decode_impl(q, num_qo_heads, pool, num_pages, page_size, num_kv_heads, head_dim, dtype,
                    PKV_LAYOUT_HND, pkv::csr_view(page_indptr, last_page_len), page_indices,
                    batch, sm_scale, N,
@@ -882,7 +886,8 @@ pkv_status pkv_cascade_decode(const void* q, int num_qo_heads, const void* pool,
                    state_o + (size_t)P.splits * num_qo_heads * kDecodeHeadDim,
                    state_lse + (size_t)P.splits * num_qo_heads, error_word, stream, 1,
                    (long long)P.states * num_qo_heads * kDecodeHeadDim,
-                   (long long)P.states * num_qo_heads);
+                   (long long)P.states * num_qo_heads, -1, 1.f, 1.f, nullptr, 0, 1, nullptr,
+                   nullptr, nullptr, 0, /*early_table=*/1);
   if (st != PKV_OK) return st;
   // 3. merge the prefix and suffix states of every (request, head)
   pkv::MergeArgs ma;

@@ -209,6 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   umma::fence_after_sync();
   const uint32_t tbase = ctl.tmem_base;
   grid_dependency_wait();
+  // the shared-prefix step (one wave) lets the next launch -- the cascade's
+  // own-page decode, which does not read its output -- start on the SMs it
+  // leaves idle; append attention, whose CTAs come in several waves, does not
+  if (a.prefix_pages != nullptr) grid_dependents_launch();
 
   // ---- this CTA's row block and the keys its rows may see
   const bool prefix = a.prefix_pages != nullptr;

@@ -488,7 +488,12 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
     carry += chunk_total;
   }
   __syncthreads();
-  if (f0 >= f1 || ctl.b0 < 0) return;
+  if (f0 >= f1 || ctl.b0 < 0) {
+    // no work: still wait, so that this launch never completes before the
+    // kernels it depends on (a dependent launch relies on that)
+    if (early) grid_dependency_wait();
+    return;
+  }
 
   const int G = a.group;
 

@@ -108,6 +108,26 @@ def test_cascade_requests_without_own_tokens(N):
     assert_parity(out, lse, ref_o, ref_l, what=f"empty own, N={N}")
 
 
+@pytest.mark.parametrize("N", [0, 3])
+def test_cascade_with_no_own_tokens_at_all(N):
+    """Every request holds only the prefix: the own-page decode has no work, and
+    its CTAs (which read their table before the dependency wait) must still not
+    let the launch complete before the prefix step, whose states the merge
+    reads right after.  A long prefix keeps the prefix step running."""
+    batch = 16
+    full = 128 * 16
+    w = wl.make_workload("cascade-prefix-only", np.full(batch, full), num_qo_heads=32,
+                         num_kv_heads=8, page_size=16, dtype="bf16", seed=62,
+                         shared_prefix_len=full, pool_factor=1.2)
+    prefix, _, ip, ix, ll = wl.cascade_view(w)
+    q, pool, _, _ = wl.make_tensors(w, "cpu")
+    qd, pd = q.cuda(), pool.cuda()
+    ref_o, ref_l = repacked_oracle(w, wl.bits(q), wl.bits(pool), prefix, full, ip, ix, ll)
+    for _ in range(3):
+        out, lse = run_cascade(w, qd, pd, prefix, full, ip, ix, ll, num_partitions=N)
+        assert_parity(out, lse, ref_o, ref_l, what=f"prefix only, N={N}")
+
+
 def test_cascade_equals_decode_on_shared_prefix_workload():
     w = wl.named(5)
     q, pool, _, _ = wl.make_tensors(w, "cuda")
