@@ -103,11 +103,20 @@ static_assert(kMaxStages <= kConsumerWarps * (kQBufs - 1) &&
 // for 48 slots)
 constexpr int kFp8Warps = 12;
 constexpr int kFp8WarpsStages = 36;
+// Short chunks with two column tiles (q_len * G up to 16): twice the MMA work
+// per tile on 168 registers, so again the consumers set the pace; 10 consumer
+// warps (three warps of 168 registers per scheduler still fit) on a 20-slot
+// ring (160 KiB in flight), with 4 staged query blocks to make the room
+constexpr int kChunkWarps = 10;
+constexpr int kChunkWarpsStages = 20;
+constexpr int kChunkQBufs = 4;
 // ring slots of a variant: 16-bit tiles (8 KiB), 8-bit tiles (4 KiB)
 __host__ __device__ constexpr int ring_slots(int gc, bool fp8, int cw) {
-  return !fp8 ? (gc <= 4 ? kStagesNarrow : kStages)
+  return !fp8 ? (cw == kChunkWarps ? kChunkWarpsStages : (gc <= 4 ? kStagesNarrow : kStages))
               : (cw == kFp8Warps ? kFp8WarpsStages : 2 * (gc <= 4 ? kStagesNarrow : kStages));
 }
+// staged query blocks of a variant
+__host__ __device__ constexpr int q_bufs(int cw) { return cw == kChunkWarps ? kChunkQBufs : kQBufs; }
 constexpr int kScratchStride = kD + 4;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -166,11 +175,12 @@ constexpr size_t scratch_bytes(int gc, int cw) {
 }
 constexpr size_t smem_bytes(int nq, int gc, bool fp8 = false, int cw = kConsumerWarps) {
   return 1024 /*alignment slack*/ + (size_t)ring_slots(gc, fp8, cw) * (fp8 ? kSlotBytes / 2 : kSlotBytes) +
-         (size_t)kQBufs * q_buf_bytes(nq, gc) + sizeof(Ctl) + scratch_bytes(gc <= 4 ? 4 : kMaxGroup, cw);
+         (size_t)q_bufs(cw) * q_buf_bytes(nq, gc) + sizeof(Ctl) + scratch_bytes(gc <= 4 ? 4 : kMaxGroup, cw);
 }
 static_assert(smem_bytes(1, 4) <= 227 * 1024 && smem_bytes(1, kMaxGroup) <= 227 * 1024 &&
                   smem_bytes(2, kMaxGroup) <= 227 * 1024 &&
-                  smem_bytes(1, 4, true, kFp8Warps) <= 227 * 1024,
+                  smem_bytes(1, 4, true, kFp8Warps) <= 227 * 1024 &&
+                  smem_bytes(2, kMaxGroup, false, kChunkWarps) <= 227 * 1024,
               "shared memory per CTA");
 
 // output of (request b, query head h): 16-bit final outputs, or fp32 attention
@@ -353,8 +363,12 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeArgs a) {
   constexpr bool FP8 = KV != kKv16;
   constexpr int kThreads = (CW + 1) * 32;  // CW consumer warps, then the producer warp
-  static_assert(CW == kConsumerWarps || (CW == kFp8Warps && FP8 && GC == 4),
-                "12 consumer warps: 8-bit pools, narrow groups");
+  static_assert(CW == kConsumerWarps || (CW == kFp8Warps && FP8 && GC == 4) ||
+                    (CW == kChunkWarps && CHUNK && NQ == 2),
+                "12 consumer warps: 8-bit pools, narrow groups; 10: short chunks, two column tiles");
+  constexpr int kQB = q_bufs(CW);  // staged query blocks (a power of two)
+  static_assert((kQB & (kQB - 1)) == 0 && kQB <= kQBufs && kSegRecs % (2 * kQB) == 0,
+                "query blocks");
   static_assert(CW + 1 <= kMaxWarps, "warp count");
   static_assert(NQ == 1 || (NQ == 2 && !FP8), "two column tiles only for 16-bit pools");
   static_assert(!CHUNK || !FP8, "short chunks only for 16-bit pools");
@@ -371,7 +385,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
   constexpr int kIssue = kSt < 16 ? kSt : 16;
   static_assert(kSt % CW == 0 && 32 % kIssue == 0 && kSt <= kMaxStages,
                 "each ring slot must have a single consumer warp");
-  static_assert(kSt <= CW * (kQBufs - 1) && kSt <= CW * (kSegRecs - 1),
+  static_assert(kSt <= CW * (kQB - 1) && kSt <= CW * (kSegRecs - 1),
                 "a query buffer or segment record could be refilled before every warp read it");
   // MMA operand type: 16-bit pools use their own type; E4M3 codes are widened
   // to fp16 (exact), so those tiles run the fp16 MMA
@@ -381,7 +395,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* ring = smem;
   uint8_t* qbuf = smem + kRingBytes;
-  Ctl& ctl = *reinterpret_cast<Ctl*>(qbuf + (size_t)kQBufs * kQBufBytes);
+  Ctl& ctl = *reinterpret_cast<Ctl*>(qbuf + (size_t)kQB * kQBufBytes);
   Scratch<GC, CW>& scr =
       *reinterpret_cast<Scratch<GC, CW>*>(reinterpret_cast<uint8_t*>(&ctl) + sizeof(Ctl));
 
@@ -398,7 +412,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
       mbar_init(smem_u32(&ctl.empty[s]), 32);
     }
     mbar_init(smem_u32(&ctl.cons), CW * 32);
-    for (int i = 0; i < kQBufs; ++i) mbar_init(smem_u32(&ctl.qfull[i]), 1);
+    for (int i = 0; i < kQB; ++i) mbar_init(smem_u32(&ctl.qfull[i]), 1);
     for (int s = 0; s < kSt; ++s) ctl.last_it[s] = -1;
     for (int k = 0; k < kMaxPending; ++k) {
       ctl.pend_last[k] = 0;
@@ -570,7 +584,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
         r.ncol = q_len * G;
         r.q_row = q_row;
         // stage them (G contiguous rows per token) for the consumers
-        const int qb = seg & (kQBufs - 1);
+        const int qb = seg & (kQB - 1);
         const uint32_t qbar = smem_u32(&ctl.qfull[qb]);
         const uint32_t qbytes = (uint32_t)G * kD * 2;
         mbar_arrive_expect_tx(qbar, qbytes * (uint32_t)q_len);
@@ -699,11 +713,11 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
                global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
-      for (int qb = 0; qb < kQBufs && qb < seg; ++qb) {
-        const int last = seg - 1 - ((seg - 1 - qb) % kQBufs);  // latest segment using qbuf qb
+      for (int qb = 0; qb < kQB && qb < seg; ++qb) {
+        const int last = seg - 1 - ((seg - 1 - qb) % kQB);  // latest segment using qbuf qb
         const uint32_t bar = smem_u32(&ctl.qfull[qb]);
         const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bar, (uint32_t)(last / kQBufs) & 1u) &&
+        while (!mbar_try_wait(bar, (uint32_t)(last / kQB) & 1u) &&
                global_timer_ns() - t0 < kWaitLimitNs) {
         }
       }
@@ -764,8 +778,8 @@ __global__ void __launch_bounds__((CW + 1) * 32, kDecodeCtasPerSm)
         break;
       }
       // the segment's query rows, staged by the producer
-      const int qb = sid & (kQBufs - 1);
-      if (!mbar_wait_bounded(smem_u32(&ctl.qfull[qb]), (uint32_t)(sid / kQBufs) & 1u, &ctl.abort,
+      const int qb = sid & (kQB - 1);
+      if (!mbar_wait_bounded(smem_u32(&ctl.qfull[qb]), (uint32_t)(sid / kQB) & 1u, &ctl.abort,
                              a.err, a.wait_ns)) {
         clean = false;
         break;
@@ -1174,7 +1188,8 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
       decode_kernel<false, kKvE4M3, 1, false, 8>, decode_kernel<true, kKvE4M3, 1, false, 8>,
       decode_kernel<false, kKvE5M2, 1, false, 8>, decode_kernel<true, kKvE5M2, 1, false, 8>,
       decode_kernel<false, kKv16, 1, true, 8>,    decode_kernel<true, kKv16, 1, true, 8>,
-      decode_kernel<false, kKv16, 2, true, 8>,    decode_kernel<true, kKv16, 2, true, 8>,
+      decode_kernel<false, kKv16, 2, true, 8, kChunkWarps>,
+      decode_kernel<true, kKv16, 2, true, 8, kChunkWarps>,
       decode_kernel<false, kKv16, 1, false, 4>,   decode_kernel<true, kKv16, 1, false, 4>,
       decode_kernel<false, kKvE4M3, 1, false, 4, kFp8Warps>,
       decode_kernel<true, kKvE4M3, 1, false, 4, kFp8Warps>,
@@ -1187,7 +1202,7 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const DecodeArgs& a, bool bf1
   const int variant = (chunk ? 4 + 2 * nq : 2 * kv + (narrow ? 10 : 0)) + (bf16 ? 1 : 0);
   const Kern kern = kKerns[variant];
   const bool fp8 = kv != kKv16;
-  const int cw = narrow && fp8 ? kFp8Warps : kConsumerWarps;
+  const int cw = chunk && nq == 2 ? kChunkWarps : narrow && fp8 ? kFp8Warps : kConsumerWarps;
   const size_t smem = smem_bytes(nq, narrow ? 4 : kMaxGroup, fp8, cw);
   cudaError_t e = ensure_smem_opt_in(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;

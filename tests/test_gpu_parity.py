@@ -197,11 +197,12 @@ def test_append_overflow_sets_error_bit():
 
 # ------------------------------------------------------------------ merge
 
-# whole rows through shared memory (S * H a multiple of 4, rows up to 112 KiB),
-# one warp per (row, head) with 16-byte loads (40 states: five batches of 8;
-# 3 x 3 heads), per-dim loads (head_dim 64, 200)
+# whole rows through shared memory (S * H a multiple of 4, rows up to 112 KiB:
+# 5 and 20 states of 8 heads), one warp per (row, head) with 16-byte loads (40
+# states: five batches of 8; 3 x 3 heads), per-dim loads (head_dim 64, 200)
 @pytest.mark.parametrize("out_dtype,S,D,H", [(torch.float32, 5, 128, 8), (torch.bfloat16, 5, 128, 8),
-                                             (torch.float16, 5, 128, 8), (torch.float32, 40, 128, 8),
+                                             (torch.float16, 5, 128, 8), (torch.float32, 20, 128, 8),
+                                             (torch.float32, 40, 128, 8),
                                              (torch.bfloat16, 3, 128, 3), (torch.float32, 3, 64, 8),
                                              (torch.float32, 7, 200, 8)])
 def test_merge_states_matches_oracle(out_dtype, S, D, H):
